@@ -1,0 +1,553 @@
+#!/usr/bin/env python
+"""Benchmark of the paged KV attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one pass of the hot path over one batch: for the default workload
+(Qwen3-0.6B attention shape, 28 layers, batch 64, lengths U[128, 2048]) that
+is, for every layer, the KV store of the 64 new tokens into that layer's pool
+followed by paged decode attention over the page table.  Each layer has its
+own 200k-slot pool, so a step reads ~8 GB of KV: inputs larger than L2, no
+flush needed.  With N GPUs every rank runs its own replica with its own seed
+(weak scaling, no collective on the data path); the reported time is the max
+over ranks.
+
+The JSON line: `value` = algorithmic bytes (K/V rows once per GQA group, q,
+out, page-table entries, plus the store's reads and writes) per step summed
+over ranks / step time, in GB/s; `e2e` = the same through the public API with
+the step's inputs copied from pinned host memory and the outputs copied back
+inside the timed region; `roofline` = the decode kernel pair (split + merge)
+timed with CUDA events inside the timed region against the measured HBM copy
+bandwidth; `cpu_baseline` = the fp64 oracle on this host's cores on a bounded
+sample of the same workload.
+
+--impl reference times the oracle itself (there is no other implementation
+of this path to run) on the same metric, rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+from concurrent.futures import ThreadPoolExecutor
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from paged_kv_attention_mg_b200 import roofline as rf  # noqa: E402
+from paged_kv_attention_mg_b200 import workload as wl  # noqa: E402
+
+METRIC = "paged decode-attention KV GB/s (% of HBM peak) and decode tokens/s, 1 B200"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+KERNEL_SOURCES = ["include/mg.h", "paged_kv_attention_mg_b200/csrc/mg.cu",
+                  "paged_kv_attention_mg_b200/csrc/common.cuh", "paged_kv_attention_mg_b200/csrc/ptx.cuh",
+                  "paged_kv_attention_mg_b200/csrc/store_kv.cuh", "paged_kv_attention_mg_b200/csrc/decode.cuh",
+                  "paged_kv_attention_mg_b200/csrc/extend.cuh"]
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="qwen3_0.6b_decode_28l", choices=sorted(wl.BY_NAME))
+    ap.add_argument("--kv-chunk", type=int, default=0, help="decode keys per split (0 = automatic plan)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="bound of the cpu_baseline sample")
+    ap.add_argument("--soak-seconds", type=float, default=1.5,
+                    help="extra untimed warm-up so the clock sampler sees the GPU under load")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------- plumbing
+
+class Dist:
+    def __init__(self, want: int):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        if want != self.world:
+            raise SystemExit(f"--gpus {want} but WORLD_SIZE={self.world}: launch N>1 with torchrun")
+        self.pg = None
+        if self.world > 1:
+            import torch.distributed as dist
+            torch.cuda.set_device(self.local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
+                                    device_id=torch.device("cuda", self.local))
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg:
+            self.pg.barrier()
+
+    def max(self, x: float) -> float:
+        if not self.pg:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def sum(self, x: float) -> float:
+        if not self.pg:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.SUM)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            self.pg.barrier()
+            self.pg.destroy_process_group()
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            m = json.load(f)
+        return float(m["hbm_gbs"]), float(m["bf16_tflops"]), float(m.get("bf16_tflops_sustained", 0)), "measured"
+    return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+def source_digest() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch of the dominant kernel from a committed ncu summary,
+    or None if there is none or the kernels changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        entries = json.load(f)
+    e = entries.get(workload)
+    if not e or e.get("source_digest") != source_digest():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.proc = None
+        sel = []
+        try:
+            bus = torch.cuda.get_device_properties(device_index).pci_bus_id
+            sel = ["-i", f"{torch.cuda.get_device_properties(device_index).pci_domain_id:08x}:{bus:02x}:"
+                   f"{torch.cuda.get_device_properties(device_index).pci_device_id:02x}.0"]
+        except Exception:
+            sel = []
+        self.sel = sel
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", *self.sel, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.file, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.file.flush()
+        self.file.seek(0)
+        rows = [ln.strip().split(",") for ln in self.file.read().splitlines() if ln.strip()]
+        os.unlink(self.file.name)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [x.strip() for x in r]
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, r[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- workloads
+
+def rank_spec(spec, rank: int):
+    return dataclasses.replace(spec, seed=spec.seed + 7919 * rank) if rank else spec
+
+
+def make_layers(step, num_layers, device):
+    """Per-layer device tensors.  Host generation runs on a thread pool (each
+    layer has its own generator, so the result does not depend on threading)."""
+    def one(layer):
+        data = wl.make_layer(step, layer)
+        k = wl.build_pool(step, data.hist_slots, data.k_hist, device)
+        v = wl.build_pool(step, data.hist_slots, data.v_hist, device)
+        return dict(q=data.q.to(device), k_new=data.k_new.to(device), v_new=data.v_new.to(device),
+                    k_cache=k, v_cache=v, q_host=data.q.pin_memory(), k_new_host=data.k_new.pin_memory(),
+                    v_new_host=data.v_new.pin_memory())
+    with ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
+        return list(ex.map(one, range(num_layers)))
+
+
+class DecodeBench:
+    def __init__(self, spec, step, device, kv_chunk):
+        from paged_kv_attention_mg_b200 import mg
+        self.mg = mg
+        self.spec, self.step, self.device = spec, step, device
+        self.layers = make_layers(step, spec.num_layers, device)
+        self.meta = {n: getattr(step, n).to(device) for n in ("page_table", "table_idx", "seq_len", "out_loc")}
+        self.meta_host = {n: getattr(step, n).pin_memory() for n in ("page_table", "table_idx", "seq_len",
+                                                                      "out_loc")}
+        self.max_seq_len = step.max_seq_len
+        self.kv_chunk = kv_chunk
+        B, hq, hkv = step.batch, spec.num_q_heads, spec.num_kv_heads
+        self.chunk, self.num_splits = mg.decode_plan(B, hkv, self.max_seq_len, kv_chunk)
+        ws = mg.decode_workspace_bytes(B, hq, hkv, self.max_seq_len, kv_chunk)
+        self.workspace = torch.empty(max(ws, 16), dtype=torch.uint8, device=device)
+        self.outs = [torch.empty((B, hq, spec.head_dim), dtype=torch.bfloat16, device=device)
+                     for _ in range(spec.num_layers)]
+        self.outs_host = [torch.empty_like(o, device="cpu").pin_memory() for o in self.outs]
+        L = step.seq_len.tolist()
+        self.decode_bytes = rf.decode_bytes(L, hq, hkv, spec.head_dim)
+        self.store_bytes = rf.store_bytes(step.num_new_tokens, hkv, spec.head_dim)
+        self.step_bytes = spec.num_layers * (self.decode_bytes + self.store_bytes)
+        self.tokens_per_step = B
+        self.launches_per_step = spec.num_layers * (2 + (1 if self.num_splits > 1 else 0))
+        self.h2d_bytes = sum(t.numel() * t.element_size() for t in self.meta_host.values()) + spec.num_layers * (
+            self.layers[0]["q"].numel() * 2 + 2 * self.layers[0]["k_new"].numel() * 2)
+        self.d2h_bytes = sum(o.numel() * 2 for o in self.outs)
+        self.ev = None
+
+    def layer(self, lay, out, meta, events=None):
+        mg = self.mg
+        mg.store_kv(lay["k_new"], lay["v_new"], meta["out_loc"], lay["k_cache"], lay["v_cache"])
+        if events:
+            events[0].record()
+        mg.decode_attn(lay["q"], lay["k_cache"], lay["v_cache"], meta["page_table"], meta["table_idx"],
+                       meta["seq_len"], self.max_seq_len, self.spec.scale, kv_chunk=self.kv_chunk, out=out,
+                       workspace=self.workspace)
+        if events:
+            events[1].record()
+
+    def run_step(self, events=None):
+        for i, lay in enumerate(self.layers):
+            self.layer(lay, self.outs[i], self.meta, events[i] if events else None)
+
+    def make_events(self):
+        return [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in self.layers]
+
+    def run_step_e2e(self):
+        """Inputs from pinned host memory, outputs back to pinned host memory."""
+        for n, t in self.meta_host.items():
+            self.meta[n].copy_(t, non_blocking=True)
+        for i, lay in enumerate(self.layers):
+            lay["q"].copy_(lay["q_host"], non_blocking=True)
+            lay["k_new"].copy_(lay["k_new_host"], non_blocking=True)
+            lay["v_new"].copy_(lay["v_new_host"], non_blocking=True)
+            self.layer(lay, self.outs[i], self.meta)
+            self.outs_host[i].copy_(self.outs[i], non_blocking=True)
+
+    def kernel_bytes(self):
+        return self.decode_bytes
+
+    def describe(self):
+        s, st = self.spec, self.step
+        return {"workload": s.name, "batch": st.batch, "layers": s.num_layers, "q_heads": s.num_q_heads,
+                "kv_heads": s.num_kv_heads, "head_dim": s.head_dim, "pool_slots": s.num_slots,
+                "mean_seq_len": round(float(st.seq_len.double().mean()), 1), "max_seq_len": st.max_seq_len,
+                "kv_chunk": self.chunk, "num_splits": self.num_splits,
+                "l2": f"inputs larger than L2: {s.num_layers} per-layer pools, "
+                      f"{self.spec.num_layers * self.decode_bytes / 1e9:.2f} GB read per step"}
+
+
+class ExtendBench:
+    def __init__(self, spec, step, device, kv_chunk):
+        from paged_kv_attention_mg_b200 import mg
+        self.mg = mg
+        self.spec, self.step, self.device = spec, step, device
+        self.layers = make_layers(step, spec.num_layers, device)
+        names = ("page_table", "table_idx", "seq_len", "cached_len", "q_offset", "out_loc")
+        self.meta = {n: getattr(step, n).to(device) for n in names}
+        self.meta_host = {n: getattr(step, n).pin_memory() for n in names}
+        self.outs = [torch.empty_like(lay["q"]) for lay in self.layers]
+        self.outs_host = [torch.empty_like(o, device="cpu").pin_memory() for o in self.outs]
+        c, s = step.cached_len.tolist(), step.seq_len.tolist()
+        self.flops = rf.extend_flops(c, s, spec.num_q_heads, spec.head_dim)
+        self.extend_bytes = rf.extend_bytes(c, s, spec.num_q_heads, spec.num_kv_heads, spec.head_dim)
+        self.store_bytes = rf.store_bytes(step.num_new_tokens, spec.num_kv_heads, spec.head_dim)
+        self.tokens_per_step = step.num_new_tokens
+        self.launches_per_step = spec.num_layers * 2
+        self.h2d_bytes = sum(t.numel() * t.element_size() for t in self.meta_host.values()) + spec.num_layers * (
+            self.layers[0]["q"].numel() * 2 + 2 * self.layers[0]["k_new"].numel() * 2)
+        self.d2h_bytes = sum(o.numel() * 2 for o in self.outs)
+        self.chunk = self.num_splits = None
+
+    def layer(self, lay, out, meta, events=None):
+        mg, st = self.mg, self.step
+        mg.store_kv(lay["k_new"], lay["v_new"], meta["out_loc"], lay["k_cache"], lay["v_cache"])
+        if events:
+            events[0].record()
+        mg.extend_attn(lay["q"], lay["k_cache"], lay["v_cache"], meta["page_table"], meta["table_idx"],
+                       meta["cached_len"], meta["seq_len"], meta["q_offset"], st.max_q_len, st.max_seq_len,
+                       self.spec.scale, out=out)
+        if events:
+            events[1].record()
+
+    run_step = DecodeBench.run_step
+    make_events = DecodeBench.make_events
+    run_step_e2e = DecodeBench.run_step_e2e
+
+    def describe(self):
+        s, st = self.spec, self.step
+        n = (st.seq_len - st.cached_len)
+        return {"workload": s.name, "batch": st.batch, "layers": s.num_layers, "q_heads": s.num_q_heads,
+                "kv_heads": s.num_kv_heads, "head_dim": s.head_dim, "pool_slots": s.num_slots,
+                "new_tokens": int(n.sum()), "mean_cached_len": round(float(st.cached_len.double().mean()), 1),
+                "l2": "L2 flushed between timed steps (256 MB write)"}
+
+
+# ----------------------------------------------------------------------------- cpu baseline
+
+def oracle_sample(spec, step, seconds: float, threads: int, layers_from: int = 0):
+    """Run the oracle on whole layers of the workload (decode) or on requests
+    (extend) until `seconds` of wall time are spent; returns (bytes_or_flops, time, sample, kind)."""
+    import oracle
+    done_units, total_t = 0, 0.0
+    work, sample = 0, []
+    if spec.kind == "decode":
+        L = step.seq_len.tolist()
+        per_layer = rf.decode_bytes(L, spec.num_q_heads, spec.num_kv_heads, spec.head_dim)
+        for layer in range(layers_from, layers_from + spec.num_layers):
+            data = wl.make_layer(step, layer % spec.num_layers)
+            k = wl.build_pool(step, data.hist_slots, data.k_hist)
+            v = wl.build_pool(step, data.hist_slots, data.v_hist)
+            loc = step.out_loc.to(torch.int64)
+            k.index_copy_(0, loc, data.k_new)
+            v.index_copy_(0, loc, data.v_new)
+            args = (wl.bits(data.q), wl.bits(k), wl.bits(v), step.page_table.numpy(), step.table_idx.numpy(),
+                    step.seq_len.numpy())
+            t0 = time.perf_counter()
+            oracle.decode(*args, spec.scale, threads=threads)
+            total_t += time.perf_counter() - t0
+            work += per_layer
+            done_units += 1
+            if total_t >= seconds:
+                break
+        return work, total_t, f"{done_units} of {spec.num_layers} layers, all {step.batch} requests", "GB/s"
+    # extend: whole requests until the time bound
+    data = wl.make_layer(step, layers_from)
+    k = wl.build_pool(step, data.hist_slots, data.k_hist)
+    v = wl.build_pool(step, data.hist_slots, data.v_hist)
+    loc = step.out_loc.to(torch.int64)
+    k.index_copy_(0, loc, data.k_new)
+    v.index_copy_(0, loc, data.v_new)
+    c, s = step.cached_len.tolist(), step.seq_len.tolist()
+    for r in range(step.batch):
+        t0 = time.perf_counter()
+        oracle.extend(wl.bits(data.q), wl.bits(k), wl.bits(v), step.page_table.numpy(), step.table_idx.numpy(),
+                      step.cached_len.numpy(), step.seq_len.numpy(), step.q_offset.numpy(), spec.scale,
+                      requests=[r], threads=threads)
+        total_t += time.perf_counter() - t0
+        work += rf.extend_flops([c[r]], [s[r]], spec.num_q_heads, spec.head_dim)
+        done_units += 1
+        if total_t >= seconds:
+            break
+    return work, total_t, f"{done_units} of {step.batch} requests of one layer", "TFLOP/s"
+
+
+def cpu_threads():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# ----------------------------------------------------------------------------- arms
+
+def run_reference(args):
+    """The oracle as the reference arm: rank 0 only, on the host cores."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    spec = wl.BY_NAME[args.workload]
+    step = wl.make_step(spec)
+    threads = cpu_threads()
+    per_step_seconds = max(0.5, min(6.0, 150.0 / max(1, args.steps + args.warmup)))
+    for i in range(args.warmup):
+        oracle_sample(spec, step, per_step_seconds, threads, layers_from=i)
+    work, secs = 0, 0.0
+    sample = unit = None
+    for i in range(args.steps):
+        w, t, sample, unit = oracle_sample(spec, step, per_step_seconds, threads, layers_from=i)
+        work += w
+        secs += t
+    value = (work / secs / 1e9) if unit == "GB/s" else (work / secs / 1e12)
+    line = {"impl": "reference", "metric": METRIC if spec.kind == "decode" else "extend attention TFLOP/s",
+            "value": round(value, 4), "unit": unit, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(1e3 * secs / args.steps, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": spec.name, "parallelism": "host cores (oracle)"},
+            "cpu_baseline": {"value": round(value, 4), "unit": unit, "cores": threads, "kind": "oracle",
+                             "sample": f"per step: {sample}"},
+            "e2e": {"value": round(value, 4), "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args):
+    dist = Dist(args.gpus)
+    device = torch.device("cuda", dist.local)
+    torch.cuda.set_device(device)
+    spec = rank_spec(wl.BY_NAME[args.workload], dist.rank)
+    step = wl.make_step(spec)
+    bench = (DecodeBench if spec.kind == "decode" else ExtendBench)(spec, step, device, args.kv_chunk)
+    flush = None
+    if spec.kind == "extend":
+        flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(dist.local)
+    sampler.start()
+    # warm-up (W steps) plus a short soak so clocks are sampled under load
+    for _ in range(max(3, args.warmup)):
+        bench.run_step()
+    torch.cuda.synchronize()
+    t_end = time.perf_counter() + args.soak_seconds
+    while time.perf_counter() < t_end:
+        bench.run_step()
+        torch.cuda.synchronize()
+
+    events = [bench.make_events() for _ in range(args.steps)]
+    flush_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                    for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    flush_ms = 0.0
+    dist.barrier()
+    torch.cuda.synchronize()
+    start.record()
+    for k in range(args.steps):
+        if flush is not None:
+            flush_events[k][0].record()
+            flush.fill_(k & 0xFF)
+            flush_events[k][1].record()
+        bench.run_step(events[k])
+    stop.record()
+    torch.cuda.synchronize()
+    dist.barrier()
+    clocks = sampler.stop()
+    total_ms = start.elapsed_time(stop)
+    if flush is not None:
+        flush_ms = sum(a.elapsed_time(b) for a, b in flush_events)
+    step_ms_local = (total_ms - flush_ms) / args.steps
+    kernel_ms_local = sum(a.elapsed_time(b) for ev in events for (a, b) in ev) / (
+        args.steps * spec.num_layers)
+    step_ms = dist.max(step_ms_local)
+    kernel_ms = dist.max(kernel_ms_local)
+
+    # end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        for _ in range(2):
+            bench.run_step_e2e()
+        torch.cuda.synchronize()
+        dist.barrier()
+        ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e2e_steps = max(3, min(args.steps, 20))
+        ea.record()
+        for _ in range(e2e_steps):
+            bench.run_step_e2e()
+        eb.record()
+        torch.cuda.synchronize()
+        e2e_ms = dist.max(ea.elapsed_time(eb) / e2e_steps)
+        e2e = e2e_ms
+
+    hbm, tflops, tflops_sus, peak_src = measured_peaks()
+    n = args.gpus
+    if spec.kind == "decode":
+        value = n * bench.step_bytes / (step_ms * 1e-3) / 1e9
+        unit = "GB/s"
+        metric = METRIC
+        achieved = bench.decode_bytes / (kernel_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "kernel": "decode_split_kernel + decode_merge_kernel (one mg_decode_attn call)",
+                "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s", "frac": round(achieved / hbm, 4),
+                "peak_source": f"{peak_src} HBM copy bandwidth",
+                "traffic": profiled_traffic(spec.name)}
+        extra = {"tokens_per_s": round(n * bench.tokens_per_step / (step_ms * 1e-3), 1),
+                 "frac_of_8tbs_nominal": round(value / n / 8000.0, 4),
+                 "frac_of_measured_hbm": round(value / n / hbm, 4)}
+    else:
+        value = n * bench.flops / (step_ms * 1e-3) / 1e12
+        unit = "TFLOP/s"
+        metric = "chunked-prefill extend attention TFLOP/s (unmasked QK^T + PV flops), 1 B200"
+        achieved = bench.flops / (kernel_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "kernel": "extend_kernel", "achieved": round(achieved, 1), "peak": tflops,
+                "unit": "TFLOP/s", "frac": round(achieved / tflops, 4),
+                "peak_source": f"{peak_src} dense bf16 (burst)", "traffic": profiled_traffic(spec.name)}
+        extra = {"tokens_per_s": round(n * bench.tokens_per_step / (step_ms * 1e-3), 1),
+                 "frac_of_sustained_bf16": round(achieved / tflops_sus, 4) if tflops_sus else None}
+
+    cpu = None
+    if dist.rank == 0 and n == 1 and not args.no_cpu_baseline:
+        threads = cpu_threads()
+        w, secs, sample, cunit = oracle_sample(spec, step, args.cpu_seconds, threads)
+        cval = w / secs / (1e9 if cunit == "GB/s" else 1e12)
+        cpu = {"value": round(cval, 4), "unit": cunit, "cores": threads, "kind": "oracle",
+               "sample": sample, "seconds": round(secs, 2)}
+
+    if dist.rank == 0:
+        cfg = bench.describe()
+        cfg["parallelism"] = f"dp{n} (independent replicas, no collective)" if n > 1 else "single GPU"
+        line = {"metric": metric, "value": round(value, 2), "unit": unit, "n_gpus": n, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": round(step_ms, 4), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg,
+                **extra, "roofline": roof, "cpu_baseline": cpu,
+                "e2e": ({"value": round(n * (bench.step_bytes / 1e9 if spec.kind == 'decode' else bench.flops / 1e12)
+                                       / (e2e * 1e-3), 2),
+                         "unit": unit, "ms_per_step": round(e2e, 4), "h2d_bytes_per_step": bench.h2d_bytes,
+                         "d2h_bytes_per_step": bench.d2h_bytes} if e2e else None),
+                "gpu_launches": bench.launches_per_step * args.steps, "clocks": clocks,
+                "kernel_source_digest": source_digest()}
+        print(json.dumps(line), flush=True)
+    dist.close()
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

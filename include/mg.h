@@ -1,0 +1,188 @@
+/*
+ * mg.h -- C ABI of the B200 (sm_100a) paged KV attention library (libmg.so).
+ *
+ * Three operations make up the per-layer attention hot path of the
+ * mini-sglang engine, in the order the engine runs them (Mini-SGLang tag
+ * page, Engine post, §一 "GPU inference is not only matrix multiplication":
+ * ... RoPE -> write KV cache -> attention -> o_proj):
+ *
+ *   mg_store_kv     write the new tokens' K/V into pool slots at out_loc;
+ *   mg_decode_attn  one query token per request against its paged history
+ *                   (split-KV kernel + merge kernel);
+ *   mg_extend_attn  a chunk of new tokens per request (chunked prefill),
+ *                   causal over cached_len + i, on tcgen05 tensor cores.
+ *
+ * Data structures ("手写 mini-sglang 阶段一 · Engine 与采样器" (Stage 1, Engine and
+ * sampler), §初始化的顺序 and §手工驱动引擎):
+ *   - KV pool, per layer, K and V separately: [num_slots, num_kv_heads, head_dim]
+ *     bf16, row-major.  This is the engine's [pages, page_size, heads, dim]
+ *     pool flattened with page_size 1, so a page-table entry is a slot.
+ *   - page_table: int32 [page_table_rows, page_table_stride], row-major.  Row
+ *     table_idx[r] holds the slot of every token of request r, position 0 first.
+ *   - a request has cached_len tokens already in the pool and seq_len tokens
+ *     after this step (seq_len is the engine's device_len); its new tokens sit
+ *     at positions cached_len .. seq_len-1.
+ *   - q head h reads KV head h / (num_q_heads / num_kv_heads) (grouped-query
+ *     attention with consecutive q heads sharing a KV head).
+ *
+ * Conventions for every entry point:
+ *   - Pointers named as tensors are DEVICE pointers (the current CUDA device);
+ *     bf16 data is passed as void*.  Every tensor is dense and row-major, and
+ *     every bf16 tensor must start on a 16-byte boundary.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  All work is
+ *     enqueued on it; no entry point synchronises the host, allocates device
+ *     memory or keeps state between calls, so calls can be captured in a CUDA
+ *     graph (mg_read_device_error excepted, which synchronises).
+ *   - The caller owns every buffer.  Inputs are read-only except the pools
+ *     in mg_store_kv; outputs are written in full for every real (request,
+ *     head) row.
+ *   - Errors found on the host (null pointer, bad size, unsupported shape,
+ *     misalignment, workspace too small) return a status BEFORE anything is
+ *     launched.  A failed launch returns MG_ERR_CUDA.  Metadata that can only
+ *     be checked on the device (a slot outside the pool, a page-table row
+ *     outside the table, a length beyond the page-table width or the
+ *     max_seq_len hint) never makes a kernel read or write out of bounds: the
+ *     offending token or request is skipped, a bit is set in a device error
+ *     word, and mg_read_device_error reports it.
+ */
+#ifndef MG_H
+#define MG_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum mg_status {
+    MG_OK = 0,
+    MG_ERR_INVALID_ARGUMENT = 1,    /* null pointer, negative or zero size, bad hint */
+    MG_ERR_UNSUPPORTED_SHAPE = 2,   /* head_dim != 128, Hq % Hkv != 0, group > 16 */
+    MG_ERR_MISALIGNED = 3,          /* a bf16 tensor not on a 16-byte boundary */
+    MG_ERR_WORKSPACE_TOO_SMALL = 4, /* decode workspace below mg_decode_workspace_bytes */
+    MG_ERR_CUDA = 5,                /* a CUDA runtime call or launch failed */
+    MG_ERR_DEVICE_CHECK = 6,        /* device-side metadata check failed (see bits) */
+    MG_ERR_DEVICE_TIMEOUT = 7       /* a bounded device wait gave up (see bits) */
+} mg_status;
+
+/* Bits of the device error word (mg_read_device_error). */
+#define MG_DEVERR_SLOT_RANGE 0x1u    /* a slot (out_loc or page-table entry) outside [0, num_slots) */
+#define MG_DEVERR_ROW_RANGE 0x2u     /* table_idx outside [0, page_table_rows) */
+#define MG_DEVERR_LENGTH 0x4u        /* seq_len / cached_len / q_offset inconsistent or beyond hints */
+#define MG_DEVERR_WAIT_TIMEOUT 0x8u  /* a pipeline wait exceeded its iteration limit */
+
+/* Human-readable name of a status. Never NULL. */
+const char *mg_status_string(mg_status status);
+
+/* ABI version: bumped on any incompatible change of a signature below. */
+int32_t mg_abi_version(void);
+
+/*
+ * mg_store_kv -- KV write (the engine's "write KV cache" step; the custom
+ * kernel of "mini-sglang from Scratch Stage 4 · Faster and bigger", §What each
+ * chapter adds, "launch overhead and memory traffic of small operations such
+ * as KV writes").
+ *
+ *   k_cache[out_loc[t], h, :] = k[t, h, :]   and   v_cache[out_loc[t], h, :] = v[t, h, :]
+ *   for t < num_tokens, h < num_kv_heads.  A bit copy.
+ *
+ *   k, v          [num_tokens, num_kv_heads, head_dim] bf16 (the new tokens,
+ *                 concatenated in request order)
+ *   out_loc       [num_tokens] int32 slots = page_table[table_idx[r], cached_len:seq_len]
+ *   k_cache/v_cache [num_slots, num_kv_heads, head_dim] bf16, updated in place
+ * num_tokens == 0 is a no-op.  Slots must be distinct except for a dummy slot
+ * that padded requests share (which write lands there is unspecified).  A slot
+ * outside [0, num_slots) is skipped and sets MG_DEVERR_SLOT_RANGE.
+ * head_dim * num_kv_heads * 2 must be a multiple of 16 bytes.
+ */
+mg_status mg_store_kv(const void *k, const void *v, const int32_t *out_loc, int32_t num_tokens,
+                      void *k_cache, void *v_cache, int64_t num_slots, int32_t num_kv_heads,
+                      int32_t head_dim, void *stream);
+
+/*
+ * mg_decode_plan -- the host-side plan of mg_decode_attn (the role FlashInfer's
+ * "plan" step plays, Stage 4 page, §Checkpoint): keys per split (`chunk`, a
+ * multiple of 64) and the number of splits of the longest request.
+ * kv_chunk > 0 forces that chunk (rounded up to a multiple of 64); kv_chunk == 0
+ * picks one from batch x num_kv_heads x max_seq_len and the SM count of the
+ * current device.  The plan depends only on these arguments, so a captured
+ * launch stays valid for any batch whose lengths stay <= max_seq_len.
+ */
+mg_status mg_decode_plan(int32_t batch, int32_t num_kv_heads, int32_t max_seq_len,
+                         int32_t kv_chunk, int32_t *chunk_out, int32_t *num_splits_out);
+
+/* Bytes of workspace mg_decode_attn needs for this plan (0 when one split). */
+size_t mg_decode_workspace_bytes(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+                                 int32_t head_dim, int32_t max_seq_len, int32_t kv_chunk);
+
+/*
+ * mg_decode_attn -- paged decode attention, one query token per request
+ * (Mini-SGLang tag page, KV Cache post §一: at step t the query attends to
+ * positions 0..t; Stage 1 page §手工驱动引擎 for the metadata).
+ *
+ *   for request r with L = seq_len[r], row = page_table[table_idx[r]], q head h,
+ *   kv head kh = h / (Hq / Hkv):
+ *     x_j = scale * <q[r, h, :], k_cache[row[j], kh, :]>,  j = 0 .. L-1
+ *     out[r, h, :] = sum_j softmax(x)_j * v_cache[row[j], kh, :]
+ *   The new token (position L-1) must already be stored (mg_store_kv).
+ *
+ *   q, out        [batch, num_q_heads, head_dim] bf16 (out rounded from fp32, RNE)
+ *   page_table    [page_table_rows, page_table_stride] int32
+ *   table_idx, seq_len  [batch] int32, 1 <= seq_len[r] <= min(max_seq_len, stride)
+ *   max_seq_len   host-side upper bound of seq_len (sizes the split grid)
+ *   kv_chunk      0 = automatic split plan; > 0 forces keys per split
+ *   workspace     device buffer of >= mg_decode_workspace_bytes(...) bytes,
+ *                 16-byte aligned; may be NULL when that is 0.  Contents on
+ *                 entry do not matter; they are scratch for the split partials.
+ * Supported: head_dim == 128, num_q_heads % num_kv_heads == 0, group <= 16.
+ */
+mg_status mg_decode_attn(const void *q, const void *k_cache, const void *v_cache, int64_t num_slots,
+                         const int32_t *page_table, int32_t page_table_rows,
+                         int32_t page_table_stride, const int32_t *table_idx,
+                         const int32_t *seq_len, int32_t batch, int32_t max_seq_len,
+                         int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, float scale,
+                         int32_t kv_chunk, void *out, void *workspace, size_t workspace_bytes,
+                         void *stream);
+
+/*
+ * mg_extend_attn -- chunked-prefill ("extend") attention over the paged pool
+ * (Stage 1 page §手工驱动引擎: positions = arange(cached_len, device_len), new
+ * tokens concatenated in request order; Mini-SGLang tag page, Scheduler post:
+ * chunked prefill).  The chunk's K/V must already be stored (mg_store_kv).
+ *
+ *   for request r: c = cached_len[r], n = seq_len[r] - c, new token i < n is
+ *   query row t = q_offset[r] + i, at position c + i, and attends to the keys at
+ *   positions 0 .. c + i of its page-table row:
+ *     out[t, h, :] = sum_{j <= c+i} softmax_j(scale * <q[t, h], k[row[j], kh]>) v[row[j], kh]
+ *
+ *   q, out        [total_q, num_q_heads, head_dim] bf16
+ *   cached_len, seq_len [batch] int32; q_offset [batch + 1] int32 prefix sums of
+ *                 n (q_offset[0] = 0, q_offset[batch] = total_q)
+ *   max_q_len     host bound of n;  max_seq_len  host bound of seq_len
+ * Requests with n == 0 are allowed and produce no rows.  Same shape limits as
+ * decode; needs no workspace.
+ */
+mg_status mg_extend_attn(const void *q, const void *k_cache, const void *v_cache, int64_t num_slots,
+                         const int32_t *page_table, int32_t page_table_rows,
+                         int32_t page_table_stride, const int32_t *table_idx,
+                         const int32_t *cached_len, const int32_t *seq_len,
+                         const int32_t *q_offset, int32_t batch, int32_t total_q,
+                         int32_t max_q_len, int32_t max_seq_len, int32_t num_q_heads,
+                         int32_t num_kv_heads, int32_t head_dim, float scale, void *out,
+                         void *stream);
+
+/*
+ * mg_read_device_error -- synchronise `stream`, return the device error word
+ * accumulated since the last call on this device (bits MG_DEVERR_*) in
+ * *bits_out (may be NULL), and clear it.  Returns MG_OK when no bit was set,
+ * MG_ERR_DEVICE_TIMEOUT if MG_DEVERR_WAIT_TIMEOUT is set, else
+ * MG_ERR_DEVICE_CHECK.  Not capturable (it synchronises).
+ */
+mg_status mg_read_device_error(void *stream, uint32_t *bits_out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MG_H */

@@ -1,0 +1,478 @@
+// extend.cuh -- chunked-prefill ("extend") attention on tcgen05 tensor cores.
+//
+// What it computes ("手写 mini-sglang 阶段一 · Engine 与采样器", §手工驱动引擎;
+// Mini-SGLang tag page, Scheduler post, chunked prefill): request r has
+// c = cached_len[r] tokens in the pool and n = seq_len[r] - c new ones, already
+// stored; new token i (query row q_offset[r] + i, position c + i) attends to the
+// keys at positions 0 .. c + i of its page-table row.
+//
+// Work decomposition (B200 design):
+//   * one CTA per (q block, kv head, request).  A q block is two 128-row Q
+//     tiles; a row is (token, head) with the g heads that share the KV head
+//     adjacent, so one K/V tile feeds 2 x 128 query rows (GQA packing).
+//   * warp 0 loads: Q tiles with 3-D TMA, K and V tiles (128 keys each) with
+//     TMA tile::gather4 straight from the paged pool (4 page-table rows per
+//     instruction, 128-byte swizzle), double-buffered behind mbarriers.
+//   * warp 1, one thread: issues tcgen05.mma (M=128, N=128, K=16, bf16 in,
+//     fp32 accumulate in TMEM).  S_t = Q_t K^T lands in TMEM; P_t (bf16) is
+//     written back over S_t and consumed straight from TMEM as the A operand
+//     of O_t += P_t V.  The two Q tiles ping-pong so the tensor core works on
+//     one tile while the softmax warps work on the other.
+//   * warps 2-5 / 6-9: softmax for Q tile 0 / 1, one TMEM lane (= one query
+//     row) per thread: causal mask key <= c + i, online softmax in the exp2
+//     domain, O rescaled in TMEM only when the running max grows by more than
+//     2^8 (exact: the same stale max is used for P and for the row sum),
+//     epilogue O / l -> bf16 -> global.
+// TMEM: S0 [0,128)  S1 [128,256)  O0 [256,384)  O1 [384,512) columns.
+#pragma once
+
+#include <cuda.h>
+
+#include "common.cuh"
+
+namespace mg {
+namespace extend {
+
+constexpr int kM = 128;                     // query rows per Q tile
+constexpr int kN = 128;                     // keys per KV tile
+constexpr int kQTiles = 2;
+constexpr int kStages = 2;
+constexpr int kThreads = 320;               // 10 warps
+constexpr int kHalfBytes = 128 * 128;       // 128 rows x 128 B (64 bf16): one swizzle column
+constexpr int kTileBytes = 2 * kHalfBytes;  // 128 rows x 256 B
+constexpr int kTmemCols = 512;
+__device__ __forceinline__ uint32_t col_s(int t) { return (uint32_t)t * 128u; }
+__device__ __forceinline__ uint32_t col_o(int t) { return 256u + (uint32_t)t * 128u; }
+constexpr float kRescaleThreshold = 8.0f;   // log2 units
+
+// shared memory map (offsets from a 1024-byte aligned base)
+constexpr int kOffQ = 0;
+constexpr int kOffK = kOffQ + kQTiles * kTileBytes;
+constexpr int kOffV = kOffK + kStages * kTileBytes;
+constexpr int kOffBar = kOffV + kStages * kTileBytes;
+constexpr int kNumBars = 1 + 3 * kStages + 3 * kQTiles;
+constexpr int kOffMisc = kOffBar + kNumBars * 8;
+constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
+
+struct Params {
+    const __nv_bfloat16 *q;
+    const __nv_bfloat16 *k_cache;
+    const __nv_bfloat16 *v_cache;
+    const int32_t *page_table;
+    const int32_t *table_idx;
+    const int32_t *cached_len;
+    const int32_t *seq_len;
+    const int32_t *q_offset;
+    __nv_bfloat16 *out;
+    int64_t num_slots;
+    int32_t pt_rows, pt_stride;
+    int32_t batch, total_q, max_q_len, max_seq_len;
+    int32_t num_q_heads, num_kv_heads, group;
+    int32_t tokens_per_qtile;  // floor(128 / group)
+    float scale_log2;
+};
+
+// UMMA shared-memory descriptor, 128-byte swizzle, sm_100 version bits.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;  // descriptor version (Blackwell)
+    d |= (uint64_t)2 << 61;  // SWIZZLE_128B
+    return d;
+}
+
+// Instruction descriptor, kind::f16: bf16 x bf16 -> f32, M = 128, N = 128.
+__host__ __device__ constexpr uint32_t idesc_bf16(bool b_mn_major) {
+    return (1u << 4)                         // D format f32
+           | (1u << 7)                       // A bf16
+           | (1u << 10)                      // B bf16
+           | ((b_mn_major ? 1u : 0u) << 16)  // B major
+           | ((uint32_t)(kN >> 3) << 17)     // N / 8
+           | ((uint32_t)(kM >> 4) << 24);    // M / 16
+}
+
+struct Sync {
+    uint32_t q_full;
+    uint32_t k_full[kStages], v_full[kStages], kv_empty[kStages];
+    uint32_t s_full[kQTiles], p_full[kQTiles], o_done[kQTiles];
+};
+
+// Waits with a time bound; on timeout records the error, raises the CTA abort
+// flag and returns false.  Once the flag is up every later wait returns false
+// at once, so all roles drain to the final barrier.
+__device__ __forceinline__ bool wait_or_abort_thread(uint32_t bar, uint32_t parity, volatile int *abort_flag) {
+    if (*abort_flag) return false;
+    uint64_t t0 = 0;
+    for (uint32_t it = 0;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 1023u) == 1023u) {
+            uint64_t now;
+            asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(now));
+            if (t0 == 0) t0 = now;
+            else if (now - t0 > 2000000000ull || *abort_flag) {  // 2 s
+                *abort_flag = 1;
+                atomicOr(&g_mg_device_error, MG_DEVERR_WAIT_TIMEOUT);
+                return false;
+            }
+        }
+    }
+}
+
+// Warp-uniform form: every lane waits, and the warp proceeds only if all did
+// (tcgen05.ld/st and __syncwarp need the whole warp to stay converged).
+__device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, volatile int *abort_flag) {
+    const bool ok = wait_or_abort_thread(bar, parity, abort_flag);
+    return __all_sync(0xffffffffu, ok);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    extend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffMisc);
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + kOffMisc + 4);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int r = blockIdx.z, kvh = blockIdx.y;
+    const int qb = gridDim.x - 1 - blockIdx.x;  // heaviest (latest) q blocks first
+
+    // ---- request metadata (uniform across the CTA; exit before any barrier)
+    const int row = __ldg(p.table_idx + r);
+    const int c = __ldg(p.cached_len + r);
+    const int L = __ldg(p.seq_len + r);
+    const int qo = __ldg(p.q_offset + r);
+    const int n = L - c;
+    {
+        unsigned bad = 0;
+        if (row < 0 || row >= p.pt_rows) bad |= MG_DEVERR_ROW_RANGE;
+        if (c < 0 || n < 0 || L > p.pt_stride || L > p.max_seq_len || n > p.max_q_len || qo < 0 ||
+            qo + n > p.total_q || __ldg(p.q_offset + r + 1) - qo != n)
+            bad |= MG_DEVERR_LENGTH;
+        if (bad) {
+            if (threadIdx.x == 0 && blockIdx.x == 0 && kvh == 0) atomicOr(&g_mg_device_error, bad);
+            return;
+        }
+    }
+    const int tpq = p.tokens_per_qtile;
+    const int g = p.group;
+    const int tok0 = qb * kQTiles * tpq;
+    if (tok0 >= n) return;
+    const int last_tok = min(tok0 + kQTiles * tpq, n) - 1;
+    const int kv_len = c + last_tok + 1;  // keys this CTA needs: positions [0, kv_len)
+    const int n_kv = (kv_len + kN - 1) / kN;
+    const bool has_q1 = tok0 + tpq < n;
+
+    Sync sy;
+    {
+        uint32_t b = sbase + kOffBar;
+        sy.q_full = b; b += 8;
+        for (int s = 0; s < kStages; ++s) { sy.k_full[s] = b; b += 8; }
+        for (int s = 0; s < kStages; ++s) { sy.v_full[s] = b; b += 8; }
+        for (int s = 0; s < kStages; ++s) { sy.kv_empty[s] = b; b += 8; }
+        for (int t = 0; t < kQTiles; ++t) { sy.s_full[t] = b; b += 8; }
+        for (int t = 0; t < kQTiles; ++t) { sy.p_full[t] = b; b += 8; }
+        for (int t = 0; t < kQTiles; ++t) { sy.o_done[t] = b; b += 8; }
+    }
+    if (threadIdx.x == 0) {
+        *abort_flag = 0;
+        mbar_init(sy.q_full, 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(sy.k_full[s], 1);
+            mbar_init(sy.v_full[s], 1);
+            mbar_init(sy.kv_empty[s], 1);
+        }
+        for (int t = 0; t < kQTiles; ++t) {
+            mbar_init(sy.s_full[t], 1);
+            mbar_init(sy.p_full[t], 128);
+            mbar_init(sy.o_done[t], 1);
+        }
+        fence_mbarrier_init();
+    }
+    if (warp == 1) {  // TMEM allocation is warp-wide
+        tmem_alloc(smem_u32(tmem_holder), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    if (warp == 0) {
+        // =============================================================== loads
+        if (lane == 0) {
+            prefetch_tmap(&tm_q);
+            prefetch_tmap(&tm_k);
+            prefetch_tmap(&tm_v);
+            const uint32_t qbytes = (uint32_t)(kQTiles * 2 * 128 * g * tpq);
+            mbar_arrive_expect_tx(sy.q_full, qbytes);
+            for (int t = 0; t < kQTiles; ++t)
+                for (int h = 0; h < 2; ++h)
+                    tma_load_3d(sbase + kOffQ + t * kTileBytes + h * kHalfBytes, &tm_q, sy.q_full, h * 64,
+                                kvh * g, qo + tok0 + t * tpq);
+        }
+        const int32_t *pt = p.page_table + (int64_t)row * p.pt_stride;
+        const int oob_row = (int)(p.num_slots * p.num_kv_heads);  // reads as zeros
+        for (int j = 0; j < n_kv; ++j) {
+            const int s = j % kStages;
+            if (j >= kStages && !wait_or_abort(sy.kv_empty[s], ((j / kStages) - 1) & 1, abort_flag)) break;
+            int rows[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int key = j * kN + lane * 4 + e;
+                int slot = key < kv_len ? __ldg(pt + key) : -1;
+                if (key < kv_len && (slot < 0 || (int64_t)slot >= p.num_slots)) {
+                    atomicOr(&g_mg_device_error, MG_DEVERR_SLOT_RANGE);
+                    slot = -1;
+                }
+                rows[e] = slot < 0 ? oob_row : slot * p.num_kv_heads + kvh;
+            }
+            if (lane == 0) mbar_arrive_expect_tx(sy.k_full[s], kTileBytes);
+            __syncwarp();
+            const uint32_t kdst = sbase + kOffK + s * kTileBytes + lane * 4 * 128;
+            tma_gather4(kdst, &tm_k, sy.k_full[s], 0, rows[0], rows[1], rows[2], rows[3]);
+            tma_gather4(kdst + kHalfBytes, &tm_k, sy.k_full[s], 64, rows[0], rows[1], rows[2], rows[3]);
+            if (lane == 0) mbar_arrive_expect_tx(sy.v_full[s], kTileBytes);
+            __syncwarp();
+            const uint32_t vdst = sbase + kOffV + s * kTileBytes + lane * 4 * 128;
+            tma_gather4(vdst, &tm_v, sy.v_full[s], 0, rows[0], rows[1], rows[2], rows[3]);
+            tma_gather4(vdst + kHalfBytes, &tm_v, sy.v_full[s], 64, rows[0], rows[1], rows[2], rows[3]);
+        }
+    } else if (warp == 1) {
+        // =============================================================== MMA issue
+        if (lane == 0) {
+            constexpr uint32_t idesc_qk = idesc_bf16(false);
+            constexpr uint32_t idesc_pv = idesc_bf16(true);
+            auto issue_s = [&](int t, int j) {
+                const int s = j % kStages;
+                const uint32_t qa = sbase + kOffQ + t * kTileBytes;
+                const uint32_t ka = sbase + kOffK + s * kTileBytes;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+                    umma_ss(tmem + col_s(t), sw128_desc(qa + off, 16, 1024), sw128_desc(ka + off, 16, 1024),
+                            idesc_qk, kk > 0);
+                }
+                umma_commit(sy.s_full[t]);
+            };
+            auto issue_pv = [&](int t, int j) {
+                const int s = j % kStages;
+                const uint32_t va = sbase + kOffV + s * kTileBytes;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    umma_ts(tmem + col_o(t), tmem + col_s(t) + kk * 8,
+                            sw128_desc(va + kk * 2048, kHalfBytes, 1024), idesc_pv, (j > 0 || kk > 0));
+                umma_commit(sy.o_done[t]);
+            };
+            bool ok = wait_or_abort(sy.q_full, 0, abort_flag) && wait_or_abort(sy.k_full[0], 0, abort_flag);
+            if (ok) {
+                tc_fence_after();
+                issue_s(0, 0);
+                if (has_q1) issue_s(1, 0);
+            }
+            for (int j = 0; ok && j < n_kv; ++j) {
+                const int s = j % kStages;
+                const uint32_t ph = (j / kStages) & 1;
+                if (!(ok = wait_or_abort(sy.v_full[s], ph, abort_flag))) break;
+                if (!(ok = wait_or_abort(sy.p_full[0], j & 1, abort_flag))) break;
+                tc_fence_after();
+                issue_pv(0, j);
+                const bool more = j + 1 < n_kv;
+                if (more) {
+                    const int s1 = (j + 1) % kStages;
+                    if (!(ok = wait_or_abort(sy.k_full[s1], ((j + 1) / kStages) & 1, abort_flag))) break;
+                    tc_fence_after();
+                    issue_s(0, j + 1);
+                }
+                if (has_q1) {
+                    if (!(ok = wait_or_abort(sy.p_full[1], j & 1, abort_flag))) break;
+                    tc_fence_after();
+                    issue_pv(1, j);
+                }
+                umma_commit(sy.kv_empty[s]);
+                if (more && has_q1) issue_s(1, j + 1);
+            }
+        }
+        __syncwarp();
+    } else {
+        // =============================================================== softmax
+        const int t = (warp - 2) >> 2;  // Q tile
+        const int wq = warp & 3;        // TMEM lane quarter this warp may access
+        const int qrow = wq * 32 + lane;
+        const int tok_local = qrow / g, head_local = qrow - tok_local * g;
+        const int i = tok0 + t * tpq + tok_local;  // new-token index within the request
+        const bool valid = tok_local < tpq && i < n;
+        const int lim = valid ? c + i : kv_len - 1;  // last visible key position
+        const bool active = t == 0 || has_q1;
+        const uint32_t lane_addr = (uint32_t)(wq * 32) << 16;
+        const uint32_t tS = tmem + lane_addr + col_s(t);
+        const uint32_t tO = tmem + lane_addr + col_o(t);
+        float m_run = -INFINITY, l_run = 0.f;
+        bool ok = active;
+        for (int j = 0; ok && j < n_kv; ++j) {
+            if (!(ok = wait_or_abort(sy.s_full[t], j & 1, abort_flag))) break;
+            tc_fence_after();
+            uint32_t sv[128];
+            tmem_ld_32x32b_x32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+            tmem_ld_32x32b_x32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+            tmem_ld_32x32b_x32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[64]));
+            tmem_ld_32x32b_x32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
+            tmem_ld_wait();
+            const int key0 = j * kN;
+            const int nvis = min(max(lim - key0 + 1, 0), kN);  // visible keys in this tile
+            float mx = -INFINITY;
+#pragma unroll
+            for (int e = 0; e < 128; ++e) {
+                float x = __uint_as_float(sv[e]) * p.scale_log2;
+                x = e < nvis ? x : -INFINITY;
+                sv[e] = __float_as_uint(x);
+                mx = fmaxf(mx, x);
+            }
+            const float m_new = fmaxf(m_run, mx);
+            const bool need = m_new > m_run + kRescaleThreshold;  // also true for the first tile
+            const bool warp_need = __any_sync(0xffffffffu, need);
+            float corr = 1.f;
+            if (warp_need) {
+                const float m_tgt = need ? m_new : m_run;
+                corr = m_run == -INFINITY ? 0.f : fast_exp2(m_run - m_tgt);
+                m_run = m_tgt;
+                l_run *= corr;
+            }
+            const float mu = m_run == -INFINITY ? 0.f : m_run;
+            float rs = 0.f;
+#pragma unroll
+            for (int cb = 0; cb < 4; ++cb) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const float p0 = fast_exp2(__uint_as_float(sv[cb * 32 + 2 * e]) - mu);
+                    const float p1 = fast_exp2(__uint_as_float(sv[cb * 32 + 2 * e + 1]) - mu);
+                    rs += p0 + p1;
+                    pk[e] = pack_bf16x2(p0, p1);
+                }
+                tmem_st_32x32b_x16(tS + cb * 16, pk);
+            }
+            l_run += rs;
+            if (warp_need && j > 0) {
+                // O holds the sum up to tile j-1; rescale it once that PV is done
+                if (!(ok = wait_or_abort(sy.o_done[t], (j - 1) & 1, abort_flag))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int cb = 0; cb < 4; ++cb) {
+                    uint32_t ov[32];
+                    tmem_ld_32x32b_x32(tO + cb * 32, ov);
+                    tmem_ld_wait();
+                    uint32_t lo[16], hi[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        lo[e] = __float_as_uint(__uint_as_float(ov[e]) * corr);
+                        hi[e] = __float_as_uint(__uint_as_float(ov[16 + e]) * corr);
+                    }
+                    tmem_st_32x32b_x16(tO + cb * 32, lo);
+                    tmem_st_32x32b_x16(tO + cb * 32 + 16, hi);
+                }
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(sy.p_full[t]);
+        }
+        // ---- epilogue: O / l -> bf16 -> out
+        if (ok && wait_or_abort(sy.o_done[t], (n_kv - 1) & 1, abort_flag)) {
+            tc_fence_after();
+            const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+            __nv_bfloat16 *dst = p.out + ((int64_t)(qo + i) * p.num_q_heads + kvh * g + head_local) * kHeadDim;
+#pragma unroll
+            for (int cb = 0; cb < 4; ++cb) {
+                uint32_t ov[32];
+                tmem_ld_32x32b_x32(tO + cb * 32, ov);
+                tmem_ld_wait();
+                if (valid) {
+                    uint4 *d4 = reinterpret_cast<uint4 *>(dst + cb * 32);
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) {
+                        uint4 w;
+                        w.x = pack_bf16x2(__uint_as_float(ov[8 * v + 0]) * inv, __uint_as_float(ov[8 * v + 1]) * inv);
+                        w.y = pack_bf16x2(__uint_as_float(ov[8 * v + 2]) * inv, __uint_as_float(ov[8 * v + 3]) * inv);
+                        w.z = pack_bf16x2(__uint_as_float(ov[8 * v + 4]) * inv, __uint_as_float(ov[8 * v + 5]) * inv);
+                        w.w = pack_bf16x2(__uint_as_float(ov[8 * v + 6]) * inv, __uint_as_float(ov[8 * v + 7]) * inv);
+                        d4[v] = w;
+                    }
+                }
+            }
+        }
+    }
+
+    // ---- teardown: everyone meets here, even after an abort
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------- host side
+
+inline cudaError_t set_attributes() {
+    return cudaFuncSetAttribute(extend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
+                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                   CUtensorMapFloatOOBfill);
+
+inline EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    return fn;
+}
+
+inline mg_status launch(Params &p, cudaStream_t stream) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return MG_ERR_CUDA;
+    const int g = p.group;
+    p.tokens_per_qtile = kM / g;
+    CUtensorMap tq, tk, tv;
+    {
+        cuuint64_t dims[3] = {(cuuint64_t)kHeadDim, (cuuint64_t)p.num_q_heads, (cuuint64_t)p.total_q};
+        cuuint64_t strides[2] = {(cuuint64_t)kHeadDim * 2, (cuuint64_t)p.num_q_heads * kHeadDim * 2};
+        cuuint32_t box[3] = {64, (cuuint32_t)g, (cuuint32_t)p.tokens_per_qtile};
+        cuuint32_t es[3] = {1, 1, 1};
+        if (enc(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<__nv_bfloat16 *>(p.q), dims, strides, box, es,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return MG_ERR_CUDA;
+    }
+    const cuuint64_t pool_rows = (cuuint64_t)p.num_slots * (cuuint64_t)p.num_kv_heads;
+    if (pool_rows >= (1ull << 31)) return MG_ERR_UNSUPPORTED_SHAPE;  // gather4 row coordinates are int32
+    for (int which = 0; which < 2; ++which) {
+        cuuint64_t dims[2] = {(cuuint64_t)kHeadDim, pool_rows};
+        cuuint64_t strides[1] = {(cuuint64_t)kHeadDim * 2};
+        cuuint32_t box[2] = {64, 1};
+        cuuint32_t es[2] = {1, 1};
+        void *base = const_cast<__nv_bfloat16 *>(which == 0 ? p.k_cache : p.v_cache);
+        if (enc(which == 0 ? &tk : &tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, es,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return MG_ERR_CUDA;
+    }
+    const int tokens_per_cta = kQTiles * p.tokens_per_qtile;
+    const int nqb = (p.max_q_len + tokens_per_cta - 1) / tokens_per_cta;
+    if (nqb > 0x7fffffff || p.batch > 65535 || p.num_kv_heads > 65535) return MG_ERR_INVALID_ARGUMENT;
+    dim3 grid((unsigned)nqb, (unsigned)p.num_kv_heads, (unsigned)p.batch);
+    extend_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tq, tk, tv, p);
+    return cudaGetLastError() == cudaSuccess ? MG_OK : MG_ERR_CUDA;
+}
+
+}  // namespace extend
+}  // namespace mg

@@ -1,0 +1,290 @@
+// mg.cu -- the C ABI of libmg (declared in include/mg.h): argument checks,
+// the decode split plan, and kernel launches on the caller's stream.
+//
+// Everything is one translation unit so the kernels share the device error
+// word without relocatable device code.
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "decode.cuh"
+#include "extend.cuh"
+#include "store_kv.cuh"
+
+namespace mg {
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kDecodeStages = 3;
+
+int g_sm_count[kMaxDevices];
+bool g_attr_done[kMaxDevices];
+std::mutex g_attr_mutex;
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+mg_status current_device(int &dev) {
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MG_ERR_CUDA;
+    return MG_OK;
+}
+
+mg_status sm_count(int &sms) {
+    int dev;
+    if (current_device(dev) != MG_OK) return MG_ERR_CUDA;
+    if (g_sm_count[dev] == 0) {
+        int v = 0;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+            return MG_ERR_CUDA;
+        g_sm_count[dev] = v;
+    }
+    sms = g_sm_count[dev];
+    return MG_OK;
+}
+
+// Opt the kernels with large dynamic shared memory in, once per device.
+mg_status ensure_kernel_attributes() {
+    int dev;
+    if (current_device(dev) != MG_OK) return MG_ERR_CUDA;
+    if (g_attr_done[dev]) return MG_OK;
+    std::lock_guard<std::mutex> lock(g_attr_mutex);
+    if (g_attr_done[dev]) return MG_OK;
+    if (cudaFuncSetAttribute(decode::decode_split_kernel<kDecodeStages>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             decode::Smem<kDecodeStages>::kBytes) != cudaSuccess)
+        return MG_ERR_CUDA;
+    if (extend::set_attributes() != cudaSuccess) return MG_ERR_CUDA;
+    g_attr_done[dev] = true;
+    return MG_OK;
+}
+
+mg_status launched() {
+    return cudaGetLastError() == cudaSuccess ? MG_OK : MG_ERR_CUDA;
+}
+
+// Split plan: keys per split (multiple of the 64-key tile, <= 2048) and the
+// number of splits of a max_seq_len request.  Aim for ~4 waves of 2 CTAs per
+// SM if every request were max_seq_len long; shorter requests end early and
+// leave room, longer splits would leave a long tail.
+mg_status decode_plan(int batch, int hkv, int max_seq_len, int kv_chunk, int &chunk, int &nsplits) {
+    if (batch <= 0 || hkv <= 0 || max_seq_len <= 0 || kv_chunk < 0) return MG_ERR_INVALID_ARGUMENT;
+    const int tile = decode::kTile;
+    if (kv_chunk > 0) {
+        chunk = (kv_chunk + tile - 1) / tile * tile;
+        if (chunk > decode::kMaxChunk) return MG_ERR_INVALID_ARGUMENT;
+    } else {
+        int sms;
+        if (sm_count(sms) != MG_OK) return MG_ERR_CUDA;
+        const double target_ctas = (double)sms * 2.0 * 4.0;
+        const double work = (double)max_seq_len * (double)batch * (double)hkv;
+        long long c = (long long)((work / target_ctas) + tile - 1) / tile * tile;
+        if (c < 256) c = 256;
+        if (c > decode::kMaxChunk) c = decode::kMaxChunk;
+        chunk = (int)c;
+    }
+    nsplits = (max_seq_len + chunk - 1) / chunk;
+    if (nsplits > 65535) return MG_ERR_INVALID_ARGUMENT;
+    return MG_OK;
+}
+
+size_t decode_ws_bytes(int batch, int hq, int nsplits) {
+    if (nsplits <= 1) return 0;
+    const size_t rows = (size_t)batch * hq * nsplits;
+    return rows * kHeadDim * sizeof(float) + ((rows * sizeof(float) + 255) / 256) * 256;
+}
+
+mg_status check_attention_shape(int hq, int hkv, int head_dim) {
+    if (hq <= 0 || hkv <= 0 || head_dim <= 0) return MG_ERR_INVALID_ARGUMENT;
+    if (head_dim != kHeadDim || hq % hkv != 0 || hq / hkv > decode::kRows) return MG_ERR_UNSUPPORTED_SHAPE;
+    return MG_OK;
+}
+
+}  // namespace
+}  // namespace mg
+
+using namespace mg;
+
+extern "C" {
+
+const char *mg_status_string(mg_status s) {
+    switch (s) {
+        case MG_OK: return "MG_OK";
+        case MG_ERR_INVALID_ARGUMENT: return "MG_ERR_INVALID_ARGUMENT";
+        case MG_ERR_UNSUPPORTED_SHAPE: return "MG_ERR_UNSUPPORTED_SHAPE";
+        case MG_ERR_MISALIGNED: return "MG_ERR_MISALIGNED";
+        case MG_ERR_WORKSPACE_TOO_SMALL: return "MG_ERR_WORKSPACE_TOO_SMALL";
+        case MG_ERR_CUDA: return "MG_ERR_CUDA";
+        case MG_ERR_DEVICE_CHECK: return "MG_ERR_DEVICE_CHECK";
+        case MG_ERR_DEVICE_TIMEOUT: return "MG_ERR_DEVICE_TIMEOUT";
+    }
+    return "MG_ERR_UNKNOWN";
+}
+
+int32_t mg_abi_version(void) { return 1; }
+
+mg_status mg_store_kv(const void *k, const void *v, const int32_t *out_loc, int32_t num_tokens,
+                      void *k_cache, void *v_cache, int64_t num_slots, int32_t num_kv_heads,
+                      int32_t head_dim, void *stream) {
+    if (num_tokens < 0 || num_slots <= 0 || num_kv_heads <= 0 || head_dim <= 0)
+        return MG_ERR_INVALID_ARGUMENT;
+    if (num_tokens == 0) return MG_OK;
+    if (!k || !v || !out_loc || !k_cache || !v_cache) return MG_ERR_INVALID_ARGUMENT;
+    const int64_t row_bytes = (int64_t)num_kv_heads * head_dim * 2;
+    if (row_bytes % 16 != 0) return MG_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache))
+        return MG_ERR_MISALIGNED;
+    int sms;
+    if (sm_count(sms) != MG_OK) return MG_ERR_CUDA;
+    StoreParams p;
+    p.k = static_cast<const uint4 *>(k);
+    p.v = static_cast<const uint4 *>(v);
+    p.out_loc = out_loc;
+    p.k_cache = static_cast<uint4 *>(k_cache);
+    p.v_cache = static_cast<uint4 *>(v_cache);
+    p.num_slots = num_slots;
+    p.vecs_per_token = (int32_t)(row_bytes / 16);
+    p.total_vecs = (int64_t)num_tokens * p.vecs_per_token;
+    const int threads = 256;
+    long long blocks = (p.total_vecs + threads - 1) / threads;
+    const long long cap = (long long)sms * 8;
+    if (blocks > cap) blocks = cap;
+    store_kv_kernel<<<(unsigned)blocks, threads, 0, static_cast<cudaStream_t>(stream)>>>(p);
+    return launched();
+}
+
+mg_status mg_decode_plan(int32_t batch, int32_t num_kv_heads, int32_t max_seq_len, int32_t kv_chunk,
+                         int32_t *chunk_out, int32_t *num_splits_out) {
+    int chunk, ns;
+    mg_status st = decode_plan(batch, num_kv_heads, max_seq_len, kv_chunk, chunk, ns);
+    if (st != MG_OK) return st;
+    if (chunk_out) *chunk_out = chunk;
+    if (num_splits_out) *num_splits_out = ns;
+    return MG_OK;
+}
+
+size_t mg_decode_workspace_bytes(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+                                 int32_t head_dim, int32_t max_seq_len, int32_t kv_chunk) {
+    (void)head_dim;
+    int chunk, ns;
+    if (decode_plan(batch, num_kv_heads, max_seq_len, kv_chunk, chunk, ns) != MG_OK) return 0;
+    return decode_ws_bytes(batch, num_q_heads, ns);
+}
+
+mg_status mg_decode_attn(const void *q, const void *k_cache, const void *v_cache, int64_t num_slots,
+                         const int32_t *page_table, int32_t page_table_rows,
+                         int32_t page_table_stride, const int32_t *table_idx,
+                         const int32_t *seq_len, int32_t batch, int32_t max_seq_len,
+                         int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, float scale,
+                         int32_t kv_chunk, void *out, void *workspace, size_t workspace_bytes,
+                         void *stream) {
+    mg_status st = check_attention_shape(num_q_heads, num_kv_heads, head_dim);
+    if (st != MG_OK) return st;
+    if (batch <= 0 || num_slots <= 0 || page_table_rows <= 0 || page_table_stride <= 0 ||
+        max_seq_len <= 0 || max_seq_len > page_table_stride)
+        return MG_ERR_INVALID_ARGUMENT;
+    if (!q || !k_cache || !v_cache || !page_table || !table_idx || !seq_len || !out)
+        return MG_ERR_INVALID_ARGUMENT;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
+        return MG_ERR_MISALIGNED;
+    int chunk, ns;
+    st = decode_plan(batch, num_kv_heads, max_seq_len, kv_chunk, chunk, ns);
+    if (st != MG_OK) return st;
+    const size_t need = decode_ws_bytes(batch, num_q_heads, ns);
+    if (need > 0) {
+        if (!workspace || workspace_bytes < need) return MG_ERR_WORKSPACE_TOO_SMALL;
+        if (!aligned16(workspace)) return MG_ERR_MISALIGNED;
+    }
+    if (ensure_kernel_attributes() != MG_OK) return MG_ERR_CUDA;
+
+    decode::Params p;
+    p.q = static_cast<const __nv_bfloat16 *>(q);
+    p.k_cache = static_cast<const __nv_bfloat16 *>(k_cache);
+    p.v_cache = static_cast<const __nv_bfloat16 *>(v_cache);
+    p.page_table = page_table;
+    p.table_idx = table_idx;
+    p.seq_len = seq_len;
+    p.out = static_cast<__nv_bfloat16 *>(out);
+    const size_t rows = (size_t)batch * num_q_heads * ns;
+    p.part_o = need ? static_cast<float *>(workspace) : nullptr;
+    p.part_lse = need ? static_cast<float *>(workspace) + rows * kHeadDim : nullptr;
+    p.num_slots = num_slots;
+    p.pt_rows = page_table_rows;
+    p.pt_stride = page_table_stride;
+    p.batch = batch;
+    p.num_q_heads = num_q_heads;
+    p.num_kv_heads = num_kv_heads;
+    p.group = num_q_heads / num_kv_heads;
+    p.chunk = chunk;
+    p.num_splits = ns;
+    p.max_seq_len = max_seq_len;
+    p.scale_log2 = scale * kLog2e;
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    dim3 grid(num_kv_heads, ns, batch);
+    decode::decode_split_kernel<kDecodeStages>
+        <<<grid, decode::kThreads, decode::Smem<kDecodeStages>::kBytes, s>>>(p);
+    if ((st = launched()) != MG_OK) return st;
+    if (ns > 1) {
+        const int warps = batch * num_q_heads;
+        decode::decode_merge_kernel<<<(warps + 3) / 4, 128, 0, s>>>(p);
+        if ((st = launched()) != MG_OK) return st;
+    }
+    return MG_OK;
+}
+
+mg_status mg_extend_attn(const void *q, const void *k_cache, const void *v_cache, int64_t num_slots,
+                         const int32_t *page_table, int32_t page_table_rows,
+                         int32_t page_table_stride, const int32_t *table_idx,
+                         const int32_t *cached_len, const int32_t *seq_len,
+                         const int32_t *q_offset, int32_t batch, int32_t total_q,
+                         int32_t max_q_len, int32_t max_seq_len, int32_t num_q_heads,
+                         int32_t num_kv_heads, int32_t head_dim, float scale, void *out,
+                         void *stream) {
+    mg_status st = check_attention_shape(num_q_heads, num_kv_heads, head_dim);
+    if (st != MG_OK) return st;
+    if (batch <= 0 || total_q < 0 || max_q_len < 0 || num_slots <= 0 || page_table_rows <= 0 ||
+        page_table_stride <= 0 || max_seq_len <= 0 || max_seq_len > page_table_stride)
+        return MG_ERR_INVALID_ARGUMENT;
+    if (total_q == 0 || max_q_len == 0) return MG_OK;
+    if (!q || !k_cache || !v_cache || !page_table || !table_idx || !cached_len || !seq_len ||
+        !q_offset || !out)
+        return MG_ERR_INVALID_ARGUMENT;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
+        return MG_ERR_MISALIGNED;
+    if (ensure_kernel_attributes() != MG_OK) return MG_ERR_CUDA;
+    extend::Params p;
+    p.q = static_cast<const __nv_bfloat16 *>(q);
+    p.k_cache = static_cast<const __nv_bfloat16 *>(k_cache);
+    p.v_cache = static_cast<const __nv_bfloat16 *>(v_cache);
+    p.page_table = page_table;
+    p.table_idx = table_idx;
+    p.cached_len = cached_len;
+    p.seq_len = seq_len;
+    p.q_offset = q_offset;
+    p.out = static_cast<__nv_bfloat16 *>(out);
+    p.num_slots = num_slots;
+    p.pt_rows = page_table_rows;
+    p.pt_stride = page_table_stride;
+    p.batch = batch;
+    p.total_q = total_q;
+    p.max_q_len = max_q_len;
+    p.max_seq_len = max_seq_len;
+    p.num_q_heads = num_q_heads;
+    p.num_kv_heads = num_kv_heads;
+    p.group = num_q_heads / num_kv_heads;
+    p.scale_log2 = scale * kLog2e;
+    return extend::launch(p, static_cast<cudaStream_t>(stream));
+}
+
+mg_status mg_read_device_error(void *stream, uint32_t *bits_out) {
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MG_ERR_CUDA;
+    unsigned int bits = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&bits, g_mg_device_error, sizeof bits) != cudaSuccess) return MG_ERR_CUDA;
+    if (bits && cudaMemcpyToSymbol(g_mg_device_error, &zero, sizeof zero) != cudaSuccess)
+        return MG_ERR_CUDA;
+    if (bits_out) *bits_out = bits;
+    if (bits & MG_DEVERR_WAIT_TIMEOUT) return MG_ERR_DEVICE_TIMEOUT;
+    return bits ? MG_ERR_DEVICE_CHECK : MG_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,183 @@
+"""Python binding of libmg (include/mg.h): argument marshalling only.
+
+Every operation runs in the CUDA library; this module checks tensor dtypes,
+shapes and devices, passes raw pointers and the current CUDA stream through
+ctypes, and raises ``MgError`` on a non-OK status.  There is no fallback: if
+libmg.so is missing, the first call raises.  PyTorch is used for device
+memory and streams only.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional
+
+import torch
+
+LIBRARY = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmg.so")
+
+STATUS = {
+    0: "MG_OK",
+    1: "MG_ERR_INVALID_ARGUMENT",
+    2: "MG_ERR_UNSUPPORTED_SHAPE",
+    3: "MG_ERR_MISALIGNED",
+    4: "MG_ERR_WORKSPACE_TOO_SMALL",
+    5: "MG_ERR_CUDA",
+    6: "MG_ERR_DEVICE_CHECK",
+    7: "MG_ERR_DEVICE_TIMEOUT",
+}
+DEVERR_SLOT_RANGE = 0x1
+DEVERR_ROW_RANGE = 0x2
+DEVERR_LENGTH = 0x4
+DEVERR_WAIT_TIMEOUT = 0x8
+
+# name -> (restype, argtypes), the exact list of include/mg.h
+_P, _I32, _I64, _F32, _SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+SIGNATURES = {
+    "mg_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "mg_abi_version": (_I32, []),
+    "mg_store_kv": (ctypes.c_int, [_P, _P, _P, _I32, _P, _P, _I64, _I32, _I32, _P]),
+    "mg_decode_plan": (ctypes.c_int, [_I32, _I32, _I32, _I32, ctypes.POINTER(_I32), ctypes.POINTER(_I32)]),
+    "mg_decode_workspace_bytes": (_SZ, [_I32, _I32, _I32, _I32, _I32, _I32]),
+    "mg_decode_attn": (ctypes.c_int, [_P, _P, _P, _I64, _P, _I32, _I32, _P, _P, _I32, _I32, _I32, _I32,
+                                      _I32, _F32, _I32, _P, _P, _SZ, _P]),
+    "mg_extend_attn": (ctypes.c_int, [_P, _P, _P, _I64, _P, _I32, _I32, _P, _P, _P, _P, _I32, _I32, _I32,
+                                      _I32, _I32, _I32, _I32, _F32, _P, _P]),
+    "mg_read_device_error": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_uint32)]),
+}
+
+_lock = threading.Lock()
+_lib = None
+
+
+class MgError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {STATUS.get(status, status)}")
+        self.status = status
+
+
+def load(path: str = LIBRARY):
+    """Load libmg.so once; raises if it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(path):
+                raise RuntimeError(f"libmg.so not built ({path}); run python -m paged_kv_attention_mg_b200.build")
+            lib = ctypes.CDLL(path)
+            for name, (res, args) in SIGNATURES.items():
+                fn = getattr(lib, name)
+                fn.restype = res
+                fn.argtypes = args
+            _lib = lib
+        return _lib
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        raise MgError(status, what)
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _dev(t: torch.Tensor, dtype, name: str) -> int:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def store_kv(k: torch.Tensor, v: torch.Tensor, out_loc: torch.Tensor, k_cache: torch.Tensor,
+             v_cache: torch.Tensor, stream=None) -> None:
+    """k_cache[out_loc[t]] = k[t]; v_cache[out_loc[t]] = v[t] (bf16 rows)."""
+    t, hkv, d = k.shape
+    if v.shape != k.shape or k_cache.shape[1:] != (hkv, d) or v_cache.shape != k_cache.shape:
+        raise ValueError("store_kv: shape mismatch")
+    if out_loc.shape != (t,):
+        raise ValueError("store_kv: out_loc must be [num_tokens]")
+    _check(load().mg_store_kv(_dev(k, torch.bfloat16, "k"), _dev(v, torch.bfloat16, "v"),
+                              _dev(out_loc, torch.int32, "out_loc"), t,
+                              _dev(k_cache, torch.bfloat16, "k_cache"),
+                              _dev(v_cache, torch.bfloat16, "v_cache"), k_cache.shape[0], hkv, d,
+                              _stream(stream)), "mg_store_kv")
+
+
+def decode_plan(batch: int, num_kv_heads: int, max_seq_len: int, kv_chunk: int = 0):
+    """(keys per split, number of splits) that mg_decode_attn will use."""
+    chunk, ns = _I32(), _I32()
+    _check(load().mg_decode_plan(batch, num_kv_heads, max_seq_len, kv_chunk, ctypes.byref(chunk),
+                                 ctypes.byref(ns)), "mg_decode_plan")
+    return chunk.value, ns.value
+
+
+def decode_workspace_bytes(batch: int, num_q_heads: int, num_kv_heads: int, max_seq_len: int,
+                           kv_chunk: int = 0, head_dim: int = 128) -> int:
+    return int(load().mg_decode_workspace_bytes(batch, num_q_heads, num_kv_heads, head_dim, max_seq_len,
+                                                 kv_chunk))
+
+
+def decode_attn(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, page_table: torch.Tensor,
+                table_idx: torch.Tensor, seq_len: torch.Tensor, max_seq_len: int, scale: float,
+                kv_chunk: int = 0, out: Optional[torch.Tensor] = None,
+                workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Paged decode attention; returns out [B, Hq, D] bf16."""
+    b, hq, d = q.shape
+    hkv = k_cache.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    need = decode_workspace_bytes(b, hq, hkv, max_seq_len, kv_chunk, d)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = _dev(workspace, torch.uint8, "workspace") if workspace is not None else None
+    ws_bytes = workspace.numel() if workspace is not None else 0
+    _check(load().mg_decode_attn(_dev(q, torch.bfloat16, "q"), _dev(k_cache, torch.bfloat16, "k_cache"),
+                                 _dev(v_cache, torch.bfloat16, "v_cache"), k_cache.shape[0],
+                                 _dev(page_table, torch.int32, "page_table"), page_table.shape[0],
+                                 page_table.shape[1], _dev(table_idx, torch.int32, "table_idx"),
+                                 _dev(seq_len, torch.int32, "seq_len"), b, max_seq_len, hq, hkv, d,
+                                 float(scale), kv_chunk, _dev(out, torch.bfloat16, "out"), ws_ptr, ws_bytes,
+                                 _stream(stream)), "mg_decode_attn")
+    return out
+
+
+def extend_attn(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, page_table: torch.Tensor,
+                table_idx: torch.Tensor, cached_len: torch.Tensor, seq_len: torch.Tensor,
+                q_offset: torch.Tensor, max_q_len: int, max_seq_len: int, scale: float,
+                out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Chunked-prefill extend attention; returns out [total_q, Hq, D] bf16."""
+    total_q, hq, d = q.shape
+    hkv = k_cache.shape[1]
+    b = seq_len.shape[0]
+    if q_offset.shape != (b + 1,):
+        raise ValueError("extend_attn: q_offset must be [batch + 1]")
+    if out is None:
+        out = torch.empty_like(q)
+    _check(load().mg_extend_attn(_dev(q, torch.bfloat16, "q"), _dev(k_cache, torch.bfloat16, "k_cache"),
+                                 _dev(v_cache, torch.bfloat16, "v_cache"), k_cache.shape[0],
+                                 _dev(page_table, torch.int32, "page_table"), page_table.shape[0],
+                                 page_table.shape[1], _dev(table_idx, torch.int32, "table_idx"),
+                                 _dev(cached_len, torch.int32, "cached_len"),
+                                 _dev(seq_len, torch.int32, "seq_len"), _dev(q_offset, torch.int32, "q_offset"),
+                                 b, total_q, max_q_len, max_seq_len, hq, hkv, d, float(scale),
+                                 _dev(out, torch.bfloat16, "out"), _stream(stream)), "mg_extend_attn")
+    return out
+
+
+def read_device_error(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device error bits."""
+    bits = ctypes.c_uint32(0)
+    st = load().mg_read_device_error(_stream(stream), ctypes.byref(bits))
+    if st not in (0, 6, 7):
+        raise MgError(st, "mg_read_device_error")
+    return bits.value

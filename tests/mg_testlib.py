@@ -101,3 +101,85 @@ def dense_extend(q, k_pool, v_pool, page_table, table_idx, cached_len, seq_len, 
 
 def bf16_to_f64(t: torch.Tensor) -> np.ndarray:
     return t.detach().to("cpu").to(torch.float64).numpy()
+
+
+# ----------------------------------------------------------------------------- GPU side
+
+MAX_ABS_TOL = 1e-2   # bf16 attention outputs vs the fp64 oracle (max |err|)
+MEAN_ABS_TOL = 1e-3  # ... and mean |err| over all real rows
+
+
+def assert_matches_oracle(got: torch.Tensor, ref: np.ndarray, what: str = ""):
+    """got: bf16 kernel output (any device); ref: fp64 oracle, NaN rows = not computed."""
+    g = got.detach().to("cpu").to(torch.float64).numpy()
+    sel = ~np.isnan(ref).any(axis=-1)
+    assert sel.any(), "oracle computed no rows"
+    gs, rs = g[sel], ref[sel]
+    assert np.isfinite(gs).all(), f"{what}: non-finite kernel output"
+    diff = np.abs(gs - rs)
+    assert diff.max() <= MAX_ABS_TOL, f"{what}: max abs err {diff.max():.3e} (mean {diff.mean():.3e})"
+    assert diff.mean() <= MEAN_ABS_TOL, f"{what}: mean abs err {diff.mean():.3e}"
+    return float(diff.max()), float(diff.mean())
+
+
+class GpuStep:
+    """Device copies of one (step, layer): pools before the store, new K/V, metadata."""
+
+    def __init__(self, step, data, device="cuda"):
+        self.step, self.data = step, data
+        spec = step.spec
+        self.k_cache = wl.build_pool(step, data.hist_slots, data.k_hist, device)
+        self.v_cache = wl.build_pool(step, data.hist_slots, data.v_hist, device)
+        self.k_new = data.k_new.to(device)
+        self.v_new = data.v_new.to(device)
+        self.q = data.q.to(device)
+        self.out_loc = step.out_loc.to(device)
+        self.page_table = step.page_table.to(device)
+        self.table_idx = step.table_idx.to(device)
+        self.seq_len = step.seq_len.to(device)
+        self.cached_len = step.cached_len.to(device)
+        self.q_offset = step.q_offset.to(device)
+        self.scale = spec.scale
+
+    def store(self):
+        from paged_kv_attention_mg_b200 import mg
+        mg.store_kv(self.k_new, self.v_new, self.out_loc, self.k_cache, self.v_cache)
+
+    def decode(self, kv_chunk=0, max_seq_len=None, out=None):
+        from paged_kv_attention_mg_b200 import mg
+        msl = max_seq_len or self.step.max_seq_len
+        return mg.decode_attn(self.q, self.k_cache, self.v_cache, self.page_table, self.table_idx, self.seq_len,
+                              msl, self.scale, kv_chunk=kv_chunk, out=out)
+
+    def extend(self, out=None):
+        from paged_kv_attention_mg_b200 import mg
+        s = self.step
+        return mg.extend_attn(self.q, self.k_cache, self.v_cache, self.page_table, self.table_idx,
+                              self.cached_len, self.seq_len, self.q_offset, max(s.max_q_len, 1),
+                              max(s.max_seq_len, 1), self.scale, out=out)
+
+
+def host_pools_after_store(step, data):
+    """Host pools with the new tokens stored (by index_copy_, independent of the kernels)."""
+    k = wl.build_pool(step, data.hist_slots, data.k_hist)
+    v = wl.build_pool(step, data.hist_slots, data.v_hist)
+    loc = step.out_loc.to(torch.int64)
+    if loc.numel():
+        k.index_copy_(0, loc, data.k_new)
+        v.index_copy_(0, loc, data.v_new)
+    return k, v
+
+
+def oracle_decode(step, data, requests=None):
+    import oracle
+    k, v = host_pools_after_store(step, data)
+    return oracle.decode(wl.bits(data.q), wl.bits(k), wl.bits(v), step.page_table.numpy(),
+                         step.table_idx.numpy(), step.seq_len.numpy(), step.spec.scale, requests=requests)
+
+
+def oracle_extend(step, data, requests=None):
+    import oracle
+    k, v = host_pools_after_store(step, data)
+    return oracle.extend(wl.bits(data.q), wl.bits(k), wl.bits(v), step.page_table.numpy(),
+                         step.table_idx.numpy(), step.cached_len.numpy(), step.seq_len.numpy(),
+                         step.q_offset.numpy(), step.spec.scale, requests=requests)

@@ -1,0 +1,110 @@
+"""The C ABI library, without a GPU: it builds, loads, exports exactly what
+include/mg.h declares, and rejects bad arguments on the host before any CUDA
+work (these calls return before touching the device)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from paged_kv_attention_mg_b200 import build, mg
+
+HEADER = os.path.join(build.INCLUDE, "mg.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(mg_\w+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build_library()
+    return mg.load()
+
+
+def test_header_and_binding_agree():
+    assert declared_functions() == sorted(mg.SIGNATURES)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", mg.LIBRARY], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(re.findall(r"\bT (mg_\w+)$", out, flags=re.M))
+    assert set(declared_functions()) <= exported
+    for name in declared_functions():
+        assert hasattr(lib, name)
+
+
+def test_build_targets_sm100a_only():
+    flags = " ".join(build.NVCC_FLAGS)
+    assert "arch=compute_100a,code=sm_100a" in flags and "-lineinfo" in flags
+    assert flags.count("-gencode") == 1
+
+
+def test_status_strings(lib):
+    for code, name in mg.STATUS.items():
+        assert lib.mg_status_string(code).decode() == name
+    assert lib.mg_abi_version() == 1
+
+
+def test_store_zero_tokens_is_noop(lib):
+    assert lib.mg_store_kv(None, None, None, 0, None, None, 10, 8, 128, None) == 0
+
+
+@pytest.mark.parametrize("args,expect", [
+    (dict(num_tokens=-1), 1),
+    (dict(num_slots=0), 1),
+    (dict(num_kv_heads=0), 1),
+    (dict(k=None), 1),
+    (dict(num_kv_heads=1, head_dim=4), 2),   # 8-byte rows are not 16-byte vectors
+    (dict(k=8), 3),                          # misaligned
+])
+def test_store_host_validation(lib, args, expect):
+    base = dict(k=4096, v=4096, out_loc=4096, num_tokens=3, k_cache=4096, v_cache=4096, num_slots=10,
+                num_kv_heads=8, head_dim=128)
+    base.update(args)
+    st = lib.mg_store_kv(base["k"], base["v"], base["out_loc"], base["num_tokens"], base["k_cache"],
+                         base["v_cache"], base["num_slots"], base["num_kv_heads"], base["head_dim"], None)
+    assert st == expect
+
+
+@pytest.mark.parametrize("hq,hkv,d,expect", [(16, 8, 64, 2), (12, 8, 128, 2), (64, 2, 128, 2),
+                                             (0, 8, 128, 1)])
+def test_decode_rejects_shapes(lib, hq, hkv, d, expect):
+    st = lib.mg_decode_attn(4096, 4096, 4096, 100, 4096, 5, 32, 4096, 4096, 4, 32, hq, hkv, d, 0.1, 0,
+                            4096, None, 0, None)
+    assert st == expect
+
+
+def test_decode_rejects_bad_hints(lib):
+    # max_seq_len above the page-table width
+    assert lib.mg_decode_attn(4096, 4096, 4096, 100, 4096, 5, 32, 4096, 4096, 4, 33, 16, 8, 128, 0.1, 0,
+                              4096, None, 0, None) == 1
+    # forced chunk above the prefetch capacity
+    assert lib.mg_decode_attn(4096, 4096, 4096, 100, 4096, 5, 4096, 4096, 4096, 4, 4096, 16, 8, 128, 0.1,
+                              4096, 4096, None, 0, None) == 1
+
+
+def test_decode_plan_with_forced_chunk_needs_no_device(lib):
+    chunk, ns = ctypes.c_int32(), ctypes.c_int32()
+    assert lib.mg_decode_plan(8, 4, 32768, 1000, ctypes.byref(chunk), ctypes.byref(ns)) == 0
+    assert chunk.value == 1024 and ns.value == 32
+    assert lib.mg_decode_workspace_bytes(8, 32, 4, 128, 32768, 1000) >= 8 * 32 * 32 * (128 + 1) * 4
+    assert lib.mg_decode_workspace_bytes(8, 32, 4, 128, 1000, 1024) == 0  # one split
+
+
+def test_extend_rejects_shapes_and_empty_is_noop(lib):
+    assert lib.mg_extend_attn(4096, 4096, 4096, 100, 4096, 5, 32, 4096, 4096, 4096, 4096, 4, 10, 4, 32,
+                              16, 8, 64, 0.1, 4096, None) == 2
+    # no new tokens at all: nothing to launch
+    assert lib.mg_extend_attn(4096, 4096, 4096, 100, 4096, 5, 32, 4096, 4096, 4096, 4096, 4, 0, 0, 32,
+                              16, 8, 128, 0.1, 4096, None) == 0
+
+
+def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    monkeypatch.setattr(mg, "_lib", None)
+    with pytest.raises(RuntimeError, match="not built"):
+        mg.load(str(tmp_path / "missing.so"))
