@@ -120,8 +120,9 @@ __device__ __forceinline__ bool wait_or_abort_thread(uint32_t bar, uint32_t pari
     }
 }
 
-// Warp-uniform form: every lane waits, and the warp proceeds only if all did
-// (tcgen05.ld/st and __syncwarp need the whole warp to stay converged).
+// Warp-uniform form for roles where all 32 lanes wait together: the warp
+// proceeds only if every lane did (tcgen05.ld/st and __syncwarp need the whole
+// warp converged).  The single-thread MMA issuer uses wait_or_abort_thread.
 __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, volatile int *abort_flag) {
     const bool ok = wait_or_abort_thread(bar, parity, abort_flag);
     return __all_sync(0xffffffffu, ok);
@@ -267,7 +268,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             sw128_desc(va + kk * 2048, kHalfBytes, 1024), idesc_pv, (j > 0 || kk > 0));
                 umma_commit(sy.o_done[t]);
             };
-            bool ok = wait_or_abort(sy.q_full, 0, abort_flag) && wait_or_abort(sy.k_full[0], 0, abort_flag);
+            bool ok = wait_or_abort_thread(sy.q_full, 0, abort_flag) && wait_or_abort_thread(sy.k_full[0], 0, abort_flag);
             if (ok) {
                 tc_fence_after();
                 issue_s(0, 0);
@@ -276,19 +277,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int j = 0; ok && j < n_kv; ++j) {
                 const int s = j % kStages;
                 const uint32_t ph = (j / kStages) & 1;
-                if (!(ok = wait_or_abort(sy.v_full[s], ph, abort_flag))) break;
-                if (!(ok = wait_or_abort(sy.p_full[0], j & 1, abort_flag))) break;
+                if (!(ok = wait_or_abort_thread(sy.v_full[s], ph, abort_flag))) break;
+                if (!(ok = wait_or_abort_thread(sy.p_full[0], j & 1, abort_flag))) break;
                 tc_fence_after();
                 issue_pv(0, j);
                 const bool more = j + 1 < n_kv;
                 if (more) {
                     const int s1 = (j + 1) % kStages;
-                    if (!(ok = wait_or_abort(sy.k_full[s1], ((j + 1) / kStages) & 1, abort_flag))) break;
+                    if (!(ok = wait_or_abort_thread(sy.k_full[s1], ((j + 1) / kStages) & 1, abort_flag))) break;
                     tc_fence_after();
                     issue_s(0, j + 1);
                 }
                 if (has_q1) {
-                    if (!(ok = wait_or_abort(sy.p_full[1], j & 1, abort_flag))) break;
+                    if (!(ok = wait_or_abort_thread(sy.p_full[1], j & 1, abort_flag))) break;
                     tc_fence_after();
                     issue_pv(1, j);
                 }
