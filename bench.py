@@ -64,6 +64,8 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="qwen3_0.6b_decode_28l", choices=sorted(wl.BY_NAME))
     ap.add_argument("--kv-chunk", type=int, default=0, help="decode keys per split (0 = automatic plan)")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="run only the first N layers (small cases for profiling; 0 = the workload's own)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="bound of the cpu_baseline sample")
@@ -429,6 +431,8 @@ def run_ours(args):
     device = torch.device("cuda", dist.local)
     torch.cuda.set_device(device)
     spec = rank_spec(wl.BY_NAME[args.workload], dist.rank)
+    if args.layers:
+        spec = dataclasses.replace(spec, num_layers=min(args.layers, spec.num_layers))
     step = wl.make_step(spec)
     bench = (DecodeBench if spec.kind == "decode" else ExtendBench)(spec, step, device, args.kv_chunk)
     flush = None

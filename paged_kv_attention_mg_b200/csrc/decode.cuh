@@ -80,8 +80,12 @@ __device__ __forceinline__ int checked_length(const Params &p, int r, int &row) 
     return L;
 }
 
+#ifndef MG_DECODE_MIN_BLOCKS
+#define MG_DECODE_MIN_BLOCKS 2  // resident CTAs per SM the register budget is sized for
+#endif
+
 template <int STAGES>
-__global__ void __launch_bounds__(kThreads, 2) decode_split_kernel(const Params p) {
+__global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS) decode_split_kernel(const Params p) {
     using S = Smem<STAGES>;
     extern __shared__ __align__(1024) uint8_t smem[];
     int32_t *idx = reinterpret_cast<int32_t *>(smem + S::kIdxOffset);

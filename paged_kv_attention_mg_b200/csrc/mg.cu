@@ -16,7 +16,10 @@ namespace mg {
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr int kDecodeStages = 3;
+#ifndef MG_DECODE_STAGES
+#define MG_DECODE_STAGES 3  // cp.async ring depth of the decode split kernel (build-time tunable)
+#endif
+constexpr int kDecodeStages = MG_DECODE_STAGES;
 
 int g_sm_count[kMaxDevices];
 bool g_attr_done[kMaxDevices];

@@ -156,10 +156,13 @@ def test_decode_split_count_independence_and_determinism():
     a = g.decode(kv_chunk=64).float()
     b = g.decode(kv_chunk=2048).float()
     c = g.decode().float()
-    # different split counts only reorder fp32 sums: at most a bf16 ulp apart
-    tol = torch.maximum(a.abs(), b.abs()) * 2.0 ** -7 + 1e-6
+    # different split counts change the running max each P is scaled by before
+    # its bf16 rounding, so results differ by rounding noise, not by a fixed ulp
+    tol = torch.maximum(a.abs(), b.abs()) * 2.0 ** -7 + 2e-3
     assert bool(((a - b).abs() <= tol).all())
     assert bool(((a - c).abs() <= tol).all())
+    assert_matches_oracle(a, oracle_decode(step, data), "chunk 64")
+    assert_matches_oracle(b, oracle_decode(step, data), "chunk 2048")
     c2 = g.decode().float()
     assert torch.equal(c, c2)
 
@@ -192,15 +195,16 @@ def test_decode_flags_bad_metadata_without_faulting():
 
 
 def test_decode_host_errors():
-    step, data = _custom("decode", [9], [10], 16, 8, seed=9)
+    step, data = _custom("decode", [299], [300], 16, 8, seed=9)
     g = GpuStep(step, data)
+    assert mg.decode_workspace_bytes(1, 16, 8, 300, kv_chunk=64) > 16  # 5 splits need partials
     with pytest.raises(mg.MgError) as e:
-        mg.decode_attn(g.q, g.k_cache, g.v_cache, g.page_table, g.table_idx, g.seq_len, 10, 0.1,
+        mg.decode_attn(g.q, g.k_cache, g.v_cache, g.page_table, g.table_idx, g.seq_len, 300, 0.1,
                        kv_chunk=64, workspace=torch.empty(16, dtype=torch.uint8, device="cuda"))
     assert e.value.status == 4
     qm = torch.empty(g.q.numel() + 8, dtype=torch.bfloat16, device="cuda")[1:1 + g.q.numel()].view(g.q.shape)
     with pytest.raises(mg.MgError) as e:
-        mg.decode_attn(qm, g.k_cache, g.v_cache, g.page_table, g.table_idx, g.seq_len, 10, 0.1)
+        mg.decode_attn(qm, g.k_cache, g.v_cache, g.page_table, g.table_idx, g.seq_len, 300, 0.1)
     assert e.value.status == 3
 
 
