@@ -28,7 +28,6 @@ from __future__ import annotations
 
 import argparse
 import dataclasses
-import datetime
 import hashlib
 import json
 import os
@@ -45,6 +44,7 @@ sys.path.insert(0, ROOT)
 import torch  # noqa: E402
 
 from paged_kv_attention_mg_b200 import roofline as rf  # noqa: E402
+from paged_kv_attention_mg_b200.replicas import Replicas, rank_spec  # noqa: E402
 from paged_kv_attention_mg_b200 import workload as wl  # noqa: E402
 
 METRIC = "paged decode-attention KV GB/s (% of HBM peak) and decode tokens/s, 1 B200"
@@ -63,7 +63,7 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="qwen3_0.6b_decode_28l", choices=sorted(wl.BY_NAME))
-    ap.add_argument("--kv-chunk", type=int, default=0, help="decode keys per split (0 = automatic plan)")
+    ap.add_argument("--partitions", type=int, default=0, help="decode workers (0 = automatic plan)")
     ap.add_argument("--layers", type=int, default=0,
                     help="run only the first N layers (small cases for profiling; 0 = the workload's own)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -75,45 +75,6 @@ def parse_args():
 
 
 # ----------------------------------------------------------------------------- plumbing
-
-class Dist:
-    def __init__(self, want: int):
-        self.world = int(os.environ.get("WORLD_SIZE", "1"))
-        self.rank = int(os.environ.get("RANK", "0"))
-        self.local = int(os.environ.get("LOCAL_RANK", "0"))
-        if want != self.world:
-            raise SystemExit(f"--gpus {want} but WORLD_SIZE={self.world}: launch N>1 with torchrun")
-        self.pg = None
-        if self.world > 1:
-            import torch.distributed as dist
-            torch.cuda.set_device(self.local)
-            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
-                                    device_id=torch.device("cuda", self.local))
-            self.pg = dist
-
-    def barrier(self):
-        if self.pg:
-            self.pg.barrier()
-
-    def max(self, x: float) -> float:
-        if not self.pg:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
-        return float(t.item())
-
-    def sum(self, x: float) -> float:
-        if not self.pg:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        self.pg.all_reduce(t, op=self.pg.ReduceOp.SUM)
-        return float(t.item())
-
-    def close(self):
-        if self.pg:
-            self.pg.barrier()
-            self.pg.destroy_process_group()
-
 
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -203,10 +164,6 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- workloads
 
-def rank_spec(spec, rank: int):
-    return dataclasses.replace(spec, seed=spec.seed + 7919 * rank) if rank else spec
-
-
 def make_layers(step, num_layers, device):
     """Per-layer device tensors.  Host generation runs on a thread pool (each
     layer has its own generator, so the result does not depend on threading)."""
@@ -222,7 +179,7 @@ def make_layers(step, num_layers, device):
 
 
 class DecodeBench:
-    def __init__(self, spec, step, device, kv_chunk):
+    def __init__(self, spec, step, device, partitions):
         from paged_kv_attention_mg_b200 import mg
         self.mg = mg
         self.spec, self.step, self.device = spec, step, device
@@ -231,10 +188,10 @@ class DecodeBench:
         self.meta_host = {n: getattr(step, n).pin_memory() for n in ("page_table", "table_idx", "seq_len",
                                                                       "out_loc")}
         self.max_seq_len = step.max_seq_len
-        self.kv_chunk = kv_chunk
+        self.partitions = partitions
         B, hq, hkv = step.batch, spec.num_q_heads, spec.num_kv_heads
-        self.chunk, self.num_splits = mg.decode_plan(B, hkv, self.max_seq_len, kv_chunk)
-        ws = mg.decode_workspace_bytes(B, hq, hkv, self.max_seq_len, kv_chunk)
+        self.workers, self.slots = mg.decode_plan(B, hkv, self.max_seq_len, partitions)
+        ws = mg.decode_workspace_bytes(B, hq, hkv, self.max_seq_len, partitions)
         self.workspace = torch.empty(max(ws, 16), dtype=torch.uint8, device=device)
         self.outs = [torch.empty((B, hq, spec.head_dim), dtype=torch.bfloat16, device=device)
                      for _ in range(spec.num_layers)]
@@ -244,7 +201,7 @@ class DecodeBench:
         self.store_bytes = rf.store_bytes(step.num_new_tokens, hkv, spec.head_dim)
         self.step_bytes = spec.num_layers * (self.decode_bytes + self.store_bytes)
         self.tokens_per_step = B
-        self.launches_per_step = spec.num_layers * (2 + (1 if self.num_splits > 1 else 0))
+        self.launches_per_step = spec.num_layers * 3  # store, decode workers, merge
         self.h2d_bytes = sum(t.numel() * t.element_size() for t in self.meta_host.values()) + spec.num_layers * (
             self.layers[0]["q"].numel() * 2 + 2 * self.layers[0]["k_new"].numel() * 2)
         self.d2h_bytes = sum(o.numel() * 2 for o in self.outs)
@@ -256,7 +213,7 @@ class DecodeBench:
         if events:
             events[0].record()
         mg.decode_attn(lay["q"], lay["k_cache"], lay["v_cache"], meta["page_table"], meta["table_idx"],
-                       meta["seq_len"], self.max_seq_len, self.spec.scale, kv_chunk=self.kv_chunk, out=out,
+                       meta["seq_len"], self.max_seq_len, self.spec.scale, num_partitions=self.partitions, out=out,
                        workspace=self.workspace)
         if events:
             events[1].record()
@@ -288,13 +245,13 @@ class DecodeBench:
         return {"workload": s.name, "batch": st.batch, "layers": s.num_layers, "q_heads": s.num_q_heads,
                 "kv_heads": s.num_kv_heads, "head_dim": s.head_dim, "pool_slots": s.num_slots,
                 "mean_seq_len": round(float(st.seq_len.double().mean()), 1), "max_seq_len": st.max_seq_len,
-                "kv_chunk": self.chunk, "num_splits": self.num_splits,
+                "decode_workers": self.workers,
                 "l2": f"inputs larger than L2: {s.num_layers} per-layer pools, "
                       f"{self.spec.num_layers * self.decode_bytes / 1e9:.2f} GB read per step"}
 
 
 class ExtendBench:
-    def __init__(self, spec, step, device, kv_chunk):
+    def __init__(self, spec, step, device, partitions):
         from paged_kv_attention_mg_b200 import mg
         self.mg = mg
         self.spec, self.step, self.device = spec, step, device
@@ -313,7 +270,7 @@ class ExtendBench:
         self.h2d_bytes = sum(t.numel() * t.element_size() for t in self.meta_host.values()) + spec.num_layers * (
             self.layers[0]["q"].numel() * 2 + 2 * self.layers[0]["k_new"].numel() * 2)
         self.d2h_bytes = sum(o.numel() * 2 for o in self.outs)
-        self.chunk = self.num_splits = None
+        self.workers = None
 
     def layer(self, lay, out, meta, events=None):
         mg, st = self.mg, self.step
@@ -427,14 +384,14 @@ def run_reference(args):
 
 
 def run_ours(args):
-    dist = Dist(args.gpus)
+    dist = Replicas(args.gpus, backend="nccl")
     device = torch.device("cuda", dist.local)
     torch.cuda.set_device(device)
     spec = rank_spec(wl.BY_NAME[args.workload], dist.rank)
     if args.layers:
         spec = dataclasses.replace(spec, num_layers=min(args.layers, spec.num_layers))
     step = wl.make_step(spec)
-    bench = (DecodeBench if spec.kind == "decode" else ExtendBench)(spec, step, device, args.kv_chunk)
+    bench = (DecodeBench if spec.kind == "decode" else ExtendBench)(spec, step, device, args.partitions)
     flush = None
     if spec.kind == "extend":
         flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
@@ -502,7 +459,7 @@ def run_ours(args):
         unit = "GB/s"
         metric = METRIC
         achieved = bench.decode_bytes / (kernel_ms * 1e-3) / 1e9
-        roof = {"bound": "hbm", "kernel": "decode_split_kernel + decode_merge_kernel (one mg_decode_attn call)",
+        roof = {"bound": "hbm", "kernel": "decode_kernel + decode_merge_kernel (one mg_decode_attn call)",
                 "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s", "frac": round(achieved / hbm, 4),
                 "peak_source": f"{peak_src} HBM copy bandwidth",
                 "traffic": profiled_traffic(spec.name)}

@@ -102,19 +102,21 @@ mg_status mg_store_kv(const void *k, const void *v, const int32_t *out_loc, int3
 
 /*
  * mg_decode_plan -- the host-side plan of mg_decode_attn (the role FlashInfer's
- * "plan" step plays, Stage 4 page, §Checkpoint): keys per split (`chunk`, a
- * multiple of 64) and the number of splits of the longest request.
- * kv_chunk > 0 forces that chunk (rounded up to a multiple of 64); kv_chunk == 0
- * picks one from batch x num_kv_heads x max_seq_len and the SM count of the
- * current device.  The plan depends only on these arguments, so a captured
- * launch stays valid for any batch whose lengths stay <= max_seq_len.
+ * "plan" step plays, Stage 4 page, §Checkpoint).  The decode work is cut into
+ * units of 16 keys of one (request, kv head) pair; `workers` warps share the
+ * units equally and in order, so a pair may be split across workers, whose
+ * partial results a merge kernel combines.  num_partitions == 0 picks one
+ * worker per resident warp slot of the current device (SMs x 12); > 0 forces
+ * that many workers.  slots_out = batch * num_kv_heads + workers partial slots.
+ * The plan depends only on these arguments (never on the lengths), so a
+ * captured launch stays valid for any batch with lengths <= max_seq_len.
  */
 mg_status mg_decode_plan(int32_t batch, int32_t num_kv_heads, int32_t max_seq_len,
-                         int32_t kv_chunk, int32_t *chunk_out, int32_t *num_splits_out);
+                         int32_t num_partitions, int32_t *workers_out, int64_t *slots_out);
 
-/* Bytes of workspace mg_decode_attn needs for this plan (0 when one split). */
+/* Bytes of workspace mg_decode_attn needs for this plan (0 on bad arguments). */
 size_t mg_decode_workspace_bytes(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
-                                 int32_t head_dim, int32_t max_seq_len, int32_t kv_chunk);
+                                 int32_t head_dim, int32_t max_seq_len, int32_t num_partitions);
 
 /*
  * mg_decode_attn -- paged decode attention, one query token per request
@@ -130,19 +132,21 @@ size_t mg_decode_workspace_bytes(int32_t batch, int32_t num_q_heads, int32_t num
  *   q, out        [batch, num_q_heads, head_dim] bf16 (out rounded from fp32, RNE)
  *   page_table    [page_table_rows, page_table_stride] int32
  *   table_idx, seq_len  [batch] int32, 1 <= seq_len[r] <= min(max_seq_len, stride)
- *   max_seq_len   host-side upper bound of seq_len (sizes the split grid)
- *   kv_chunk      0 = automatic split plan; > 0 forces keys per split
+ *   max_seq_len   host-side upper bound of seq_len
+ *   num_partitions 0 = automatic plan; > 0 forces the number of workers
  *   workspace     device buffer of >= mg_decode_workspace_bytes(...) bytes,
- *                 16-byte aligned; may be NULL when that is 0.  Contents on
- *                 entry do not matter; they are scratch for the split partials.
- * Supported: head_dim == 128, num_q_heads % num_kv_heads == 0, group <= 16.
+ *                 16-byte aligned.  Contents on entry do not matter; it holds
+ *                 the per-request unit prefix and the partial results.
+ * Launches two kernels on `stream` (workers, then merge).
+ * Supported: head_dim == 128, num_q_heads % num_kv_heads == 0, group <= 16,
+ * batch <= 131072.
  */
 mg_status mg_decode_attn(const void *q, const void *k_cache, const void *v_cache, int64_t num_slots,
                          const int32_t *page_table, int32_t page_table_rows,
                          int32_t page_table_stride, const int32_t *table_idx,
                          const int32_t *seq_len, int32_t batch, int32_t max_seq_len,
                          int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, float scale,
-                         int32_t kv_chunk, void *out, void *workspace, size_t workspace_bytes,
+                         int32_t num_partitions, void *out, void *workspace, size_t workspace_bytes,
                          void *stream);
 
 /*

@@ -16,10 +16,7 @@ namespace mg {
 namespace {
 
 constexpr int kMaxDevices = 64;
-#ifndef MG_DECODE_STAGES
-#define MG_DECODE_STAGES 3  // cp.async ring depth of the decode split kernel (build-time tunable)
-#endif
-constexpr int kDecodeStages = MG_DECODE_STAGES;
+constexpr int kMaxDecodeWorkers = 1 << 22;
 
 int g_sm_count[kMaxDevices];
 bool g_attr_done[kMaxDevices];
@@ -52,9 +49,8 @@ mg_status ensure_kernel_attributes() {
     if (g_attr_done[dev]) return MG_OK;
     std::lock_guard<std::mutex> lock(g_attr_mutex);
     if (g_attr_done[dev]) return MG_OK;
-    if (cudaFuncSetAttribute(decode::decode_split_kernel<kDecodeStages>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             decode::Smem<kDecodeStages>::kBytes) != cudaSuccess)
+    if (cudaFuncSetAttribute(decode::decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             decode::kSmemBytes) != cudaSuccess)
         return MG_ERR_CUDA;
     if (extend::set_attributes() != cudaSuccess) return MG_ERR_CUDA;
     g_attr_done[dev] = true;
@@ -65,35 +61,39 @@ mg_status launched() {
     return cudaGetLastError() == cudaSuccess ? MG_OK : MG_ERR_CUDA;
 }
 
-// Split plan: keys per split (multiple of the 64-key tile, <= 2048) and the
-// number of splits of a max_seq_len request.  Aim for ~4 waves of 2 CTAs per
-// SM if every request were max_seq_len long; shorter requests end early and
-// leave room, longer splits would leave a long tail.
-mg_status decode_plan(int batch, int hkv, int max_seq_len, int kv_chunk, int &chunk, int &nsplits) {
-    if (batch <= 0 || hkv <= 0 || max_seq_len <= 0 || kv_chunk < 0) return MG_ERR_INVALID_ARGUMENT;
-    const int tile = decode::kTile;
-    if (kv_chunk > 0) {
-        chunk = (kv_chunk + tile - 1) / tile * tile;
-        if (chunk > decode::kMaxChunk) return MG_ERR_INVALID_ARGUMENT;
+// Decode plan: the number of workers (warps) that share the work equally.
+// Automatic: one per warp slot the device keeps resident (SMs x resident CTAs
+// x 4), i.e. a single persistent wave.  Forced: num_partitions workers.
+mg_status decode_plan(int batch, int hkv, int max_seq_len, int num_partitions, int &workers) {
+    if (batch <= 0 || hkv <= 0 || max_seq_len <= 0 || num_partitions < 0) return MG_ERR_INVALID_ARGUMENT;
+    if (batch > decode::kMaxScanChunks * decode::kScanChunk) return MG_ERR_UNSUPPORTED_SHAPE;
+    if (num_partitions > 0) {
+        if (num_partitions > kMaxDecodeWorkers) return MG_ERR_INVALID_ARGUMENT;
+        workers = num_partitions;
     } else {
         int sms;
         if (sm_count(sms) != MG_OK) return MG_ERR_CUDA;
-        const double target_ctas = (double)sms * 2.0 * 4.0;
-        const double work = (double)max_seq_len * (double)batch * (double)hkv;
-        long long c = (long long)((work / target_ctas) + tile - 1) / tile * tile;
-        if (c < 256) c = 256;
-        if (c > decode::kMaxChunk) c = decode::kMaxChunk;
-        chunk = (int)c;
+        workers = sms * MG_DECODE_MIN_BLOCKS * decode::kWarps;
     }
-    nsplits = (max_seq_len + chunk - 1) / chunk;
-    if (nsplits > 65535) return MG_ERR_INVALID_ARGUMENT;
     return MG_OK;
 }
 
-size_t decode_ws_bytes(int batch, int hq, int nsplits) {
-    if (nsplits <= 1) return 0;
-    const size_t rows = (size_t)batch * hq * nsplits;
-    return rows * kHeadDim * sizeof(float) + ((rows * sizeof(float) + 255) / 256) * 256;
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+// Workspace: per-request unit prefix (int64), then per-slot log-sum-exp and
+// partial outputs (fp32); slots = pairs + workers.
+struct DecodeWorkspace {
+    size_t prefix, lse, o, total;
+};
+DecodeWorkspace decode_ws_layout(int batch, int hq, int hkv, int workers) {
+    const size_t slots = (size_t)batch * hkv + (size_t)workers;
+    const size_t g = (size_t)(hq / hkv);
+    DecodeWorkspace w;
+    w.prefix = 0;
+    w.lse = align256((size_t)(batch + 1) * sizeof(int64_t));
+    w.o = w.lse + align256(slots * g * sizeof(float));
+    w.total = w.o + slots * g * kHeadDim * sizeof(float);
+    return w;
 }
 
 mg_status check_attention_shape(int hq, int hkv, int head_dim) {
@@ -155,22 +155,22 @@ mg_status mg_store_kv(const void *k, const void *v, const int32_t *out_loc, int3
     return launched();
 }
 
-mg_status mg_decode_plan(int32_t batch, int32_t num_kv_heads, int32_t max_seq_len, int32_t kv_chunk,
-                         int32_t *chunk_out, int32_t *num_splits_out) {
-    int chunk, ns;
-    mg_status st = decode_plan(batch, num_kv_heads, max_seq_len, kv_chunk, chunk, ns);
+mg_status mg_decode_plan(int32_t batch, int32_t num_kv_heads, int32_t max_seq_len,
+                         int32_t num_partitions, int32_t *workers_out, int64_t *slots_out) {
+    int workers;
+    mg_status st = decode_plan(batch, num_kv_heads, max_seq_len, num_partitions, workers);
     if (st != MG_OK) return st;
-    if (chunk_out) *chunk_out = chunk;
-    if (num_splits_out) *num_splits_out = ns;
+    if (workers_out) *workers_out = workers;
+    if (slots_out) *slots_out = (int64_t)batch * num_kv_heads + workers;
     return MG_OK;
 }
 
 size_t mg_decode_workspace_bytes(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
-                                 int32_t head_dim, int32_t max_seq_len, int32_t kv_chunk) {
-    (void)head_dim;
-    int chunk, ns;
-    if (decode_plan(batch, num_kv_heads, max_seq_len, kv_chunk, chunk, ns) != MG_OK) return 0;
-    return decode_ws_bytes(batch, num_q_heads, ns);
+                                 int32_t head_dim, int32_t max_seq_len, int32_t num_partitions) {
+    int workers;
+    if (check_attention_shape(num_q_heads, num_kv_heads, head_dim) != MG_OK) return 0;
+    if (decode_plan(batch, num_kv_heads, max_seq_len, num_partitions, workers) != MG_OK) return 0;
+    return decode_ws_layout(batch, num_q_heads, num_kv_heads, workers).total;
 }
 
 mg_status mg_decode_attn(const void *q, const void *k_cache, const void *v_cache, int64_t num_slots,
@@ -178,7 +178,7 @@ mg_status mg_decode_attn(const void *q, const void *k_cache, const void *v_cache
                          int32_t page_table_stride, const int32_t *table_idx,
                          const int32_t *seq_len, int32_t batch, int32_t max_seq_len,
                          int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, float scale,
-                         int32_t kv_chunk, void *out, void *workspace, size_t workspace_bytes,
+                         int32_t num_partitions, void *out, void *workspace, size_t workspace_bytes,
                          void *stream) {
     mg_status st = check_attention_shape(num_q_heads, num_kv_heads, head_dim);
     if (st != MG_OK) return st;
@@ -189,14 +189,12 @@ mg_status mg_decode_attn(const void *q, const void *k_cache, const void *v_cache
         return MG_ERR_INVALID_ARGUMENT;
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
         return MG_ERR_MISALIGNED;
-    int chunk, ns;
-    st = decode_plan(batch, num_kv_heads, max_seq_len, kv_chunk, chunk, ns);
+    int workers;
+    st = decode_plan(batch, num_kv_heads, max_seq_len, num_partitions, workers);
     if (st != MG_OK) return st;
-    const size_t need = decode_ws_bytes(batch, num_q_heads, ns);
-    if (need > 0) {
-        if (!workspace || workspace_bytes < need) return MG_ERR_WORKSPACE_TOO_SMALL;
-        if (!aligned16(workspace)) return MG_ERR_MISALIGNED;
-    }
+    const DecodeWorkspace ws = decode_ws_layout(batch, num_q_heads, num_kv_heads, workers);
+    if (!workspace || workspace_bytes < ws.total) return MG_ERR_WORKSPACE_TOO_SMALL;
+    if (!aligned16(workspace)) return MG_ERR_MISALIGNED;
     if (ensure_kernel_attributes() != MG_OK) return MG_ERR_CUDA;
 
     decode::Params p;
@@ -207,9 +205,10 @@ mg_status mg_decode_attn(const void *q, const void *k_cache, const void *v_cache
     p.table_idx = table_idx;
     p.seq_len = seq_len;
     p.out = static_cast<__nv_bfloat16 *>(out);
-    const size_t rows = (size_t)batch * num_q_heads * ns;
-    p.part_o = need ? static_cast<float *>(workspace) : nullptr;
-    p.part_lse = need ? static_cast<float *>(workspace) + rows * kHeadDim : nullptr;
+    uint8_t *wsb = static_cast<uint8_t *>(workspace);
+    p.prefix = reinterpret_cast<int64_t *>(wsb + ws.prefix);
+    p.part_lse = reinterpret_cast<float *>(wsb + ws.lse);
+    p.part_o = reinterpret_cast<float *>(wsb + ws.o);
     p.num_slots = num_slots;
     p.pt_rows = page_table_rows;
     p.pt_stride = page_table_stride;
@@ -217,22 +216,17 @@ mg_status mg_decode_attn(const void *q, const void *k_cache, const void *v_cache
     p.num_q_heads = num_q_heads;
     p.num_kv_heads = num_kv_heads;
     p.group = num_q_heads / num_kv_heads;
-    p.chunk = chunk;
-    p.num_splits = ns;
+    p.num_workers = workers;
     p.max_seq_len = max_seq_len;
     p.scale_log2 = scale * kLog2e;
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    dim3 grid(num_kv_heads, ns, batch);
-    decode::decode_split_kernel<kDecodeStages>
-        <<<grid, decode::kThreads, decode::Smem<kDecodeStages>::kBytes, s>>>(p);
+    const int ctas = (workers + decode::kWarps - 1) / decode::kWarps;
+    decode::decode_kernel<<<ctas, decode::kThreads, decode::kSmemBytes, s>>>(p);
     if ((st = launched()) != MG_OK) return st;
-    if (ns > 1) {
-        const int warps = batch * num_q_heads;
-        decode::decode_merge_kernel<<<(warps + 3) / 4, 128, 0, s>>>(p);
-        if ((st = launched()) != MG_OK) return st;
-    }
-    return MG_OK;
+    const int warps = batch * num_q_heads;
+    decode::decode_merge_kernel<<<(warps + 3) / 4, 128, 0, s>>>(p);
+    return launched();
 }
 
 mg_status mg_extend_attn(const void *q, const void *k_cache, const void *v_cache, int64_t num_slots,

@@ -38,7 +38,7 @@ SIGNATURES = {
     "mg_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "mg_abi_version": (_I32, []),
     "mg_store_kv": (ctypes.c_int, [_P, _P, _P, _I32, _P, _P, _I64, _I32, _I32, _P]),
-    "mg_decode_plan": (ctypes.c_int, [_I32, _I32, _I32, _I32, ctypes.POINTER(_I32), ctypes.POINTER(_I32)]),
+    "mg_decode_plan": (ctypes.c_int, [_I32, _I32, _I32, _I32, ctypes.POINTER(_I32), ctypes.POINTER(_I64)]),
     "mg_decode_workspace_bytes": (_SZ, [_I32, _I32, _I32, _I32, _I32, _I32]),
     "mg_decode_attn": (ctypes.c_int, [_P, _P, _P, _I64, _P, _I32, _I32, _P, _P, _I32, _I32, _I32, _I32,
                                       _I32, _F32, _I32, _P, _P, _SZ, _P]),
@@ -113,30 +113,30 @@ def store_kv(k: torch.Tensor, v: torch.Tensor, out_loc: torch.Tensor, k_cache: t
                               _stream(stream)), "mg_store_kv")
 
 
-def decode_plan(batch: int, num_kv_heads: int, max_seq_len: int, kv_chunk: int = 0):
-    """(keys per split, number of splits) that mg_decode_attn will use."""
-    chunk, ns = _I32(), _I32()
-    _check(load().mg_decode_plan(batch, num_kv_heads, max_seq_len, kv_chunk, ctypes.byref(chunk),
-                                 ctypes.byref(ns)), "mg_decode_plan")
-    return chunk.value, ns.value
+def decode_plan(batch: int, num_kv_heads: int, max_seq_len: int, num_partitions: int = 0):
+    """(workers, partial slots) that mg_decode_attn will use."""
+    workers, slots = _I32(), _I64()
+    _check(load().mg_decode_plan(batch, num_kv_heads, max_seq_len, num_partitions, ctypes.byref(workers),
+                                 ctypes.byref(slots)), "mg_decode_plan")
+    return workers.value, slots.value
 
 
 def decode_workspace_bytes(batch: int, num_q_heads: int, num_kv_heads: int, max_seq_len: int,
-                           kv_chunk: int = 0, head_dim: int = 128) -> int:
+                           num_partitions: int = 0, head_dim: int = 128) -> int:
     return int(load().mg_decode_workspace_bytes(batch, num_q_heads, num_kv_heads, head_dim, max_seq_len,
-                                                 kv_chunk))
+                                                 num_partitions))
 
 
 def decode_attn(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, page_table: torch.Tensor,
                 table_idx: torch.Tensor, seq_len: torch.Tensor, max_seq_len: int, scale: float,
-                kv_chunk: int = 0, out: Optional[torch.Tensor] = None,
+                num_partitions: int = 0, out: Optional[torch.Tensor] = None,
                 workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """Paged decode attention; returns out [B, Hq, D] bf16."""
     b, hq, d = q.shape
     hkv = k_cache.shape[1]
     if out is None:
         out = torch.empty_like(q)
-    need = decode_workspace_bytes(b, hq, hkv, max_seq_len, kv_chunk, d)
+    need = decode_workspace_bytes(b, hq, hkv, max_seq_len, num_partitions, d)
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_ptr = _dev(workspace, torch.uint8, "workspace") if workspace is not None else None
@@ -146,7 +146,7 @@ def decode_attn(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, p
                                  _dev(page_table, torch.int32, "page_table"), page_table.shape[0],
                                  page_table.shape[1], _dev(table_idx, torch.int32, "table_idx"),
                                  _dev(seq_len, torch.int32, "seq_len"), b, max_seq_len, hq, hkv, d,
-                                 float(scale), kv_chunk, _dev(out, torch.bfloat16, "out"), ws_ptr, ws_bytes,
+                                 float(scale), num_partitions, _dev(out, torch.bfloat16, "out"), ws_ptr, ws_bytes,
                                  _stream(stream)), "mg_decode_attn")
     return out
 

@@ -145,11 +145,11 @@ class GpuStep:
         from paged_kv_attention_mg_b200 import mg
         mg.store_kv(self.k_new, self.v_new, self.out_loc, self.k_cache, self.v_cache)
 
-    def decode(self, kv_chunk=0, max_seq_len=None, out=None):
+    def decode(self, num_partitions=0, max_seq_len=None, out=None):
         from paged_kv_attention_mg_b200 import mg
         msl = max_seq_len or self.step.max_seq_len
         return mg.decode_attn(self.q, self.k_cache, self.v_cache, self.page_table, self.table_idx, self.seq_len,
-                              msl, self.scale, kv_chunk=kv_chunk, out=out)
+                              msl, self.scale, num_partitions=num_partitions, out=out)
 
     def extend(self, out=None):
         from paged_kv_attention_mg_b200 import mg

@@ -83,17 +83,24 @@ def test_decode_rejects_bad_hints(lib):
     # max_seq_len above the page-table width
     assert lib.mg_decode_attn(4096, 4096, 4096, 100, 4096, 5, 32, 4096, 4096, 4, 33, 16, 8, 128, 0.1, 0,
                               4096, None, 0, None) == 1
-    # forced chunk above the prefetch capacity
+    # negative partition count
     assert lib.mg_decode_attn(4096, 4096, 4096, 100, 4096, 5, 4096, 4096, 4096, 4, 4096, 16, 8, 128, 0.1,
-                              4096, 4096, None, 0, None) == 1
+                              -3, 4096, None, 0, None) == 1
+    # batch beyond the in-kernel scan capacity
+    assert lib.mg_decode_attn(4096, 4096, 4096, 100, 4096, 5, 4096, 4096, 4096, 131073, 4096, 16, 8, 128,
+                              0.1, 8, 4096, 4096, 1 << 40, None) == 2
 
 
-def test_decode_plan_with_forced_chunk_needs_no_device(lib):
-    chunk, ns = ctypes.c_int32(), ctypes.c_int32()
-    assert lib.mg_decode_plan(8, 4, 32768, 1000, ctypes.byref(chunk), ctypes.byref(ns)) == 0
-    assert chunk.value == 1024 and ns.value == 32
-    assert lib.mg_decode_workspace_bytes(8, 32, 4, 128, 32768, 1000) >= 8 * 32 * 32 * (128 + 1) * 4
-    assert lib.mg_decode_workspace_bytes(8, 32, 4, 128, 1000, 1024) == 0  # one split
+def test_decode_plan_with_forced_partitions_needs_no_device(lib):
+    workers, slots = ctypes.c_int32(), ctypes.c_int64()
+    assert lib.mg_decode_plan(8, 4, 32768, 1000, ctypes.byref(workers), ctypes.byref(slots)) == 0
+    assert workers.value == 1000 and slots.value == 8 * 4 + 1000
+    # prefix (B+1 int64, 256-aligned) + lse (slots x g fp32, 256-aligned) + partial O (slots x g x 128 fp32)
+    g = 32 // 4
+    a256 = lambda x: (x + 255) // 256 * 256
+    want = a256(9 * 8) + a256(1032 * g * 4) + 1032 * g * 128 * 4
+    assert lib.mg_decode_workspace_bytes(8, 32, 4, 128, 32768, 1000) == want
+    assert lib.mg_decode_workspace_bytes(8, 12, 8, 128, 32768, 1000) == 0  # unsupported shape
 
 
 def test_extend_rejects_shapes_and_empty_is_noop(lib):

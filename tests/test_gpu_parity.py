@@ -89,14 +89,14 @@ DECODE_SMALL = [
 
 
 @pytest.mark.parametrize("lengths,hq,hkv", DECODE_SMALL)
-@pytest.mark.parametrize("kv_chunk", [0, 64, 128])
-def test_decode_small_matches_oracle(lengths, hq, hkv, kv_chunk):
+@pytest.mark.parametrize("parts", [0, 1, 7])
+def test_decode_small_matches_oracle(lengths, hq, hkv, parts):
     step, data = _custom("decode", [L - 1 for L in lengths], lengths, hq, hkv, seed=len(lengths) * 31 + hq)
     g = GpuStep(step, data)
     g.store()
-    out = g.decode(kv_chunk=kv_chunk)
+    out = g.decode(num_partitions=parts)
     assert mg.read_device_error() == 0
-    assert_matches_oracle(out, oracle_decode(step, data), f"decode {lengths} chunk {kv_chunk}")
+    assert_matches_oracle(out, oracle_decode(step, data), f"decode {lengths} partitions {parts}")
 
 
 def test_decode_tiny_workload():
@@ -119,8 +119,8 @@ def test_decode_random_sweep():
         step, data = _custom("decode", [L - 1 for L in lengths], lengths, hkv * grp, hkv, seed=100 + it)
         g = GpuStep(step, data)
         g.store()
-        chunk = int(rng.choice([0, 64, 192]))
-        out = g.decode(kv_chunk=chunk)
+        parts = int(rng.choice([0, 1, 5, 33, 4096]))
+        out = g.decode(num_partitions=parts)
         assert_matches_oracle(out, oracle_decode(step, data), f"sweep {it}: {lengths} hkv {hkv} g {grp}")
 
 
@@ -153,16 +153,16 @@ def test_decode_split_count_independence_and_determinism():
     step, data = _custom("decode", [1500, 2047, 3, 700], [1501, 2048, 4, 701], 32, 8, seed=5)
     g = GpuStep(step, data)
     g.store()
-    a = g.decode(kv_chunk=64).float()
-    b = g.decode(kv_chunk=2048).float()
+    a = g.decode(num_partitions=1).float()
+    b = g.decode(num_partitions=997).float()
     c = g.decode().float()
-    # different split counts change the running max each P is scaled by before
+    # different partitions change the running max each P is scaled by before
     # its bf16 rounding, so results differ by rounding noise, not by a fixed ulp
     tol = torch.maximum(a.abs(), b.abs()) * 2.0 ** -7 + 2e-3
     assert bool(((a - b).abs() <= tol).all())
     assert bool(((a - c).abs() <= tol).all())
-    assert_matches_oracle(a, oracle_decode(step, data), "chunk 64")
-    assert_matches_oracle(b, oracle_decode(step, data), "chunk 2048")
+    assert_matches_oracle(a, oracle_decode(step, data), "1 worker")
+    assert_matches_oracle(b, oracle_decode(step, data), "997 workers")
     c2 = g.decode().float()
     assert torch.equal(c, c2)
 
@@ -197,10 +197,10 @@ def test_decode_flags_bad_metadata_without_faulting():
 def test_decode_host_errors():
     step, data = _custom("decode", [299], [300], 16, 8, seed=9)
     g = GpuStep(step, data)
-    assert mg.decode_workspace_bytes(1, 16, 8, 300, kv_chunk=64) > 16  # 5 splits need partials
+    assert mg.decode_workspace_bytes(1, 16, 8, 300, num_partitions=64) > 16
     with pytest.raises(mg.MgError) as e:
         mg.decode_attn(g.q, g.k_cache, g.v_cache, g.page_table, g.table_idx, g.seq_len, 300, 0.1,
-                       kv_chunk=64, workspace=torch.empty(16, dtype=torch.uint8, device="cuda"))
+                       num_partitions=64, workspace=torch.empty(16, dtype=torch.uint8, device="cuda"))
     assert e.value.status == 4
     qm = torch.empty(g.q.numel() + 8, dtype=torch.bfloat16, device="cuda")[1:1 + g.q.numel()].view(g.q.shape)
     with pytest.raises(mg.MgError) as e:
