@@ -16,10 +16,12 @@
 //     all workers finish together whatever the length mix (no tail of long
 //     splits).  A worker's share covers one or a few "segments" (its part of a
 //     pair).
-//   * per tile a worker gathers the 16 K and 16 V rows (256 B each) with
-//     16-byte cp.async into its own STAGES-deep ring, one full row per 16
-//     lanes, XOR-swizzled so ldmatrix is conflict-free; page-table entries of
-//     the next tile are prefetched one step ahead.
+//   * per tile a worker gathers the 16 K and 16 V rows (256 B each) straight
+//     from the pool with TMA tile::gather4 (4 page-table rows per instruction,
+//     128-byte swizzle, 16 instructions per tile issued by 16 lanes at once)
+//     into its own STAGES-deep ring, completion counted on one mbarrier per
+//     stage; page-table entries of the next tile are prefetched one step
+//     ahead.  Few warps with deep rings keep most of shared memory in flight.
 //   * the GQA group is the M dimension of warp-level bf16 tensor-core MMAs
 //     (m16n8k16, fp32 accumulate, g <= 16 rows, zero padded), so each K/V row
 //     is read from HBM once for all g heads: S = Q K^T, online softmax in the
@@ -33,13 +35,18 @@
 //     the scan that locates their first unit.
 #pragma once
 
+#include <cuda.h>
+
 #include "common.cuh"
 
 namespace mg {
 namespace decode {
 
 constexpr int kKeys = 16;          // keys per unit / pipeline tile
-constexpr int kWarps = 4;          // workers per CTA
+#ifndef MG_DECODE_WARPS
+#define MG_DECODE_WARPS 4  // workers per CTA (build-time tunable)
+#endif
+constexpr int kWarps = MG_DECODE_WARPS;
 constexpr int kThreads = kWarps * 32;
 constexpr int kRows = 16;          // MMA M: GQA group padded to 16
 constexpr int kRowBytes = kHeadDim * 2;
@@ -48,13 +55,15 @@ constexpr int kScanChunk = 4 * kThreads;           // requests per scan step
 constexpr int kMaxScanChunks = 256;                // requests <= 131072
 
 #ifndef MG_DECODE_STAGES
-#define MG_DECODE_STAGES 2  // per-worker cp.async ring depth (build-time tunable)
+#define MG_DECODE_STAGES 3  // per-worker ring depth (build-time tunable)
 #endif
 #ifndef MG_DECODE_MIN_BLOCKS
-#define MG_DECODE_MIN_BLOCKS 3  // resident CTAs per SM the register budget is sized for
+#define MG_DECODE_MIN_BLOCKS 2  // resident CTAs per SM (the shared memory is sized for it)
 #endif
 constexpr int kStages = MG_DECODE_STAGES;
-constexpr int kSmemBytes = kWarps * kStages * kTileBytes;
+constexpr int kRingBytes = kWarps * kStages * kTileBytes;
+constexpr int kSmemBytes = kRingBytes + 1024;  // + alignment slack (128-byte swizzle atoms)
+constexpr int kHalfRows = kKeys * 128;          // one 64-column half of a 16-row tile: 2 KB
 
 struct Params {
     const __nv_bfloat16 *q;
@@ -74,8 +83,10 @@ struct Params {
     float scale_log2;  // softmax scale * log2(e)
 };
 
+// byte offset of 16-byte chunk c (0..15) of row `row` in a [16 rows x 256 B]
+// tile stored as two 64-column halves with the 128-byte TMA swizzle
 __device__ __forceinline__ uint32_t swz(int row, int c) {
-    return (uint32_t)(row * kRowBytes + ((c ^ (row & 7)) << 4));
+    return (uint32_t)((c >> 3) * kHalfRows + row * 128 + (((c & 7) ^ (row & 7)) << 4));
 }
 
 // Units of request r (0 for a request whose metadata is invalid).
@@ -142,8 +153,34 @@ __device__ __forceinline__ void cursor_advance(const Params &p, Cursor &c) {
     if (c.r < p.batch) cursor_load_request(p, c);
 }
 
-__global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS) decode_kernel(const Params p) {
-    extern __shared__ __align__(128) uint8_t smem[];
+// Warp-uniform bounded wait on an mbarrier phase: gives up after ~2 s of
+// %globaltimer, sets MG_DEVERR_WAIT_TIMEOUT and returns false.
+__device__ __forceinline__ bool warp_wait_bounded(uint32_t bar, uint32_t parity) {
+    bool done = false;
+    uint64_t t0 = 0;
+    for (uint32_t it = 0; !done; ++it) {
+        done = mbar_try_wait(bar, parity);
+        if (!done && (it & 255u) == 255u) {
+            uint64_t now;
+            asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(now));
+            if (t0 == 0) {
+                t0 = now;
+            } else if (now - t0 > 2000000000ull) {
+                atomicOr(&g_mg_device_error, MG_DEVERR_WAIT_TIMEOUT);
+                break;
+            }
+        }
+    }
+    return __all_sync(0xffffffffu, done);
+}
+
+__global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
+    decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                  const Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ __align__(8) uint64_t full_bar[kWarps][kStages];
+    __shared__ int64_t sh_bound[kWarps + 1];
     __shared__ int64_t sh_scan[kWarps];
     __shared__ int64_t sh_chunk_excl[kMaxScanChunks + 1];
     __shared__ int sh_start_r[kWarps];
@@ -177,15 +214,16 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS) decode_kernel(
 
     // ---- pass 2: locate the request holding each worker's first unit (CTA 0
     // scans every chunk and also publishes the per-request prefix for the merge)
+    if (tid <= kWarps) sh_bound[tid] = worker_begin(T, blockIdx.x * kWarps + tid, W);
+    __syncthreads();
     {
-        const int64_t b0 = worker_begin(T, blockIdx.x * kWarps, W);
-        const int64_t b3 = worker_begin(T, blockIdx.x * kWarps + kWarps - 1, W);
+        const int64_t b0 = sh_bound[0], b3 = sh_bound[kWarps - 1];
         for (int ch = 0; ch < nchunks; ++ch) {
             const int64_t lo = sh_chunk_excl[ch], hi = sh_chunk_excl[ch + 1];
             const bool needed = blockIdx.x == 0 || (hi > b0 && lo <= b3);
             if (!needed) continue;  // uniform across the CTA
             int64_t u[4], v = 0;
-            int r0 = ch * kScanChunk + tid * 4;
+            const int r0 = ch * kScanChunk + tid * 4;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 int L, row;
@@ -203,7 +241,7 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS) decode_kernel(
                     if (blockIdx.x == 0) p.prefix[r] = pre;
 #pragma unroll
                     for (int k = 0; k < kWarps; ++k) {
-                        const int64_t bk = worker_begin(T, blockIdx.x * kWarps + k, W);
+                        const int64_t bk = sh_bound[k];
                         if (u[i] > 0 && bk >= pre && bk < pre + u[i]) {
                             sh_start_r[k] = r;
                             sh_start_prefix[k] = pre;
@@ -215,18 +253,26 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS) decode_kernel(
         }
         if (blockIdx.x == 0 && tid == 0) p.prefix[p.batch] = T;
     }
+    if (tid < kWarps * kStages) {
+        mbar_init(smem_u32(&full_bar[tid / kStages][tid % kStages]), 1);
+        fence_mbarrier_init();
+    }
     __syncthreads();
 
     // ---- this warp's share
-    const int64_t ub = worker_begin(T, w, W), ue = worker_begin(T, w + 1, W);
+    const int64_t ub = sh_bound[warp], ue = sh_bound[warp + 1];
     if (w >= W || ub >= ue) return;
     const int n_units = (int)(ue - ub);
 
-    const int64_t head_stride = (int64_t)p.num_kv_heads * kHeadDim;
     const int g = p.group;
     const uint32_t ring = smem_u32(smem) + (uint32_t)(warp * kStages * kTileBytes);
+    const int oob_row = (int)(p.num_slots * p.num_kv_heads);  // TMA reads it as zeros
+    if (lane == 0) {
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_v);
+    }
 
-    Cursor cur;  // position of the tile being prefetched
+    Cursor cur;  // position of the tile whose indices are fetched next
     cur.r = sh_start_r[warp];
     cursor_load_request(p, cur);
     {
@@ -235,9 +281,8 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS) decode_kernel(
         cur.t = (int)(off - (int64_t)cur.kvh * cur.tiles);
     }
 
-    // per-tile descriptors travel with the pipeline in registers
+    // per-tile descriptors travel with the pipeline
     Cursor dq[kStages + 1];
-    int idx_next = -1;  // lanes 0..15: slot of key lane of the next tile to issue
 
     auto fetch_idx = [&](const Cursor &c) -> int {
         const int key = c.t * kKeys + lane;
@@ -251,24 +296,30 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS) decode_kernel(
         }
         return s;
     };
+    // One warp instruction: lanes 0..15 each issue one gather4 of 4 rows x 128 B.
+    // gather index gi: K/V = gi / 8, 64-column half = (gi / 4) % 2, row quad = gi % 4.
     auto issue = [&](Cursor &c, int slot_reg, int stage) {
         c.valid = __ballot_sync(0xffffffffu, slot_reg >= 0) & 0xFFFFu;
-        const uint32_t base = ring + (uint32_t)(stage * kTileBytes);
-        const int ch = lane & 15;
-#pragma unroll
-        for (int it = 0; it < 16; ++it) {
-            const int rr = it * 2 + (lane >> 4);  // 0..31: K rows 0-15, V rows 16-31
-            const int key = rr & (kKeys - 1);
-            const bool is_v = rr >= kKeys;
-            const int slot = __shfl_sync(0xffffffffu, slot_reg, key);
-            const __nv_bfloat16 *src = (is_v ? p.v_cache : p.k_cache) +
-                                       (int64_t)(slot < 0 ? 0 : slot) * head_stride +
-                                       (int64_t)c.kvh * kHeadDim + ch * 8;
-            cp_async_16(base + (is_v ? kKeys * kRowBytes : 0) + swz(key, ch), src, slot < 0 ? 0u : 16u);
+        const int row_id = slot_reg >= 0 ? slot_reg * p.num_kv_heads + c.kvh : oob_row;
+        const int quad = lane & 3;
+        const int r0 = __shfl_sync(0xffffffffu, row_id, quad * 4 + 0);
+        const int r1 = __shfl_sync(0xffffffffu, row_id, quad * 4 + 1);
+        const int r2 = __shfl_sync(0xffffffffu, row_id, quad * 4 + 2);
+        const int r3 = __shfl_sync(0xffffffffu, row_id, quad * 4 + 3);
+        const uint32_t bar = smem_u32(&full_bar[warp][stage]);
+        if (lane == 0) mbar_arrive_expect_tx(bar, kTileBytes);
+        __syncwarp();
+        if (lane < 16) {
+            const int kind = lane >> 3, half = (lane >> 2) & 1;
+            const uint32_t dst = ring + (uint32_t)(stage * kTileBytes + kind * 2 * kHalfRows + half * kHalfRows +
+                                                   quad * 4 * 128);
+            fence_proxy_async_smem();
+            tma_gather4(dst, kind ? (const void *)&tm_v : (const void *)&tm_k, bar, half * 64, r0, r1, r2, r3);
         }
     };
 
     // prologue: tiles 0 .. STAGES-2 in flight, indices of tile STAGES-1 in registers
+    int idx_next;
     {
         int idx0 = fetch_idx(cur);
 #pragma unroll
@@ -279,7 +330,6 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS) decode_kernel(
                 cursor_advance(p, cur);
                 if (s + 1 < n_units) idx0 = fetch_idx(cur);
             }
-            cp_async_commit();
         }
         idx_next = idx0;
     }
@@ -289,9 +339,12 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS) decode_kernel(
     uint32_t qf[8][4];
     const int ra = lane >> 2, rb = ra + 8;
     int seg_first_t = 0;
+    bool ok = true;
+    int k = 0;
 
-    for (int k = 0; k < n_units; ++k) {
-        // issue tile k + STAGES - 1, prefetch the indices of the tile after it
+    for (; k < n_units; ++k) {
+        // issue tile k + STAGES - 1 (its stage was freed at the end of tile k - 1),
+        // then prefetch the indices of the tile after it
         {
             const int j = k + kStages - 1;
             if (j < n_units) {
@@ -300,7 +353,6 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS) decode_kernel(
                 cursor_advance(p, cur);
                 if (j + 1 < n_units) idx_next = fetch_idx(cur);
             }
-            cp_async_commit();
         }
         const Cursor c = dq[k % (kStages + 1)];
         const bool first = k == 0 || c.t == 0;
@@ -326,11 +378,14 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS) decode_kernel(
             l0 = l1 = 0.f;
             seg_first_t = c.t;
         }
-        cp_async_wait<kStages - 1>();
-        __syncwarp();
+        // wait for tile k (bounded: a lost transfer sets the timeout bit and ends this worker)
+        if (!warp_wait_bounded(smem_u32(&full_bar[warp][k % kStages]), (k / kStages) & 1)) {
+            ok = false;
+            break;
+        }
 
         const uint32_t kt = ring + (uint32_t)((k % kStages) * kTileBytes);
-        const uint32_t vt = kt + kKeys * kRowBytes;
+        const uint32_t vt = kt + 2 * kHalfRows;
 
         float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
         {
@@ -351,9 +406,9 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS) decode_kernel(
             for (int e = 0; e < 2; ++e) {
                 const int key = nt * 8 + (lane & 3) * 2 + e;
                 // keys past the end, or whose slot was rejected (zero-filled), are masked
-                const bool ok = (c.valid >> key) & 1u;
-                const float s0 = ok ? sc[nt][e] * p.scale_log2 : -INFINITY;
-                const float s1 = ok ? sc[nt][e + 2] * p.scale_log2 : -INFINITY;
+                const bool kv_ok = (c.valid >> key) & 1u;
+                const float s0 = kv_ok ? sc[nt][e] * p.scale_log2 : -INFINITY;
+                const float s1 = kv_ok ? sc[nt][e + 2] * p.scale_log2 : -INFINITY;
                 sc[nt][e] = s0;
                 sc[nt][e + 2] = s1;
                 mx0 = fmaxf(mx0, s0);
@@ -367,7 +422,7 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS) decode_kernel(
         const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
         const float mu0 = mn0 == -INFINITY ? 0.f : mn0;
         const float mu1 = mn1 == -INFINITY ? 0.f : mn1;
-        if (mn0 != m0 || mn1 != m1) {
+        if (__any_sync(0xffffffffu, mn0 != m0 || mn1 != m1)) {
             const float corr0 = fast_exp2(m0 - mu0), corr1 = fast_exp2(m1 - mu1);
             l0 *= corr0;
             l1 *= corr1;
@@ -447,7 +502,12 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS) decode_kernel(
             }
         }
     }
-    cp_async_wait<0>();
+    if (!ok) {
+        // give this worker's outstanding transfers (tiles k .. k+STAGES-2) a
+        // bounded chance to land before its shared memory can be released
+        for (int t = k; t < n_units && t < k + kStages - 1; ++t)
+            (void)mbar_wait_bounded(smem_u32(&full_bar[warp][t % kStages]), (t / kStages) & 1, 1u << 20);
+    }
 }
 
 // One warp per (request, q head): combine the partials of a pair that more

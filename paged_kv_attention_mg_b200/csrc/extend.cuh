@@ -421,23 +421,6 @@ inline cudaError_t set_attributes() {
     return cudaFuncSetAttribute(extend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
 }
 
-using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
-                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
-                                   CUtensorMapFloatOOBfill);
-
-inline EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void *ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(ptr);
-    }
-    return fn;
-}
-
 inline mg_status launch(Params &p, cudaStream_t stream) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return MG_ERR_CUDA;
@@ -454,19 +437,10 @@ inline mg_status launch(Params &p, cudaStream_t stream) {
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return MG_ERR_CUDA;
     }
-    const cuuint64_t pool_rows = (cuuint64_t)p.num_slots * (cuuint64_t)p.num_kv_heads;
-    if (pool_rows >= (1ull << 31)) return MG_ERR_UNSUPPORTED_SHAPE;  // gather4 row coordinates are int32
-    for (int which = 0; which < 2; ++which) {
-        cuuint64_t dims[2] = {(cuuint64_t)kHeadDim, pool_rows};
-        cuuint64_t strides[1] = {(cuuint64_t)kHeadDim * 2};
-        cuuint32_t box[2] = {64, 1};
-        cuuint32_t es[2] = {1, 1};
-        void *base = const_cast<__nv_bfloat16 *>(which == 0 ? p.k_cache : p.v_cache);
-        if (enc(which == 0 ? &tk : &tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, es,
-                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            return MG_ERR_CUDA;
-    }
+    if ((uint64_t)p.num_slots * (uint64_t)p.num_kv_heads >= (1ull << 31)) return MG_ERR_UNSUPPORTED_SHAPE;
+    if (!make_pool_tmap(&tk, p.k_cache, p.num_slots, p.num_kv_heads) ||
+        !make_pool_tmap(&tv, p.v_cache, p.num_slots, p.num_kv_heads))
+        return MG_ERR_CUDA;
     const int tokens_per_cta = kQTiles * p.tokens_per_qtile;
     const int nqb = (p.max_q_len + tokens_per_cta - 1) / tokens_per_cta;
     if (nqb > 0x7fffffff || p.batch > 65535 || p.num_kv_heads > 65535) return MG_ERR_INVALID_ARGUMENT;

@@ -220,9 +220,14 @@ mg_status mg_decode_attn(const void *q, const void *k_cache, const void *v_cache
     p.max_seq_len = max_seq_len;
     p.scale_log2 = scale * kLog2e;
 
+    if ((uint64_t)num_slots * (uint64_t)num_kv_heads >= (1ull << 31)) return MG_ERR_UNSUPPORTED_SHAPE;
+    CUtensorMap tk, tv;
+    if (!make_pool_tmap(&tk, k_cache, num_slots, num_kv_heads) ||
+        !make_pool_tmap(&tv, v_cache, num_slots, num_kv_heads))
+        return MG_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int ctas = (workers + decode::kWarps - 1) / decode::kWarps;
-    decode::decode_kernel<<<ctas, decode::kThreads, decode::kSmemBytes, s>>>(p);
+    decode::decode_kernel<<<ctas, decode::kThreads, decode::kSmemBytes, s>>>(tk, tv, p);
     if ((st = launched()) != MG_OK) return st;
     const int warps = batch * num_q_heads;
     decode::decode_merge_kernel<<<(warps + 3) / 4, 128, 0, s>>>(p);
