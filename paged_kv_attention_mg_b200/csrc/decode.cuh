@@ -60,7 +60,13 @@ constexpr int kMaxScanChunks = 256;                // requests <= 131072
 #ifndef MG_DECODE_MIN_BLOCKS
 #define MG_DECODE_MIN_BLOCKS 2  // resident CTAs per SM (the shared memory is sized for it)
 #endif
+#ifndef MG_DECODE_IDX_AHEAD
+#define MG_DECODE_IDX_AHEAD 8  // tiles of page-table entries fetched ahead of the K/V issue
+#endif
 constexpr int kStages = MG_DECODE_STAGES;
+constexpr int kIdxAhead = MG_DECODE_IDX_AHEAD;
+constexpr int kDescRing = 16;  // per-warp ring of tile descriptors / index rows
+static_assert(kDescRing >= kIdxAhead + kStages, "descriptor ring too small");
 constexpr int kRingBytes = kWarps * kStages * kTileBytes;
 constexpr int kSmemBytes = kRingBytes + 1024;  // + alignment slack (128-byte swizzle atoms)
 constexpr int kHalfRows = kKeys * 128;          // one 64-column half of a 16-row tile: 2 KB
@@ -128,15 +134,35 @@ __device__ __forceinline__ int64_t block_scan_excl(int64_t v, int64_t &excl, int
 // The walk along a worker's units: pair (r, kvh), tile t of the pair.
 struct Cursor {
     int r, kvh, t, tiles, L, row;
-    unsigned valid;  // bit i: key i of the tile has an accepted slot (set when issued)
+    int next_L, next_row;  // metadata of request r + 1, loaded ahead of the boundary
 };
 
+// What the pipeline stages need to know about one tile.
+struct TileDesc {
+    int r, kvh, t, tiles, L, row;
+    unsigned valid;  // bit i: key i has an accepted slot (set when the tile is issued)
+    int pad;
+};
+
+__device__ __forceinline__ bool metadata_ok(const Params &p, int L, int row) {
+    return row >= 0 && row < p.pt_rows && L >= 1 && L <= p.pt_stride && L <= p.max_seq_len;
+}
+
+__device__ __forceinline__ void cursor_prefetch_next(const Params &p, Cursor &c) {
+    if (c.r + 1 < p.batch) {
+        c.next_L = __ldg(p.seq_len + c.r + 1);  // consumed only at the next request boundary
+        c.next_row = __ldg(p.table_idx + c.r + 1);
+    }
+}
+
+// Position the cursor on the first request >= c.r that owns units.
 __device__ __forceinline__ void cursor_load_request(const Params &p, Cursor &c) {
     for (;;) {
         unsigned bad = 0;
         const int64_t u = request_units(p, c.r, c.L, c.row, bad);
         if (u > 0) {
             c.tiles = (c.L + kKeys - 1) / kKeys;
+            cursor_prefetch_next(p, c);
             return;
         }
         ++c.r;  // zero-unit (rejected) request: it owns no units, skip it
@@ -150,7 +176,15 @@ __device__ __forceinline__ void cursor_advance(const Params &p, Cursor &c) {
     if (++c.kvh < p.num_kv_heads) return;
     c.kvh = 0;
     ++c.r;
-    if (c.r < p.batch) cursor_load_request(p, c);
+    if (c.r >= p.batch) return;
+    if (metadata_ok(p, c.next_L, c.next_row)) {  // the common case: no stall at the boundary
+        c.L = c.next_L;
+        c.row = c.next_row;
+        c.tiles = (c.L + kKeys - 1) / kKeys;
+        cursor_prefetch_next(p, c);
+    } else {
+        cursor_load_request(p, c);
+    }
 }
 
 // Warp-uniform bounded wait on an mbarrier phase: gives up after ~2 s of
@@ -180,6 +214,8 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     __shared__ __align__(8) uint64_t full_bar[kWarps][kStages];
+    __shared__ __align__(16) int idx_ring[kWarps][kDescRing][kKeys];
+    __shared__ __align__(16) TileDesc desc_ring[kWarps][kDescRing];
     __shared__ int64_t sh_bound[kWarps + 1];
     __shared__ int64_t sh_scan[kWarps];
     __shared__ int64_t sh_chunk_excl[kMaxScanChunks + 1];
@@ -272,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
         prefetch_tmap(&tm_v);
     }
 
-    Cursor cur;  // position of the tile whose indices are fetched next
+    Cursor cur;  // position of the next tile whose page-table entries are fetched
     cur.r = sh_start_r[warp];
     cursor_load_request(p, cur);
     {
@@ -280,27 +316,47 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
         cur.kvh = (int)(off / cur.tiles);
         cur.t = (int)(off - (int64_t)cur.kvh * cur.tiles);
     }
+    int (*my_idx)[kKeys] = idx_ring[warp];
+    TileDesc *my_desc = desc_ring[warp];
 
-    // per-tile descriptors travel with the pipeline
-    Cursor dq[kStages + 1];
-
-    auto fetch_idx = [&](const Cursor &c) -> int {
-        const int key = c.t * kKeys + lane;
-        int s = -1;
-        if (lane < kKeys && key < c.L) {
-            s = __ldg(p.page_table + (int64_t)c.row * p.pt_stride + key);
-            if (s < 0 || (int64_t)s >= p.num_slots) {
+    // Fetch stage: record tile j's descriptor and start copying its 16
+    // page-table entries into the index ring (one cp.async group per tile).
+    auto fetch = [&](int j) {
+        if (j < n_units) {
+            const int e = j % kDescRing;
+            if (lane == 0) {
+                TileDesc d;
+                d.r = cur.r; d.kvh = cur.kvh; d.t = cur.t; d.tiles = cur.tiles; d.L = cur.L; d.row = cur.row;
+                d.valid = 0; d.pad = 0;
+                my_desc[e] = d;
+            }
+            const int key = cur.t * kKeys + lane;
+            if (lane < kKeys) {
+                if (key < cur.L)
+                    cp_async_4(smem_u32(&my_idx[e][lane]), p.page_table + (int64_t)cur.row * p.pt_stride + key);
+                else
+                    my_idx[e][lane] = -1;
+            }
+            cursor_advance(p, cur);
+        }
+        cp_async_commit();
+    };
+    // Issue stage: read tile j's entries, check them, and let lanes 0..15 each
+    // issue one gather4 (K/V = lane / 8, 64-column half = (lane / 4) % 2, row quad = lane % 4).
+    auto issue = [&](int j) {
+        const int e = j % kDescRing, stage = j % kStages;
+        const TileDesc d = my_desc[e];
+        int slot = -1;
+        if (lane < kKeys && d.t * kKeys + lane < d.L) {
+            slot = my_idx[e][lane];
+            if (slot < 0 || (int64_t)slot >= p.num_slots) {
                 atomicOr(&g_mg_device_error, MG_DEVERR_SLOT_RANGE);
-                s = -1;
+                slot = -1;
             }
         }
-        return s;
-    };
-    // One warp instruction: lanes 0..15 each issue one gather4 of 4 rows x 128 B.
-    // gather index gi: K/V = gi / 8, 64-column half = (gi / 4) % 2, row quad = gi % 4.
-    auto issue = [&](Cursor &c, int slot_reg, int stage) {
-        c.valid = __ballot_sync(0xffffffffu, slot_reg >= 0) & 0xFFFFu;
-        const int row_id = slot_reg >= 0 ? slot_reg * p.num_kv_heads + c.kvh : oob_row;
+        const unsigned valid = __ballot_sync(0xffffffffu, slot >= 0) & 0xFFFFu;
+        if (lane == 0) my_desc[e].valid = valid;
+        const int row_id = slot >= 0 ? slot * p.num_kv_heads + d.kvh : oob_row;
         const int quad = lane & 3;
         const int r0 = __shfl_sync(0xffffffffu, row_id, quad * 4 + 0);
         const int r1 = __shfl_sync(0xffffffffu, row_id, quad * 4 + 1);
@@ -318,20 +374,18 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
         }
     };
 
-    // prologue: tiles 0 .. STAGES-2 in flight, indices of tile STAGES-1 in registers
-    int idx_next;
-    {
-        int idx0 = fetch_idx(cur);
+    // prologue: entries of tiles 0 .. IDX_AHEAD+STAGES-2 requested, tiles
+    // 0 .. STAGES-2 issued
+    constexpr int kPre = kIdxAhead + kStages - 1;
 #pragma unroll
-        for (int s = 0; s < kStages - 1; ++s) {
-            if (s < n_units) {
-                issue(cur, idx0, s);
-                dq[s] = cur;
-                cursor_advance(p, cur);
-                if (s + 1 < n_units) idx0 = fetch_idx(cur);
-            }
+    for (int j = 0; j < kPre; ++j) fetch(j);
+#pragma unroll
+    for (int j = 0; j < kStages - 1; ++j) {
+        if (j < n_units) {
+            cp_async_wait_dyn(kPre - 1 - j);
+            __syncwarp();
+            issue(j);
         }
-        idx_next = idx0;
     }
 
     float o[16][4];
@@ -343,18 +397,16 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
     int k = 0;
 
     for (; k < n_units; ++k) {
-        // issue tile k + STAGES - 1 (its stage was freed at the end of tile k - 1),
-        // then prefetch the indices of the tile after it
-        {
-            const int j = k + kStages - 1;
-            if (j < n_units) {
-                issue(cur, idx_next, j % kStages);
-                dq[j % (kStages + 1)] = cur;
-                cursor_advance(p, cur);
-                if (j + 1 < n_units) idx_next = fetch_idx(cur);
-            }
+        // fetch the entries of tile k + kPre; issue tile k + STAGES - 1 (its
+        // stage was freed at the end of tile k - 1; its entries are the group
+        // committed kIdxAhead fetches ago)
+        fetch(k + kPre);
+        if (k + kStages - 1 < n_units) {
+            cp_async_wait<kIdxAhead>();
+            __syncwarp();
+            issue(k + kStages - 1);
         }
-        const Cursor c = dq[k % (kStages + 1)];
+        const TileDesc c = my_desc[k % kDescRing];
         const bool first = k == 0 || c.t == 0;
         const bool last = k == n_units - 1 || c.t == c.tiles - 1;
         if (first) {
@@ -508,6 +560,7 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
         for (int t = k; t < n_units && t < k + kStages - 1; ++t)
             (void)mbar_wait_bounded(smem_u32(&full_bar[warp][t % kStages]), (t / kStages) & 1, 1u << 20);
     }
+    cp_async_wait<0>();  // page-table copies still in flight
 }
 
 // One warp per (request, q head): combine the partials of a pair that more
