@@ -60,6 +60,9 @@ constexpr int kMaxScanChunks = 256;                // requests <= 131072
 #ifndef MG_DECODE_MIN_BLOCKS
 #define MG_DECODE_MIN_BLOCKS 2  // resident CTAs per SM (the shared memory is sized for it)
 #endif
+#ifndef MG_DECODE_TMA
+#define MG_DECODE_TMA 0  // 1: K/V tiles by TMA gather4 + mbarrier; 0: 16-byte cp.async
+#endif
 #ifndef MG_DECODE_IDX_AHEAD
 #define MG_DECODE_IDX_AHEAD 8  // tiles of page-table entries fetched ahead of the K/V issue
 #endif
@@ -303,6 +306,9 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
     const int g = p.group;
     const uint32_t ring = smem_u32(smem) + (uint32_t)(warp * kStages * kTileBytes);
     const int oob_row = (int)(p.num_slots * p.num_kv_heads);  // TMA reads it as zeros
+    const int64_t head_stride = (int64_t)p.num_kv_heads * kHeadDim;
+    (void)oob_row;
+    (void)head_stride;
     if (lane == 0) {
         prefetch_tmap(&tm_k);
         prefetch_tmap(&tm_v);
@@ -339,7 +345,6 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
             }
             cursor_advance(p, cur);
         }
-        cp_async_commit();
     };
     // Issue stage: read tile j's entries, check them, and let lanes 0..15 each
     // issue one gather4 (K/V = lane / 8, 64-column half = (lane / 4) % 2, row quad = lane % 4).
@@ -356,6 +361,7 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
         }
         const unsigned valid = __ballot_sync(0xffffffffu, slot >= 0) & 0xFFFFu;
         if (lane == 0) my_desc[e].valid = valid;
+#if MG_DECODE_TMA
         const int row_id = slot >= 0 ? slot * p.num_kv_heads + d.kvh : oob_row;
         const int quad = lane & 3;
         const int r0 = __shfl_sync(0xffffffffu, row_id, quad * 4 + 0);
@@ -372,21 +378,25 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
             fence_proxy_async_smem();
             tma_gather4(dst, kind ? (const void *)&tm_v : (const void *)&tm_k, bar, half * 64, r0, r1, r2, r3);
         }
+#else
+        // 16-byte cp.async: each warp instruction moves two whole 256-byte rows
+        // (lanes 0-15 and 16-31); 32 rows per tile (16 K then 16 V)
+        const uint32_t base = ring + (uint32_t)(stage * kTileBytes);
+        const int ch = lane & 15;
+        const int64_t head_off = (int64_t)d.kvh * kHeadDim + ch * 8;
+#pragma unroll
+        for (int it = 0; it < 16; ++it) {
+            const int rr = it * 2 + (lane >> 4);
+            const int key = rr & (kKeys - 1);
+            const bool is_v = rr >= kKeys;
+            const int sl = __shfl_sync(0xffffffffu, slot, key);
+            const __nv_bfloat16 *src = (is_v ? p.v_cache : p.k_cache) + (int64_t)(sl < 0 ? 0 : sl) * head_stride + head_off;
+            cp_async_16(base + (is_v ? 2 * kHalfRows : 0) + swz(key, ch), src, sl < 0 ? 0u : 16u);
+        }
+#endif
     };
 
-    // prologue: entries of tiles 0 .. IDX_AHEAD+STAGES-2 requested, tiles
-    // 0 .. STAGES-2 issued
-    constexpr int kPre = kIdxAhead + kStages - 1;
-#pragma unroll
-    for (int j = 0; j < kPre; ++j) fetch(j);
-#pragma unroll
-    for (int j = 0; j < kStages - 1; ++j) {
-        if (j < n_units) {
-            cp_async_wait_dyn(kPre - 1 - j);
-            __syncwarp();
-            issue(j);
-        }
-    }
+    constexpr int kPre = kIdxAhead + kStages - 1;  // fetch runs this many tiles ahead of compute
 
     float o[16][4];
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;  // rows lane/4 and lane/4+8
@@ -394,18 +404,31 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
     const int ra = lane >> 2, rb = ra + 8;
     int seg_first_t = 0;
     bool ok = true;
-    int k = 0;
+    int k = -kPre;
 
+    // One software pipeline, one cp.async group per iteration k: fetch the
+    // page-table entries of tile k + kPre; issue the K/V loads of tile
+    // k + STAGES - 1 (its stage was freed when tile k - 1 finished, its entries
+    // were fetched kIdxAhead iterations ago); compute tile k.
     for (; k < n_units; ++k) {
-        // fetch the entries of tile k + kPre; issue tile k + STAGES - 1 (its
-        // stage was freed at the end of tile k - 1; its entries are the group
-        // committed kIdxAhead fetches ago)
         fetch(k + kPre);
-        if (k + kStages - 1 < n_units) {
+        const int j = k + kStages - 1;
+#if MG_DECODE_TMA
+        cp_async_commit();
+        if (j >= 0 && j < n_units) {
             cp_async_wait<kIdxAhead>();
             __syncwarp();
-            issue(k + kStages - 1);
+            issue(j);
         }
+#else
+        if (j >= 0 && j < n_units) {
+            cp_async_wait<kIdxAhead - 1>();
+            __syncwarp();
+            issue(j);
+        }
+        cp_async_commit();
+#endif
+        if (k < 0) continue;
         const TileDesc c = my_desc[k % kDescRing];
         const bool first = k == 0 || c.t == 0;
         const bool last = k == n_units - 1 || c.t == c.tiles - 1;
@@ -430,11 +453,16 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
             l0 = l1 = 0.f;
             seg_first_t = c.t;
         }
+#if MG_DECODE_TMA
         // wait for tile k (bounded: a lost transfer sets the timeout bit and ends this worker)
         if (!warp_wait_bounded(smem_u32(&full_bar[warp][k % kStages]), (k / kStages) & 1)) {
             ok = false;
             break;
         }
+#else
+        cp_async_wait<kStages - 1>();
+        __syncwarp();
+#endif
 
         const uint32_t kt = ring + (uint32_t)((k % kStages) * kTileBytes);
         const uint32_t vt = kt + 2 * kHalfRows;
@@ -560,6 +588,7 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
         for (int t = k; t < n_units && t < k + kStages - 1; ++t)
             (void)mbar_wait_bounded(smem_u32(&full_bar[warp][t % kStages]), (t / kStages) & 1, 1u << 20);
     }
+    (void)ok;
     cp_async_wait<0>();  // page-table copies still in flight
 }
 
