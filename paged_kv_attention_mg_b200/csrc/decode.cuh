@@ -16,12 +16,15 @@
 //     all workers finish together whatever the length mix (no tail of long
 //     splits).  A worker's share covers one or a few "segments" (its part of a
 //     pair).
-//   * per tile a worker gathers the 16 K and 16 V rows (256 B each) straight
-//     from the pool with TMA tile::gather4 (4 page-table rows per instruction,
-//     128-byte swizzle, 16 instructions per tile issued by 16 lanes at once)
-//     into its own STAGES-deep ring, completion counted on one mbarrier per
-//     stage; page-table entries of the next tile are prefetched one step
-//     ahead.  Few warps with deep rings keep most of shared memory in flight.
+//   * three prefetch distances per worker: page-table entries of tile
+//     k + IDX_AHEAD are copied (cp.async) into a per-warp index ring; the K/V
+//     rows of tile k + L2_AHEAD are prefetched into L2 (bulk prefetch, one
+//     256-byte row per lane), which keeps many DRAM requests in flight without
+//     holding shared memory; tile k + STAGES - 1 is copied from L2 into the
+//     warp's STAGES-deep shared-memory ring, in the 128-byte-swizzled layout
+//     ldmatrix reads without bank conflicts.  Loads used TMA tile::gather4
+//     into the ring with an mbarrier per
+//     stage (build switch MG_DECODE_TMA), or with 16-byte cp.async (default).
 //   * the GQA group is the M dimension of warp-level bf16 tensor-core MMAs
 //     (m16n8k16, fp32 accumulate, g <= 16 rows, zero padded), so each K/V row
 //     is read from HBM once for all g heads: S = Q K^T, online softmax in the
@@ -64,12 +67,18 @@ constexpr int kMaxScanChunks = 256;                // requests <= 131072
 #define MG_DECODE_TMA 0  // 1: K/V tiles by TMA gather4 + mbarrier; 0: 16-byte cp.async
 #endif
 #ifndef MG_DECODE_IDX_AHEAD
-#define MG_DECODE_IDX_AHEAD 8  // tiles of page-table entries fetched ahead of the K/V issue
+#define MG_DECODE_IDX_AHEAD 12  // tiles of page-table entries fetched ahead of compute
+#endif
+#ifndef MG_DECODE_L2_AHEAD
+#define MG_DECODE_L2_AHEAD 8  // tiles of K/V rows prefetched into L2 ahead of compute (0: off)
 #endif
 constexpr int kStages = MG_DECODE_STAGES;
 constexpr int kIdxAhead = MG_DECODE_IDX_AHEAD;
+constexpr int kL2Ahead = MG_DECODE_L2_AHEAD;
 constexpr int kDescRing = 16;  // per-warp ring of tile descriptors / index rows
-static_assert(kDescRing >= kIdxAhead + kStages, "descriptor ring too small");
+static_assert(kDescRing >= kIdxAhead + 1, "descriptor ring too small");
+static_assert(kIdxAhead > kL2Ahead && kL2Ahead >= kStages - 1 || kL2Ahead == 0, "prefetch distances out of order");
+static_assert(kIdxAhead >= kStages, "page-table entries must lead the K/V loads");
 constexpr int kRingBytes = kWarps * kStages * kTileBytes;
 constexpr int kSmemBytes = kRingBytes + 1024;  // + alignment slack (128-byte swizzle atoms)
 constexpr int kHalfRows = kKeys * 128;          // one 64-column half of a 16-row tile: 2 KB
@@ -396,7 +405,22 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
 #endif
     };
 
-    constexpr int kPre = kIdxAhead + kStages - 1;  // fetch runs this many tiles ahead of compute
+    constexpr int kPre = kIdxAhead;  // page-table fetch runs this many tiles ahead of compute
+
+    // L2 stage: prefetch tile j's 32 K/V rows (one 256-byte row per lane).
+    auto l2prefetch = [&](int j) {
+        if (j < 0 || j >= n_units) return;
+        const int e = j % kDescRing;
+        const TileDesc d = my_desc[e];
+        const int key = lane & (kKeys - 1);
+        if (d.t * kKeys + key < d.L) {
+            const int sl = my_idx[e][key];
+            if (sl >= 0 && (int64_t)sl < p.num_slots)
+                prefetch_l2_bulk(((lane >> 4) ? p.v_cache : p.k_cache) + (int64_t)sl * head_stride +
+                                     (int64_t)d.kvh * kHeadDim,
+                                 kRowBytes);
+        }
+    };
 
     float o[16][4];
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;  // rows lane/4 and lane/4+8
@@ -407,25 +431,30 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
     int k = -kPre;
 
     // One software pipeline, one cp.async group per iteration k: fetch the
-    // page-table entries of tile k + kPre; issue the K/V loads of tile
-    // k + STAGES - 1 (its stage was freed when tile k - 1 finished, its entries
-    // were fetched kIdxAhead iterations ago); compute tile k.
+    // page-table entries of tile k + IDX_AHEAD; prefetch tile k + L2_AHEAD
+    // into L2 (its entries arrived: their group is IDX_AHEAD - L2_AHEAD
+    // iterations old); copy tile k + STAGES - 1 into its shared-memory stage
+    // (freed when tile k - 1 finished); compute tile k.
     for (; k < n_units; ++k) {
         fetch(k + kPre);
         const int j = k + kStages - 1;
 #if MG_DECODE_TMA
         cp_async_commit();
         if (j >= 0 && j < n_units) {
-            cp_async_wait<kIdxAhead>();
+            cp_async_wait<kIdxAhead - kStages + 1>();
             __syncwarp();
             issue(j);
         }
 #else
-        if (j >= 0 && j < n_units) {
-            cp_async_wait<kIdxAhead - 1>();
+        if (kL2Ahead > 0) {
+            cp_async_wait<(kL2Ahead > 0 ? kIdxAhead - kL2Ahead - 1 : 0)>();
             __syncwarp();
-            issue(j);
+            l2prefetch(k + kL2Ahead);
+        } else {
+            cp_async_wait<kIdxAhead - kStages>();
+            __syncwarp();
         }
+        if (j >= 0 && j < n_units) issue(j);
         cp_async_commit();
 #endif
         if (k < 0) continue;
