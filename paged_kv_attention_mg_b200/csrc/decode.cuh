@@ -70,14 +70,17 @@ constexpr int kMaxScanChunks = 256;                // requests <= 131072
 #define MG_DECODE_IDX_AHEAD 12  // tiles of page-table entries fetched ahead of compute
 #endif
 #ifndef MG_DECODE_L2_AHEAD
-#define MG_DECODE_L2_AHEAD 8  // tiles of K/V rows prefetched into L2 ahead of compute (0: off)
+#define MG_DECODE_L2_AHEAD 0  // tiles of K/V rows prefetched into L2 ahead of compute (0: off)
+#endif
+#ifndef MG_DECODE_L2_MODE
+#define MG_DECODE_L2_MODE 2  // 1: bulk prefetch (one 256-B request), 2: two 128-B line prefetches
 #endif
 constexpr int kStages = MG_DECODE_STAGES;
 constexpr int kIdxAhead = MG_DECODE_IDX_AHEAD;
 constexpr int kL2Ahead = MG_DECODE_L2_AHEAD;
 constexpr int kDescRing = 16;  // per-warp ring of tile descriptors / index rows
 static_assert(kDescRing >= kIdxAhead + 1, "descriptor ring too small");
-static_assert(kIdxAhead > kL2Ahead && kL2Ahead >= kStages - 1 || kL2Ahead == 0, "prefetch distances out of order");
+static_assert((kIdxAhead > kL2Ahead && kL2Ahead >= kStages - 1) || kL2Ahead == 0, "prefetch distances out of order");
 static_assert(kIdxAhead >= kStages, "page-table entries must lead the K/V loads");
 constexpr int kRingBytes = kWarps * kStages * kTileBytes;
 constexpr int kSmemBytes = kRingBytes + 1024;  // + alignment slack (128-byte swizzle atoms)
@@ -415,10 +418,16 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
         const int key = lane & (kKeys - 1);
         if (d.t * kKeys + key < d.L) {
             const int sl = my_idx[e][key];
-            if (sl >= 0 && (int64_t)sl < p.num_slots)
-                prefetch_l2_bulk(((lane >> 4) ? p.v_cache : p.k_cache) + (int64_t)sl * head_stride +
-                                     (int64_t)d.kvh * kHeadDim,
-                                 kRowBytes);
+            if (sl >= 0 && (int64_t)sl < p.num_slots) {
+                const __nv_bfloat16 *row = ((lane >> 4) ? p.v_cache : p.k_cache) + (int64_t)sl * head_stride +
+                                           (int64_t)d.kvh * kHeadDim;
+#if MG_DECODE_L2_MODE == 1
+                prefetch_l2_bulk(row, kRowBytes);
+#else
+                prefetch_l2_line(row);
+                prefetch_l2_line(row + 64);
+#endif
+            }
         }
     };
 

@@ -38,6 +38,11 @@ __device__ __forceinline__ void prefetch_l2_bulk(const void *src, uint32_t bytes
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(src), "r"(bytes) : "memory");
 }
 
+// Prefetch the 128-byte line holding `addr` into L2 (an ordinary LSU request).
+__device__ __forceinline__ void prefetch_l2_line(const void *addr) {
+    asm volatile("prefetch.global.L2 [%0];\n" ::"l"(addr));
+}
+
 // wait_group with a run-time count (0..15)
 __device__ __forceinline__ void cp_async_wait_dyn(int n) {
     switch (n) {
