@@ -223,6 +223,7 @@ __device__ __forceinline__ bool warp_wait_bounded(uint32_t bar, uint32_t parity)
     return __all_sync(0xffffffffu, done);
 }
 
+template <int NT>  // n-tiles of 8 GQA heads: 1 for g <= 8, 2 for g <= 16
 __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
     decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                   const Params p) {
@@ -231,6 +232,7 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
     __shared__ __align__(8) uint64_t full_bar[kWarps][kStages];
     __shared__ __align__(16) int idx_ring[kWarps][kDescRing][kKeys];
     __shared__ __align__(16) TileDesc desc_ring[kWarps][kDescRing];
+    __shared__ float sh_lse[kWarps][16];
     __shared__ int64_t sh_bound[kWarps + 1];
     __shared__ int64_t sh_scan[kWarps];
     __shared__ int64_t sh_chunk_excl[kMaxScanChunks + 1];
@@ -431,10 +433,15 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
         }
     };
 
-    float o[16][4];
-    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;  // rows lane/4 and lane/4+8
-    uint32_t qf[8][4];
-    const int ra = lane >> 2, rb = ra + 8;
+    // Transposed tile products: S^T[key, head] = K Q^T and O^T[dim, head] +=
+    // V^T P^T, keys / dims in the MMA M dimension and the GQA heads in N (8 per
+    // n-tile), so a g <= 8 group needs 16 m16n8k16 MMAs per 16-key tile.
+    // Fragment ownership: lane l holds heads nt*8 + 2(l%4) + {0,1} of the keys
+    // (or dims) l/4 and l/4 + 8.
+    float o[NT][8][4];
+    float mh[NT][2], lh[NT][2];  // running max / partial sum of this lane's two heads per n-tile
+    uint32_t qb[NT][8][2];       // Q^T as B fragments
+    const int quad = lane & 3;
     int seg_first_t = 0;
     bool ok = true;
     int k = -kPre;
@@ -471,24 +478,23 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
         const bool first = k == 0 || c.t == 0;
         const bool last = k == n_units - 1 || c.t == c.tiles - 1;
         if (first) {
-            // new segment: load this pair's q as MMA A fragments, reset the state
-            const int h0 = c.kvh * g;
-            const int cq = (lane & 3) * 2;
-            const __nv_bfloat16 *qa = p.q + ((int64_t)c.r * p.num_q_heads + h0 + ra) * kHeadDim;
-            const __nv_bfloat16 *qb = p.q + ((int64_t)c.r * p.num_q_heads + h0 + rb) * kHeadDim;
-            const bool va = ra < g, vb = rb < g;
+            // new segment: this pair's q as B fragments (head l/4 of each n-tile), reset the state
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const int c0 = kk * 16 + cq;
-                qf[kk][0] = va ? __ldg(reinterpret_cast<const uint32_t *>(qa + c0)) : 0u;
-                qf[kk][1] = vb ? __ldg(reinterpret_cast<const uint32_t *>(qb + c0)) : 0u;
-                qf[kk][2] = va ? __ldg(reinterpret_cast<const uint32_t *>(qa + c0 + 8)) : 0u;
-                qf[kk][3] = vb ? __ldg(reinterpret_cast<const uint32_t *>(qb + c0 + 8)) : 0u;
+            for (int nt = 0; nt < NT; ++nt) {
+                const int hl = nt * 8 + (lane >> 2);
+                const bool hv = hl < g;
+                const __nv_bfloat16 *qh = p.q + ((int64_t)c.r * p.num_q_heads + (int64_t)c.kvh * g + hl) * kHeadDim +
+                                          quad * 2;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    qb[nt][kk][0] = hv ? __ldg(reinterpret_cast<const uint32_t *>(qh + kk * 16)) : 0u;
+                    qb[nt][kk][1] = hv ? __ldg(reinterpret_cast<const uint32_t *>(qh + kk * 16 + 8)) : 0u;
+                }
+#pragma unroll
+                for (int dt = 0; dt < 8; ++dt) o[nt][dt][0] = o[nt][dt][1] = o[nt][dt][2] = o[nt][dt][3] = 0.f;
+                mh[nt][0] = mh[nt][1] = -INFINITY;
+                lh[nt][0] = lh[nt][1] = 0.f;
             }
-#pragma unroll
-            for (int jj = 0; jj < 16; ++jj) o[jj][0] = o[jj][1] = o[jj][2] = o[jj][3] = 0.f;
-            m0 = m1 = -INFINITY;
-            l0 = l1 = 0.f;
             seg_first_t = c.t;
         }
 #if MG_DECODE_TMA
@@ -505,119 +511,148 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
         const uint32_t kt = ring + (uint32_t)((k % kStages) * kTileBytes);
         const uint32_t vt = kt + 2 * kHalfRows;
 
-        float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-        {
-            const int mi = lane >> 3;
-            const int key = (mi >> 1) * 8 + (lane & 7);
+        // ---- S^T = K Q^T: two accumulators (even / odd k-steps) halve the MMA chain
+        float sa[NT][4], sb[NT][4];
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                uint32_t b0, b1, b2, b3;
-                ldmatrix_x4(kt + swz(key, 2 * kk + (mi & 1)), b0, b1, b2, b3);
-                mma_bf16_16816(sc[0], qf[kk], b0, b1);
-                mma_bf16_16816(sc[1], qf[kk], b2, b3);
-            }
-        }
-        float mx0 = -INFINITY, mx1 = -INFINITY;
+        for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int key = nt * 8 + (lane & 3) * 2 + e;
-                // keys past the end, or whose slot was rejected (zero-filled), are masked
-                const bool kv_ok = (c.valid >> key) & 1u;
-                const float s0 = kv_ok ? sc[nt][e] * p.scale_log2 : -INFINITY;
-                const float s1 = kv_ok ? sc[nt][e + 2] * p.scale_log2 : -INFINITY;
-                sc[nt][e] = s0;
-                sc[nt][e + 2] = s1;
-                mx0 = fmaxf(mx0, s0);
-                mx1 = fmaxf(mx1, s1);
-            }
-        }
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-        const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-        const float mu0 = mn0 == -INFINITY ? 0.f : mn0;
-        const float mu1 = mn1 == -INFINITY ? 0.f : mn1;
-        if (__any_sync(0xffffffffu, mn0 != m0 || mn1 != m1)) {
-            const float corr0 = fast_exp2(m0 - mu0), corr1 = fast_exp2(m1 - mu1);
-            l0 *= corr0;
-            l1 *= corr1;
-#pragma unroll
-            for (int jj = 0; jj < 16; ++jj) {
-                o[jj][0] *= corr0;
-                o[jj][1] *= corr0;
-                o[jj][2] *= corr1;
-                o[jj][3] *= corr1;
-            }
-            m0 = mn0;
-            m1 = mn1;
-        }
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-            sc[nt][0] = fast_exp2(sc[nt][0] - mu0);
-            sc[nt][1] = fast_exp2(sc[nt][1] - mu0);
-            sc[nt][2] = fast_exp2(sc[nt][2] - mu1);
-            sc[nt][3] = fast_exp2(sc[nt][3] - mu1);
-            l0 += sc[nt][0] + sc[nt][1];
-            l1 += sc[nt][2] + sc[nt][3];
-        }
-        uint32_t pa[4];
-        pa[0] = pack_bf16x2(sc[0][0], sc[0][1]);
-        pa[1] = pack_bf16x2(sc[0][2], sc[0][3]);
-        pa[2] = pack_bf16x2(sc[1][0], sc[1][1]);
-        pa[3] = pack_bf16x2(sc[1][2], sc[1][3]);
+            for (int e = 0; e < 4; ++e) sa[nt][e] = sb[nt][e] = 0.f;
         {
             const int mi = lane >> 3;
             const int key = (mi & 1) * 8 + (lane & 7);
 #pragma unroll
-            for (int dp = 0; dp < 8; ++dp) {
-                uint32_t b0, b1, b2, b3;
-                ldmatrix_x4_trans(vt + swz(key, 2 * dp + (mi >> 1)), b0, b1, b2, b3);
-                mma_bf16_16816(o[2 * dp], pa, b0, b1);
-                mma_bf16_16816(o[2 * dp + 1], pa, b2, b3);
+            for (int kk = 0; kk < 8; ++kk) {
+                uint32_t a[4];
+                ldmatrix_x4(kt + swz(key, 2 * kk + (mi >> 1)), a[0], a[1], a[2], a[3]);
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    if (kk & 1) mma_bf16_16816(sb[nt], a, qb[nt][kk][0], qb[nt][kk][1]);
+                    else mma_bf16_16816(sa[nt], a, qb[nt][kk][0], qb[nt][kk][1]);
+                }
             }
         }
-        __syncwarp();  // every lane is done with this stage before it is refilled
+        // keys past the end, or whose slot was rejected (zero-filled), are masked
+        const bool v0 = (c.valid >> (lane >> 2)) & 1u, v1 = (c.valid >> ((lane >> 2) + 8)) & 1u;
+        bool changed = false;
+        float sc[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            sc[nt][0] = v0 ? (sa[nt][0] + sb[nt][0]) * p.scale_log2 : -INFINITY;  // key l/4,   head even
+            sc[nt][1] = v0 ? (sa[nt][1] + sb[nt][1]) * p.scale_log2 : -INFINITY;  // key l/4,   head odd
+            sc[nt][2] = v1 ? (sa[nt][2] + sb[nt][2]) * p.scale_log2 : -INFINITY;  // key l/4+8, head even
+            sc[nt][3] = v1 ? (sa[nt][3] + sb[nt][3]) * p.scale_log2 : -INFINITY;  // key l/4+8, head odd
+            float x0 = fmaxf(sc[nt][0], sc[nt][2]), x1 = fmaxf(sc[nt][1], sc[nt][3]);
+#pragma unroll
+            for (int off = 4; off < 32; off <<= 1) {
+                x0 = fmaxf(x0, __shfl_xor_sync(0xffffffffu, x0, off));
+                x1 = fmaxf(x1, __shfl_xor_sync(0xffffffffu, x1, off));
+            }
+            const float n0 = fmaxf(mh[nt][0], x0), n1 = fmaxf(mh[nt][1], x1);
+            changed |= (n0 != mh[nt][0]) || (n1 != mh[nt][1]);
+            sa[nt][0] = n0;  // reuse: new maxima
+            sa[nt][1] = n1;
+        }
+        if (__any_sync(0xffffffffu, changed)) {
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const float n0 = sa[nt][0], n1 = sa[nt][1];
+                const float c0 = mh[nt][0] == -INFINITY ? 0.f : fast_exp2(mh[nt][0] - (n0 == -INFINITY ? 0.f : n0));
+                const float c1 = mh[nt][1] == -INFINITY ? 0.f : fast_exp2(mh[nt][1] - (n1 == -INFINITY ? 0.f : n1));
+                lh[nt][0] *= c0;
+                lh[nt][1] *= c1;
+#pragma unroll
+                for (int dt = 0; dt < 8; ++dt) {
+                    o[nt][dt][0] *= c0;
+                    o[nt][dt][1] *= c1;
+                    o[nt][dt][2] *= c0;
+                    o[nt][dt][3] *= c1;
+                }
+                mh[nt][0] = n0;
+                mh[nt][1] = n1;
+            }
+        }
+        // ---- P^T (bf16) as B fragments: lane l needs keys 2(l%4), +1 (and +8)
+        // of head l/4, which sit in lanes 8(l%4) + l/8 and that + 4
+        uint32_t pb[NT][2];
+        {
+            const int s0 = 8 * quad + (lane >> 3);
+            const uint32_t sel = ((lane >> 2) & 1) ? 0x7632u : 0x5410u;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const float mu0 = mh[nt][0] == -INFINITY ? 0.f : mh[nt][0];
+                const float mu1 = mh[nt][1] == -INFINITY ? 0.f : mh[nt][1];
+                const float p0 = fast_exp2(sc[nt][0] - mu0), p1 = fast_exp2(sc[nt][1] - mu1);
+                const float p2 = fast_exp2(sc[nt][2] - mu0), p3 = fast_exp2(sc[nt][3] - mu1);
+                lh[nt][0] += p0 + p2;
+                lh[nt][1] += p1 + p3;
+                const uint32_t X = pack_bf16x2(p0, p1), Y = pack_bf16x2(p2, p3);
+                const uint32_t xa = __shfl_sync(0xffffffffu, X, s0), xb = __shfl_sync(0xffffffffu, X, s0 + 4);
+                const uint32_t ya = __shfl_sync(0xffffffffu, Y, s0), yb = __shfl_sync(0xffffffffu, Y, s0 + 4);
+                pb[nt][0] = __byte_perm(xa, xb, sel);
+                pb[nt][1] = __byte_perm(ya, yb, sel);
+            }
+        }
+        // ---- O^T += V^T P^T
+        {
+            const int mi = lane >> 3;
+            const int key = (mi >> 1) * 8 + (lane & 7);
+#pragma unroll
+            for (int dt = 0; dt < 8; ++dt) {
+                uint32_t a[4];
+                ldmatrix_x4_trans(vt + swz(key, 2 * dt + (mi & 1)), a[0], a[1], a[2], a[3]);
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(o[nt][dt], a, pb[nt][0], pb[nt][1]);
+            }
+        }
+        __syncwarp();  // every lane is done reading this stage
 
         if (last) {
-            // ---- finish the segment: whole pair -> bf16 out, else a partial
-            float la = l0 + __shfl_xor_sync(0xffffffffu, l0, 1);
-            la += __shfl_xor_sync(0xffffffffu, la, 2);
-            float lb = l1 + __shfl_xor_sync(0xffffffffu, l1, 1);
-            lb += __shfl_xor_sync(0xffffffffu, lb, 2);
-            const float ia = la > 0.f ? 1.f / la : 0.f, ib = lb > 0.f ? 1.f / lb : 0.f;
+            // ---- finish the segment through the (now idle) stage as fp32 scratch
+            // [heads][dims + 4]: whole pair -> bf16 out, else a partial
+            float *scr = reinterpret_cast<float *>(smem + (size_t)(warp * kStages + k % kStages) * kTileBytes);
+            constexpr int kPitch = NT == 1 ? kHeadDim + 4 : kHeadDim;  // pad when there is room
+            static_assert(NT * 8 * kPitch * 4 <= kTileBytes, "scratch must fit in one stage");
+            float *lse_scr = sh_lse[warp];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                float l0 = lh[nt][0], l1 = lh[nt][1];
+#pragma unroll
+                for (int off = 4; off < 32; off <<= 1) {
+                    l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+                    l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+                }
+                const float i0 = l0 > 0.f ? 1.f / l0 : 0.f, i1 = l1 > 0.f ? 1.f / l1 : 0.f;
+                const int h0 = nt * 8 + 2 * quad;
+#pragma unroll
+                for (int dt = 0; dt < 8; ++dt) {
+                    const int d0 = dt * 16 + (lane >> 2);
+                    scr[h0 * kPitch + d0] = o[nt][dt][0] * i0;
+                    scr[(h0 + 1) * kPitch + d0] = o[nt][dt][1] * i1;
+                    scr[h0 * kPitch + d0 + 8] = o[nt][dt][2] * i0;
+                    scr[(h0 + 1) * kPitch + d0 + 8] = o[nt][dt][3] * i1;
+                }
+                if (lane < 4) {  // log2-sum-exp of heads h0, h0 + 1
+                    lse_scr[h0] = l0 > 0.f ? mh[nt][0] + __log2f(l0) : -INFINITY;
+                    lse_scr[h0 + 1] = l1 > 0.f ? mh[nt][1] + __log2f(l1) : -INFINITY;
+                }
+            }
+            __syncwarp();
             const bool whole = seg_first_t == 0 && c.t == c.tiles - 1;
             const int64_t head0 = (int64_t)c.r * p.num_q_heads + (int64_t)c.kvh * g;
             const int64_t slot = (int64_t)c.r * p.num_kv_heads + c.kvh + w;
-            const int dcol = (lane & 3) * 2;
-            if (whole) {
-#pragma unroll
-                for (int jj = 0; jj < 16; ++jj) {
-                    if (ra < g)
-                        *reinterpret_cast<uint32_t *>(p.out + (head0 + ra) * kHeadDim + jj * 8 + dcol) =
-                            pack_bf16x2(o[jj][0] * ia, o[jj][1] * ia);
-                    if (rb < g)
-                        *reinterpret_cast<uint32_t *>(p.out + (head0 + rb) * kHeadDim + jj * 8 + dcol) =
-                            pack_bf16x2(o[jj][2] * ib, o[jj][3] * ib);
-                }
-            } else {
-                float *po = p.part_o + slot * g * kHeadDim;
-#pragma unroll
-                for (int jj = 0; jj < 16; ++jj) {
-                    if (ra < g)
-                        *reinterpret_cast<float2 *>(po + ra * kHeadDim + jj * 8 + dcol) =
-                            make_float2(o[jj][0] * ia, o[jj][1] * ia);
-                    if (rb < g)
-                        *reinterpret_cast<float2 *>(po + rb * kHeadDim + jj * 8 + dcol) =
-                            make_float2(o[jj][2] * ib, o[jj][3] * ib);
-                }
-                if ((lane & 3) == 0) {
-                    if (ra < g) p.part_lse[slot * g + ra] = la > 0.f ? m0 + __log2f(la) : -INFINITY;
-                    if (rb < g) p.part_lse[slot * g + rb] = lb > 0.f ? m1 + __log2f(lb) : -INFINITY;
+            for (int h = 0; h < g; ++h) {
+                const float4 v = *reinterpret_cast<const float4 *>(scr + h * kPitch + lane * 4);
+                if (whole) {
+                    uint2 packed;
+                    packed.x = pack_bf16x2(v.x, v.y);
+                    packed.y = pack_bf16x2(v.z, v.w);
+                    *reinterpret_cast<uint2 *>(p.out + (head0 + h) * kHeadDim + lane * 4) = packed;
+                } else {
+                    *reinterpret_cast<float4 *>(p.part_o + (slot * g + h) * kHeadDim + lane * 4) = v;
                 }
             }
+            if (!whole && lane < g) p.part_lse[slot * g + lane] = lse_scr[lane];
+            __syncwarp();  // scratch reads done before the stage is refilled
         }
     }
     if (!ok) {

@@ -49,7 +49,9 @@ mg_status ensure_kernel_attributes() {
     if (g_attr_done[dev]) return MG_OK;
     std::lock_guard<std::mutex> lock(g_attr_mutex);
     if (g_attr_done[dev]) return MG_OK;
-    if (cudaFuncSetAttribute(decode::decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(decode::decode_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             decode::kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(decode::decode_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              decode::kSmemBytes) != cudaSuccess)
         return MG_ERR_CUDA;
     if (extend::set_attributes() != cudaSuccess) return MG_ERR_CUDA;
@@ -227,7 +229,10 @@ mg_status mg_decode_attn(const void *q, const void *k_cache, const void *v_cache
         return MG_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int ctas = (workers + decode::kWarps - 1) / decode::kWarps;
-    decode::decode_kernel<<<ctas, decode::kThreads, decode::kSmemBytes, s>>>(tk, tv, p);
+    if (p.group <= 8)
+        decode::decode_kernel<1><<<ctas, decode::kThreads, decode::kSmemBytes, s>>>(tk, tv, p);
+    else
+        decode::decode_kernel<2><<<ctas, decode::kThreads, decode::kSmemBytes, s>>>(tk, tv, p);
     if ((st = launched()) != MG_OK) return st;
     const int warps = batch * num_q_heads;
     decode::decode_merge_kernel<<<(warps + 3) / 4, 128, 0, s>>>(p);
