@@ -12,12 +12,16 @@ flush needed.  With N GPUs every rank runs its own replica with its own seed
 (weak scaling, no collective on the data path); the reported time is the max
 over ranks.
 
+The step is recorded once into a CUDA graph over fixed buffers and replayed,
+as the engine runs decode (--no-graph launches it eagerly instead).
+
 The JSON line: `value` = algorithmic bytes (K/V rows once per GQA group, q,
 out, page-table entries, plus the store's reads and writes) per step summed
 over ranks / step time, in GB/s; `e2e` = the same through the public API with
-the step's inputs copied from pinned host memory and the outputs copied back
-inside the timed region; `roofline` = the decode kernel pair (split + merge)
-timed with CUDA events inside the timed region against the measured HBM copy
+the step's inputs copied from pinned host memory into the fixed buffers and
+the outputs copied back inside the timed region; `roofline` = one
+mg_decode_attn call (worker kernel + merge kernel), timed by CUDA events
+recorded inside the step around every call, against the measured HBM copy
 bandwidth; `cpu_baseline` = the fp64 oracle on this host's cores on a bounded
 sample of the same workload.
 
@@ -68,6 +72,7 @@ def parse_args():
                     help="run only the first N layers (small cases for profiling; 0 = the workload's own)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="launch every step eagerly instead of a CUDA graph")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="bound of the cpu_baseline sample")
     ap.add_argument("--soak-seconds", type=float, default=1.5,
                     help="extra untimed warm-up so the clock sampler sees the GPU under load")
@@ -222,20 +227,18 @@ class DecodeBench:
         for i, lay in enumerate(self.layers):
             self.layer(lay, self.outs[i], self.meta, events[i] if events else None)
 
-    def make_events(self):
-        return [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                for _ in self.layers]
-
-    def run_step_e2e(self):
-        """Inputs from pinned host memory, outputs back to pinned host memory."""
+    def copy_in(self):
+        """This step's inputs from pinned host memory into the fixed device buffers."""
         for n, t in self.meta_host.items():
             self.meta[n].copy_(t, non_blocking=True)
-        for i, lay in enumerate(self.layers):
+        for lay in self.layers:
             lay["q"].copy_(lay["q_host"], non_blocking=True)
             lay["k_new"].copy_(lay["k_new_host"], non_blocking=True)
             lay["v_new"].copy_(lay["v_new_host"], non_blocking=True)
-            self.layer(lay, self.outs[i], self.meta)
-            self.outs_host[i].copy_(self.outs[i], non_blocking=True)
+
+    def copy_out(self):
+        for i, o in enumerate(self.outs):
+            self.outs_host[i].copy_(o, non_blocking=True)
 
     def kernel_bytes(self):
         return self.decode_bytes
@@ -284,8 +287,8 @@ class ExtendBench:
             events[1].record()
 
     run_step = DecodeBench.run_step
-    make_events = DecodeBench.make_events
-    run_step_e2e = DecodeBench.run_step_e2e
+    copy_in = DecodeBench.copy_in
+    copy_out = DecodeBench.copy_out
 
     def describe(self):
         s, st = self.spec, self.step
@@ -397,60 +400,90 @@ def run_ours(args):
         flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
     torch.cuda.synchronize()
 
+    # The step as the engine runs decode: recorded once into a CUDA graph over
+    # fixed buffers, then replayed (--no-graph: launched eagerly every step).
+    # Timing events around every attention call are recorded inside the step
+    # (graph-capturable "external" events), so the kernel time is measured in
+    # the timed region itself, free of host launch gaps.
+    use_graph = not args.no_graph
+    kev = [(torch.cuda.Event(enable_timing=True, external=use_graph),
+            torch.cuda.Event(enable_timing=True, external=use_graph)) for _ in range(spec.num_layers)]
+    fev = (torch.cuda.Event(enable_timing=True, external=use_graph),
+           torch.cuda.Event(enable_timing=True, external=use_graph))
+
+    def enqueue_step():
+        if flush is not None:
+            fev[0].record()
+            flush.fill_(0x5A)
+            fev[1].record()
+        bench.run_step(kev)
+
+    for _ in range(2):  # eager warm-up: module load, kernel attributes
+        enqueue_step()
+    torch.cuda.synchronize()
+    graphs = []
+    if use_graph:
+        g_timed, g_plain = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_timed):
+            enqueue_step()
+        with torch.cuda.graph(g_plain):
+            bench.run_step()
+        graphs = [g_timed, g_plain]
+        run_timed, run_plain = g_timed.replay, g_plain.replay
+    else:
+        run_timed, run_plain = enqueue_step, bench.run_step
+    torch.cuda.synchronize()
+
     sampler = ClockSampler(dist.local)
     sampler.start()
     # warm-up (W steps) plus a short soak so clocks are sampled under load
     for _ in range(max(3, args.warmup)):
-        bench.run_step()
+        run_timed()
     torch.cuda.synchronize()
     t_end = time.perf_counter() + args.soak_seconds
     while time.perf_counter() < t_end:
-        bench.run_step()
+        for _ in range(10):
+            run_timed()
         torch.cuda.synchronize()
 
-    events = [bench.make_events() for _ in range(args.steps)]
-    flush_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                    for _ in range(args.steps)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    flush_ms = 0.0
     dist.barrier()
     torch.cuda.synchronize()
     start.record()
-    for k in range(args.steps):
-        if flush is not None:
-            flush_events[k][0].record()
-            flush.fill_(k & 0xFF)
-            flush_events[k][1].record()
-        bench.run_step(events[k])
+    for _ in range(args.steps):
+        run_timed()
     stop.record()
     torch.cuda.synchronize()
     dist.barrier()
     clocks = sampler.stop()
     total_ms = start.elapsed_time(stop)
-    if flush is not None:
-        flush_ms = sum(a.elapsed_time(b) for a, b in flush_events)
-    step_ms_local = (total_ms - flush_ms) / args.steps
-    kernel_ms_local = sum(a.elapsed_time(b) for ev in events for (a, b) in ev) / (
-        args.steps * spec.num_layers)
+    flush_ms = fev[0].elapsed_time(fev[1]) if flush is not None else 0.0  # last step's flush
+    step_ms_local = total_ms / args.steps - flush_ms
+    kernel_ms_local = sum(a.elapsed_time(b) for a, b in kev) / spec.num_layers  # last step's calls
     step_ms = dist.max(step_ms_local)
     kernel_ms = dist.max(kernel_ms_local)
 
-    # end to end through the public API with host buffers
+    # end to end through the public API with host buffers: this step's inputs
+    # copied from pinned host memory into the fixed device buffers, the step,
+    # the outputs copied back to pinned host memory
     e2e = None
     if not args.no_e2e:
+        def e2e_step():
+            bench.copy_in()
+            run_plain()
+            bench.copy_out()
         for _ in range(2):
-            bench.run_step_e2e()
+            e2e_step()
         torch.cuda.synchronize()
         dist.barrier()
         ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e2e_steps = max(3, min(args.steps, 20))
+        e2e_steps = max(3, args.steps)
         ea.record()
         for _ in range(e2e_steps):
-            bench.run_step_e2e()
+            e2e_step()
         eb.record()
         torch.cuda.synchronize()
-        e2e_ms = dist.max(ea.elapsed_time(eb) / e2e_steps)
-        e2e = e2e_ms
+        e2e = dist.max(ea.elapsed_time(eb) / e2e_steps)
 
     hbm, tflops, tflops_sus, peak_src = measured_peaks()
     n = args.gpus
@@ -497,8 +530,10 @@ def run_ours(args):
                          "unit": unit, "ms_per_step": round(e2e, 4), "h2d_bytes_per_step": bench.h2d_bytes,
                          "d2h_bytes_per_step": bench.d2h_bytes} if e2e else None),
                 "gpu_launches": bench.launches_per_step * args.steps, "clocks": clocks,
+                "launch": "cuda graph per step" if use_graph else "eager",
                 "kernel_source_digest": source_digest()}
         print(json.dumps(line), flush=True)
+    del graphs
     dist.close()
 
 
