@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cstdint>
+#include <utility>
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -17,6 +18,27 @@ __device__ unsigned int g_mg_device_error;
 
 constexpr int kHeadDim = 128;
 constexpr float kLog2e = 1.4426950408889634f;
+
+// ---------------------------------------------------------------- host: launches
+
+// Launch with programmatic stream serialization: the kernel may start while
+// the previous kernel in the stream finishes; it calls griddepcontrol.wait
+// before touching anything that kernel wrote.
+template <typename... KArgs, typename... Args>
+inline mg_status launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                            Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) == cudaSuccess ? MG_OK : MG_ERR_CUDA;
+}
 
 // ---------------------------------------------------------------- host: TMA tensor maps
 

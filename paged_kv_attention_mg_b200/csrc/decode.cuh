@@ -47,7 +47,7 @@ namespace decode {
 
 constexpr int kKeys = 16;          // keys per unit / pipeline tile
 #ifndef MG_DECODE_WARPS
-#define MG_DECODE_WARPS 4  // workers per CTA (build-time tunable)
+#define MG_DECODE_WARPS 6  // workers per CTA (build-time tunable)
 #endif
 constexpr int kWarps = MG_DECODE_WARPS;
 constexpr int kThreads = kWarps * 32;
@@ -58,10 +58,10 @@ constexpr int kScanChunk = 4 * kThreads;           // requests per scan step
 constexpr int kMaxScanChunks = 256;                // requests <= 131072
 
 #ifndef MG_DECODE_STAGES
-#define MG_DECODE_STAGES 3  // per-worker ring depth (build-time tunable)
+#define MG_DECODE_STAGES 4  // per-worker ring depth (build-time tunable)
 #endif
 #ifndef MG_DECODE_MIN_BLOCKS
-#define MG_DECODE_MIN_BLOCKS 2  // resident CTAs per SM (the shared memory is sized for it)
+#define MG_DECODE_MIN_BLOCKS 1  // resident CTAs per SM (the shared memory is sized for it)
 #endif
 #ifndef MG_DECODE_TMA
 #define MG_DECODE_TMA 0  // 1: K/V tiles by TMA gather4 + mbarrier; 0: 16-byte cp.async
@@ -119,8 +119,10 @@ __device__ __forceinline__ int64_t request_units(const Params &p, int r, int &L,
     return (int64_t)((L + kKeys - 1) / kKeys) * p.num_kv_heads;
 }
 
+// First unit of worker w out of W over `total` units (the host guarantees
+// total * W < 2^62, so the product fits 64 bits).
 __device__ __forceinline__ int64_t worker_begin(int64_t total, int w, int W) {
-    return (int64_t)(((__int128)total * w) / W);
+    return total * (int64_t)w / (int64_t)W;
 }
 
 // Block-wide exclusive scan of one int64 per thread; returns the block total.
@@ -243,6 +245,8 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
     const int W = p.num_workers;
     const int w = blockIdx.x * kWarps + warp;
     const int nchunks = (p.batch + kScanChunk - 1) / kScanChunk;
+    griddep_launch_dependents();  // the merge kernel may launch and wait on us
+    griddep_wait();               // inputs written by the previous kernel (e.g. the KV store)
 
     // ---- pass 1: units per scan chunk (and the total T)
     unsigned bad = 0;
@@ -670,6 +674,8 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
 __global__ void __launch_bounds__(128) decode_merge_kernel(const Params p) {
     const int wg = blockIdx.x * 4 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
+    griddep_launch_dependents();
+    griddep_wait();  // the decode kernel's partials
     if (wg >= p.batch * p.num_q_heads) return;
     const int r = wg / p.num_q_heads, h = wg - r * p.num_q_heads;
     const int g = p.group;
@@ -680,8 +686,8 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const Params p) {
     const int64_t tiles = units_r / p.num_kv_heads;
     const int64_t u0 = pr + kvh * tiles, u1 = u0 + tiles;  // this pair's units
     const int W = p.num_workers;
-    auto worker_of = [&](int64_t u) -> int {
-        const int64_t wv = (int64_t)((((__int128)(u + 1)) * W - 1) / T);
+    auto worker_of = [&](int64_t u) -> int {  // the worker whose share holds unit u
+        const int64_t wv = ((u + 1) * (int64_t)W - 1) / T;
         return (int)(wv < W - 1 ? wv : W - 1);
     };
     const int wf = worker_of(u0), wl = worker_of(u1 - 1);

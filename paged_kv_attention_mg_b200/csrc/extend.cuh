@@ -139,6 +139,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int r = blockIdx.z, kvh = blockIdx.y;
+    griddep_launch_dependents();
+    griddep_wait();  // inputs written by the previous kernel (e.g. the KV store)
     const int qb = gridDim.x - 1 - blockIdx.x;  // heaviest (latest) q blocks first
 
     // ---- request metadata (uniform across the CTA; exit before any barrier)
@@ -445,8 +447,7 @@ inline mg_status launch(Params &p, cudaStream_t stream) {
     const int nqb = (p.max_q_len + tokens_per_cta - 1) / tokens_per_cta;
     if (nqb > 0x7fffffff || p.batch > 65535 || p.num_kv_heads > 65535) return MG_ERR_INVALID_ARGUMENT;
     dim3 grid((unsigned)nqb, (unsigned)p.num_kv_heads, (unsigned)p.batch);
-    extend_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tq, tk, tv, p);
-    return cudaGetLastError() == cudaSuccess ? MG_OK : MG_ERR_CUDA;
+    return launch_pdl(extend_kernel, grid, dim3(kThreads), kSmemBytes, stream, tq, tk, tv, p);
 }
 
 }  // namespace extend

@@ -59,10 +59,6 @@ mg_status ensure_kernel_attributes() {
     return MG_OK;
 }
 
-mg_status launched() {
-    return cudaGetLastError() == cudaSuccess ? MG_OK : MG_ERR_CUDA;
-}
-
 // Decode plan: the number of workers (warps) that share the work equally.
 // Automatic: one per warp slot the device keeps resident (SMs x resident CTAs
 // x 4), i.e. a single persistent wave.  Forced: num_partitions workers.
@@ -153,8 +149,7 @@ mg_status mg_store_kv(const void *k, const void *v, const int32_t *out_loc, int3
     long long blocks = (p.total_vecs + threads - 1) / threads;
     const long long cap = (long long)sms * 8;
     if (blocks > cap) blocks = cap;
-    store_kv_kernel<<<(unsigned)blocks, threads, 0, static_cast<cudaStream_t>(stream)>>>(p);
-    return launched();
+    return launch_pdl(store_kv_kernel, dim3((unsigned)blocks), dim3(threads), 0, static_cast<cudaStream_t>(stream), p);
 }
 
 mg_status mg_decode_plan(int32_t batch, int32_t num_kv_heads, int32_t max_seq_len,
@@ -194,6 +189,9 @@ mg_status mg_decode_attn(const void *q, const void *k_cache, const void *v_cache
     int workers;
     st = decode_plan(batch, num_kv_heads, max_seq_len, num_partitions, workers);
     if (st != MG_OK) return st;
+    // units <= batch * Hkv * ceil(max_seq_len / 16); the partition math multiplies by workers
+    const double max_units = (double)batch * num_kv_heads * ((max_seq_len + 15) / 16);
+    if (max_units * (double)(workers + 1) >= 4.0e18) return MG_ERR_UNSUPPORTED_SHAPE;
     const DecodeWorkspace ws = decode_ws_layout(batch, num_q_heads, num_kv_heads, workers);
     if (!workspace || workspace_bytes < ws.total) return MG_ERR_WORKSPACE_TOO_SMALL;
     if (!aligned16(workspace)) return MG_ERR_MISALIGNED;
@@ -230,13 +228,12 @@ mg_status mg_decode_attn(const void *q, const void *k_cache, const void *v_cache
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int ctas = (workers + decode::kWarps - 1) / decode::kWarps;
     if (p.group <= 8)
-        decode::decode_kernel<1><<<ctas, decode::kThreads, decode::kSmemBytes, s>>>(tk, tv, p);
+        st = launch_pdl(decode::decode_kernel<1>, dim3(ctas), dim3(decode::kThreads), decode::kSmemBytes, s, tk, tv, p);
     else
-        decode::decode_kernel<2><<<ctas, decode::kThreads, decode::kSmemBytes, s>>>(tk, tv, p);
-    if ((st = launched()) != MG_OK) return st;
+        st = launch_pdl(decode::decode_kernel<2>, dim3(ctas), dim3(decode::kThreads), decode::kSmemBytes, s, tk, tv, p);
+    if (st != MG_OK) return st;
     const int warps = batch * num_q_heads;
-    decode::decode_merge_kernel<<<(warps + 3) / 4, 128, 0, s>>>(p);
-    return launched();
+    return launch_pdl(decode::decode_merge_kernel, dim3((warps + 3) / 4), dim3(128), 0, s, p);
 }
 
 mg_status mg_extend_attn(const void *q, const void *k_cache, const void *v_cache, int64_t num_slots,

@@ -26,6 +26,8 @@ struct StoreParams {
 };
 
 __global__ void __launch_bounds__(256) store_kv_kernel(const StoreParams p) {
+    griddep_launch_dependents();  // attention may launch and wait on the store
+    griddep_wait();               // k / v / out_loc written by the previous kernel
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < p.total_vecs; i += stride) {
         const int64_t t = i / p.vecs_per_token;
