@@ -54,8 +54,7 @@ constexpr int kThreads = kWarps * 32;
 constexpr int kRows = 16;          // MMA M: GQA group padded to 16
 constexpr int kRowBytes = kHeadDim * 2;
 constexpr int kTileBytes = 2 * kKeys * kRowBytes;  // K + V rows of one tile: 8 KB
-constexpr int kScanChunk = 4 * kThreads;           // requests per scan step
-constexpr int kMaxScanChunks = 256;                // requests <= 131072
+constexpr int kMaxBatch = 131072;                  // requests per call
 
 #ifndef MG_DECODE_STAGES
 #define MG_DECODE_STAGES 4  // per-worker ring depth (build-time tunable)
@@ -76,6 +75,8 @@ constexpr int kMaxScanChunks = 256;                // requests <= 131072
 #define MG_DECODE_L2_MODE 2  // 1: bulk prefetch (one 256-B request), 2: two 128-B line prefetches
 #endif
 constexpr int kStages = MG_DECODE_STAGES;
+constexpr int kScanChunk = 4 * kThreads;  // requests per scan step
+constexpr int kMaxScanChunks = (kMaxBatch + kScanChunk - 1) / kScanChunk;
 constexpr int kIdxAhead = MG_DECODE_IDX_AHEAD;
 constexpr int kL2Ahead = MG_DECODE_L2_AHEAD;
 constexpr int kDescRing = 16;  // per-warp ring of tile descriptors / index rows

@@ -64,7 +64,7 @@ mg_status ensure_kernel_attributes() {
 // x 4), i.e. a single persistent wave.  Forced: num_partitions workers.
 mg_status decode_plan(int batch, int hkv, int max_seq_len, int num_partitions, int &workers) {
     if (batch <= 0 || hkv <= 0 || max_seq_len <= 0 || num_partitions < 0) return MG_ERR_INVALID_ARGUMENT;
-    if (batch > decode::kMaxScanChunks * decode::kScanChunk) return MG_ERR_UNSUPPORTED_SHAPE;
+    if (batch > decode::kMaxBatch) return MG_ERR_UNSUPPORTED_SHAPE;
     if (num_partitions > 0) {
         if (num_partitions > kMaxDecodeWorkers) return MG_ERR_INVALID_ARGUMENT;
         workers = num_partitions;
