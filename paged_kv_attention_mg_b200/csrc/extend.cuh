@@ -36,7 +36,10 @@ namespace extend {
 constexpr int kM = 128;                     // query rows per Q tile
 constexpr int kN = 128;                     // keys per KV tile
 constexpr int kQTiles = 2;
-constexpr int kStages = 2;
+constexpr int kKStages = 3;                 // K ring: S of a tile needs K before P V needs V
+constexpr int kVStages = 2;                 // V ring
+constexpr int kIdxAhead = 3;                // tiles of page-table entries in flight ahead of the K issue
+constexpr int kIdxRing = 4;                 // >= kIdxAhead + 1
 constexpr int kThreads = 320;               // 10 warps
 constexpr int kHalfBytes = 128 * 128;       // 128 rows x 128 B (64 bf16): one swizzle column
 constexpr int kTileBytes = 2 * kHalfBytes;  // 128 rows x 256 B
@@ -45,14 +48,18 @@ __device__ __forceinline__ uint32_t col_s(int t) { return (uint32_t)t * 128u; }
 __device__ __forceinline__ uint32_t col_o(int t) { return 256u + (uint32_t)t * 128u; }
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
 
-// shared memory map (offsets from a 1024-byte aligned base)
+// shared memory map.  The kernel has no static shared memory, so its dynamic
+// shared memory starts on a 1024-byte boundary (checked at run time), as the
+// 128-byte swizzle atoms require; every region below keeps that alignment.
 constexpr int kOffQ = 0;
 constexpr int kOffK = kOffQ + kQTiles * kTileBytes;
-constexpr int kOffV = kOffK + kStages * kTileBytes;
-constexpr int kOffBar = kOffV + kStages * kTileBytes;
-constexpr int kNumBars = 1 + 3 * kStages + 3 * kQTiles;
+constexpr int kOffV = kOffK + kKStages * kTileBytes;
+constexpr int kOffIdx = kOffV + kVStages * kTileBytes;
+constexpr int kOffBar = kOffIdx + kIdxRing * kN * 4;
+constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 3 * kQTiles;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
-constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
+constexpr int kSmemBytes = kOffMisc + 16;
+static_assert(kSmemBytes <= 227 * 1024, "extend shared memory over the per-CTA limit");
 
 struct Params {
     const __nv_bfloat16 *q;
@@ -95,7 +102,7 @@ __host__ __device__ constexpr uint32_t idesc_bf16(bool b_mn_major) {
 
 struct Sync {
     uint32_t q_full;
-    uint32_t k_full[kStages], v_full[kStages], kv_empty[kStages];
+    uint32_t k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
     uint32_t s_full[kQTiles], p_full[kQTiles], o_done[kQTiles];
 };
 
@@ -131,9 +138,12 @@ __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, vol
 __global__ void __launch_bounds__(kThreads, 1)
     extend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const Params p) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    extern __shared__ __align__(1024) uint8_t smem[];
     const uint32_t sbase = smem_u32(smem);
+    if (sbase & 1023u) {  // the swizzled layouts need 1024-byte alignment: refuse, never fault
+        if (threadIdx.x == 0) atomicOr(&g_mg_device_error, MG_DEVERR_WAIT_TIMEOUT);
+        return;
+    }
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffMisc);
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + kOffMisc + 4);
 
@@ -173,9 +183,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     {
         uint32_t b = sbase + kOffBar;
         sy.q_full = b; b += 8;
-        for (int s = 0; s < kStages; ++s) { sy.k_full[s] = b; b += 8; }
-        for (int s = 0; s < kStages; ++s) { sy.v_full[s] = b; b += 8; }
-        for (int s = 0; s < kStages; ++s) { sy.kv_empty[s] = b; b += 8; }
+        for (int s = 0; s < kKStages; ++s) { sy.k_full[s] = b; b += 8; }
+        for (int s = 0; s < kKStages; ++s) { sy.k_empty[s] = b; b += 8; }
+        for (int s = 0; s < kVStages; ++s) { sy.v_full[s] = b; b += 8; }
+        for (int s = 0; s < kVStages; ++s) { sy.v_empty[s] = b; b += 8; }
         for (int t = 0; t < kQTiles; ++t) { sy.s_full[t] = b; b += 8; }
         for (int t = 0; t < kQTiles; ++t) { sy.p_full[t] = b; b += 8; }
         for (int t = 0; t < kQTiles; ++t) { sy.o_done[t] = b; b += 8; }
@@ -183,10 +194,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         *abort_flag = 0;
         mbar_init(sy.q_full, 1);
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < kKStages; ++s) {
             mbar_init(sy.k_full[s], 1);
+            mbar_init(sy.k_empty[s], 1);
+        }
+        for (int s = 0; s < kVStages; ++s) {
             mbar_init(sy.v_full[s], 1);
-            mbar_init(sy.kv_empty[s], 1);
+            mbar_init(sy.v_empty[s], 1);
         }
         for (int t = 0; t < kQTiles; ++t) {
             mbar_init(sy.s_full[t], 1);
@@ -219,40 +233,71 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const int32_t *pt = p.page_table + (int64_t)row * p.pt_stride;
         const int oob_row = (int)(p.num_slots * p.num_kv_heads);  // reads as zeros
-        for (int j = 0; j < n_kv; ++j) {
-            const int s = j % kStages;
-            if (j >= kStages && !wait_or_abort(sy.kv_empty[s], ((j / kStages) - 1) & 1, abort_flag)) break;
-            int rows[4];
+        int *idx_ring = reinterpret_cast<int *>(smem + kOffIdx);
+        // page-table entries of tile j: lane l copies keys 4l .. 4l+3 (one cp.async group per tile)
+        auto fetch_idx = [&](int j) {
+            if (j < n_kv) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int key = j * kN + lane * 4 + e;
+                    int *dst = idx_ring + (j % kIdxRing) * kN + lane * 4 + e;
+                    if (key < kv_len) cp_async_4(smem_u32(dst), pt + key);
+                    else *dst = -1;
+                }
+            }
+            cp_async_commit();
+        };
+        auto rows_of = [&](int j, int (&rows)[4]) {
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int key = j * kN + lane * 4 + e;
-                int slot = key < kv_len ? __ldg(pt + key) : -1;
+                int slot = key < kv_len ? idx_ring[(j % kIdxRing) * kN + lane * 4 + e] : -1;
                 if (key < kv_len && (slot < 0 || (int64_t)slot >= p.num_slots)) {
                     atomicOr(&g_mg_device_error, MG_DEVERR_SLOT_RANGE);
                     slot = -1;
                 }
                 rows[e] = slot < 0 ? oob_row : slot * p.num_kv_heads + kvh;
             }
-            if (lane == 0) mbar_arrive_expect_tx(sy.k_full[s], kTileBytes);
+        };
+        auto gather = [&](const CUtensorMap *tm, uint32_t tile_base, uint32_t bar, const int (&rows)[4]) {
+            if (lane == 0) mbar_arrive_expect_tx(bar, kTileBytes);
             __syncwarp();
-            const uint32_t kdst = sbase + kOffK + s * kTileBytes + lane * 4 * 128;
-            tma_gather4(kdst, &tm_k, sy.k_full[s], 0, rows[0], rows[1], rows[2], rows[3]);
-            tma_gather4(kdst + kHalfBytes, &tm_k, sy.k_full[s], 64, rows[0], rows[1], rows[2], rows[3]);
-            if (lane == 0) mbar_arrive_expect_tx(sy.v_full[s], kTileBytes);
-            __syncwarp();
-            const uint32_t vdst = sbase + kOffV + s * kTileBytes + lane * 4 * 128;
-            tma_gather4(vdst, &tm_v, sy.v_full[s], 0, rows[0], rows[1], rows[2], rows[3]);
-            tma_gather4(vdst + kHalfBytes, &tm_v, sy.v_full[s], 64, rows[0], rows[1], rows[2], rows[3]);
+            const uint32_t dst = tile_base + lane * 4 * 128;
+            tma_gather4(dst, tm, bar, 0, rows[0], rows[1], rows[2], rows[3]);
+            tma_gather4(dst + kHalfBytes, tm, bar, 64, rows[0], rows[1], rows[2], rows[3]);
+        };
+#pragma unroll
+        for (int j = 0; j < kIdxAhead; ++j) fetch_idx(j);
+        // iteration j: entries of tile j + kIdxAhead requested; K of tile j
+        // issued; V of tile j - 1 issued (K leads V by one tile)
+        int prev_rows[4] = {oob_row, oob_row, oob_row, oob_row};
+        for (int j = 0; j <= n_kv; ++j) {
+            fetch_idx(j + kIdxAhead);
+            int rows[4] = {oob_row, oob_row, oob_row, oob_row};
+            if (j < n_kv) {
+                const int s = j % kKStages;
+                if (j >= kKStages && !wait_or_abort(sy.k_empty[s], ((j / kKStages) - 1) & 1, abort_flag)) break;
+                cp_async_wait<kIdxAhead>();
+                rows_of(j, rows);
+                gather(&tm_k, sbase + kOffK + s * kTileBytes, sy.k_full[s], rows);
+            }
+            if (j >= 1) {
+                const int jv = j - 1, s = jv % kVStages;
+                if (jv >= kVStages && !wait_or_abort(sy.v_empty[s], ((jv / kVStages) - 1) & 1, abort_flag)) break;
+                gather(&tm_v, sbase + kOffV + s * kTileBytes, sy.v_full[s], prev_rows);
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) prev_rows[e] = rows[e];
         }
+        cp_async_wait<0>();
     } else if (warp == 1) {
         // =============================================================== MMA issue
         if (lane == 0) {
             constexpr uint32_t idesc_qk = idesc_bf16(false);
             constexpr uint32_t idesc_pv = idesc_bf16(true);
             auto issue_s = [&](int t, int j) {
-                const int s = j % kStages;
                 const uint32_t qa = sbase + kOffQ + t * kTileBytes;
-                const uint32_t ka = sbase + kOffK + s * kTileBytes;
+                const uint32_t ka = sbase + kOffK + (j % kKStages) * kTileBytes;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
@@ -262,8 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 umma_commit(sy.s_full[t]);
             };
             auto issue_pv = [&](int t, int j) {
-                const int s = j % kStages;
-                const uint32_t va = sbase + kOffV + s * kTileBytes;
+                const uint32_t va = sbase + kOffV + (j % kVStages) * kTileBytes;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     umma_ts(tmem + col_o(t), tmem + col_s(t) + kk * 8,
@@ -275,18 +319,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 issue_s(0, 0);
                 if (has_q1) issue_s(1, 0);
+                umma_commit(sy.k_empty[0]);
             }
             for (int j = 0; ok && j < n_kv; ++j) {
-                const int s = j % kStages;
-                const uint32_t ph = (j / kStages) & 1;
-                if (!(ok = wait_or_abort_thread(sy.v_full[s], ph, abort_flag))) break;
+                const int sv = j % kVStages;
+                if (!(ok = wait_or_abort_thread(sy.v_full[sv], (j / kVStages) & 1, abort_flag))) break;
                 if (!(ok = wait_or_abort_thread(sy.p_full[0], j & 1, abort_flag))) break;
                 tc_fence_after();
                 issue_pv(0, j);
                 const bool more = j + 1 < n_kv;
                 if (more) {
-                    const int s1 = (j + 1) % kStages;
-                    if (!(ok = wait_or_abort_thread(sy.k_full[s1], ((j + 1) / kStages) & 1, abort_flag))) break;
+                    const int sk = (j + 1) % kKStages;
+                    if (!(ok = wait_or_abort_thread(sy.k_full[sk], ((j + 1) / kKStages) & 1, abort_flag))) break;
                     tc_fence_after();
                     issue_s(0, j + 1);
                 }
@@ -295,8 +339,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_fence_after();
                     issue_pv(1, j);
                 }
-                umma_commit(sy.kv_empty[s]);
-                if (more && has_q1) issue_s(1, j + 1);
+                umma_commit(sy.v_empty[sv]);
+                if (more) {
+                    if (has_q1) issue_s(1, j + 1);
+                    umma_commit(sy.k_empty[(j + 1) % kKStages]);
+                }
             }
         }
         __syncwarp();
