@@ -8,7 +8,8 @@
  *
  *   mg_store_kv     write the new tokens' K/V into pool slots at out_loc;
  *   mg_decode_attn  one query token per request against its paged history
- *                   (split-KV kernel + merge kernel);
+ *                   (balanced split-KV kernel + merge kernel);
+ *   mg_store_decode_attn  the two above fused into one decode launch;
  *   mg_extend_attn  a chunk of new tokens per request (chunked prefill),
  *                   causal over cached_len + i, on tcgen05 tensor cores.
  *
@@ -148,6 +149,33 @@ mg_status mg_decode_attn(const void *q, const void *k_cache, const void *v_cache
                          int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, float scale,
                          int32_t num_partitions, void *out, void *workspace, size_t workspace_bytes,
                          void *stream);
+
+/*
+ * mg_store_decode_attn -- mg_store_kv of the step's new tokens followed by
+ * mg_decode_attn, in one launch of the decode kernel (plus the merge kernel)
+ * instead of two.  The engine runs exactly this pair in every layer of a
+ * decode step (Mini-SGLang tag page, Engine post §一: write KV cache ->
+ * attention); fusing it removes a launch and a pool round trip per layer
+ * ("mini-sglang from Scratch Stage 4 · Faster and bigger", §What each chapter
+ * adds: launch overhead of small operations such as KV writes).
+ *
+ *   k_new, v_new  [batch, num_kv_heads, head_dim] bf16: request r's new token
+ *   out_loc       [batch] int32, out_loc[r] = page_table[table_idx[r]][seq_len[r]-1]
+ *   k_cache, v_cache  updated in place exactly as mg_store_kv would
+ * Every other argument and the output are those of mg_decode_attn.  The new
+ * token's K/V enter attention from k_new / v_new directly; its pool slot is
+ * written by the one worker that owns that (request, kv head) tile.  An
+ * out_loc[r] that differs from the page-table entry of position seq_len-1 sets
+ * MG_DEVERR_LENGTH (the store and the attention would disagree); one outside
+ * the pool sets MG_DEVERR_SLOT_RANGE and is not written.
+ */
+mg_status mg_store_decode_attn(const void *q, const void *k_new, const void *v_new, const int32_t *out_loc,
+                               void *k_cache, void *v_cache, int64_t num_slots, const int32_t *page_table,
+                               int32_t page_table_rows, int32_t page_table_stride, const int32_t *table_idx,
+                               const int32_t *seq_len, int32_t batch, int32_t max_seq_len,
+                               int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, float scale,
+                               int32_t num_partitions, void *out, void *workspace, size_t workspace_bytes,
+                               void *stream);
 
 /*
  * mg_extend_attn -- chunked-prefill ("extend") attention over the paged pool

@@ -6,7 +6,7 @@
 algorithmic byte / FLOP formulas.
 """
 from .mg import (MgError, decode_attn, decode_plan, decode_workspace_bytes, extend_attn, load,
-                 read_device_error, store_kv)
+                 read_device_error, store_decode_attn, store_kv)
 
 __all__ = ["MgError", "decode_attn", "decode_plan", "decode_workspace_bytes", "extend_attn", "load",
-           "read_device_error", "store_kv"]
+           "read_device_error", "store_decode_attn", "store_kv"]

@@ -96,6 +96,14 @@ struct Params {
     const int32_t *seq_len;
     __nv_bfloat16 *out;
     int64_t *prefix;  // [B + 1] units before request r (written by CTA 0 for the merge)
+    // fused KV store (store + decode in one launch), else null: the new token
+    // of request r is row r of k_new / v_new [B, Hkv, 128], destined for
+    // pool slot out_loc[r], which must be the page-table entry of position L-1
+    const __nv_bfloat16 *k_new;
+    const __nv_bfloat16 *v_new;
+    const int32_t *out_loc;
+    __nv_bfloat16 *k_store;  // the pools, writable
+    __nv_bfloat16 *v_store;
     float *part_lse;  // [slots, group]
     float *part_o;    // [slots, group, 128]
     int64_t num_slots;
@@ -159,7 +167,7 @@ struct Cursor {
 struct TileDesc {
     int r, kvh, t, tiles, L, row;
     unsigned valid;  // bit i: key i has an accepted slot (set when the tile is issued)
-    int pad;
+    int store_slot;  // fused store: out_loc[r] when this is the pair's last tile
 };
 
 __device__ __forceinline__ bool metadata_ok(const Params &p, int L, int row) {
@@ -226,7 +234,9 @@ __device__ __forceinline__ bool warp_wait_bounded(uint32_t bar, uint32_t parity)
     return __all_sync(0xffffffffu, done);
 }
 
-template <int NT>  // n-tiles of 8 GQA heads: 1 for g <= 8, 2 for g <= 16
+// NT: n-tiles of 8 GQA heads (1 for g <= 8, 2 for g <= 16).
+// FUSED: the KV store of the step's new tokens happens in the same launch.
+template <int NT, bool FUSED>
 __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
     decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                   const Params p) {
@@ -352,8 +362,10 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
             if (lane == 0) {
                 TileDesc d;
                 d.r = cur.r; d.kvh = cur.kvh; d.t = cur.t; d.tiles = cur.tiles; d.L = cur.L; d.row = cur.row;
-                d.valid = 0; d.pad = 0;
+                d.valid = 0; d.store_slot = -1;
                 my_desc[e] = d;
+                if (FUSED && cur.t == cur.tiles - 1)  // the pair's last tile holds the new token
+                    cp_async_4(smem_u32(&my_desc[e].store_slot), p.out_loc + cur.r);
             }
             const int key = cur.t * kKeys + lane;
             if (lane < kKeys) {
@@ -403,6 +415,10 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
         const uint32_t base = ring + (uint32_t)(stage * kTileBytes);
         const int ch = lane & 15;
         const int64_t head_off = (int64_t)d.kvh * kHeadDim + ch * 8;
+        // fused store: the new token (position L-1) is read from k_new / v_new,
+        // the pool slot is written only after this tile lands
+        const int new_key = (FUSED && d.t == d.tiles - 1) ? d.L - 1 - d.t * kKeys : -1;
+        const int64_t new_off = ((int64_t)d.r * p.num_kv_heads + d.kvh) * kHeadDim + ch * 8;
 #pragma unroll
         for (int it = 0; it < 16; ++it) {
             const int rr = it * 2 + (lane >> 4);
@@ -410,6 +426,7 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
             const bool is_v = rr >= kKeys;
             const int sl = __shfl_sync(0xffffffffu, slot, key);
             const __nv_bfloat16 *src = (is_v ? p.v_cache : p.k_cache) + (int64_t)(sl < 0 ? 0 : sl) * head_stride + head_off;
+            if (key == new_key) src = (is_v ? p.v_new : p.k_new) + new_off;
             cp_async_16(base + (is_v ? 2 * kHalfRows : 0) + swz(key, ch), src, sl < 0 ? 0u : 16u);
         }
 #endif
@@ -607,6 +624,27 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
                 ldmatrix_x4_trans(vt + swz(key, 2 * dt + (mi & 1)), a[0], a[1], a[2], a[3]);
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(o[nt][dt], a, pb[nt][0], pb[nt][1]);
+            }
+        }
+        if (FUSED && c.t == c.tiles - 1) {
+            // fused store: lanes 0-15 copy the new token's K row, lanes 16-31 its V row,
+            // 16 bytes each, from the landed stage into pool slot out_loc[r]
+            const int nk = c.L - 1 - c.t * kKeys;
+            const int ss = c.store_slot;
+            const int pt_slot = my_idx[k % kDescRing][nk];
+            if (ss < 0 || (int64_t)ss >= p.num_slots) {
+                if (lane == 0) atomicOr(&g_mg_device_error, MG_DEVERR_SLOT_RANGE);
+            } else {
+                if (lane == 0 && ss != pt_slot) atomicOr(&g_mg_device_error, MG_DEVERR_LENGTH);
+                const int ch = lane & 15;
+                const bool is_v = lane >= 16;
+                uint4 v;
+                asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];\n"
+                             : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                             : "r"(kt + (is_v ? 2 * kHalfRows : 0) + swz(nk, ch)));
+                __nv_bfloat16 *dst = (is_v ? p.v_store : p.k_store) + (int64_t)ss * head_stride +
+                                     (int64_t)c.kvh * kHeadDim + ch * 8;
+                *reinterpret_cast<uint4 *>(dst) = v;
             }
         }
         __syncwarp();  // every lane is done reading this stage

@@ -49,9 +49,13 @@ mg_status ensure_kernel_attributes() {
     if (g_attr_done[dev]) return MG_OK;
     std::lock_guard<std::mutex> lock(g_attr_mutex);
     if (g_attr_done[dev]) return MG_OK;
-    if (cudaFuncSetAttribute(decode::decode_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(decode::decode_kernel<1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              decode::kSmemBytes) != cudaSuccess ||
-        cudaFuncSetAttribute(decode::decode_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaFuncSetAttribute(decode::decode_kernel<2, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             decode::kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(decode::decode_kernel<1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             decode::kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(decode::decode_kernel<2, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              decode::kSmemBytes) != cudaSuccess)
         return MG_ERR_CUDA;
     if (extend::set_attributes() != cudaSuccess) return MG_ERR_CUDA;
@@ -100,6 +104,89 @@ mg_status check_attention_shape(int hq, int hkv, int head_dim) {
     return MG_OK;
 }
 
+}  // namespace
+}  // namespace mg
+
+namespace mg {
+namespace {
+// Decode attention; with k_new != nullptr the KV store of the step's new
+// tokens (one per request) is fused into the same launch.
+mg_status decode_impl(const void *q, const void *k_new, const void *v_new, const int32_t *out_loc,
+                      const void *k_cache, const void *v_cache, int64_t num_slots, const int32_t *page_table,
+                      int32_t page_table_rows, int32_t page_table_stride, const int32_t *table_idx,
+                      const int32_t *seq_len, int32_t batch, int32_t max_seq_len, int32_t num_q_heads,
+                      int32_t num_kv_heads, int32_t head_dim, float scale, int32_t num_partitions, void *out,
+                      void *workspace, size_t workspace_bytes, void *stream) {
+    const bool fused = k_new != nullptr;
+    mg_status st = check_attention_shape(num_q_heads, num_kv_heads, head_dim);
+    if (st != MG_OK) return st;
+    if (batch <= 0 || num_slots <= 0 || page_table_rows <= 0 || page_table_stride <= 0 ||
+        max_seq_len <= 0 || max_seq_len > page_table_stride)
+        return MG_ERR_INVALID_ARGUMENT;
+    if (!q || !k_cache || !v_cache || !page_table || !table_idx || !seq_len || !out)
+        return MG_ERR_INVALID_ARGUMENT;
+    if (fused && (!v_new || !out_loc)) return MG_ERR_INVALID_ARGUMENT;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
+        return MG_ERR_MISALIGNED;
+    if (fused && (!aligned16(k_new) || !aligned16(v_new))) return MG_ERR_MISALIGNED;
+    int workers;
+    st = decode_plan(batch, num_kv_heads, max_seq_len, num_partitions, workers);
+    if (st != MG_OK) return st;
+    // units <= batch * Hkv * ceil(max_seq_len / 16); the partition math multiplies by workers
+    const double max_units = (double)batch * num_kv_heads * ((max_seq_len + 15) / 16);
+    if (max_units * (double)(workers + 1) >= 4.0e18) return MG_ERR_UNSUPPORTED_SHAPE;
+    const DecodeWorkspace ws = decode_ws_layout(batch, num_q_heads, num_kv_heads, workers);
+    if (!workspace || workspace_bytes < ws.total) return MG_ERR_WORKSPACE_TOO_SMALL;
+    if (!aligned16(workspace)) return MG_ERR_MISALIGNED;
+    if (ensure_kernel_attributes() != MG_OK) return MG_ERR_CUDA;
+
+    decode::Params p;
+    p.q = static_cast<const __nv_bfloat16 *>(q);
+    p.k_cache = static_cast<const __nv_bfloat16 *>(k_cache);
+    p.v_cache = static_cast<const __nv_bfloat16 *>(v_cache);
+    p.page_table = page_table;
+    p.table_idx = table_idx;
+    p.seq_len = seq_len;
+    p.out = static_cast<__nv_bfloat16 *>(out);
+    uint8_t *wsb = static_cast<uint8_t *>(workspace);
+    p.prefix = reinterpret_cast<int64_t *>(wsb + ws.prefix);
+    p.part_lse = reinterpret_cast<float *>(wsb + ws.lse);
+    p.part_o = reinterpret_cast<float *>(wsb + ws.o);
+    p.k_new = static_cast<const __nv_bfloat16 *>(k_new);
+    p.v_new = static_cast<const __nv_bfloat16 *>(v_new);
+    p.out_loc = out_loc;
+    p.k_store = const_cast<__nv_bfloat16 *>(p.k_cache);
+    p.v_store = const_cast<__nv_bfloat16 *>(p.v_cache);
+    p.num_slots = num_slots;
+    p.pt_rows = page_table_rows;
+    p.pt_stride = page_table_stride;
+    p.batch = batch;
+    p.num_q_heads = num_q_heads;
+    p.num_kv_heads = num_kv_heads;
+    p.group = num_q_heads / num_kv_heads;
+    p.num_workers = workers;
+    p.max_seq_len = max_seq_len;
+    p.scale_log2 = scale * kLog2e;
+
+    if ((uint64_t)num_slots * (uint64_t)num_kv_heads >= (1ull << 31)) return MG_ERR_UNSUPPORTED_SHAPE;
+    CUtensorMap tk, tv;
+    if (!make_pool_tmap(&tk, k_cache, num_slots, num_kv_heads) ||
+        !make_pool_tmap(&tv, v_cache, num_slots, num_kv_heads))
+        return MG_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int ctas = (workers + decode::kWarps - 1) / decode::kWarps;
+    const dim3 grid(ctas), block(decode::kThreads);
+    const size_t smem = decode::kSmemBytes;
+    if (p.group <= 8)
+        st = fused ? launch_pdl(decode::decode_kernel<1, true>, grid, block, smem, s, tk, tv, p)
+                   : launch_pdl(decode::decode_kernel<1, false>, grid, block, smem, s, tk, tv, p);
+    else
+        st = fused ? launch_pdl(decode::decode_kernel<2, true>, grid, block, smem, s, tk, tv, p)
+                   : launch_pdl(decode::decode_kernel<2, false>, grid, block, smem, s, tk, tv, p);
+    if (st != MG_OK) return st;
+    const int warps = batch * num_q_heads;
+    return launch_pdl(decode::decode_merge_kernel, dim3((warps + 3) / 4), dim3(128), 0, s, p);
+}
 }  // namespace
 }  // namespace mg
 
@@ -177,63 +264,22 @@ mg_status mg_decode_attn(const void *q, const void *k_cache, const void *v_cache
                          int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, float scale,
                          int32_t num_partitions, void *out, void *workspace, size_t workspace_bytes,
                          void *stream) {
-    mg_status st = check_attention_shape(num_q_heads, num_kv_heads, head_dim);
-    if (st != MG_OK) return st;
-    if (batch <= 0 || num_slots <= 0 || page_table_rows <= 0 || page_table_stride <= 0 ||
-        max_seq_len <= 0 || max_seq_len > page_table_stride)
-        return MG_ERR_INVALID_ARGUMENT;
-    if (!q || !k_cache || !v_cache || !page_table || !table_idx || !seq_len || !out)
-        return MG_ERR_INVALID_ARGUMENT;
-    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
-        return MG_ERR_MISALIGNED;
-    int workers;
-    st = decode_plan(batch, num_kv_heads, max_seq_len, num_partitions, workers);
-    if (st != MG_OK) return st;
-    // units <= batch * Hkv * ceil(max_seq_len / 16); the partition math multiplies by workers
-    const double max_units = (double)batch * num_kv_heads * ((max_seq_len + 15) / 16);
-    if (max_units * (double)(workers + 1) >= 4.0e18) return MG_ERR_UNSUPPORTED_SHAPE;
-    const DecodeWorkspace ws = decode_ws_layout(batch, num_q_heads, num_kv_heads, workers);
-    if (!workspace || workspace_bytes < ws.total) return MG_ERR_WORKSPACE_TOO_SMALL;
-    if (!aligned16(workspace)) return MG_ERR_MISALIGNED;
-    if (ensure_kernel_attributes() != MG_OK) return MG_ERR_CUDA;
+    return decode_impl(q, nullptr, nullptr, nullptr, k_cache, v_cache, num_slots, page_table, page_table_rows,
+                       page_table_stride, table_idx, seq_len, batch, max_seq_len, num_q_heads, num_kv_heads,
+                       head_dim, scale, num_partitions, out, workspace, workspace_bytes, stream);
+}
 
-    decode::Params p;
-    p.q = static_cast<const __nv_bfloat16 *>(q);
-    p.k_cache = static_cast<const __nv_bfloat16 *>(k_cache);
-    p.v_cache = static_cast<const __nv_bfloat16 *>(v_cache);
-    p.page_table = page_table;
-    p.table_idx = table_idx;
-    p.seq_len = seq_len;
-    p.out = static_cast<__nv_bfloat16 *>(out);
-    uint8_t *wsb = static_cast<uint8_t *>(workspace);
-    p.prefix = reinterpret_cast<int64_t *>(wsb + ws.prefix);
-    p.part_lse = reinterpret_cast<float *>(wsb + ws.lse);
-    p.part_o = reinterpret_cast<float *>(wsb + ws.o);
-    p.num_slots = num_slots;
-    p.pt_rows = page_table_rows;
-    p.pt_stride = page_table_stride;
-    p.batch = batch;
-    p.num_q_heads = num_q_heads;
-    p.num_kv_heads = num_kv_heads;
-    p.group = num_q_heads / num_kv_heads;
-    p.num_workers = workers;
-    p.max_seq_len = max_seq_len;
-    p.scale_log2 = scale * kLog2e;
-
-    if ((uint64_t)num_slots * (uint64_t)num_kv_heads >= (1ull << 31)) return MG_ERR_UNSUPPORTED_SHAPE;
-    CUtensorMap tk, tv;
-    if (!make_pool_tmap(&tk, k_cache, num_slots, num_kv_heads) ||
-        !make_pool_tmap(&tv, v_cache, num_slots, num_kv_heads))
-        return MG_ERR_CUDA;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const int ctas = (workers + decode::kWarps - 1) / decode::kWarps;
-    if (p.group <= 8)
-        st = launch_pdl(decode::decode_kernel<1>, dim3(ctas), dim3(decode::kThreads), decode::kSmemBytes, s, tk, tv, p);
-    else
-        st = launch_pdl(decode::decode_kernel<2>, dim3(ctas), dim3(decode::kThreads), decode::kSmemBytes, s, tk, tv, p);
-    if (st != MG_OK) return st;
-    const int warps = batch * num_q_heads;
-    return launch_pdl(decode::decode_merge_kernel, dim3((warps + 3) / 4), dim3(128), 0, s, p);
+mg_status mg_store_decode_attn(const void *q, const void *k_new, const void *v_new, const int32_t *out_loc,
+                               void *k_cache, void *v_cache, int64_t num_slots, const int32_t *page_table,
+                               int32_t page_table_rows, int32_t page_table_stride, const int32_t *table_idx,
+                               const int32_t *seq_len, int32_t batch, int32_t max_seq_len,
+                               int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, float scale,
+                               int32_t num_partitions, void *out, void *workspace, size_t workspace_bytes,
+                               void *stream) {
+    if (!k_new) return MG_ERR_INVALID_ARGUMENT;
+    return decode_impl(q, k_new, v_new, out_loc, k_cache, v_cache, num_slots, page_table, page_table_rows,
+                       page_table_stride, table_idx, seq_len, batch, max_seq_len, num_q_heads, num_kv_heads,
+                       head_dim, scale, num_partitions, out, workspace, workspace_bytes, stream);
 }
 
 mg_status mg_extend_attn(const void *q, const void *k_cache, const void *v_cache, int64_t num_slots,

@@ -42,6 +42,8 @@ SIGNATURES = {
     "mg_decode_workspace_bytes": (_SZ, [_I32, _I32, _I32, _I32, _I32, _I32]),
     "mg_decode_attn": (ctypes.c_int, [_P, _P, _P, _I64, _P, _I32, _I32, _P, _P, _I32, _I32, _I32, _I32,
                                       _I32, _F32, _I32, _P, _P, _SZ, _P]),
+    "mg_store_decode_attn": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _P, _I32, _I32, _P, _P, _I32, _I32,
+                                            _I32, _I32, _I32, _F32, _I32, _P, _P, _SZ, _P]),
     "mg_extend_attn": (ctypes.c_int, [_P, _P, _P, _I64, _P, _I32, _I32, _P, _P, _P, _P, _I32, _I32, _I32,
                                       _I32, _I32, _I32, _I32, _F32, _P, _P]),
     "mg_read_device_error": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_uint32)]),
@@ -148,6 +150,35 @@ def decode_attn(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, p
                                  _dev(seq_len, torch.int32, "seq_len"), b, max_seq_len, hq, hkv, d,
                                  float(scale), num_partitions, _dev(out, torch.bfloat16, "out"), ws_ptr, ws_bytes,
                                  _stream(stream)), "mg_decode_attn")
+    return out
+
+
+def store_decode_attn(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor, out_loc: torch.Tensor,
+                      k_cache: torch.Tensor, v_cache: torch.Tensor, page_table: torch.Tensor,
+                      table_idx: torch.Tensor, seq_len: torch.Tensor, max_seq_len: int, scale: float,
+                      num_partitions: int = 0, out: Optional[torch.Tensor] = None,
+                      workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """store_kv(k_new, v_new, out_loc) then decode_attn, fused into one decode launch."""
+    b, hq, d = q.shape
+    hkv = k_cache.shape[1]
+    if k_new.shape != (b, hkv, d) or v_new.shape != k_new.shape or out_loc.shape != (b,):
+        raise ValueError("store_decode_attn: one new token per request expected")
+    if out is None:
+        out = torch.empty_like(q)
+    need = decode_workspace_bytes(b, hq, hkv, max_seq_len, num_partitions, d)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = _dev(workspace, torch.uint8, "workspace") if workspace is not None else None
+    ws_bytes = workspace.numel() if workspace is not None else 0
+    _check(load().mg_store_decode_attn(_dev(q, torch.bfloat16, "q"), _dev(k_new, torch.bfloat16, "k_new"),
+                                       _dev(v_new, torch.bfloat16, "v_new"), _dev(out_loc, torch.int32, "out_loc"),
+                                       _dev(k_cache, torch.bfloat16, "k_cache"),
+                                       _dev(v_cache, torch.bfloat16, "v_cache"), k_cache.shape[0],
+                                       _dev(page_table, torch.int32, "page_table"), page_table.shape[0],
+                                       page_table.shape[1], _dev(table_idx, torch.int32, "table_idx"),
+                                       _dev(seq_len, torch.int32, "seq_len"), b, max_seq_len, hq, hkv, d,
+                                       float(scale), num_partitions, _dev(out, torch.bfloat16, "out"), ws_ptr,
+                                       ws_bytes, _stream(stream)), "mg_store_decode_attn")
     return out
 
 

@@ -151,6 +151,14 @@ class GpuStep:
         return mg.decode_attn(self.q, self.k_cache, self.v_cache, self.page_table, self.table_idx, self.seq_len,
                               msl, self.scale, num_partitions=num_partitions, out=out)
 
+    def store_decode(self, num_partitions=0, max_seq_len=None, out=None):
+        """The fused store + decode of one new token per request."""
+        from paged_kv_attention_mg_b200 import mg
+        msl = max_seq_len or self.step.max_seq_len
+        return mg.store_decode_attn(self.q, self.k_new, self.v_new, self.out_loc, self.k_cache, self.v_cache,
+                                    self.page_table, self.table_idx, self.seq_len, msl, self.scale,
+                                    num_partitions=num_partitions, out=out)
+
     def extend(self, out=None):
         from paged_kv_attention_mg_b200 import mg
         s = self.step

@@ -208,6 +208,59 @@ def test_decode_host_errors():
     assert e.value.status == 3
 
 
+# ----------------------------------------------------------------------------- fused store + decode
+
+@pytest.mark.parametrize("lengths,hq,hkv", DECODE_SMALL)
+@pytest.mark.parametrize("parts", [0, 1, 7])
+def test_store_decode_fused_matches_oracle_and_stores(lengths, hq, hkv, parts):
+    step, data = _custom("decode", [L - 1 for L in lengths], lengths, hq, hkv, seed=len(lengths) * 37 + hq)
+    g = GpuStep(step, data)
+    out = g.store_decode(num_partitions=parts)
+    assert mg.read_device_error() == 0
+    assert_matches_oracle(out, oracle_decode(step, data), f"fused {lengths} partitions {parts}")
+    k_ref, v_ref = host_pools_after_store(step, data)  # the pool as mg_store_kv leaves it
+    assert torch.equal(g.k_cache.cpu().view(torch.int16), k_ref.view(torch.int16))
+    assert torch.equal(g.v_cache.cpu().view(torch.int16), v_ref.view(torch.int16))
+
+
+@pytest.mark.parametrize("name", ["qwen3_0.6b_decode_28l", "batch256_gqa4_decode", "longctx_gqa8_decode"])
+def test_store_decode_fused_full_size(name):
+    spec = wl.BY_NAME[name]
+    step = wl.make_step(spec)
+    data = wl.make_layer(step, 3 if spec.num_layers > 3 else 0)
+    g = GpuStep(step, data)
+    out = g.store_decode()
+    assert mg.read_device_error() == 0
+    req = _sample(step, k=3 if name.startswith("longctx") else 6, seed=1)
+    assert_matches_oracle(out, oracle_decode(step, data, requests=req), f"fused {name}")
+    # the new tokens' slots now hold k_new / v_new
+    loc = step.out_loc.long()
+    assert torch.equal(g.k_cache[loc.cuda()].cpu().view(torch.int16), data.k_new.view(torch.int16))
+    assert torch.equal(g.v_cache[loc.cuda()].cpu().view(torch.int16), data.v_new.view(torch.int16))
+
+
+def test_store_decode_fused_equals_separate_calls():
+    step, data = _custom("decode", [130, 5, 999], [131, 6, 1000], 32, 8, seed=41)
+    a = GpuStep(step, data)
+    a.store()
+    sep = a.decode(num_partitions=9)
+    b = GpuStep(step, data)
+    fused = b.store_decode(num_partitions=9)
+    assert torch.equal(sep, fused)  # same partition, same arithmetic order
+    assert torch.equal(a.k_cache, b.k_cache) and torch.equal(a.v_cache, b.v_cache)
+
+
+def test_store_decode_flags_out_loc_mismatch():
+    step, data = _custom("decode", [9, 19], [10, 20], 16, 8, seed=42)
+    g = GpuStep(step, data)
+    mg.read_device_error()
+    bad = g.out_loc.clone()
+    bad[0] = int(step.dummy_slot)  # not the page-table entry of position L-1
+    mg.store_decode_attn(g.q, g.k_new, g.v_new, bad, g.k_cache, g.v_cache, g.page_table, g.table_idx,
+                         g.seq_len, 20, g.scale)
+    assert mg.read_device_error() & mg.DEVERR_LENGTH
+
+
 # ----------------------------------------------------------------------------- extend
 
 EXTEND_SMALL = [
