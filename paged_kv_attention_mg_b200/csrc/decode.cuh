@@ -732,26 +732,34 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const Params p) {
     const int wf = worker_of(u0), wl = worker_of(u1 - 1);
     if (wf == wl) return;  // one worker held the whole pair and wrote the output
     const int64_t pair = (int64_t)r * p.num_kv_heads + kvh;
-    float mx = -INFINITY;
-    for (int wk = wf + lane; wk <= wl; wk += 32) {
-        if (worker_begin(T, wk, W) == worker_begin(T, wk + 1, W)) continue;
-        mx = fmaxf(mx, p.part_lse[(pair + wk) * g + j]);
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-    float wsum = 0.f;
+    // online combine, four segments per round so their loads are in flight together
+    float mx = -INFINITY, wsum = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int wk = wf; wk <= wl; ++wk) {
-        if (worker_begin(T, wk, W) == worker_begin(T, wk + 1, W)) continue;
-        const int64_t s = pair + wk;
-        const float ls = p.part_lse[s * g + j];
-        const float wt = ls == -INFINITY ? 0.f : fast_exp2(ls - mx);
-        const float4 v = reinterpret_cast<const float4 *>(p.part_o + (s * g + j) * kHeadDim)[lane];
-        wsum += wt;
-        acc.x += wt * v.x;
-        acc.y += wt * v.y;
-        acc.z += wt * v.z;
-        acc.w += wt * v.w;
+    for (int w0 = wf; w0 <= wl; w0 += 4) {
+        float ls[4];
+        float4 v[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int wk = w0 + i;
+            const bool use = wk <= wl && worker_begin(T, wk, W) != worker_begin(T, wk + 1, W);
+            const int64_t s = pair + wk;
+            ls[i] = use ? p.part_lse[s * g + j] : -INFINITY;
+            v[i] = use ? reinterpret_cast<const float4 *>(p.part_o + (s * g + j) * kHeadDim)[lane]
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            if (ls[i] == -INFINITY) continue;
+            const float mn = fmaxf(mx, ls[i]);
+            const float c = mx == -INFINITY ? 0.f : fast_exp2(mx - mn);
+            const float wt = fast_exp2(ls[i] - mn);
+            wsum = wsum * c + wt;
+            acc.x = acc.x * c + wt * v[i].x;
+            acc.y = acc.y * c + wt * v[i].y;
+            acc.z = acc.z * c + wt * v[i].z;
+            acc.w = acc.w * c + wt * v[i].w;
+            mx = mn;
+        }
     }
     const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
     uint2 packed;
