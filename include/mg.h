@@ -205,6 +205,43 @@ mg_status mg_extend_attn(const void *q, const void *k_cache, const void *v_cache
                          void *stream);
 
 /*
+ * mg_decode_attn_static_workspace -- mg_decode_attn for callers that cannot
+ * pass device scratch memory.  (The pages have no counterpart: this is a
+ * deployment convenience of this library, not a step of the method.)
+ *
+ * Who needs it: callers whose device memory is all owned by another allocator
+ * (a serving engine's pre-sized pool, a framework's caching allocator), so an
+ * extra cudaMalloc would fail or fragment it; plug-ins that are given only
+ * their inputs and outputs; step loops that must not pay an allocation, which
+ * can synchronise the device, in the middle of a step.
+ *
+ * Same arguments and result as mg_decode_attn, without workspace and
+ * workspace_bytes.  The workspace is a fixed array of
+ * MG_DECODE_STATIC_WORKSPACE_BYTES in device global memory inside this library;
+ * every device that loads the library holds it until the process exits.
+ *   - Limit: a plan needing more than MG_DECODE_STATIC_WORKSPACE_BYTES (see
+ *     mg_decode_workspace_bytes) returns MG_ERR_WORKSPACE_TOO_SMALL before any
+ *     launch; use mg_decode_attn with your own workspace instead.
+ *   - Nothing is allocated: no cudaMalloc, cudaFree or allocating library call.
+ *   - The first call on each device looks up the array's device address (with
+ *     that device current) and caches it; make that first call before any
+ *     stream capture.
+ *   - All calls share the one array, which keeps the last call's contents.
+ *     Nothing in it needs to start at zero (every value is written before it is
+ *     read within a call), but calls that overlap on the GPU (e.g. on two
+ *     streams, or from two host threads) race on it and corrupt each other:
+ *     serialise them.
+ */
+#define MG_DECODE_STATIC_WORKSPACE_BYTES (16u << 20)
+mg_status mg_decode_attn_static_workspace(const void *q, const void *k_cache, const void *v_cache,
+                                          int64_t num_slots, const int32_t *page_table,
+                                          int32_t page_table_rows, int32_t page_table_stride,
+                                          const int32_t *table_idx, const int32_t *seq_len, int32_t batch,
+                                          int32_t max_seq_len, int32_t num_q_heads, int32_t num_kv_heads,
+                                          int32_t head_dim, float scale, int32_t num_partitions, void *out,
+                                          void *stream);
+
+/*
  * mg_read_device_error -- synchronise `stream`, return the device error word
  * accumulated since the last call on this device (bits MG_DEVERR_*) in
  * *bits_out (may be NULL), and clear it.  Returns MG_OK when no bit was set,

@@ -338,3 +338,62 @@ mg_status mg_read_device_error(void *stream, uint32_t *bits_out) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- decode without a caller workspace
+//
+// Some callers cannot hand the library device scratch memory: code whose
+// device memory is entirely owned by another allocator (a serving engine's
+// pre-sized pool, a framework's caching allocator) where an extra cudaMalloc
+// would fail or fragment it, plug-ins that receive only their inputs and
+// outputs, and step loops that must not pay an allocation (which can
+// synchronise the device) in the middle of a step.  For them decode can use a
+// workspace that lives in this library: a fixed-size array in device global
+// memory that every device which loads the library holds until the process
+// exits.
+namespace mg {
+namespace {
+
+constexpr size_t kStaticDecodeWorkspaceBytes = MG_DECODE_STATIC_WORKSPACE_BYTES;
+static __device__ __align__(256) unsigned char g_decode_static_workspace[kStaticDecodeWorkspaceBytes];
+
+void *g_static_ws_ptr[kMaxDevices];
+std::mutex g_static_ws_mutex;
+
+// The array's device address on the current device.  In host code the
+// array's name is only a host-side stand-in, so the address is looked up once
+// per device, with that device current, and cached.
+mg_status static_workspace(void *&ptr) {
+    int dev;
+    if (current_device(dev) != MG_OK) return MG_ERR_CUDA;
+    if (!g_static_ws_ptr[dev]) {
+        std::lock_guard<std::mutex> lock(g_static_ws_mutex);
+        if (!g_static_ws_ptr[dev]) {
+            void *p = nullptr;
+            if (cudaGetSymbolAddress(&p, g_decode_static_workspace) != cudaSuccess || p == nullptr)
+                return MG_ERR_CUDA;
+            g_static_ws_ptr[dev] = p;
+        }
+    }
+    ptr = g_static_ws_ptr[dev];
+    return MG_OK;
+}
+
+}  // namespace
+}  // namespace mg
+
+extern "C" mg_status mg_decode_attn_static_workspace(
+    const void *q, const void *k_cache, const void *v_cache, int64_t num_slots, const int32_t *page_table,
+    int32_t page_table_rows, int32_t page_table_stride, const int32_t *table_idx, const int32_t *seq_len,
+    int32_t batch, int32_t max_seq_len, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+    float scale, int32_t num_partitions, void *out, void *stream) {
+    // the plan's workspace must fit the fixed array: refuse larger batches up front
+    const size_t need = mg_decode_workspace_bytes(batch, num_q_heads, num_kv_heads, head_dim, max_seq_len,
+                                                  num_partitions);
+    if (need > kStaticDecodeWorkspaceBytes) return MG_ERR_WORKSPACE_TOO_SMALL;
+    void *ws = nullptr;
+    const mg_status st = static_workspace(ws);
+    if (st != MG_OK) return st;
+    return mg_decode_attn(q, k_cache, v_cache, num_slots, page_table, page_table_rows, page_table_stride,
+                          table_idx, seq_len, batch, max_seq_len, num_q_heads, num_kv_heads, head_dim, scale,
+                          num_partitions, out, ws, kStaticDecodeWorkspaceBytes, stream);
+}

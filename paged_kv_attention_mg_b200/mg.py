@@ -46,6 +46,8 @@ SIGNATURES = {
                                             _I32, _I32, _I32, _F32, _I32, _P, _P, _SZ, _P]),
     "mg_extend_attn": (ctypes.c_int, [_P, _P, _P, _I64, _P, _I32, _I32, _P, _P, _P, _P, _I32, _I32, _I32,
                                       _I32, _I32, _I32, _I32, _F32, _P, _P]),
+    "mg_decode_attn_static_workspace": (ctypes.c_int, [_P, _P, _P, _I64, _P, _I32, _I32, _P, _P, _I32, _I32,
+                                                       _I32, _I32, _I32, _F32, _I32, _P, _P]),
     "mg_read_device_error": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_uint32)]),
 }
 
@@ -202,6 +204,31 @@ def extend_attn(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, p
                                  _dev(seq_len, torch.int32, "seq_len"), _dev(q_offset, torch.int32, "q_offset"),
                                  b, total_q, max_q_len, max_seq_len, hq, hkv, d, float(scale),
                                  _dev(out, torch.bfloat16, "out"), _stream(stream)), "mg_extend_attn")
+    return out
+
+
+STATIC_WORKSPACE_BYTES = 16 << 20  # MG_DECODE_STATIC_WORKSPACE_BYTES in include/mg.h
+
+
+def decode_attn_static_workspace(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                                 page_table: torch.Tensor, table_idx: torch.Tensor, seq_len: torch.Tensor,
+                                 max_seq_len: int, scale: float, num_partitions: int = 0,
+                                 out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """decode_attn for callers that cannot pass device scratch memory: the
+    library's own fixed workspace is used (shared by all calls; overlapping
+    calls race).  Raises MgError(MG_ERR_WORKSPACE_TOO_SMALL) when the plan
+    needs more than STATIC_WORKSPACE_BYTES.  Allocates nothing on the device
+    except `out` when it is not given."""
+    b, hq, d = q.shape
+    hkv = k_cache.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    _check(load().mg_decode_attn_static_workspace(
+        _dev(q, torch.bfloat16, "q"), _dev(k_cache, torch.bfloat16, "k_cache"),
+        _dev(v_cache, torch.bfloat16, "v_cache"), k_cache.shape[0], _dev(page_table, torch.int32, "page_table"),
+        page_table.shape[0], page_table.shape[1], _dev(table_idx, torch.int32, "table_idx"),
+        _dev(seq_len, torch.int32, "seq_len"), b, max_seq_len, hq, hkv, d, float(scale), num_partitions,
+        _dev(out, torch.bfloat16, "out"), _stream(stream)), "mg_decode_attn_static_workspace")
     return out
 
 
