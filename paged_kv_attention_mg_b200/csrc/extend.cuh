@@ -195,11 +195,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         *abort_flag = 0;
         mbar_init(sy.q_full, 1);
         for (int s = 0; s < kKStages; ++s) {
-            mbar_init(sy.k_full[s], 1);
+            mbar_init(sy.k_full[s], 32);  // one arrival per producer lane
             mbar_init(sy.k_empty[s], 1);
         }
         for (int s = 0; s < kVStages; ++s) {
-            mbar_init(sy.v_full[s], 1);
+            mbar_init(sy.v_full[s], 32);
             mbar_init(sy.v_empty[s], 1);
         }
         for (int t = 0; t < kQTiles; ++t) {
@@ -232,10 +232,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 kvh * g, qo + tok0 + t * tpq);
         }
         const int32_t *pt = p.page_table + (int64_t)row * p.pt_stride;
-        const int oob_row = (int)(p.num_slots * p.num_kv_heads);  // reads as zeros
+        const int64_t head_stride = (int64_t)p.num_kv_heads * kHeadDim;
         int *idx_ring = reinterpret_cast<int *>(smem + kOffIdx);
-        // page-table entries of tile j: lane l copies keys 4l .. 4l+3 (one cp.async group per tile)
-        auto fetch_idx = [&](int j) {
+        // One cp.async group per iteration j: the page-table entries of tile
+        // j + kIdxAhead, K of tile j, V of tile j - 1 (K leads V by one tile).
+        // A group's tiles are published one iteration later: wait for it,
+        // fence the generic-proxy writes for the tensor cores' async proxy,
+        // arrive on the full barriers (one arrival per lane).
+        auto fetch_idx = [&](int j) {  // lane l copies keys 4l .. 4l+3
             if (j < n_kv) {
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
@@ -245,51 +249,69 @@ __global__ void __launch_bounds__(kThreads, 1)
                     else *dst = -1;
                 }
             }
-            cp_async_commit();
         };
-        auto rows_of = [&](int j, int (&rows)[4]) {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int key = j * kN + lane * 4 + e;
-                int slot = key < kv_len ? idx_ring[(j % kIdxRing) * kN + lane * 4 + e] : -1;
-                if (key < kv_len && (slot < 0 || (int64_t)slot >= p.num_slots)) {
-                    atomicOr(&g_mg_device_error, MG_DEVERR_SLOT_RANGE);
-                    slot = -1;
-                }
-                rows[e] = slot < 0 ? oob_row : slot * p.num_kv_heads + kvh;
+        // 128 rows x 256 B of K or V into a tile stored as two 64-column halves with
+        // the 128-byte swizzle; each warp instruction moves two whole rows.
+        auto copy_tile = [&](int j, const __nv_bfloat16 *pool, uint32_t tile_base) {
+            const int *ids = idx_ring + (j % kIdxRing) * kN;
+            const int c = lane & 15, half = c >> 3, cc = c & 7;
+#pragma unroll 8
+            for (int i = 0; i < kN / 2; ++i) {
+                const int key = i * 2 + (lane >> 4);
+                int slot = j * kN + key < kv_len ? ids[key] : -1;
+                if (slot >= 0 && (int64_t)slot >= p.num_slots) slot = -1;  // flagged by check_tile
+                const __nv_bfloat16 *src = pool + (int64_t)(slot < 0 ? 0 : slot) * head_stride +
+                                           (int64_t)kvh * kHeadDim + c * 8;
+                const uint32_t dst = tile_base + half * kHalfBytes + key * 128 + ((cc ^ (key & 7)) << 4);
+                cp_async_16(dst, src, slot < 0 ? 0u : 16u);
             }
         };
-        auto gather = [&](const CUtensorMap *tm, uint32_t tile_base, uint32_t bar, const int (&rows)[4]) {
-            if (lane == 0) mbar_arrive_expect_tx(bar, kTileBytes);
-            __syncwarp();
-            const uint32_t dst = tile_base + lane * 4 * 128;
-            tma_gather4(dst, tm, bar, 0, rows[0], rows[1], rows[2], rows[3]);
-            tma_gather4(dst + kHalfBytes, tm, bar, 64, rows[0], rows[1], rows[2], rows[3]);
+        auto check_tile = [&](int j) {  // record rejected page-table entries (they were zero-filled)
+            const int *ids = idx_ring + (j % kIdxRing) * kN;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int key = lane * 4 + e;
+                const int slot = j * kN + key < kv_len ? ids[key] : 0;
+                if (slot < 0 || (int64_t)slot >= p.num_slots) atomicOr(&g_mg_device_error, MG_DEVERR_SLOT_RANGE);
+            }
+        };
+        auto publish = [&](int j) {  // tiles of iteration j's group have landed
+            fence_proxy_async_smem();
+            if (j < n_kv) mbar_arrive(sy.k_full[j % kKStages]);
+            if (j >= 1) mbar_arrive(sy.v_full[(j - 1) % kVStages]);
         };
 #pragma unroll
-        for (int j = 0; j < kIdxAhead; ++j) fetch_idx(j);
-        // iteration j: entries of tile j + kIdxAhead requested; K of tile j
-        // issued; V of tile j - 1 issued (K leads V by one tile)
-        int prev_rows[4] = {oob_row, oob_row, oob_row, oob_row};
+        for (int j = 0; j < kIdxAhead; ++j) {
+            fetch_idx(j);
+            cp_async_commit();
+        }
+        bool ok = true;
         for (int j = 0; j <= n_kv; ++j) {
-            fetch_idx(j + kIdxAhead);
-            int rows[4] = {oob_row, oob_row, oob_row, oob_row};
+            // entries of tile j (fetched kIdxAhead groups ago) are needed by K_j
             if (j < n_kv) {
                 const int s = j % kKStages;
-                if (j >= kKStages && !wait_or_abort(sy.k_empty[s], ((j / kKStages) - 1) & 1, abort_flag)) break;
-                cp_async_wait<kIdxAhead>();
-                rows_of(j, rows);
-                gather(&tm_k, sbase + kOffK + s * kTileBytes, sy.k_full[s], rows);
+                if (j >= kKStages && !(ok = wait_or_abort(sy.k_empty[s], ((j / kKStages) - 1) & 1, abort_flag))) break;
             }
             if (j >= 1) {
                 const int jv = j - 1, s = jv % kVStages;
-                if (jv >= kVStages && !wait_or_abort(sy.v_empty[s], ((jv / kVStages) - 1) & 1, abort_flag)) break;
-                gather(&tm_v, sbase + kOffV + s * kTileBytes, sy.v_full[s], prev_rows);
+                if (jv >= kVStages && !(ok = wait_or_abort(sy.v_empty[s], ((jv / kVStages) - 1) & 1, abort_flag))) break;
             }
-#pragma unroll
-            for (int e = 0; e < 4; ++e) prev_rows[e] = rows[e];
+            cp_async_wait<kIdxAhead - 1>();
+            __syncwarp();
+            fetch_idx(j + kIdxAhead);
+            if (j < n_kv) {
+                check_tile(j);
+                copy_tile(j, p.k_cache, sbase + kOffK + (j % kKStages) * kTileBytes);
+            }
+            if (j >= 1) copy_tile(j - 1, p.v_cache, sbase + kOffV + ((j - 1) % kVStages) * kTileBytes);
+            cp_async_commit();
+            if (j >= 1) {  // publish iteration j-1's group
+                cp_async_wait<1>();
+                publish(j - 1);
+            }
         }
         cp_async_wait<0>();
+        if (ok) publish(n_kv);
     } else if (warp == 1) {
         // =============================================================== MMA issue
         if (lane == 0) {
