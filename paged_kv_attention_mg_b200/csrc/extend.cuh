@@ -6,7 +6,8 @@
 // stored; new token i (query row q_offset[r] + i, position c + i) attends to the
 // keys at positions 0 .. c + i of its page-table row.
 //
-// Work decomposition (B200 design):
+// Work decomposition (B200 design; warps 0 and 10 load, warp 1 issues MMAs,
+// warps 2-9 run the softmax):
 //   * one CTA per (q block, kv head, request).  A q block is two 128-row Q
 //     tiles; a row is (token, head) with the g heads that share the KV head
 //     adjacent, so one K/V tile feeds 2 x 128 query rows (GQA packing).
@@ -40,7 +41,8 @@ constexpr int kKStages = 3;                 // K ring: S of a tile needs K befor
 constexpr int kVStages = 2;                 // V ring
 constexpr int kIdxAhead = 3;                // tiles of page-table entries in flight ahead of the K issue
 constexpr int kIdxRing = 4;                 // >= kIdxAhead + 1
-constexpr int kThreads = 320;               // 10 warps
+constexpr int kThreads = 352;               // 11 warps: 2 load, 1 MMA, 8 softmax
+constexpr int kLoadWarp2 = 10;              // the second load warp (warp 0 is the first)
 constexpr int kHalfBytes = 128 * 128;       // 128 rows x 128 B (64 bf16): one swizzle column
 constexpr int kTileBytes = 2 * kHalfBytes;  // 128 rows x 256 B
 constexpr int kTmemCols = 512;
@@ -195,11 +197,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         *abort_flag = 0;
         mbar_init(sy.q_full, 1);
         for (int s = 0; s < kKStages; ++s) {
-            mbar_init(sy.k_full[s], 32);  // one arrival per producer lane
+            mbar_init(sy.k_full[s], 64);  // one arrival per lane of the two load warps
             mbar_init(sy.k_empty[s], 1);
         }
         for (int s = 0; s < kVStages; ++s) {
-            mbar_init(sy.v_full[s], 32);
+            mbar_init(sy.v_full[s], 64);
             mbar_init(sy.v_empty[s], 1);
         }
         for (int t = 0; t < kQTiles; ++t) {
@@ -218,12 +220,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
 
-    if (warp == 0) {
+    if (warp == 0 || warp == kLoadWarp2) {
         // =============================================================== loads
-        if (lane == 0) {
+        const int pi = warp == 0 ? 0 : 1;  // this load warp's half of every tile's 128 keys
+        if (warp == 0 && lane == 0) {
             prefetch_tmap(&tm_q);
-            prefetch_tmap(&tm_k);
-            prefetch_tmap(&tm_v);
             const uint32_t qbytes = (uint32_t)(kQTiles * 2 * 128 * g * tpq);
             mbar_arrive_expect_tx(sy.q_full, qbytes);
             for (int t = 0; t < kQTiles; ++t)
@@ -234,48 +235,49 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int32_t *pt = p.page_table + (int64_t)row * p.pt_stride;
         const int64_t head_stride = (int64_t)p.num_kv_heads * kHeadDim;
         int *idx_ring = reinterpret_cast<int *>(smem + kOffIdx);
-        // One cp.async group per iteration j: the page-table entries of tile
-        // j + kIdxAhead, K of tile j, V of tile j - 1 (K leads V by one tile).
-        // A group's tiles are published one iteration later: wait for it,
-        // fence the generic-proxy writes for the tensor cores' async proxy,
-        // arrive on the full barriers (one arrival per lane).
-        auto fetch_idx = [&](int j) {  // lane l copies keys 4l .. 4l+3
+        const int k_lo = pi * (kN / 2);  // keys k_lo .. k_lo + 63 of each tile
+        // One cp.async group per iteration j: this warp's page-table entries of
+        // tile j + kIdxAhead, its K rows of tile j, its V rows of tile j - 1
+        // (K leads V by one tile).  A group is published one iteration later:
+        // wait for it, fence the generic-proxy writes for the tensor cores'
+        // async proxy, arrive on the full barriers (one arrival per lane).
+        auto fetch_idx = [&](int j) {  // lane l copies keys k_lo + 2l, k_lo + 2l + 1
             if (j < n_kv) {
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int key = j * kN + lane * 4 + e;
-                    int *dst = idx_ring + (j % kIdxRing) * kN + lane * 4 + e;
+                for (int e = 0; e < 2; ++e) {
+                    const int key = j * kN + k_lo + lane * 2 + e;
+                    int *dst = idx_ring + (j % kIdxRing) * kN + k_lo + lane * 2 + e;
                     if (key < kv_len) cp_async_4(smem_u32(dst), pt + key);
                     else *dst = -1;
                 }
             }
         };
-        // 128 rows x 256 B of K or V into a tile stored as two 64-column halves with
+        // 64 rows x 256 B of K or V into a tile stored as two 64-column halves with
         // the 128-byte swizzle; each warp instruction moves two whole rows.
-        auto copy_tile = [&](int j, const __nv_bfloat16 *pool, uint32_t tile_base) {
+        auto copy_rows = [&](int j, const __nv_bfloat16 *pool, uint32_t tile_base) {
             const int *ids = idx_ring + (j % kIdxRing) * kN;
             const int c = lane & 15, half = c >> 3, cc = c & 7;
 #pragma unroll 8
-            for (int i = 0; i < kN / 2; ++i) {
-                const int key = i * 2 + (lane >> 4);
+            for (int i = 0; i < kN / 4; ++i) {
+                const int key = k_lo + i * 2 + (lane >> 4);
                 int slot = j * kN + key < kv_len ? ids[key] : -1;
-                if (slot >= 0 && (int64_t)slot >= p.num_slots) slot = -1;  // flagged by check_tile
+                if (slot >= 0 && (int64_t)slot >= p.num_slots) slot = -1;  // flagged by check_rows
                 const __nv_bfloat16 *src = pool + (int64_t)(slot < 0 ? 0 : slot) * head_stride +
                                            (int64_t)kvh * kHeadDim + c * 8;
                 const uint32_t dst = tile_base + half * kHalfBytes + key * 128 + ((cc ^ (key & 7)) << 4);
                 cp_async_16(dst, src, slot < 0 ? 0u : 16u);
             }
         };
-        auto check_tile = [&](int j) {  // record rejected page-table entries (they were zero-filled)
+        auto check_rows = [&](int j) {  // record rejected page-table entries (they were zero-filled)
             const int *ids = idx_ring + (j % kIdxRing) * kN;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int key = lane * 4 + e;
+            for (int e = 0; e < 2; ++e) {
+                const int key = k_lo + lane * 2 + e;
                 const int slot = j * kN + key < kv_len ? ids[key] : 0;
                 if (slot < 0 || (int64_t)slot >= p.num_slots) atomicOr(&g_mg_device_error, MG_DEVERR_SLOT_RANGE);
             }
         };
-        auto publish = [&](int j) {  // tiles of iteration j's group have landed
+        auto publish = [&](int j) {  // this warp's rows of iteration j's group have landed
             fence_proxy_async_smem();
             if (j < n_kv) mbar_arrive(sy.k_full[j % kKStages]);
             if (j >= 1) mbar_arrive(sy.v_full[(j - 1) % kVStages]);
@@ -287,7 +289,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         bool ok = true;
         for (int j = 0; j <= n_kv; ++j) {
-            // entries of tile j (fetched kIdxAhead groups ago) are needed by K_j
             if (j < n_kv) {
                 const int s = j % kKStages;
                 if (j >= kKStages && !(ok = wait_or_abort(sy.k_empty[s], ((j / kKStages) - 1) & 1, abort_flag))) break;
@@ -296,14 +297,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int jv = j - 1, s = jv % kVStages;
                 if (jv >= kVStages && !(ok = wait_or_abort(sy.v_empty[s], ((jv / kVStages) - 1) & 1, abort_flag))) break;
             }
-            cp_async_wait<kIdxAhead - 1>();
+            cp_async_wait<kIdxAhead - 1>();  // entries of tile j (kIdxAhead groups old) landed
             __syncwarp();
-            fetch_idx(j + kIdxAhead);
             if (j < n_kv) {
-                check_tile(j);
-                copy_tile(j, p.k_cache, sbase + kOffK + (j % kKStages) * kTileBytes);
+                check_rows(j);
+                copy_rows(j, p.k_cache, sbase + kOffK + (j % kKStages) * kTileBytes);
             }
-            if (j >= 1) copy_tile(j - 1, p.v_cache, sbase + kOffV + ((j - 1) % kVStages) * kTileBytes);
+            if (j >= 1) copy_rows(j - 1, p.v_cache, sbase + kOffV + ((j - 1) % kVStages) * kTileBytes);
+            // only now reuse the ring slot of tile j - 1 (its V rows were just issued)
+            fetch_idx(j + kIdxAhead);
             cp_async_commit();
             if (j >= 1) {  // publish iteration j-1's group
                 cp_async_wait<1>();
