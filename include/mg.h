@@ -134,6 +134,7 @@ size_t mg_decode_workspace_bytes(int32_t batch, int32_t num_q_heads, int32_t num
  *   page_table    [page_table_rows, page_table_stride] int32
  *   table_idx, seq_len  [batch] int32, 1 <= seq_len[r] <= min(max_seq_len, stride)
  *   max_seq_len   host-side upper bound of seq_len
+ *   scale         softmax scale, finite and > 0 (else MG_ERR_INVALID_ARGUMENT)
  *   num_partitions 0 = automatic plan; > 0 forces the number of workers
  *   workspace     device buffer of >= mg_decode_workspace_bytes(...) bytes,
  *                 16-byte aligned.  Contents on entry do not matter; it holds
@@ -192,6 +193,7 @@ mg_status mg_store_decode_attn(const void *q, const void *k_new, const void *v_n
  *   cached_len, seq_len [batch] int32; q_offset [batch + 1] int32 prefix sums of
  *                 n (q_offset[0] = 0, q_offset[batch] = total_q)
  *   max_q_len     host bound of n;  max_seq_len  host bound of seq_len
+ *   scale         softmax scale, finite and > 0 (else MG_ERR_INVALID_ARGUMENT)
  * Requests with n == 0 are allowed and produce no rows.  Same shape limits as
  * decode; needs no workspace.
  */

@@ -6,20 +6,24 @@
 // stored; new token i (query row q_offset[r] + i, position c + i) attends to the
 // keys at positions 0 .. c + i of its page-table row.
 //
-// Work decomposition (B200 design; warps 0 and 10 load, warp 1 issues MMAs,
-// warps 2-9 run the softmax):
+// Work decomposition (B200 design; 16 warps in four warpgroups with their
+// register budgets moved by setmaxnreg: warpgroups 0 and 3 load and issue
+// MMAs on 72 registers a thread, warpgroups 1 and 2 run the softmax on 184):
 //   * one CTA per (q block, kv head, request).  A q block is two 128-row Q
 //     tiles; a row is (token, head) with the g heads that share the KV head
 //     adjacent, so one K/V tile feeds 2 x 128 query rows (GQA packing).
-//   * warp 0 loads: Q tiles with 3-D TMA, K and V tiles (128 keys each) with
-//     TMA tile::gather4 straight from the paged pool (4 page-table rows per
-//     instruction, 128-byte swizzle), double-buffered behind mbarriers.
-//   * warp 1, one thread: issues tcgen05.mma (M=128, N=128, K=16, bf16 in,
+//   * seven load warps (0-3, 13-15): the Q tiles with 3-D TMA, the K and V
+//     tiles (128 keys each) with 16-byte cp.async straight from the paged pool
+//     into the 128-byte swizzled layout, behind mbarriers.  A warp keeps about
+//     one 512-byte cp.async in flight per 70 cycles whatever the SM does, so
+//     the copy rate grows with the number of issuing warps; every load warp
+//     owns every seventh pair of rows of each tile.
+//   * warp 12, one thread: issues tcgen05.mma (M=128, N=128, K=16, bf16 in,
 //     fp32 accumulate in TMEM).  S_t = Q_t K^T lands in TMEM; P_t (bf16) is
 //     written back over S_t and consumed straight from TMEM as the A operand
 //     of O_t += P_t V.  The two Q tiles ping-pong so the tensor core works on
 //     one tile while the softmax warps work on the other.
-//   * warps 2-5 / 6-9: softmax for Q tile 0 / 1, one TMEM lane (= one query
+//   * warpgroups 1 / 2: softmax for Q tile 0 / 1, one TMEM lane (= one query
 //     row) per thread: causal mask key <= c + i, online softmax in the exp2
 //     domain, O rescaled in TMEM only when the running max grows by more than
 //     2^8 (exact: the same stale max is used for P and for the row sum),
@@ -41,8 +45,16 @@ constexpr int kKStages = 3;                 // K ring: S of a tile needs K befor
 constexpr int kVStages = 2;                 // V ring
 constexpr int kIdxAhead = 3;                // tiles of page-table entries in flight ahead of the K issue
 constexpr int kIdxRing = 4;                 // >= kIdxAhead + 1
-constexpr int kThreads = 352;               // 11 warps: 2 load, 1 MMA, 8 softmax
-constexpr int kLoadWarp2 = 10;              // the second load warp (warp 0 is the first)
+constexpr int kThreads = 512;               // 16 warps: 7 load, 1 MMA, 8 softmax
+constexpr int kLoaders = 7;                 // load warps 0-3 and 13-15
+constexpr int kMmaWarp = 12;
+constexpr int kPairs = kN / 2;              // row pairs per tile (one warp instruction moves a pair)
+constexpr int kMaxPairsPerLoader = (kPairs + kLoaders - 1) / kLoaders;
+constexpr int kRegsLoad = 72;               // registers a thread in warpgroups 0 and 3
+constexpr int kRegsSoftmax = 184;           // registers a thread in warpgroups 1 and 2
+static_assert(2 * 128 * kRegsLoad + 2 * 128 * kRegsSoftmax == 65536 && 65536 / kThreads == 128,
+              "the register split must add up to what the block is launched with");
+static_assert(2 * kMaxPairsPerLoader <= 32, "a load warp fetches one page-table entry per lane");
 constexpr int kHalfBytes = 128 * 128;       // 128 rows x 128 B (64 bf16): one swizzle column
 constexpr int kTileBytes = 2 * kHalfBytes;  // 128 rows x 256 B
 constexpr int kTmemCols = 512;
@@ -197,11 +209,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         *abort_flag = 0;
         mbar_init(sy.q_full, 1);
         for (int s = 0; s < kKStages; ++s) {
-            mbar_init(sy.k_full[s], 64);  // one arrival per lane of the two load warps
+            mbar_init(sy.k_full[s], kLoaders * 32);  // one arrival per lane of the load warps
             mbar_init(sy.k_empty[s], 1);
         }
         for (int s = 0; s < kVStages; ++s) {
-            mbar_init(sy.v_full[s], 64);
+            mbar_init(sy.v_full[s], kLoaders * 32);
             mbar_init(sy.v_empty[s], 1);
         }
         for (int t = 0; t < kQTiles; ++t) {
@@ -211,7 +223,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         fence_mbarrier_init();
     }
-    if (warp == 1) {  // TMEM allocation is warp-wide
+    if (warp == kMmaWarp) {  // TMEM allocation is warp-wide
         tmem_alloc(smem_u32(tmem_holder), kTmemCols);
         tmem_relinquish();
     }
@@ -220,160 +232,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
 
-    if (warp == 0 || warp == kLoadWarp2) {
-        // =============================================================== loads
-        const int pi = warp == 0 ? 0 : 1;  // this load warp's half of every tile's 128 keys
-        if (warp == 0 && lane == 0) {
-            prefetch_tmap(&tm_q);
-            const uint32_t qbytes = (uint32_t)(kQTiles * 2 * 128 * g * tpq);
-            mbar_arrive_expect_tx(sy.q_full, qbytes);
-            for (int t = 0; t < kQTiles; ++t)
-                for (int h = 0; h < 2; ++h)
-                    tma_load_3d(sbase + kOffQ + t * kTileBytes + h * kHalfBytes, &tm_q, sy.q_full, h * 64,
-                                kvh * g, qo + tok0 + t * tpq);
-        }
-        const int32_t *pt = p.page_table + (int64_t)row * p.pt_stride;
-        const int64_t head_stride = (int64_t)p.num_kv_heads * kHeadDim;
-        int *idx_ring = reinterpret_cast<int *>(smem + kOffIdx);
-        const int k_lo = pi * (kN / 2);  // keys k_lo .. k_lo + 63 of each tile
-        // One cp.async group per iteration j: this warp's page-table entries of
-        // tile j + kIdxAhead, its K rows of tile j, its V rows of tile j - 1
-        // (K leads V by one tile).  A group is published one iteration later:
-        // wait for it, fence the generic-proxy writes for the tensor cores'
-        // async proxy, arrive on the full barriers (one arrival per lane).
-        auto fetch_idx = [&](int j) {  // lane l copies keys k_lo + 2l, k_lo + 2l + 1
-            if (j < n_kv) {
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int key = j * kN + k_lo + lane * 2 + e;
-                    int *dst = idx_ring + (j % kIdxRing) * kN + k_lo + lane * 2 + e;
-                    if (key < kv_len) cp_async_4(smem_u32(dst), pt + key);
-                    else *dst = -1;
-                }
-            }
-        };
-        // 64 rows x 256 B of K or V into a tile stored as two 64-column halves with
-        // the 128-byte swizzle; each warp instruction moves two whole rows.
-        auto copy_rows = [&](int j, const __nv_bfloat16 *pool, uint32_t tile_base) {
-            const int *ids = idx_ring + (j % kIdxRing) * kN;
-            const int c = lane & 15, half = c >> 3, cc = c & 7;
-#pragma unroll 8
-            for (int i = 0; i < kN / 4; ++i) {
-                const int key = k_lo + i * 2 + (lane >> 4);
-                int slot = j * kN + key < kv_len ? ids[key] : -1;
-                if (slot >= 0 && (int64_t)slot >= p.num_slots) slot = -1;  // flagged by check_rows
-                const __nv_bfloat16 *src = pool + (int64_t)(slot < 0 ? 0 : slot) * head_stride +
-                                           (int64_t)kvh * kHeadDim + c * 8;
-                const uint32_t dst = tile_base + half * kHalfBytes + key * 128 + ((cc ^ (key & 7)) << 4);
-                cp_async_16(dst, src, slot < 0 ? 0u : 16u);
-            }
-        };
-        auto check_rows = [&](int j) {  // record rejected page-table entries (they were zero-filled)
-            const int *ids = idx_ring + (j % kIdxRing) * kN;
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int key = k_lo + lane * 2 + e;
-                const int slot = j * kN + key < kv_len ? ids[key] : 0;
-                if (slot < 0 || (int64_t)slot >= p.num_slots) atomicOr(&g_mg_device_error, MG_DEVERR_SLOT_RANGE);
-            }
-        };
-        auto publish = [&](int j) {  // this warp's rows of iteration j's group have landed
-            fence_proxy_async_smem();
-            if (j < n_kv) mbar_arrive(sy.k_full[j % kKStages]);
-            if (j >= 1) mbar_arrive(sy.v_full[(j - 1) % kVStages]);
-        };
-#pragma unroll
-        for (int j = 0; j < kIdxAhead; ++j) {
-            fetch_idx(j);
-            cp_async_commit();
-        }
-        bool ok = true;
-        for (int j = 0; j <= n_kv; ++j) {
-            if (j < n_kv) {
-                const int s = j % kKStages;
-                if (j >= kKStages && !(ok = wait_or_abort(sy.k_empty[s], ((j / kKStages) - 1) & 1, abort_flag))) break;
-            }
-            if (j >= 1) {
-                const int jv = j - 1, s = jv % kVStages;
-                if (jv >= kVStages && !(ok = wait_or_abort(sy.v_empty[s], ((jv / kVStages) - 1) & 1, abort_flag))) break;
-            }
-            cp_async_wait<kIdxAhead - 1>();  // entries of tile j (kIdxAhead groups old) landed
-            __syncwarp();
-            if (j < n_kv) {
-                check_rows(j);
-                copy_rows(j, p.k_cache, sbase + kOffK + (j % kKStages) * kTileBytes);
-            }
-            if (j >= 1) copy_rows(j - 1, p.v_cache, sbase + kOffV + ((j - 1) % kVStages) * kTileBytes);
-            // only now reuse the ring slot of tile j - 1 (its V rows were just issued)
-            fetch_idx(j + kIdxAhead);
-            cp_async_commit();
-            if (j >= 1) {  // publish iteration j-1's group
-                cp_async_wait<1>();
-                publish(j - 1);
-            }
-        }
-        cp_async_wait<0>();
-        if (ok) publish(n_kv);
-    } else if (warp == 1) {
-        // =============================================================== MMA issue
-        if (lane == 0) {
-            constexpr uint32_t idesc_qk = idesc_bf16(false);
-            constexpr uint32_t idesc_pv = idesc_bf16(true);
-            auto issue_s = [&](int t, int j) {
-                const uint32_t qa = sbase + kOffQ + t * kTileBytes;
-                const uint32_t ka = sbase + kOffK + (j % kKStages) * kTileBytes;
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-                    umma_ss(tmem + col_s(t), sw128_desc(qa + off, 16, 1024), sw128_desc(ka + off, 16, 1024),
-                            idesc_qk, kk > 0);
-                }
-                umma_commit(sy.s_full[t]);
-            };
-            auto issue_pv = [&](int t, int j) {
-                const uint32_t va = sbase + kOffV + (j % kVStages) * kTileBytes;
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    umma_ts(tmem + col_o(t), tmem + col_s(t) + kk * 8,
-                            sw128_desc(va + kk * 2048, kHalfBytes, 1024), idesc_pv, (j > 0 || kk > 0));
-                umma_commit(sy.o_done[t]);
-            };
-            bool ok = wait_or_abort_thread(sy.q_full, 0, abort_flag) && wait_or_abort_thread(sy.k_full[0], 0, abort_flag);
-            if (ok) {
-                tc_fence_after();
-                issue_s(0, 0);
-                if (has_q1) issue_s(1, 0);
-                umma_commit(sy.k_empty[0]);
-            }
-            for (int j = 0; ok && j < n_kv; ++j) {
-                const int sv = j % kVStages;
-                if (!(ok = wait_or_abort_thread(sy.v_full[sv], (j / kVStages) & 1, abort_flag))) break;
-                if (!(ok = wait_or_abort_thread(sy.p_full[0], j & 1, abort_flag))) break;
-                tc_fence_after();
-                issue_pv(0, j);
-                const bool more = j + 1 < n_kv;
-                if (more) {
-                    const int sk = (j + 1) % kKStages;
-                    if (!(ok = wait_or_abort_thread(sy.k_full[sk], ((j + 1) / kKStages) & 1, abort_flag))) break;
-                    tc_fence_after();
-                    issue_s(0, j + 1);
-                }
-                if (has_q1) {
-                    if (!(ok = wait_or_abort_thread(sy.p_full[1], j & 1, abort_flag))) break;
-                    tc_fence_after();
-                    issue_pv(1, j);
-                }
-                umma_commit(sy.v_empty[sv]);
-                if (more) {
-                    if (has_q1) issue_s(1, j + 1);
-                    umma_commit(sy.k_empty[(j + 1) % kKStages]);
-                }
-            }
-        }
-        __syncwarp();
-    } else {
+    // setmaxnreg is issued once per warpgroup role, at the top of its branch
+    if (warp >= 4 && warp < 12) {
+        setmaxnreg_inc<kRegsSoftmax>();
         // =============================================================== softmax
-        const int t = (warp - 2) >> 2;  // Q tile
+        const int t = (warp - 4) >> 2;  // Q tile
         const int wq = warp & 3;        // TMEM lane quarter this warp may access
         const int qrow = wq * 32 + lane;
         const int tok_local = qrow / g, head_local = qrow - tok_local * g;
@@ -397,15 +260,29 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_ld_wait();
             const int key0 = j * kN;
             const int nvis = min(max(lim - key0 + 1, 0), kN);  // visible keys in this tile
-            float mx = -INFINITY;
+            // Row max of the raw scores (scale > 0, so scaling commutes with the
+            // max); a tile every key of which is visible to the whole warp skips
+            // the mask.
+            const bool full = __all_sync(0xffffffffu, nvis == kN);
+            float mx;
+            if (full) {
+                float m0 = -INFINITY, m1 = -INFINITY;
 #pragma unroll
-            for (int e = 0; e < 128; ++e) {
-                float x = __uint_as_float(sv[e]) * p.scale_log2;
-                x = e < nvis ? x : -INFINITY;
-                sv[e] = __float_as_uint(x);
-                mx = fmaxf(mx, x);
+                for (int e = 0; e < 128; e += 4) {
+                    m0 = fmax3(m0, __uint_as_float(sv[e]), __uint_as_float(sv[e + 1]));
+                    m1 = fmax3(m1, __uint_as_float(sv[e + 2]), __uint_as_float(sv[e + 3]));
+                }
+                mx = fmaxf(m0, m1);
+            } else {
+                mx = -INFINITY;
+#pragma unroll
+                for (int e = 0; e < 128; ++e) {
+                    const float x = e < nvis ? __uint_as_float(sv[e]) : -INFINITY;
+                    sv[e] = __float_as_uint(x);
+                    mx = fmaxf(mx, x);
+                }
             }
-            const float m_new = fmaxf(m_run, mx);
+            const float m_new = fmaxf(m_run, mx * p.scale_log2);
             const bool need = m_new > m_run + kRescaleThreshold;  // also true for the first tile
             const bool warp_need = __any_sync(0xffffffffu, need);
             float corr = 1.f;
@@ -415,21 +292,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                 m_run = m_tgt;
                 l_run *= corr;
             }
+            // P = 2^(s * scale_log2 - m), one fused multiply-add per pair of keys
             const float mu = m_run == -INFINITY ? 0.f : m_run;
-            float rs = 0.f;
+            const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+            const float2 nmu2 = make_float2(-mu, -mu);
+            float2 rs2 = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int cb = 0; cb < 4; ++cb) {
+            for (int cb = 0; cb < 4; ++cb) {  // masked keys hold -inf and give exactly 0
                 uint32_t pk[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
-                    const float p0 = fast_exp2(__uint_as_float(sv[cb * 32 + 2 * e]) - mu);
-                    const float p1 = fast_exp2(__uint_as_float(sv[cb * 32 + 2 * e + 1]) - mu);
-                    rs += p0 + p1;
-                    pk[e] = pack_bf16x2(p0, p1);
+                    const float2 x = ffma2(make_float2(__uint_as_float(sv[cb * 32 + 2 * e]),
+                                                       __uint_as_float(sv[cb * 32 + 2 * e + 1])),
+                                           sc2, nmu2);
+                    const float2 pp = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+                    rs2 = fadd2(rs2, pp);
+                    pk[e] = pack_bf16x2(pp.x, pp.y);
                 }
                 tmem_st_32x32b_x16(tS + cb * 16, pk);
             }
-            l_run += rs;
+            l_run += rs2.x + rs2.y;
             if (warp_need && j > 0) {
                 // O holds the sum up to tile j-1; rescale it once that PV is done
                 if (!(ok = wait_or_abort(sy.o_done[t], (j - 1) & 1, abort_flag))) break;
@@ -477,12 +359,166 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         }
+    } else {
+        setmaxnreg_dec<kRegsLoad>();
+        if (warp == kMmaWarp) {
+            // =============================================================== MMA issue
+            if (lane == 0) {
+                constexpr uint32_t idesc_qk = idesc_bf16(false);
+                constexpr uint32_t idesc_pv = idesc_bf16(true);
+                auto issue_s = [&](int t, int j) {
+                    const uint32_t qa = sbase + kOffQ + t * kTileBytes;
+                    const uint32_t ka = sbase + kOffK + (j % kKStages) * kTileBytes;
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+                        umma_ss(tmem + col_s(t), sw128_desc(qa + off, 16, 1024), sw128_desc(ka + off, 16, 1024),
+                                idesc_qk, kk > 0);
+                    }
+                    umma_commit(sy.s_full[t]);
+                };
+                auto issue_pv = [&](int t, int j) {
+                    const uint32_t va = sbase + kOffV + (j % kVStages) * kTileBytes;
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        umma_ts(tmem + col_o(t), tmem + col_s(t) + kk * 8,
+                                sw128_desc(va + kk * 2048, kHalfBytes, 1024), idesc_pv, (j > 0 || kk > 0));
+                    umma_commit(sy.o_done[t]);
+                };
+                bool ok = wait_or_abort_thread(sy.q_full, 0, abort_flag) && wait_or_abort_thread(sy.k_full[0], 0, abort_flag);
+                if (ok) {
+                    fence_proxy_async_smem();
+                    tc_fence_after();
+                    issue_s(0, 0);
+                    if (has_q1) issue_s(1, 0);
+                    umma_commit(sy.k_empty[0]);
+                }
+                for (int j = 0; ok && j < n_kv; ++j) {
+                    const int sv = j % kVStages;
+                    if (!(ok = wait_or_abort_thread(sy.v_full[sv], (j / kVStages) & 1, abort_flag))) break;
+                    fence_proxy_async_smem();  // cp.async (generic proxy) writes -> tensor core reads
+                    if (!(ok = wait_or_abort_thread(sy.p_full[0], j & 1, abort_flag))) break;
+                    tc_fence_after();
+                    issue_pv(0, j);
+                    const bool more = j + 1 < n_kv;
+                    if (more) {
+                        const int sk = (j + 1) % kKStages;
+                        if (!(ok = wait_or_abort_thread(sy.k_full[sk], ((j + 1) / kKStages) & 1, abort_flag))) break;
+                        fence_proxy_async_smem();
+                        tc_fence_after();
+                        issue_s(0, j + 1);
+                    }
+                    if (has_q1) {
+                        if (!(ok = wait_or_abort_thread(sy.p_full[1], j & 1, abort_flag))) break;
+                        tc_fence_after();
+                        issue_pv(1, j);
+                    }
+                    umma_commit(sy.v_empty[sv]);
+                    if (more) {
+                        if (has_q1) issue_s(1, j + 1);
+                        umma_commit(sy.k_empty[(j + 1) % kKStages]);
+                    }
+                }
+            }
+            __syncwarp();
+        } else {
+            // =============================================================== loads
+            const int li = warp < 4 ? warp : warp - 9;  // load warp index 0 .. kLoaders - 1
+            if (li == 0 && lane == 0) {
+                prefetch_tmap(&tm_q);
+                const uint32_t qbytes = (uint32_t)(kQTiles * 2 * 128 * g * tpq);
+                mbar_arrive_expect_tx(sy.q_full, qbytes);
+                for (int t = 0; t < kQTiles; ++t)
+                    for (int h = 0; h < 2; ++h)
+                        tma_load_3d(sbase + kOffQ + t * kTileBytes + h * kHalfBytes, &tm_q, sy.q_full, h * 64,
+                                    kvh * g, qo + tok0 + t * tpq);
+            }
+            const int32_t *pt = p.page_table + (int64_t)row * p.pt_stride;
+            const int64_t head_stride = (int64_t)p.num_kv_heads * kHeadDim;
+            int *idx_ring = reinterpret_cast<int *>(smem + kOffIdx);
+            // this warp's row pairs of every tile: li, li + kLoaders, ... (< kPairs)
+            const int npairs = (kPairs - li + kLoaders - 1) / kLoaders;
+            // lane l < 2 * npairs owns the page-table entry of key 2 (li + kLoaders (l / 2)) + l % 2
+            const bool has_key = lane < 2 * npairs;
+            const int my_key = 2 * (li + kLoaders * (lane >> 1)) + (lane & 1);
+            // Iteration j copies this warp's K rows of tile j and V rows of tile
+            // j - 1 (K leads V by one tile); each lane then arms the tile's full
+            // barrier with cp.async.mbarrier.arrive.noinc, so the barrier
+            // completes when every load lane's copies have landed, without the
+            // load warps waiting for them.  The page-table entries of tile
+            // j + kIdxAhead ride in the iteration's commit group, the only group
+            // the warp waits for.
+            auto fetch_idx = [&](int j) {
+                if (j < n_kv && has_key) {
+                    const int key = j * kN + my_key;
+                    int *dst = idx_ring + (j % kIdxRing) * kN + my_key;
+                    if (key < kv_len) cp_async_4(smem_u32(dst), pt + key);
+                    else *dst = -1;
+                }
+            };
+            // This warp's row pairs of K or V into a tile stored as two 64-column
+            // halves with the 128-byte swizzle; each warp instruction moves one pair.
+            auto copy_rows = [&](int j, const __nv_bfloat16 *pool, uint32_t tile_base) {
+                const int *ids = idx_ring + (j % kIdxRing) * kN;
+                const int c = lane & 15, half = c >> 3, cc = c & 7;
+#pragma unroll
+                for (int m = 0; m < kMaxPairsPerLoader; ++m) {
+                    if (m < npairs) {
+                        const int key = 2 * (li + kLoaders * m) + (lane >> 4);
+                        int slot = j * kN + key < kv_len ? ids[key] : -1;
+                        if (slot >= 0 && (int64_t)slot >= p.num_slots) slot = -1;  // flagged by check_rows
+                        const __nv_bfloat16 *src = pool + (int64_t)(slot < 0 ? 0 : slot) * head_stride +
+                                                   (int64_t)kvh * kHeadDim + c * 8;
+                        const uint32_t dst = tile_base + half * kHalfBytes + key * 128 + ((cc ^ (key & 7)) << 4);
+                        cp_async_16(dst, src, slot < 0 ? 0u : 16u);
+                    }
+                }
+            };
+            auto check_rows = [&](int j) {  // record rejected page-table entries (they were zero-filled)
+                if (has_key && j * kN + my_key < kv_len) {
+                    const int slot = idx_ring[(j % kIdxRing) * kN + my_key];
+                    if (slot < 0 || (int64_t)slot >= p.num_slots) atomicOr(&g_mg_device_error, MG_DEVERR_SLOT_RANGE);
+                }
+            };
+#pragma unroll
+            for (int j = 0; j < kIdxAhead; ++j) {
+                fetch_idx(j);
+                cp_async_commit();
+            }
+            for (int j = 0; j <= n_kv; ++j) {
+                if (j < n_kv) {
+                    const int s = j % kKStages;
+                    if (j >= kKStages && !wait_or_abort(sy.k_empty[s], ((j / kKStages) - 1) & 1, abort_flag)) break;
+                }
+                if (j >= 1) {
+                    const int jv = j - 1, s = jv % kVStages;
+                    if (jv >= kVStages && !wait_or_abort(sy.v_empty[s], ((jv / kVStages) - 1) & 1, abort_flag)) break;
+                }
+                cp_async_wait<kIdxAhead - 1>();  // entries of tile j (kIdxAhead groups old) landed
+                __syncwarp();
+                if (j < n_kv) {
+                    check_rows(j);
+                    copy_rows(j, p.k_cache, sbase + kOffK + (j % kKStages) * kTileBytes);
+                    cp_async_arrive_noinc(sy.k_full[j % kKStages]);
+                }
+                if (j >= 1) {
+                    copy_rows(j - 1, p.v_cache, sbase + kOffV + ((j - 1) % kVStages) * kTileBytes);
+                    cp_async_arrive_noinc(sy.v_full[(j - 1) % kVStages]);
+                }
+                // only now reuse the ring slot of tile j - 1 (every lane has read its
+                // entries for the V rows just issued)
+                __syncwarp();
+                fetch_idx(j + kIdxAhead);
+                cp_async_commit();
+            }
+            cp_async_wait<0>();  // nothing in flight into shared memory at teardown
+        }
     }
 
     // ---- teardown: everyone meets here, even after an abort
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == kMmaWarp) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }

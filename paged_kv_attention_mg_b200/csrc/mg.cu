@@ -104,6 +104,10 @@ mg_status check_attention_shape(int hq, int hkv, int head_dim) {
     return MG_OK;
 }
 
+// A softmax scale is finite and positive; the kernels take row maxima of the
+// unscaled scores and scale them afterwards, which needs scale > 0.
+bool valid_scale(float scale) { return scale > 0.f && scale <= 3.0e38f; }
+
 }  // namespace
 }  // namespace mg
 
@@ -120,6 +124,7 @@ mg_status decode_impl(const void *q, const void *k_new, const void *v_new, const
     const bool fused = k_new != nullptr;
     mg_status st = check_attention_shape(num_q_heads, num_kv_heads, head_dim);
     if (st != MG_OK) return st;
+    if (!valid_scale(scale)) return MG_ERR_INVALID_ARGUMENT;
     if (batch <= 0 || num_slots <= 0 || page_table_rows <= 0 || page_table_stride <= 0 ||
         max_seq_len <= 0 || max_seq_len > page_table_stride)
         return MG_ERR_INVALID_ARGUMENT;
@@ -292,6 +297,7 @@ mg_status mg_extend_attn(const void *q, const void *k_cache, const void *v_cache
                          void *stream) {
     mg_status st = check_attention_shape(num_q_heads, num_kv_heads, head_dim);
     if (st != MG_OK) return st;
+    if (!valid_scale(scale)) return MG_ERR_INVALID_ARGUMENT;
     if (batch <= 0 || total_q < 0 || max_q_len < 0 || num_slots <= 0 || page_table_rows <= 0 ||
         page_table_stride <= 0 || max_seq_len <= 0 || max_seq_len > page_table_stride)
         return MG_ERR_INVALID_ARGUMENT;

@@ -115,3 +115,11 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(mg, "_lib", None)
     with pytest.raises(RuntimeError, match="not built"):
         mg.load(str(tmp_path / "missing.so"))
+
+
+@pytest.mark.parametrize("scale", [0.0, -0.1, float("nan"), float("inf")])
+def test_attention_rejects_a_scale_that_is_not_finite_and_positive(lib, scale):
+    assert lib.mg_decode_attn(4096, 4096, 4096, 100, 4096, 5, 32, 4096, 4096, 4, 32, 16, 8, 128, scale, 0,
+                              4096, None, 0, None) == 1
+    assert lib.mg_extend_attn(4096, 4096, 4096, 100, 4096, 5, 32, 4096, 4096, 4096, 4096, 4, 0, 0, 32,
+                              16, 8, 128, scale, 4096, None) == 1
