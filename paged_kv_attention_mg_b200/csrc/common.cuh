@@ -60,20 +60,4 @@ inline EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// A pool [num_slots, num_kv_heads, 128] bf16 seen as 2-D rows (slot * Hkv + head)
-// x 128 columns, box 64 columns x 1 row, 128-byte swizzle: the map tile::gather4
-// reads four (slot, head) rows through.  Rows past the end read as zeros.
-inline bool make_pool_tmap(CUtensorMap *map, const void *pool, int64_t num_slots, int num_kv_heads) {
-    EncodeTiledFn enc = encode_fn();
-    const cuuint64_t rows = (cuuint64_t)num_slots * (cuuint64_t)num_kv_heads;
-    if (!enc || rows >= (1ull << 31)) return false;  // gather4 row coordinates are int32
-    cuuint64_t dims[2] = {(cuuint64_t)kHeadDim, rows};
-    cuuint64_t strides[1] = {(cuuint64_t)kHeadDim * 2};
-    cuuint32_t box[2] = {64, 1};
-    cuuint32_t es[2] = {1, 1};
-    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(pool), dims, strides, box, es,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 }  // namespace mg

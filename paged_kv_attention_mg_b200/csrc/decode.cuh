@@ -16,25 +16,25 @@
 //     all workers finish together whatever the length mix (no tail of long
 //     splits).  A worker's share covers one or a few "segments" (its part of a
 //     pair).
-//   * three prefetch distances per worker: page-table entries of tile
-//     k + IDX_AHEAD are copied (cp.async) into a per-warp index ring; the K/V
-//     rows of tile k + L2_AHEAD are prefetched into L2 (bulk prefetch, one
-//     256-byte row per lane), which keeps many DRAM requests in flight without
-//     holding shared memory; tile k + STAGES - 1 is copied from L2 into the
-//     warp's STAGES-deep shared-memory ring, in the 128-byte-swizzled layout
-//     ldmatrix reads without bank conflicts.  Loads used TMA tile::gather4
-//     into the ring with an mbarrier per
-//     stage (build switch MG_DECODE_TMA), or with 16-byte cp.async (default).
-//   * the GQA group is the M dimension of warp-level bf16 tensor-core MMAs
-//     (m16n8k16, fp32 accumulate, g <= 16 rows, zero padded), so each K/V row
-//     is read from HBM once for all g heads: S = Q K^T, online softmax in the
-//     exp2 domain with quad shuffles, O += P V, O kept in registers.
+//   * two prefetch distances per worker: the page-table entries of tile
+//     k + IDX_AHEAD are copied (4-byte cp.async) into a per-warp index ring, and
+//     tile k + STAGES - 1 is gathered (16-byte cp.async, two 256-byte rows per
+//     warp instruction) into the warp's STAGES-deep shared-memory ring in the
+//     128-byte-swizzled layout ldmatrix reads without bank conflicts.
+//   * transposed warp-level bf16 tensor-core products (m16n8k16, fp32
+//     accumulate): S^T = K Q^T and O^T += V^T P^T with keys / head dims in M and
+//     the GQA heads in N, so each K/V row is read from HBM once for all g heads
+//     and a g <= 8 group takes 16 MMAs per 16-key tile; online softmax in the
+//     exp2 domain with quad shuffles, O kept in registers.
+//   * fused store (mg_store_decode_attn): the new token (position L-1) is read
+//     from k_new / v_new instead of the pool, and the worker that owns that tile
+//     writes it to its pool slot from shared memory once the tile has landed.
 //   * a segment that is a whole pair writes bf16 output directly; otherwise it
 //     writes (O / l, m + log2 l) partials to slot (pair + worker), a slot that
 //     is unique because along the unit sequence either the pair or the worker
 //     advances at every segment boundary.  The merge kernel combines a pair's
 //     partials: lse = log2 sum_s 2^lse_s,  o = sum_s 2^(lse_s - lse) o_s.
-//   * no CTA-wide barrier after the prologue: the 4 warps of a CTA only share
+//   * no CTA-wide barrier after the prologue: the warps of a CTA only share
 //     the scan that locates their first unit.
 #pragma once
 
@@ -47,7 +47,7 @@ namespace decode {
 
 constexpr int kKeys = 16;          // keys per unit / pipeline tile
 #ifndef MG_DECODE_WARPS
-#define MG_DECODE_WARPS 6  // workers per CTA (build-time tunable)
+#define MG_DECODE_WARPS 7  // workers per CTA (build-time tunable)
 #endif
 constexpr int kWarps = MG_DECODE_WARPS;
 constexpr int kThreads = kWarps * 32;
@@ -57,31 +57,20 @@ constexpr int kTileBytes = 2 * kKeys * kRowBytes;  // K + V rows of one tile: 8 
 constexpr int kMaxBatch = 131072;                  // requests per call
 
 #ifndef MG_DECODE_STAGES
-#define MG_DECODE_STAGES 4  // per-worker ring depth (build-time tunable)
+#define MG_DECODE_STAGES 3  // per-worker ring depth (build-time tunable)
 #endif
 #ifndef MG_DECODE_MIN_BLOCKS
 #define MG_DECODE_MIN_BLOCKS 1  // resident CTAs per SM (the shared memory is sized for it)
 #endif
-#ifndef MG_DECODE_TMA
-#define MG_DECODE_TMA 0  // 1: K/V tiles by TMA gather4 + mbarrier; 0: 16-byte cp.async
-#endif
 #ifndef MG_DECODE_IDX_AHEAD
 #define MG_DECODE_IDX_AHEAD 12  // tiles of page-table entries fetched ahead of compute
-#endif
-#ifndef MG_DECODE_L2_AHEAD
-#define MG_DECODE_L2_AHEAD 0  // tiles of K/V rows prefetched into L2 ahead of compute (0: off)
-#endif
-#ifndef MG_DECODE_L2_MODE
-#define MG_DECODE_L2_MODE 2  // 1: bulk prefetch (one 256-B request), 2: two 128-B line prefetches
 #endif
 constexpr int kStages = MG_DECODE_STAGES;
 constexpr int kScanChunk = 4 * kThreads;  // requests per scan step
 constexpr int kMaxScanChunks = (kMaxBatch + kScanChunk - 1) / kScanChunk;
 constexpr int kIdxAhead = MG_DECODE_IDX_AHEAD;
-constexpr int kL2Ahead = MG_DECODE_L2_AHEAD;
 constexpr int kDescRing = 16;  // per-warp ring of tile descriptors / index rows
 static_assert(kDescRing >= kIdxAhead + 1, "descriptor ring too small");
-static_assert((kIdxAhead > kL2Ahead && kL2Ahead >= kStages - 1) || kL2Ahead == 0, "prefetch distances out of order");
 static_assert(kIdxAhead >= kStages, "page-table entries must lead the K/V loads");
 constexpr int kRingBytes = kWarps * kStages * kTileBytes;
 constexpr int kSmemBytes = kRingBytes + 1024;  // + alignment slack (128-byte swizzle atoms)
@@ -213,36 +202,13 @@ __device__ __forceinline__ void cursor_advance(const Params &p, Cursor &c) {
     }
 }
 
-// Warp-uniform bounded wait on an mbarrier phase: gives up after ~2 s of
-// %globaltimer, sets MG_DEVERR_WAIT_TIMEOUT and returns false.
-__device__ __forceinline__ bool warp_wait_bounded(uint32_t bar, uint32_t parity) {
-    bool done = false;
-    uint64_t t0 = 0;
-    for (uint32_t it = 0; !done; ++it) {
-        done = mbar_try_wait(bar, parity);
-        if (!done && (it & 255u) == 255u) {
-            uint64_t now;
-            asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(now));
-            if (t0 == 0) {
-                t0 = now;
-            } else if (now - t0 > 2000000000ull) {
-                atomicOr(&g_mg_device_error, MG_DEVERR_WAIT_TIMEOUT);
-                break;
-            }
-        }
-    }
-    return __all_sync(0xffffffffu, done);
-}
-
 // NT: n-tiles of 8 GQA heads (1 for g <= 8, 2 for g <= 16).
 // FUSED: the KV store of the step's new tokens happens in the same launch.
 template <int NT, bool FUSED>
 __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
-    decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                  const Params p) {
+    decode_kernel(const Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    __shared__ __align__(8) uint64_t full_bar[kWarps][kStages];
     __shared__ __align__(16) int idx_ring[kWarps][kDescRing][kKeys];
     __shared__ __align__(16) TileDesc desc_ring[kWarps][kDescRing];
     __shared__ float sh_lse[kWarps][16];
@@ -321,10 +287,6 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
         }
         if (blockIdx.x == 0 && tid == 0) p.prefix[p.batch] = T;
     }
-    if (tid < kWarps * kStages) {
-        mbar_init(smem_u32(&full_bar[tid / kStages][tid % kStages]), 1);
-        fence_mbarrier_init();
-    }
     __syncthreads();
 
     // ---- this warp's share
@@ -334,14 +296,7 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
 
     const int g = p.group;
     const uint32_t ring = smem_u32(smem) + (uint32_t)(warp * kStages * kTileBytes);
-    const int oob_row = (int)(p.num_slots * p.num_kv_heads);  // TMA reads it as zeros
     const int64_t head_stride = (int64_t)p.num_kv_heads * kHeadDim;
-    (void)oob_row;
-    (void)head_stride;
-    if (lane == 0) {
-        prefetch_tmap(&tm_k);
-        prefetch_tmap(&tm_v);
-    }
 
     Cursor cur;  // position of the next tile whose page-table entries are fetched
     cur.r = sh_start_r[warp];
@@ -377,8 +332,8 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
             cursor_advance(p, cur);
         }
     };
-    // Issue stage: read tile j's entries, check them, and let lanes 0..15 each
-    // issue one gather4 (K/V = lane / 8, 64-column half = (lane / 4) % 2, row quad = lane % 4).
+    // Issue stage: read tile j's entries, check them, gather its 16 K and 16 V
+    // rows into the tile's shared-memory stage.
     auto issue = [&](int j) {
         const int e = j % kDescRing, stage = j % kStages;
         const TileDesc d = my_desc[e];
@@ -392,24 +347,6 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
         }
         const unsigned valid = __ballot_sync(0xffffffffu, slot >= 0) & 0xFFFFu;
         if (lane == 0) my_desc[e].valid = valid;
-#if MG_DECODE_TMA
-        const int row_id = slot >= 0 ? slot * p.num_kv_heads + d.kvh : oob_row;
-        const int quad = lane & 3;
-        const int r0 = __shfl_sync(0xffffffffu, row_id, quad * 4 + 0);
-        const int r1 = __shfl_sync(0xffffffffu, row_id, quad * 4 + 1);
-        const int r2 = __shfl_sync(0xffffffffu, row_id, quad * 4 + 2);
-        const int r3 = __shfl_sync(0xffffffffu, row_id, quad * 4 + 3);
-        const uint32_t bar = smem_u32(&full_bar[warp][stage]);
-        if (lane == 0) mbar_arrive_expect_tx(bar, kTileBytes);
-        __syncwarp();
-        if (lane < 16) {
-            const int kind = lane >> 3, half = (lane >> 2) & 1;
-            const uint32_t dst = ring + (uint32_t)(stage * kTileBytes + kind * 2 * kHalfRows + half * kHalfRows +
-                                                   quad * 4 * 128);
-            fence_proxy_async_smem();
-            tma_gather4(dst, kind ? (const void *)&tm_v : (const void *)&tm_k, bar, half * 64, r0, r1, r2, r3);
-        }
-#else
         // 16-byte cp.async: each warp instruction moves two whole 256-byte rows
         // (lanes 0-15 and 16-31); 32 rows per tile (16 K then 16 V)
         const uint32_t base = ring + (uint32_t)(stage * kTileBytes);
@@ -429,31 +366,9 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
             if (key == new_key) src = (is_v ? p.v_new : p.k_new) + new_off;
             cp_async_16(base + (is_v ? 2 * kHalfRows : 0) + swz(key, ch), src, sl < 0 ? 0u : 16u);
         }
-#endif
     };
 
     constexpr int kPre = kIdxAhead;  // page-table fetch runs this many tiles ahead of compute
-
-    // L2 stage: prefetch tile j's 32 K/V rows (one 256-byte row per lane).
-    auto l2prefetch = [&](int j) {
-        if (j < 0 || j >= n_units) return;
-        const int e = j % kDescRing;
-        const TileDesc d = my_desc[e];
-        const int key = lane & (kKeys - 1);
-        if (d.t * kKeys + key < d.L) {
-            const int sl = my_idx[e][key];
-            if (sl >= 0 && (int64_t)sl < p.num_slots) {
-                const __nv_bfloat16 *row = ((lane >> 4) ? p.v_cache : p.k_cache) + (int64_t)sl * head_stride +
-                                           (int64_t)d.kvh * kHeadDim;
-#if MG_DECODE_L2_MODE == 1
-                prefetch_l2_bulk(row, kRowBytes);
-#else
-                prefetch_l2_line(row);
-                prefetch_l2_line(row + 64);
-#endif
-            }
-        }
-    };
 
     // Transposed tile products: S^T[key, head] = K Q^T and O^T[dim, head] +=
     // V^T P^T, keys / dims in the MMA M dimension and the GQA heads in N (8 per
@@ -465,36 +380,20 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
     uint32_t qb[NT][8][2];       // Q^T as B fragments
     const int quad = lane & 3;
     int seg_first_t = 0;
-    bool ok = true;
     int k = -kPre;
 
     // One software pipeline, one cp.async group per iteration k: fetch the
-    // page-table entries of tile k + IDX_AHEAD; prefetch tile k + L2_AHEAD
-    // into L2 (its entries arrived: their group is IDX_AHEAD - L2_AHEAD
-    // iterations old); copy tile k + STAGES - 1 into its shared-memory stage
-    // (freed when tile k - 1 finished); compute tile k.
+    // page-table entries of tile k + IDX_AHEAD; copy tile k + STAGES - 1 into
+    // its shared-memory stage (its entries arrived: their group is
+    // IDX_AHEAD - STAGES + 1 iterations old; the stage was freed when tile
+    // k - 1 finished); compute tile k.
     for (; k < n_units; ++k) {
         fetch(k + kPre);
         const int j = k + kStages - 1;
-#if MG_DECODE_TMA
-        cp_async_commit();
-        if (j >= 0 && j < n_units) {
-            cp_async_wait<kIdxAhead - kStages + 1>();
-            __syncwarp();
-            issue(j);
-        }
-#else
-        if (kL2Ahead > 0) {
-            cp_async_wait<(kL2Ahead > 0 ? kIdxAhead - kL2Ahead - 1 : 0)>();
-            __syncwarp();
-            l2prefetch(k + kL2Ahead);
-        } else {
-            cp_async_wait<kIdxAhead - kStages>();
-            __syncwarp();
-        }
+        cp_async_wait<kIdxAhead - kStages>();
+        __syncwarp();
         if (j >= 0 && j < n_units) issue(j);
         cp_async_commit();
-#endif
         if (k < 0) continue;
         const TileDesc c = my_desc[k % kDescRing];
         const bool first = k == 0 || c.t == 0;
@@ -519,16 +418,8 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
             }
             seg_first_t = c.t;
         }
-#if MG_DECODE_TMA
-        // wait for tile k (bounded: a lost transfer sets the timeout bit and ends this worker)
-        if (!warp_wait_bounded(smem_u32(&full_bar[warp][k % kStages]), (k / kStages) & 1)) {
-            ok = false;
-            break;
-        }
-#else
-        cp_async_wait<kStages - 1>();
+        cp_async_wait<kStages - 1>();  // tile k landed
         __syncwarp();
-#endif
 
         const uint32_t kt = ring + (uint32_t)((k % kStages) * kTileBytes);
         const uint32_t vt = kt + 2 * kHalfRows;
@@ -698,13 +589,6 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
             __syncwarp();  // scratch reads done before the stage is refilled
         }
     }
-    if (!ok) {
-        // give this worker's outstanding transfers (tiles k .. k+STAGES-2) a
-        // bounded chance to land before its shared memory can be released
-        for (int t = k; t < n_units && t < k + kStages - 1; ++t)
-            (void)mbar_wait_bounded(smem_u32(&full_bar[warp][t % kStages]), (t / kStages) & 1, 1u << 20);
-    }
-    (void)ok;
     cp_async_wait<0>();  // page-table copies still in flight
 }
 

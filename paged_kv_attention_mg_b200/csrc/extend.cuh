@@ -150,8 +150,7 @@ __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, vol
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    extend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                  const __grid_constant__ CUtensorMap tm_v, const Params p) {
+    extend_kernel(const __grid_constant__ CUtensorMap tm_q, const Params p) {
     extern __shared__ __align__(1024) uint8_t smem[];
     const uint32_t sbase = smem_u32(smem);
     if (sbase & 1023u) {  // the swizzled layouts need 1024-byte alignment: refuse, never fault
@@ -535,7 +534,7 @@ inline mg_status launch(Params &p, cudaStream_t stream) {
     if (!enc) return MG_ERR_CUDA;
     const int g = p.group;
     p.tokens_per_qtile = kM / g;
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq;
     {
         cuuint64_t dims[3] = {(cuuint64_t)kHeadDim, (cuuint64_t)p.num_q_heads, (cuuint64_t)p.total_q};
         cuuint64_t strides[2] = {(cuuint64_t)kHeadDim * 2, (cuuint64_t)p.num_q_heads * kHeadDim * 2};
@@ -546,15 +545,11 @@ inline mg_status launch(Params &p, cudaStream_t stream) {
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return MG_ERR_CUDA;
     }
-    if ((uint64_t)p.num_slots * (uint64_t)p.num_kv_heads >= (1ull << 31)) return MG_ERR_UNSUPPORTED_SHAPE;
-    if (!make_pool_tmap(&tk, p.k_cache, p.num_slots, p.num_kv_heads) ||
-        !make_pool_tmap(&tv, p.v_cache, p.num_slots, p.num_kv_heads))
-        return MG_ERR_CUDA;
     const int tokens_per_cta = kQTiles * p.tokens_per_qtile;
     const int nqb = (p.max_q_len + tokens_per_cta - 1) / tokens_per_cta;
     if (nqb > 0x7fffffff || p.batch > 65535 || p.num_kv_heads > 65535) return MG_ERR_INVALID_ARGUMENT;
     dim3 grid((unsigned)nqb, (unsigned)p.num_kv_heads, (unsigned)p.batch);
-    return launch_pdl(extend_kernel, grid, dim3(kThreads), kSmemBytes, stream, tq, tk, tv, p);
+    return launch_pdl(extend_kernel, grid, dim3(kThreads), kSmemBytes, stream, tq, p);
 }
 
 }  // namespace extend

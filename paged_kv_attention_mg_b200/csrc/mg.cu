@@ -173,21 +173,16 @@ mg_status decode_impl(const void *q, const void *k_new, const void *v_new, const
     p.max_seq_len = max_seq_len;
     p.scale_log2 = scale * kLog2e;
 
-    if ((uint64_t)num_slots * (uint64_t)num_kv_heads >= (1ull << 31)) return MG_ERR_UNSUPPORTED_SHAPE;
-    CUtensorMap tk, tv;
-    if (!make_pool_tmap(&tk, k_cache, num_slots, num_kv_heads) ||
-        !make_pool_tmap(&tv, v_cache, num_slots, num_kv_heads))
-        return MG_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int ctas = (workers + decode::kWarps - 1) / decode::kWarps;
     const dim3 grid(ctas), block(decode::kThreads);
     const size_t smem = decode::kSmemBytes;
     if (p.group <= 8)
-        st = fused ? launch_pdl(decode::decode_kernel<1, true>, grid, block, smem, s, tk, tv, p)
-                   : launch_pdl(decode::decode_kernel<1, false>, grid, block, smem, s, tk, tv, p);
+        st = fused ? launch_pdl(decode::decode_kernel<1, true>, grid, block, smem, s, p)
+                   : launch_pdl(decode::decode_kernel<1, false>, grid, block, smem, s, p);
     else
-        st = fused ? launch_pdl(decode::decode_kernel<2, true>, grid, block, smem, s, tk, tv, p)
-                   : launch_pdl(decode::decode_kernel<2, false>, grid, block, smem, s, tk, tv, p);
+        st = fused ? launch_pdl(decode::decode_kernel<2, true>, grid, block, smem, s, p)
+                   : launch_pdl(decode::decode_kernel<2, false>, grid, block, smem, s, p);
     if (st != MG_OK) return st;
     const int warps = batch * num_q_heads;
     return launch_pdl(decode::decode_merge_kernel, dim3((warps + 3) / 4), dim3(128), 0, s, p);

@@ -38,39 +38,6 @@ __device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];\n" ::"r"(bar) : "memory");
 }
 
-// Bulk prefetch of `bytes` (multiple of 16, 16-byte aligned) into L2; no
-// completion to wait for.
-__device__ __forceinline__ void prefetch_l2_bulk(const void *src, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(src), "r"(bytes) : "memory");
-}
-
-// Prefetch the 128-byte line holding `addr` into L2 (an ordinary LSU request).
-__device__ __forceinline__ void prefetch_l2_line(const void *addr) {
-    asm volatile("prefetch.global.L2 [%0];\n" ::"l"(addr));
-}
-
-// wait_group with a run-time count (0..15)
-__device__ __forceinline__ void cp_async_wait_dyn(int n) {
-    switch (n) {
-        case 0: cp_async_wait<0>(); break;
-        case 1: cp_async_wait<1>(); break;
-        case 2: cp_async_wait<2>(); break;
-        case 3: cp_async_wait<3>(); break;
-        case 4: cp_async_wait<4>(); break;
-        case 5: cp_async_wait<5>(); break;
-        case 6: cp_async_wait<6>(); break;
-        case 7: cp_async_wait<7>(); break;
-        case 8: cp_async_wait<8>(); break;
-        case 9: cp_async_wait<9>(); break;
-        case 10: cp_async_wait<10>(); break;
-        case 11: cp_async_wait<11>(); break;
-        case 12: cp_async_wait<12>(); break;
-        case 13: cp_async_wait<13>(); break;
-        case 14: cp_async_wait<14>(); break;
-        default: cp_async_wait<15>(); break;
-    }
-}
-
 // ---------------------------------------------------------------- ldmatrix / mma.sync
 __device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2,
                                             uint32_t &r3) {
@@ -158,13 +125,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-// Bounded wait: returns false after `limit` failed polls (each poll itself
-// suspends for a hardware-chosen time), never spins forever.
-__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, uint32_t limit) {
-    for (uint32_t i = 0; i < limit; ++i)
-        if (mbar_try_wait(bar, parity)) return true;
-    return false;
-}
 
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void prefetch_tmap(const void *tmap) {
@@ -177,15 +137,6 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void *tmap, uint
         "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%3, %4, %5}], [%2];\n" ::"r"(dst),
         "l"(tmap), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
-        : "memory");
-}
-// gather4: four rows (row0..row3) of a 2-D tensor map, columns [col, col+box).
-__device__ __forceinline__ void tma_gather4(uint32_t dst, const void *tmap, uint32_t bar, int32_t col,
-                                            int32_t row0, int32_t row1, int32_t row2, int32_t row3) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];\n" ::"r"(dst),
-        "l"(tmap), "r"(bar), "r"(col), "r"(row0), "r"(row1), "r"(row2), "r"(row3)
         : "memory");
 }
 
