@@ -194,6 +194,36 @@ def test_decode_flags_bad_metadata_without_faulting():
     assert mg.read_device_error() & mg.DEVERR_LENGTH
 
 
+def test_decode_workspace_contents_do_not_matter():
+    """mg_decode_attn reads nothing from its workspace that the same call did
+    not write: a workspace full of 0xFF bytes, or one a call of a different
+    plan (other batch / heads) has just used, gives the oracle's output, call
+    after call."""
+    lengths = [700, 3, 1500, 64, 2049]
+    step, data = _custom("decode", [L - 1 for L in lengths], lengths, 32, 8, seed=123)
+    g = GpuStep(step, data)
+    g.store()
+    ref = oracle_decode(step, data)
+    parts = 37  # every long pair split over several workers
+    need = mg.decode_workspace_bytes(step.batch, 32, 8, step.max_seq_len, num_partitions=parts)
+    other_step, other_data = _custom("decode", [99, 4000], [100, 4001], 16, 2, seed=5)
+    other = GpuStep(other_step, other_data)
+    other.store()
+    other_need = mg.decode_workspace_bytes(other_step.batch, 16, 2, other_step.max_seq_len, num_partitions=500)
+    ws = torch.full((max(need, other_need),), 0xFF, dtype=torch.uint8, device="cuda")
+
+    def run():
+        return mg.decode_attn(g.q, g.k_cache, g.v_cache, g.page_table, g.table_idx, g.seq_len, step.max_seq_len,
+                              g.scale, num_partitions=parts, workspace=ws)
+
+    assert_matches_oracle(run(), ref, "workspace of 0xFF bytes")
+    assert_matches_oracle(run(), ref, "second call on the same workspace")
+    mg.decode_attn(other.q, other.k_cache, other.v_cache, other.page_table, other.table_idx, other.seq_len,
+                   other_step.max_seq_len, other.scale, num_partitions=500, workspace=ws)
+    assert_matches_oracle(run(), ref, "after a call of another plan")
+    assert mg.read_device_error() == 0
+
+
 def test_decode_host_errors():
     step, data = _custom("decode", [299], [300], 16, 8, seed=9)
     g = GpuStep(step, data)
