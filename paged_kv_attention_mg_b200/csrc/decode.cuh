@@ -594,6 +594,10 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
 
 // One warp per (request, q head): combine the partials of a pair that more
 // than one worker touched.
+#ifndef MG_DECODE_MERGE_BATCH
+#define MG_DECODE_MERGE_BATCH 8
+#endif
+constexpr int kMergeBatch = MG_DECODE_MERGE_BATCH;  // partial segments loaded per round
 __global__ void __launch_bounds__(128) decode_merge_kernel(const Params p) {
     const int wg = blockIdx.x * 4 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
@@ -616,23 +620,26 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const Params p) {
     const int wf = worker_of(u0), wl = worker_of(u1 - 1);
     if (wf == wl) return;  // one worker held the whole pair and wrote the output
     const int64_t pair = (int64_t)r * p.num_kv_heads + kvh;
-    // online combine, four segments per round so their loads are in flight together
+    // with at least as many units as workers every share is non-empty; else
+    // skip the workers that got no units (and wrote no partial)
+    const bool sparse = T < W;
+    // online combine, kMergeBatch segments per round so their loads are in flight together
     float mx = -INFINITY, wsum = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int w0 = wf; w0 <= wl; w0 += 4) {
-        float ls[4];
-        float4 v[4];
+    for (int w0 = wf; w0 <= wl; w0 += kMergeBatch) {
+        float ls[kMergeBatch];
+        float4 v[kMergeBatch];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < kMergeBatch; ++i) {
             const int wk = w0 + i;
-            const bool use = wk <= wl && worker_begin(T, wk, W) != worker_begin(T, wk + 1, W);
+            const bool use = wk <= wl && (!sparse || worker_begin(T, wk, W) != worker_begin(T, wk + 1, W));
             const int64_t s = pair + wk;
             ls[i] = use ? p.part_lse[s * g + j] : -INFINITY;
             v[i] = use ? reinterpret_cast<const float4 *>(p.part_o + (s * g + j) * kHeadDim)[lane]
                        : make_float4(0.f, 0.f, 0.f, 0.f);
         }
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < kMergeBatch; ++i) {
             if (ls[i] == -INFINITY) continue;
             const float mn = fmaxf(mx, ls[i]);
             const float c = mx == -INFINITY ? 0.f : fast_exp2(mx - mn);
