@@ -52,6 +52,7 @@ from paged_kv_attention_mg_b200.replicas import Replicas, rank_spec  # noqa: E40
 from paged_kv_attention_mg_b200 import workload as wl  # noqa: E402
 
 METRIC = "paged decode-attention KV GB/s (% of HBM peak) and decode tokens/s, 1 B200"
+EXTEND_METRIC = "chunked-prefill extend attention TFLOP/s (unmasked QK^T + PV flops), 1 B200"
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 KERNEL_SOURCES = ["include/mg.h", "paged_kv_attention_mg_b200/csrc/mg.cu",
@@ -258,14 +259,8 @@ class DecodeBench:
     def kernel_bytes(self):
         return self.decode_bytes
 
-    def describe(self):
-        s, st = self.spec, self.step
-        return {"workload": s.name, "batch": st.batch, "layers": s.num_layers, "q_heads": s.num_q_heads,
-                "kv_heads": s.num_kv_heads, "head_dim": s.head_dim, "pool_slots": s.num_slots,
-                "mean_seq_len": round(float(st.seq_len.double().mean()), 1), "max_seq_len": st.max_seq_len,
-                "decode_workers": self.workers, "store": "fused into decode" if self.fused else "separate launch",
-                "l2": f"inputs larger than L2: {s.num_layers} per-layer pools, "
-                      f"{self.spec.num_layers * self.decode_bytes / 1e9:.2f} GB read per step"}
+    def details(self):
+        return {"decode_workers": self.workers, "store": "fused into decode" if self.fused else "separate launch"}
 
 
 class ExtendBench:
@@ -305,13 +300,27 @@ class ExtendBench:
     copy_in = DecodeBench.copy_in
     copy_out = DecodeBench.copy_out
 
-    def describe(self):
-        s, st = self.spec, self.step
-        n = (st.seq_len - st.cached_len)
-        return {"workload": s.name, "batch": st.batch, "layers": s.num_layers, "q_heads": s.num_q_heads,
-                "kv_heads": s.num_kv_heads, "head_dim": s.head_dim, "pool_slots": s.num_slots,
-                "new_tokens": int(n.sum()), "mean_cached_len": round(float(st.cached_len.double().mean()), 1),
-                "l2": "L2 flushed between timed steps (256 MB write)"}
+    def details(self):
+        return {}
+
+
+def workload_config(spec, step, n_gpus: int) -> dict:
+    """The `config` of the JSON line: the workload and how it is run, the same
+    for this library's arm and the reference arm."""
+    common = {"workload": spec.name, "batch": step.batch, "layers": spec.num_layers, "q_heads": spec.num_q_heads,
+              "kv_heads": spec.num_kv_heads, "head_dim": spec.head_dim, "pool_slots": spec.num_slots}
+    if spec.kind == "decode":
+        per_layer = rf.decode_bytes(step.seq_len.tolist(), spec.num_q_heads, spec.num_kv_heads, spec.head_dim)
+        common.update({"mean_seq_len": round(float(step.seq_len.double().mean()), 1),
+                       "max_seq_len": step.max_seq_len,
+                       "l2": f"inputs larger than L2: {spec.num_layers} per-layer pools, "
+                             f"{spec.num_layers * per_layer / 1e9:.2f} GB read per step"})
+    else:
+        n = step.seq_len - step.cached_len
+        common.update({"new_tokens": int(n.sum()), "mean_cached_len": round(float(step.cached_len.double().mean()), 1),
+                       "l2": "L2 flushed between timed steps (256 MB write)"})
+    common["parallelism"] = f"dp{n_gpus} (independent replicas, no collective)" if n_gpus > 1 else "single GPU"
+    return common
 
 
 # ----------------------------------------------------------------------------- cpu baseline
@@ -390,11 +399,11 @@ def run_reference(args):
         work += w
         secs += t
     value = (work / secs / 1e9) if unit == "GB/s" else (work / secs / 1e12)
-    line = {"impl": "reference", "metric": METRIC if spec.kind == "decode" else "extend attention TFLOP/s",
+    line = {"impl": "reference", "metric": METRIC if spec.kind == "decode" else EXTEND_METRIC,
             "value": round(value, 4), "unit": unit, "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(1e3 * secs / args.steps, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": spec.name, "parallelism": "host cores (oracle)"},
+            "data": "synthetic", "config": workload_config(spec, step, args.gpus), "arm": "oracle on the host cores",
             "cpu_baseline": {"value": round(value, 4), "unit": unit, "cores": threads, "kind": "oracle",
                              "sample": f"per step: {sample}"},
             "e2e": {"value": round(value, 4), "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -520,7 +529,7 @@ def run_ours(args):
     else:
         value = n * bench.flops / (step_ms * 1e-3) / 1e12
         unit = "TFLOP/s"
-        metric = "chunked-prefill extend attention TFLOP/s (unmasked QK^T + PV flops), 1 B200"
+        metric = EXTEND_METRIC
         achieved = bench.flops / (kernel_ms * 1e-3) / 1e12
         roof = {"bound": "tensor", "kernel": "extend_kernel", "achieved": round(achieved, 1), "peak": tflops,
                 "unit": "TFLOP/s", "frac": round(achieved / tflops, 4),
@@ -537,12 +546,11 @@ def run_ours(args):
                "sample": sample, "seconds": round(secs, 2)}
 
     if dist.rank == 0:
-        cfg = bench.describe()
-        cfg["parallelism"] = f"dp{n} (independent replicas, no collective)" if n > 1 else "single GPU"
+        cfg = workload_config(spec, step, n)
         line = {"metric": metric, "value": round(value, 2), "unit": unit, "n_gpus": n, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": round(step_ms, 4), "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg,
-                **extra, "roofline": roof, "cpu_baseline": cpu,
+                **extra, **bench.details(), "roofline": roof, "cpu_baseline": cpu,
                 "e2e": ({"value": round(n * (bench.step_bytes / 1e9 if spec.kind == 'decode' else bench.flops / 1e12)
                                        / (e2e * 1e-3), 2),
                          "unit": unit, "ms_per_step": round(e2e, 4), "h2d_bytes_per_step": bench.h2d_bytes,
