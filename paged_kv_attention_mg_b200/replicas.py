@@ -9,7 +9,12 @@ its own seeded batch (weak scaling).  torch.distributed is used only to line
 the ranks up around the timed region and to take the max of their times.
 
 ``shard_requests`` splits one global batch across ranks instead (the strong-
-scaling alternative), as contiguous request ranges.
+scaling alternative), as contiguous request ranges.  ``shard_kv_heads`` is the
+tensor-parallel split of the same page: each rank holds a contiguous range of
+KV heads with their query heads and its own pool of those heads, and runs the
+unchanged kernels on them (``take_heads`` cuts a rank's slice out of a full
+tensor); with fewer KV heads than ranks a head is replicated and its query
+heads are divided among the ranks that hold it.
 """
 from __future__ import annotations
 
@@ -37,6 +42,41 @@ def shard_requests(batch: int, rank: int, world: int) -> Tuple[int, int]:
     base, extra = divmod(batch, world)
     begin = rank * base + min(rank, extra)
     return begin, begin + base + (1 if rank < extra else 0)
+
+
+def shard_kv_heads(num_q_heads: int, num_kv_heads: int, rank: int, world: int) -> Tuple[int, int, int, int]:
+    """KV heads [kv0, kv1) and query heads [q0, q1) of tensor-parallel `rank`.
+
+    Query head h reads KV head h // g (g = num_q_heads // num_kv_heads), so a
+    rank's query heads are those of its KV heads and the local mapping is the
+    same formula on the slice.  world <= num_kv_heads: num_kv_heads / world KV
+    heads per rank.  world > num_kv_heads: every KV head on world / num_kv_heads
+    ranks, each with an equal share of its g query heads."""
+    if world <= 0 or not 0 <= rank < world:
+        raise ValueError("bad rank/world")
+    if num_kv_heads <= 0 or num_q_heads % num_kv_heads:
+        raise ValueError("num_q_heads must be a multiple of num_kv_heads")
+    g = num_q_heads // num_kv_heads
+    if world <= num_kv_heads:
+        if num_kv_heads % world:
+            raise ValueError("num_kv_heads must divide evenly across ranks")
+        per = num_kv_heads // world
+        kv0 = rank * per
+        return kv0, kv0 + per, kv0 * g, (kv0 + per) * g
+    if world % num_kv_heads:
+        raise ValueError("ranks must be a multiple of num_kv_heads to replicate")
+    rep = world // num_kv_heads
+    if g % rep:
+        raise ValueError("each KV head's query heads must divide evenly across its replicas")
+    kv0 = rank // rep
+    q0 = kv0 * g + (rank % rep) * (g // rep)
+    return kv0, kv0 + 1, q0, q0 + g // rep
+
+
+def take_heads(x: torch.Tensor, h0: int, h1: int) -> torch.Tensor:
+    """Heads [h0, h1) of a [..., heads, head_dim] tensor, contiguous (a rank's
+    own q / k_new / v_new rows, or its pool shard)."""
+    return x[..., h0:h1, :].contiguous()
 
 
 class Replicas:

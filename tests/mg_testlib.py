@@ -105,8 +105,24 @@ def bf16_to_f64(t: torch.Tensor) -> np.ndarray:
 
 # ----------------------------------------------------------------------------- GPU side
 
-MAX_ABS_TOL = 1e-2   # bf16 attention outputs vs the fp64 oracle (max |err|)
+MAX_ABS_TOL = 1e-2   # bf16 attention outputs vs the fp64 oracle (max |err|) ...
 MEAN_ABS_TOL = 1e-3  # ... and mean |err| over all real rows
+
+
+def bf16_ulp(x: np.ndarray) -> np.ndarray:
+    """Spacing of bf16 numbers at |x| (8 significant bits): 2^(floor(log2|x|) - 7)."""
+    ax = np.maximum(np.abs(x), np.finfo(np.float32).tiny)
+    return np.exp2(np.floor(np.log2(ax)) - 7)
+
+
+def elementwise_bound(ref: np.ndarray) -> np.ndarray:
+    """The max-abs bound an output element is held to: 1e-2, or one bf16 ulp at
+    |ref| where that is larger.  A bf16 output cannot be closer to an fp64 value
+    than half an ulp in general, and that half ulp alone exceeds 1e-2 once
+    |ref| >= 4 (an attention output over few keys is about one V entry, and V
+    entries drawn from N(0, 1) reach 4 and more); below |ref| = 2 the bound is
+    exactly 1e-2."""
+    return np.maximum(MAX_ABS_TOL, bf16_ulp(ref))
 
 
 def assert_matches_oracle(got: torch.Tensor, ref: np.ndarray, what: str = ""):
@@ -117,7 +133,10 @@ def assert_matches_oracle(got: torch.Tensor, ref: np.ndarray, what: str = ""):
     gs, rs = g[sel], ref[sel]
     assert np.isfinite(gs).all(), f"{what}: non-finite kernel output"
     diff = np.abs(gs - rs)
-    assert diff.max() <= MAX_ABS_TOL, f"{what}: max abs err {diff.max():.3e} (mean {diff.mean():.3e})"
+    excess = diff - elementwise_bound(rs)
+    worst = np.unravel_index(np.argmax(excess), excess.shape)
+    assert excess.max() <= 0, (f"{what}: |err| {diff[worst]:.3e} at |ref| {abs(rs[worst]):.3f} above its bound "
+                               f"{elementwise_bound(rs[worst]):.3e} (max abs err {diff.max():.3e}, mean {diff.mean():.3e})")
     assert diff.mean() <= MEAN_ABS_TOL, f"{what}: mean abs err {diff.mean():.3e}"
     return float(diff.max()), float(diff.mean())
 

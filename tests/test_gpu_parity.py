@@ -367,3 +367,53 @@ def test_extend_deterministic():
     a = g.extend()
     b = g.extend()
     assert torch.equal(a, b)
+
+
+# --------------------------------------------------------------------------- tensor-parallel head shards
+
+@pytest.mark.parametrize("world", [2, 16])
+def test_kv_head_shards_through_the_unchanged_kernels(world):
+    """A tensor-parallel rank's slice -- its query heads and a pool holding only
+    its KV heads (world 16 over 8 KV heads: each head on two ranks, half its
+    query heads each) -- through decode, fused store+decode and extend gives the
+    oracle's rows for those heads."""
+    from paged_kv_attention_mg_b200.replicas import shard_kv_heads, take_heads
+    hq, hkv = 32, 8
+    lengths = [700, 3, 1500, 64, 2049]
+    dstep, ddata = _custom("decode", [L - 1 for L in lengths], lengths, hq, hkv, seed=321)
+    dref = oracle_decode(dstep, ddata)
+    estep, edata = _custom("extend", [0, 130, 900], [150, 400, 1000], hq, hkv, seed=322)
+    eref = oracle_extend(estep, edata)
+    for r in range(world):
+        kv0, kv1, q0, q1 = shard_kv_heads(hq, hkv, r, world)
+        # decode and fused store+decode on the rank's own pool slice (new token not yet stored)
+        d = GpuStep(dstep, ddata)
+        kc, vc = take_heads(d.k_cache, kv0, kv1), take_heads(d.v_cache, kv0, kv1)
+        q = take_heads(d.q, q0, q1)
+        out = mg.store_decode_attn(q, take_heads(d.k_new, kv0, kv1), take_heads(d.v_new, kv0, kv1), d.out_loc,
+                                   kc, vc, d.page_table, d.table_idx, d.seq_len, dstep.max_seq_len, d.scale)
+        assert_matches_oracle(out, dref[:, q0:q1], f"rank {r}/{world} fused store+decode heads {q0}..{q1}")
+        out = mg.decode_attn(q, kc, vc, d.page_table, d.table_idx, d.seq_len, dstep.max_seq_len, d.scale)
+        assert_matches_oracle(out, dref[:, q0:q1], f"rank {r}/{world} decode heads {q0}..{q1}")
+        # extend
+        e = GpuStep(estep, edata)
+        e.store()
+        out = mg.extend_attn(take_heads(e.q, q0, q1), take_heads(e.k_cache, kv0, kv1), take_heads(e.v_cache, kv0, kv1),
+                             e.page_table, e.table_idx, e.cached_len, e.seq_len, e.q_offset, estep.max_q_len,
+                             estep.max_seq_len, e.scale)
+        assert_matches_oracle(out, eref[:, q0:q1], f"rank {r}/{world} extend heads {q0}..{q1}")
+    assert mg.read_device_error() == 0
+
+
+def test_extend_serves_a_mixed_batch():
+    """One mg_extend_attn launch over a batch as a chunked-prefill scheduler forms
+    it: decode requests (one new token after a long history), chunks of a
+    prompt, a fresh prompt and a request with nothing new this step."""
+    cached = [1999, 0, 512, 3000, 77, 40]
+    seq = [2000, 700, 1024, 3001, 78, 40]  # n = 1, 700, 512, 1, 1, 0
+    step, data = _custom("extend", cached, seq, 16, 8, seed=404)
+    g = GpuStep(step, data)
+    g.store()
+    out = g.extend()
+    assert mg.read_device_error() == 0
+    assert_matches_oracle(out, oracle_extend(step, data), "mixed decode / prefill batch")
