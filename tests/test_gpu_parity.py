@@ -417,3 +417,33 @@ def test_extend_serves_a_mixed_batch():
     out = g.extend()
     assert mg.read_device_error() == 0
     assert_matches_oracle(out, oracle_extend(step, data), "mixed decode / prefill batch")
+
+
+# --------------------------------------------------------------------------- shared prefix
+
+def test_decode_and_extend_over_a_shared_prefix():
+    """Requests whose page-table rows begin with the same slots (a prefix cache
+    hit: one copy of the shared tokens in the pool) read those slots through
+    every row; decode, fused store+decode and extend match the oracle on the
+    same tables.  (The kernels read the shared keys once per request; reading
+    them once per group is not built.)"""
+    prefix = 1500
+    lengths = [prefix + 40, prefix + 1, prefix + 700, prefix + 129, 300]
+    step, data = _custom("decode", [L - 1 for L in lengths], lengths, 32, 8, seed=777)
+    pt, ti = step.page_table, step.table_idx.long()
+    for r in (1, 2, 3):  # requests 1-3 share request 0's first `prefix` slots
+        pt[ti[r], :prefix] = pt[ti[0], :prefix]
+    ref = oracle_decode(step, data)
+    g = GpuStep(step, data)
+    assert_matches_oracle(g.store_decode(), ref, "fused store+decode, shared prefix")
+    assert_matches_oracle(g.decode(num_partitions=61), ref, "decode, shared prefix, 61 workers")
+    ecached = [prefix, prefix + 64, prefix, 0]
+    eseq = [prefix + 200, prefix + 100, prefix + 1, 180]
+    estep, edata = _custom("extend", ecached, eseq, 16, 8, seed=778)
+    ept, eti = estep.page_table, estep.table_idx.long()
+    for r in (1, 2):
+        ept[eti[r], :prefix] = ept[eti[0], :prefix]
+    e = GpuStep(estep, edata)
+    e.store()
+    assert_matches_oracle(e.extend(), oracle_extend(estep, edata), "extend, shared prefix")
+    assert mg.read_device_error() == 0
