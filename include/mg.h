@@ -107,8 +107,9 @@ mg_status mg_store_kv(const void *k, const void *v, const int32_t *out_loc, int3
  * units of 16 keys of one (request, kv head) pair; `workers` warps share the
  * units equally and in order, so a pair may be split across workers, whose
  * partial results a merge kernel combines.  num_partitions == 0 picks one
- * worker per resident warp slot of the current device (SMs x 12); > 0 forces
- * that many workers.  slots_out = batch * num_kv_heads + workers partial slots.
+ * worker per warp of the decode grid on the current device (SMs x 7 warps,
+ * one CTA per SM); > 0 forces that many workers.
+ * slots_out = batch * num_kv_heads + workers partial slots.
  * The plan depends only on these arguments (never on the lengths), so a
  * captured launch stays valid for any batch with lengths <= max_seq_len.
  */

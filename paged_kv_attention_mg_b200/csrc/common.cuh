@@ -40,7 +40,7 @@ inline mg_status launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, siz
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) == cudaSuccess ? MG_OK : MG_ERR_CUDA;
 }
 
-// ---------------------------------------------------------------- host: TMA tensor maps
+// ---------------------------------------------------------------- host: TMA tensor maps (extend's Q tiles)
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                    const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,

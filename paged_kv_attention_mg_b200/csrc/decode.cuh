@@ -103,7 +103,7 @@ struct Params {
 };
 
 // byte offset of 16-byte chunk c (0..15) of row `row` in a [16 rows x 256 B]
-// tile stored as two 64-column halves with the 128-byte TMA swizzle
+// tile stored as two 64-column halves with the 128-byte XOR swizzle
 __device__ __forceinline__ uint32_t swz(int row, int c) {
     return (uint32_t)((c >> 3) * kHalfRows + row * 128 + (((c & 7) ^ (row & 7)) << 4));
 }

@@ -65,7 +65,7 @@ mg_status ensure_kernel_attributes() {
 
 // Decode plan: the number of workers (warps) that share the work equally.
 // Automatic: one per warp slot the device keeps resident (SMs x resident CTAs
-// x 4), i.e. a single persistent wave.  Forced: num_partitions workers.
+// x warps per CTA), i.e. a single persistent wave.  Forced: num_partitions workers.
 mg_status decode_plan(int batch, int hkv, int max_seq_len, int num_partitions, int &workers) {
     if (batch <= 0 || hkv <= 0 || max_seq_len <= 0 || num_partitions < 0) return MG_ERR_INVALID_ARGUMENT;
     if (batch > decode::kMaxBatch) return MG_ERR_UNSUPPORTED_SHAPE;

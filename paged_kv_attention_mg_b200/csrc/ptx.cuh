@@ -1,8 +1,9 @@
 // ptx.cuh -- thin inline-PTX wrappers for sm_100a used by the kernels.
 //
-// Only instruction wrappers live here: async copies (cp.async, TMA tensor and
-// gather4 loads), mbarriers, warp-level bf16 MMA (decode), tcgen05 / TMEM
-// (extend) and a couple of conversions.  No kernel logic.
+// Only instruction wrappers live here: async copies (cp.async, 3-D TMA tensor
+// loads), mbarriers, warp-level bf16 MMA (decode), tcgen05 / TMEM (extend),
+// packed fp32 arithmetic, register reallocation and a couple of conversions.
+// No kernel logic.
 #pragma once
 
 #include <cstdint>
