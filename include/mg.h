@@ -80,10 +80,10 @@ const char *mg_status_string(mg_status status);
 int32_t mg_abi_version(void);
 
 /*
- * mg_store_kv -- KV write (the engine's "write KV cache" step; the custom
- * kernel of "mini-sglang from Scratch Stage 4 · Faster and bigger", §What each
- * chapter adds, "launch overhead and memory traffic of small operations such
- * as KV writes").
+ * mg_store_kv -- KV write (the engine's KV-cache write step; one of the small
+ * steps whose launch and memory cost the engine's own kernels target,
+ * "mini-sglang from Scratch Stage 4 · Faster and bigger", §What each chapter
+ * adds).
  *
  *   k_cache[out_loc[t], h, :] = k[t, h, :]   and   v_cache[out_loc[t], h, :] = v[t, h, :]
  *   for t < num_tokens, h < num_kv_heads.  A bit copy.
@@ -159,7 +159,7 @@ mg_status mg_decode_attn(const void *q, const void *k_cache, const void *v_cache
  * decode step (Mini-SGLang tag page, Engine post §一: write KV cache ->
  * attention); fusing it removes a launch and a pool round trip per layer
  * ("mini-sglang from Scratch Stage 4 · Faster and bigger", §What each chapter
- * adds: launch overhead of small operations such as KV writes).
+ * adds: a step as small as the KV write costs more in launch than in work).
  *
  *   k_new, v_new  [batch, num_kv_heads, head_dim] bf16: request r's new token
  *   out_loc       [batch] int32, out_loc[r] = page_table[table_idx[r]][seq_len[r]-1]

@@ -23,13 +23,12 @@
  *       KV Cache post, §一 (why a KV cache): at step t the query attends to the
  *       keys/values of positions 0..t.
  *  [S]  "mini-sglang from Scratch Stage 4 · Faster and bigger", §What each chapter
- *       adds: attention reads paged KV directly and never materialises the
- *       score matrix (the kernels' concern; the oracle may store one row of
- *       scores, which is the plain definition).
+ *       adds: attention works on the paged pool in place and keeps the score
+ *       matrix out of memory (the kernels' concern; the oracle may store one
+ *       row of scores, which is the plain definition).
  *
- * Readings taken where the pages are silent (each is listed in the design
- * notes): page_size is 1, so the pool is [num_slots, kv_heads, head_dim] and a
- * page-table entry is a slot; q head h uses KV head h / g with g = Hq / Hkv
+ * Readings taken where the pages are silent: page_size is 1, so the pool is
+ * [num_slots, kv_heads, head_dim] and a page-table entry is a slot; q head h uses KV head h / g with g = Hq / Hkv
  * (consecutive q heads share a KV head); scores are scale * <q, k>; softmax is
  * exp(x - max) / sum; decode is the one-new-token case (cached_len = L - 1).
  *
