@@ -7,7 +7,7 @@ A step is one pass of the hot path over one batch: for the default workload
 (Qwen3-0.6B attention shape, 28 layers, batch 64, lengths U[128, 2048]) that
 is, for every layer, the KV store of the 64 new tokens into that layer's pool
 followed by paged decode attention over the page table.  Each layer has its
-own 200k-slot pool, so a step reads ~8 GB of KV: inputs larger than L2, no
+own 200k-slot pool, so a step reads ~7.3 GB of KV: inputs larger than L2, no
 flush needed.  With N GPUs every rank runs its own replica with its own seed
 (weak scaling, no collective on the data path); the reported time is the max
 over ranks.
@@ -19,11 +19,14 @@ The JSON line: `value` = algorithmic bytes (K/V rows once per GQA group, q,
 out, page-table entries, plus the store's reads and writes) per step summed
 over ranks / step time, in GB/s; `e2e` = the same through the public API with
 the step's inputs copied from pinned host memory into the fixed buffers and
-the outputs copied back inside the timed region; `roofline` = one
-mg_decode_attn call (worker kernel + merge kernel), timed by CUDA events
-recorded inside the step around every call, against the measured HBM copy
-bandwidth; `cpu_baseline` = the fp64 oracle on this host's cores on a bounded
-sample of the same workload.
+the outputs copied back inside the timed region; `roofline` = one layer's
+mg_store_decode_attn call (decode kernel with the store fused, then the merge
+kernel; --unfused: mg_decode_attn after a separate mg_store_kv), timed by CUDA
+events recorded inside the step around every call, against the measured HBM
+copy bandwidth, with the DRAM bytes per launch ncu measured for these kernel
+sources (profiles/traffic.json); `cpu_baseline` = the fp64 oracle on this
+host's cores on a bounded sample of the same workload.  --workload
+chunked_prefill_extend measures extend (TFLOP/s against the dense bf16 peak).
 
 --impl reference times the oracle itself (there is no other implementation
 of this path to run) on the same metric, rank 0 only.
