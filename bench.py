@@ -357,60 +357,64 @@ def workload_config(spec, step, n_gpus: int) -> dict:
 
 # ----------------------------------------------------------------------------- cpu baseline
 
-def oracle_sample(spec, step, seconds: float, threads: int, layers_from: int = 0):
-    """Run the oracle on whole layers of the workload (decode) or on requests
-    (extend) until `seconds` of wall time are spent; returns (bytes_or_flops, time, sample, kind)."""
-    import oracle
-    done_units, total_t = 0, 0.0
-    work, sample = 0, []
-    if spec.kind == "decode":
-        L = step.seq_len.tolist()
-        per_layer = rf.decode_bytes(L, spec.num_q_heads, spec.num_kv_heads, spec.head_dim)
-        # every layer of the step once; when a whole pass is much shorter than the
-        # time bound, each generated layer is timed `reps` times (set after the first)
-        reps = 1
-        for i, layer in enumerate(range(layers_from, layers_from + spec.num_layers)):
-            data = wl.make_layer(step, layer % spec.num_layers)
+class OracleSampler:
+    """The oracle timed on bounded samples of the workload on the host cores.
+
+    Inputs are generated once and held across samples (decode: at most
+    `max_layers` distinct layers, each a full pool; extend: one layer), so a
+    sample times the oracle and not the synthetic-input generator.  A decode
+    sample runs whole layer calls (all requests), an extend sample whole
+    requests in turn, until `seconds` of oracle time are spent."""
+
+    def __init__(self, spec, step, threads: int, max_layers: int = 2):
+        self.spec, self.step, self.threads = spec, step, threads
+        self.max_layers = max(1, min(max_layers, spec.num_layers))
+        self._layers = []
+        self._next = 0  # decode: next cached layer; extend: next request
+
+    def _inputs(self, layer: int):
+        while len(self._layers) <= layer:
+            step = self.step
+            data = wl.make_layer(step, len(self._layers))
             k = wl.build_pool(step, data.hist_slots, data.k_hist)
             v = wl.build_pool(step, data.hist_slots, data.v_hist)
             loc = step.out_loc.to(torch.int64)
             k.index_copy_(0, loc, data.k_new)
             v.index_copy_(0, loc, data.v_new)
-            args = (wl.bits(data.q), wl.bits(k), wl.bits(v), step.page_table.numpy(), step.table_idx.numpy(),
-                    step.seq_len.numpy())
-            for _ in range(reps):
+            self._layers.append((wl.bits(data.q), wl.bits(k), wl.bits(v)))
+        return self._layers[layer]
+
+    def sample(self, seconds: float):
+        """Returns (bytes_or_flops, oracle seconds, what the sample was, unit)."""
+        import oracle
+        spec, step = self.spec, self.step
+        work, total_t, calls = 0, 0.0, 0
+        if spec.kind == "decode":
+            per_layer = rf.decode_bytes(step.seq_len.tolist(), spec.num_q_heads, spec.num_kv_heads, spec.head_dim)
+            while calls == 0 or total_t < seconds:
+                q, k, v = self._inputs(self._next)
+                self._next = (self._next + 1) % self.max_layers
                 t0 = time.perf_counter()
-                oracle.decode(*args, spec.scale, threads=threads)
-                dt = time.perf_counter() - t0
-                total_t += dt
+                oracle.decode(q, k, v, step.page_table.numpy(), step.table_idx.numpy(), step.seq_len.numpy(),
+                              spec.scale, threads=self.threads)
+                total_t += time.perf_counter() - t0
                 work += per_layer
-            if i == 0:
-                reps = max(1, min(50, int(seconds / (spec.num_layers * max(dt, 1e-6)))))
-            done_units += 1
-            if total_t >= seconds:
-                break
-        rep_note = f", each timed {reps} times" if reps > 1 else ""
-        return (work, total_t, f"{done_units} of {spec.num_layers} layers, all {step.batch} requests{rep_note}",
-                "GB/s")
-    # extend: whole requests until the time bound
-    data = wl.make_layer(step, layers_from)
-    k = wl.build_pool(step, data.hist_slots, data.k_hist)
-    v = wl.build_pool(step, data.hist_slots, data.v_hist)
-    loc = step.out_loc.to(torch.int64)
-    k.index_copy_(0, loc, data.k_new)
-    v.index_copy_(0, loc, data.v_new)
-    c, s = step.cached_len.tolist(), step.seq_len.tolist()
-    for r in range(step.batch):
-        t0 = time.perf_counter()
-        oracle.extend(wl.bits(data.q), wl.bits(k), wl.bits(v), step.page_table.numpy(), step.table_idx.numpy(),
-                      step.cached_len.numpy(), step.seq_len.numpy(), step.q_offset.numpy(), spec.scale,
-                      requests=[r], threads=threads)
-        total_t += time.perf_counter() - t0
-        work += rf.extend_flops([c[r]], [s[r]], spec.num_q_heads, spec.head_dim)
-        done_units += 1
-        if total_t >= seconds:
-            break
-    return work, total_t, f"{done_units} of {step.batch} requests of one layer", "TFLOP/s"
+                calls += 1
+            return (work, total_t, f"{calls} layer calls (all {step.batch} requests each) over "
+                    f"{len(self._layers)} generated layers", "GB/s")
+        q, k, v = self._inputs(0)
+        c, s = step.cached_len.tolist(), step.seq_len.tolist()
+        while calls == 0 or total_t < seconds:
+            r = self._next
+            self._next = (self._next + 1) % step.batch
+            t0 = time.perf_counter()
+            oracle.extend(q, k, v, step.page_table.numpy(), step.table_idx.numpy(), step.cached_len.numpy(),
+                          step.seq_len.numpy(), step.q_offset.numpy(), spec.scale, requests=[r],
+                          threads=self.threads)
+            total_t += time.perf_counter() - t0
+            work += rf.extend_flops([c[r]], [s[r]], spec.num_q_heads, spec.head_dim)
+            calls += 1
+        return work, total_t, f"{calls} requests of one layer (of {step.batch}, taken in turn)", "TFLOP/s"
 
 
 def cpu_threads():
@@ -431,12 +435,13 @@ def run_reference(args):
     step = wl.make_step(spec)
     threads = cpu_threads()
     per_step_seconds = max(0.5, min(6.0, 150.0 / max(1, args.steps + args.warmup)))
-    for i in range(args.warmup):
-        oracle_sample(spec, step, per_step_seconds, threads, layers_from=i)
+    sampler = OracleSampler(spec, step, threads)
+    for _ in range(args.warmup):
+        sampler.sample(per_step_seconds)
     work, secs = 0, 0.0
     sample = unit = None
-    for i in range(args.steps):
-        w, t, sample, unit = oracle_sample(spec, step, per_step_seconds, threads, layers_from=i)
+    for _ in range(args.steps):
+        w, t, sample, unit = sampler.sample(per_step_seconds)
         work += w
         secs += t
     value = (work / secs / 1e9) if unit == "GB/s" else (work / secs / 1e12)
@@ -581,7 +586,7 @@ def run_ours(args):
     cpu = None
     if dist.rank == 0 and n == 1 and not args.no_cpu_baseline:
         threads = cpu_threads()
-        w, secs, sample, cunit = oracle_sample(spec, step, args.cpu_seconds, threads)
+        w, secs, sample, cunit = OracleSampler(spec, step, threads).sample(args.cpu_seconds)
         cval = w / secs / (1e9 if cunit == "GB/s" else 1e12)
         cpu = {"value": round(cval, 4), "unit": cunit, "cores": threads, "kind": "oracle",
                "sample": sample, "seconds": round(secs, 2)}

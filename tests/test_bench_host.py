@@ -27,3 +27,21 @@ def test_both_arms_share_the_workload_config():
         assert cfg["workload"] == name and cfg["parallelism"] == "single GPU"
         assert cfg["batch"] == spec.batch and cfg["q_heads"] == spec.num_q_heads
         assert bench.workload_config(spec, step, 4)["parallelism"].startswith("dp4")
+
+
+def test_oracle_sampler_generates_inputs_once_and_fills_its_time_bound():
+    import oracle
+    oracle.build()
+    spec = wl.BY_NAME["tiny_decode"]
+    step = wl.make_step(spec)
+    sampler = bench.OracleSampler(spec, step, threads=1, max_layers=2)
+    for _ in range(3):
+        work, secs, sample, unit = sampler.sample(0.05)
+        assert unit == "GB/s" and secs >= 0.05 and work > 0
+        assert work % bench.rf.decode_bytes(step.seq_len.tolist(), spec.num_q_heads, spec.num_kv_heads,
+                                            spec.head_dim) == 0
+    assert len(sampler._layers) == min(2, spec.num_layers)   # held across samples, never regenerated
+    ext = wl.custom_spec("extend", [0, 5], [9, 12], 4, 2, 64, seed=3)
+    es = bench.OracleSampler(ext, wl.make_step(ext), threads=1)
+    work, secs, sample, unit = es.sample(0.0)
+    assert unit == "TFLOP/s" and work > 0 and "1 requests" in sample and len(es._layers) == 1
