@@ -21,10 +21,14 @@ over ranks / step time, in GB/s; `e2e` = the same through the public API with
 the step's inputs copied from pinned host memory into the fixed buffers and
 the outputs copied back inside the timed region; `roofline` = one layer's
 mg_store_decode_attn call (decode kernel with the store fused, then the merge
-kernel; --unfused: mg_decode_attn after a separate mg_store_kv), timed by CUDA
-events recorded inside the step around every call, against the measured HBM
-copy bandwidth, with the DRAM bytes per launch ncu measured for these kernel
-sources (profiles/traffic.json); `cpu_baseline` = the fp64 oracle on this
+kernel; --unfused: mg_decode_attn after a separate mg_store_kv) against the
+measured HBM copy bandwidth, its duration the timed step's device time over
+the layer calls it holds (the decode step's graph holds nothing else), with
+the DRAM bytes per launch ncu measured for these kernel sources
+(profiles/traffic.json); `call_us_events` is the same call timed by events
+recorded around every call inside a second, instrumented copy of the step
+(each event node ends the programmatic overlap of the next call's launch, so
+it reads a few microseconds longer); `cpu_baseline` = the fp64 oracle on this
 host's cores on a bounded sample of the same workload.  --workload
 chunked_prefill_extend measures extend (TFLOP/s against the dense bf16 peak).
 
@@ -37,6 +41,7 @@ import argparse
 import dataclasses
 import hashlib
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -211,10 +216,42 @@ def make_layers(step, num_layers, device):
         k = wl.build_pool(step, data.hist_slots, data.k_hist, device)
         v = wl.build_pool(step, data.hist_slots, data.v_hist, device)
         return dict(q=data.q.to(device), k_new=data.k_new.to(device), v_new=data.v_new.to(device),
-                    k_cache=k, v_cache=v, q_host=data.q.pin_memory(), k_new_host=data.k_new.pin_memory(),
-                    v_new_host=data.v_new.pin_memory())
+                    k_cache=k, v_cache=v, q_host=data.q, k_new_host=data.k_new, v_new_host=data.v_new)
     with ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
         return list(ex.map(one, range(num_layers)))
+
+
+def pack_io(bench, out_shape):
+    """Place the step's per-layer inputs (q, k_new, v_new) in one contiguous
+    device buffer and the per-layer outputs in another, each mirrored by one
+    pinned host buffer, so the end-to-end step moves them with one copy each
+    way.  The layers' tensors become views into these buffers."""
+    names = ("q", "k_new", "v_new")
+    sizes = [bench.layers[0][n].numel() for n in names]
+    per = sum(sizes)
+    L = len(bench.layers)
+    bench.in_dev = torch.empty(L * per, dtype=torch.bfloat16, device=bench.device)
+    bench.in_host = torch.empty(L * per, dtype=torch.bfloat16, pin_memory=True)
+    for i, lay in enumerate(bench.layers):
+        off = i * per
+        for n, sz in zip(names, sizes):
+            shape = lay[n].shape
+            view = bench.in_dev[off:off + sz].view(shape)
+            view.copy_(lay[n])
+            bench.in_host[off:off + sz].view(shape).copy_(lay.pop(n + "_host"))
+            lay[n] = view
+            off += sz
+    per_out = math.prod(out_shape)
+    bench.out_dev = torch.empty(L * per_out, dtype=torch.bfloat16, device=bench.device)
+    bench.out_host = torch.empty(L * per_out, dtype=torch.bfloat16, pin_memory=True)
+    bench.outs = [bench.out_dev[i * per_out:(i + 1) * per_out].view(out_shape) for i in range(L)]
+
+
+def io_bytes(bench):
+    """Bytes the end-to-end step copies host -> device and device -> host."""
+    h2d = sum(t.numel() * t.element_size() for t in bench.meta_host.values())
+    h2d += bench.in_host.numel() * bench.in_host.element_size()
+    return h2d, bench.out_host.numel() * bench.out_host.element_size()
 
 
 class DecodeBench:
@@ -233,9 +270,7 @@ class DecodeBench:
         self.workers, self.slots = mg.decode_plan(B, hkv, self.max_seq_len, partitions)
         ws = mg.decode_workspace_bytes(B, hq, hkv, self.max_seq_len, partitions)
         self.workspace = torch.empty(max(ws, 16), dtype=torch.uint8, device=device)
-        self.outs = [torch.empty((B, hq, spec.head_dim), dtype=torch.bfloat16, device=device)
-                     for _ in range(spec.num_layers)]
-        self.outs_host = [torch.empty_like(o, device="cpu").pin_memory() for o in self.outs]
+        pack_io(self, (B, hq, spec.head_dim))
         L = step.seq_len.tolist()
         self.decode_bytes = rf.decode_bytes(L, hq, hkv, spec.head_dim)
         self.store_bytes = rf.store_bytes(step.num_new_tokens, hkv, spec.head_dim)
@@ -245,9 +280,7 @@ class DecodeBench:
         self.launches_per_step = spec.num_layers * (2 if fused else 3)
         # what one timed call moves: the fused call also does the store
         self.kernel_bytes = self.decode_bytes + (self.store_bytes if fused else 0)
-        self.h2d_bytes = sum(t.numel() * t.element_size() for t in self.meta_host.values()) + spec.num_layers * (
-            self.layers[0]["q"].numel() * 2 + 2 * self.layers[0]["k_new"].numel() * 2)
-        self.d2h_bytes = sum(o.numel() * 2 for o in self.outs)
+        self.h2d_bytes, self.d2h_bytes = io_bytes(self)
         self.ev = None
 
     def layer(self, lay, out, meta, events=None):
@@ -276,17 +309,15 @@ class DecodeBench:
             self.layer(lay, self.outs[i], self.meta, events[i] if events else None)
 
     def copy_in(self):
-        """This step's inputs from pinned host memory into the fixed device buffers."""
+        """This step's inputs from pinned host memory into the fixed device buffers:
+        the metadata, then every layer's q / k / v rows in one copy."""
         for n, t in self.meta_host.items():
             self.meta[n].copy_(t, non_blocking=True)
-        for lay in self.layers:
-            lay["q"].copy_(lay["q_host"], non_blocking=True)
-            lay["k_new"].copy_(lay["k_new_host"], non_blocking=True)
-            lay["v_new"].copy_(lay["v_new_host"], non_blocking=True)
+        self.in_dev.copy_(self.in_host, non_blocking=True)
 
     def copy_out(self):
-        for i, o in enumerate(self.outs):
-            self.outs_host[i].copy_(o, non_blocking=True)
+        """Every layer's attention output back to pinned host memory in one copy."""
+        self.out_host.copy_(self.out_dev, non_blocking=True)
 
     def kernel_bytes(self):
         return self.decode_bytes
@@ -304,17 +335,14 @@ class ExtendBench:
         names = ("page_table", "table_idx", "seq_len", "cached_len", "q_offset", "out_loc")
         self.meta = {n: getattr(step, n).to(device) for n in names}
         self.meta_host = {n: getattr(step, n).pin_memory() for n in names}
-        self.outs = [torch.empty_like(lay["q"]) for lay in self.layers]
-        self.outs_host = [torch.empty_like(o, device="cpu").pin_memory() for o in self.outs]
+        pack_io(self, tuple(self.layers[0]["q"].shape))
         c, s = step.cached_len.tolist(), step.seq_len.tolist()
         self.flops = rf.extend_flops(c, s, spec.num_q_heads, spec.head_dim)
         self.extend_bytes = rf.extend_bytes(c, s, spec.num_q_heads, spec.num_kv_heads, spec.head_dim)
         self.store_bytes = rf.store_bytes(step.num_new_tokens, spec.num_kv_heads, spec.head_dim)
         self.tokens_per_step = step.num_new_tokens
         self.launches_per_step = spec.num_layers * 2
-        self.h2d_bytes = sum(t.numel() * t.element_size() for t in self.meta_host.values()) + spec.num_layers * (
-            self.layers[0]["q"].numel() * 2 + 2 * self.layers[0]["k_new"].numel() * 2)
-        self.d2h_bytes = sum(o.numel() * 2 for o in self.outs)
+        self.h2d_bytes, self.d2h_bytes = io_bytes(self)
         self.workers = None
 
     def layer(self, lay, out, meta, events=None):
@@ -505,16 +533,22 @@ def run_ours(args):
         run_timed, run_plain = enqueue_step, bench.run_step
     torch.cuda.synchronize()
 
+    # The decode step holds only the layer calls, so it is timed without
+    # instrumentation and a call's duration is the step time over its calls;
+    # the instrumented copy is replayed afterwards for the per-call events.
+    # The extend step also holds the L2 flush, timed by its own events and
+    # taken out, so that step runs instrumented.
+    run_step = run_plain if spec.kind == "decode" else run_timed
     sampler = ClockSampler(dist.local)
     sampler.start()
     # warm-up (W steps) plus a short soak so clocks are sampled under load
     for _ in range(max(3, args.warmup)):
-        run_timed()
+        run_step()
     torch.cuda.synchronize()
     t_end = time.perf_counter() + args.soak_seconds
     while time.perf_counter() < t_end:
         for _ in range(10):
-            run_timed()
+            run_step()
         torch.cuda.synchronize()
 
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -522,7 +556,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     start.record()
     for _ in range(args.steps):
-        run_timed()
+        run_step()
     stop.record()
     torch.cuda.synchronize()
     dist.barrier()
@@ -530,9 +564,19 @@ def run_ours(args):
     total_ms = start.elapsed_time(stop)
     flush_ms = fev[0].elapsed_time(fev[1]) if flush is not None else 0.0  # last step's flush
     step_ms_local = total_ms / args.steps - flush_ms
-    kernel_ms_local = sum(a.elapsed_time(b) for a, b in kev) / spec.num_layers  # last step's calls
+    if spec.kind == "decode":
+        kernel_ms_local = step_ms_local / spec.num_layers
+        for _ in range(3):  # the instrumented copy, outside the timed region
+            run_timed()
+        torch.cuda.synchronize()
+    else:
+        kernel_ms_local = None
+    events_ms_local = sum(a.elapsed_time(b) for a, b in kev) / spec.num_layers  # last step's calls
+    if kernel_ms_local is None:
+        kernel_ms_local = events_ms_local
     step_ms = dist.max(step_ms_local)
     kernel_ms = dist.max(kernel_ms_local)
+    events_ms = dist.max(events_ms_local)
 
     # end to end through the public API with host buffers: this step's inputs
     # copied from pinned host memory into the fixed device buffers, the step,
@@ -568,6 +612,8 @@ def run_ours(args):
         roof = {"bound": "hbm", "kernel": kname,
                 "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s", "frac": round(achieved / hbm, 4),
                 "peak_source": f"{peak_src} HBM copy bandwidth",
+                "call_us": round(kernel_ms * 1e3, 3), "duration": "timed step / layer calls in it",
+                "call_us_events": round(events_ms * 1e3, 3),
                 "traffic": profiled_traffic(spec.name)}
         extra = {"tokens_per_s": round(n * bench.tokens_per_step / (step_ms * 1e-3), 1),
                  "frac_of_8tbs_nominal": round(value / n / 8000.0, 4),
