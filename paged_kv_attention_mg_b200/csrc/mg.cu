@@ -3,6 +3,7 @@
 //
 // Everything is one translation unit so the kernels share the device error
 // word without relocatable device code.
+#include <atomic>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -18,8 +19,11 @@ namespace {
 constexpr int kMaxDevices = 64;
 constexpr int kMaxDecodeWorkers = 1 << 22;
 
-int g_sm_count[kMaxDevices];
-bool g_attr_done[kMaxDevices];
+// Per-device caches, filled on first use.  They are read without the lock,
+// so they are atomics: a thread that sees a value also sees what was done
+// before it was stored (the attributes set, the count read).
+std::atomic<int> g_sm_count[kMaxDevices];
+std::atomic<bool> g_attr_done[kMaxDevices];
 std::mutex g_attr_mutex;
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -32,13 +36,13 @@ mg_status current_device(int &dev) {
 mg_status sm_count(int &sms) {
     int dev;
     if (current_device(dev) != MG_OK) return MG_ERR_CUDA;
-    if (g_sm_count[dev] == 0) {
-        int v = 0;
+    int v = g_sm_count[dev].load(std::memory_order_acquire);
+    if (v == 0) {
         if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
             return MG_ERR_CUDA;
-        g_sm_count[dev] = v;
+        g_sm_count[dev].store(v, std::memory_order_release);
     }
-    sms = g_sm_count[dev];
+    sms = v;
     return MG_OK;
 }
 
@@ -46,9 +50,9 @@ mg_status sm_count(int &sms) {
 mg_status ensure_kernel_attributes() {
     int dev;
     if (current_device(dev) != MG_OK) return MG_ERR_CUDA;
-    if (g_attr_done[dev]) return MG_OK;
+    if (g_attr_done[dev].load(std::memory_order_acquire)) return MG_OK;
     std::lock_guard<std::mutex> lock(g_attr_mutex);
-    if (g_attr_done[dev]) return MG_OK;
+    if (g_attr_done[dev].load(std::memory_order_relaxed)) return MG_OK;
     if (cudaFuncSetAttribute(decode::decode_kernel<1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              decode::kSmemBytes) != cudaSuccess ||
         cudaFuncSetAttribute(decode::decode_kernel<2, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -59,7 +63,7 @@ mg_status ensure_kernel_attributes() {
                              decode::kSmemBytes) != cudaSuccess)
         return MG_ERR_CUDA;
     if (extend::set_attributes() != cudaSuccess) return MG_ERR_CUDA;
-    g_attr_done[dev] = true;
+    g_attr_done[dev].store(true, std::memory_order_release);
     return MG_OK;
 }
 
@@ -357,7 +361,7 @@ namespace {
 constexpr size_t kStaticDecodeWorkspaceBytes = MG_DECODE_STATIC_WORKSPACE_BYTES;
 static __device__ __align__(256) unsigned char g_decode_static_workspace[kStaticDecodeWorkspaceBytes];
 
-void *g_static_ws_ptr[kMaxDevices];
+std::atomic<void *> g_static_ws_ptr[kMaxDevices];  // read without the lock, like the caches above
 std::mutex g_static_ws_mutex;
 
 // The array's device address on the current device.  In host code the
@@ -366,16 +370,17 @@ std::mutex g_static_ws_mutex;
 mg_status static_workspace(void *&ptr) {
     int dev;
     if (current_device(dev) != MG_OK) return MG_ERR_CUDA;
-    if (!g_static_ws_ptr[dev]) {
+    void *p = g_static_ws_ptr[dev].load(std::memory_order_acquire);
+    if (!p) {
         std::lock_guard<std::mutex> lock(g_static_ws_mutex);
-        if (!g_static_ws_ptr[dev]) {
-            void *p = nullptr;
+        p = g_static_ws_ptr[dev].load(std::memory_order_relaxed);
+        if (!p) {
             if (cudaGetSymbolAddress(&p, g_decode_static_workspace) != cudaSuccess || p == nullptr)
                 return MG_ERR_CUDA;
-            g_static_ws_ptr[dev] = p;
+            g_static_ws_ptr[dev].store(p, std::memory_order_release);
         }
     }
-    ptr = g_static_ws_ptr[dev];
+    ptr = p;
     return MG_OK;
 }
 

@@ -85,6 +85,8 @@ DECODE_SMALL = [
     ([257, 190], 32, 2),      # group 16
     ([33, 100], 4, 4),        # group 1
     ([511, 3, 1000, 2], 12, 4),  # group 3 (not a power of two)
+    ([130, 7, 400], 28, 4),   # group 7
+    ([66, 300], 24, 2),       # group 12 (two row blocks, not a power of two)
 ]
 
 
@@ -308,6 +310,9 @@ EXTEND_SMALL = [
     ([0, 100], [40, 260], 32, 4),               # group 8
     ([31], [200], 32, 2),                       # group 16
     ([10, 20], [10, 50], 16, 8),                # a request with no new tokens
+    ([0, 50], [130, 300], 12, 4),               # group 3: 42 tokens fill 126 of a Q tile's 128 rows
+    ([7], [260], 28, 4),                        # group 7: 18 tokens, 126 rows
+    ([0, 9], [100, 200], 12, 1),                # group 12: 10 tokens, 120 rows
 ]
 
 
