@@ -57,6 +57,8 @@ DECODE_CASES = [
     ([17, 1, 64], 16, 2),
     ([25], 32, 4),
     ([3, 31], 4, 1),
+    ([11, 4], 12, 4),       # group 3
+    ([9, 30], 28, 4),       # group 7
 ]
 
 
@@ -219,6 +221,7 @@ EXTEND_CASES = [
     ([0], [37], 8, 2),
     ([20, 0, 5], [21, 33, 70], 8, 1),
     ([64, 1], [90, 3], 32, 4),
+    ([3, 0], [10, 40], 12, 4),      # group 3
 ]
 
 
