@@ -123,3 +123,36 @@ def test_attention_rejects_a_scale_that_is_not_finite_and_positive(lib, scale):
                               4096, None, 0, None) == 1
     assert lib.mg_extend_attn(4096, 4096, 4096, 100, 4096, 5, 32, 4096, 4096, 4096, 4096, 4, 0, 0, 32,
                               16, 8, 128, scale, 4096, None) == 1
+
+
+def test_decode_partial_slots_cover_every_segment(lib):
+    """The plan's slot count holds every split segment: units (16 keys of one
+    (request, kv head) pair, request-major) are cut into equal contiguous worker
+    shares [floor(wT/W), floor((w+1)T/W)); a segment is a (pair, worker) overlap
+    and writes its partial to slot pair + worker, which must be unique and below
+    the slot count the library reports."""
+    import numpy as np
+    rng = np.random.default_rng(5)
+    for _ in range(40):
+        batch = int(rng.integers(1, 9))
+        hkv = int(rng.choice([1, 2, 4, 8]))
+        lengths = [int(x) for x in rng.integers(1, 700, size=batch)]
+        workers = int(rng.integers(1, 300))
+        w_out, s_out = ctypes.c_int32(), ctypes.c_int64()
+        assert lib.mg_decode_plan(batch, hkv, max(lengths), workers, ctypes.byref(w_out), ctypes.byref(s_out)) == 0
+        W, slots = w_out.value, s_out.value
+        assert W == workers
+        tiles = [(L + 15) // 16 for L in lengths]
+        pair_end = np.cumsum([t for t in tiles for _ in range(hkv)])   # end unit of every pair
+        T = int(pair_end[-1])
+        used = set()
+        for w in range(W):
+            u0, u1 = w * T // W, (w + 1) * T // W
+            u = u0
+            while u < u1:
+                pair = int(np.searchsorted(pair_end, u, side="right"))
+                end = min(u1, int(pair_end[pair]))
+                slot = pair + w
+                assert slot not in used and 0 <= slot < slots
+                used.add(slot)
+                u = end
