@@ -2,9 +2,10 @@
  * mg.h -- C ABI of the B200 (sm_100a) paged KV attention library (libmg.so).
  *
  * Three operations make up the per-layer attention hot path of the
- * mini-sglang engine, in the order the engine runs them (Mini-SGLang tag
- * page, Engine post, §一 "GPU inference is not only matrix multiplication":
- * ... RoPE -> write KV cache -> attention -> o_proj):
+ * mini-sglang engine.  Each layer of its forward pass runs the QKV
+ * projection, RoPE, the KV-cache write, attention and o_proj, in that order
+ * (Mini-SGLang tag page, Engine post, §一); this library covers the KV-cache
+ * write and attention:
  *
  *   mg_store_kv     write the new tokens' K/V into pool slots at out_loc;
  *   mg_decode_attn  one query token per request against its paged history
