@@ -21,8 +21,11 @@
 //   * warp 12, one thread: issues tcgen05.mma (M=128, N=128, K=16, bf16 in,
 //     fp32 accumulate in TMEM).  S_t = Q_t K^T lands in TMEM; P_t (bf16) is
 //     written back over S_t and consumed straight from TMEM as the A operand
-//     of O_t += P_t V.  The two Q tiles ping-pong so the tensor core works on
-//     one tile while the softmax warps work on the other.
+//     of O_t += P_t V.  The MMAs of the two Q tiles interleave, each issued
+//     once its inputs are ready.  (Since P_t overwrites S_t, S_t of the next
+//     KV tile waits for P_t V; measured, both Q tiles' softmaxes then wait on
+//     the same KV tile, so the softmax and the tensor core mostly alternate
+//     instead of overlapping: the kernel's present bound.)
 //   * warpgroups 1 / 2: softmax for Q tile 0 / 1, one TMEM lane (= one query
 //     row) per thread: causal mask key <= c + i, online softmax in the exp2
 //     domain, O rescaled in TMEM only when the running max grows by more than
