@@ -27,6 +27,14 @@ MUTANTS = {
     "extend_wrong_query_row": ("const int64_t t = q_offset[r] + i;", "const int64_t t = q_offset[r];"),
     "store_swaps_k_and_v": ("= k[t * row + h * head_dim + d];", "= v[t * row + h * head_dim + d];"),
     "dot_uses_wrong_dim_of_q": ("bf16_bits_to_double(q_vec[d]) *", "bf16_bits_to_double(q_vec[0]) *"),
+    "decode_row_ignores_table_idx": ("num_slots, page_table + (int64_t)table_idx[r] * pt_stride,",
+                                     "num_slots, page_table + (int64_t)r * pt_stride,"),
+    "extend_row_ignores_table_idx": ("*pt_row = page_table + (int64_t)table_idx[r] * pt_stride;",
+                                     "*pt_row = page_table + (int64_t)r * pt_stride;"),
+    "extend_attends_only_to_the_chunk": ("pt_row, c + i, h / group,", "pt_row + c, i, h / group,"),
+    "v_row_of_the_previous_key": ("v_pool + (int64_t)pt_row[j] * row", "v_pool + (int64_t)pt_row[j > 0 ? j - 1 : 0] * row"),
+    "v_from_kv_head_zero": ("row + kvh * head_dim;\n        for (int64_t d = 0; d < head_dim; ++d) o[d] +=",
+                            "row + 0 * head_dim;\n        for (int64_t d = 0; d < head_dim; ++d) o[d] +="),
 }
 
 
@@ -45,8 +53,10 @@ def _pins(lib):
     except oracle.OracleError:
         failures.append("store-error")
     # decode vs dense SDPA
-    case = decode_case([5, 9, 12, 2], 16, 4, seed=102)
+    case = decode_case([5, 9, 12, 2], 16, 4, seed=104)
     s = case.step
+    # no request reads page-table row r itself, so a mix-up of r and table_idx[r] shows
+    assert all(int(t) != r for r, t in enumerate(s.table_idx.tolist()))
     try:
         got = oracle.decode(**case.oracle_args(), scale=SCALE, lib=lib)
         ref = dense_decode(case.data.q, case.k_pool, case.v_pool, s.page_table, s.table_idx,
@@ -71,6 +81,7 @@ def _pins(lib):
     # extend vs dense causal SDPA
     case = extend_case([0, 3, 10], [4, 9, 14], 8, 2, seed=103)
     s = case.step
+    assert all(int(t) != r for r, t in enumerate(s.table_idx.tolist()))
     try:
         a = case.oracle_args()
         a.update(cached_len=s.cached_len.numpy(), q_offset=s.q_offset.numpy())
