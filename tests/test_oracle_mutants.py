@@ -33,6 +33,8 @@ MUTANTS = {
                                      "*pt_row = page_table + (int64_t)r * pt_stride;"),
     "extend_attends_only_to_the_chunk": ("pt_row, c + i, h / group,", "pt_row + c, i, h / group,"),
     "v_row_of_the_previous_key": ("v_pool + (int64_t)pt_row[j] * row", "v_pool + (int64_t)pt_row[j > 0 ? j - 1 : 0] * row"),
+    "decode_length_of_the_table_row": ("const int64_t L = seq_len[r];", "const int64_t L = seq_len[table_idx[r]];"),
+    "store_tokens_in_reverse": ("int64_t slot = out_loc[t];", "int64_t slot = out_loc[num_tokens - 1 - t];"),
     "v_from_kv_head_zero": ("row + kvh * head_dim;\n        for (int64_t d = 0; d < head_dim; ++d) o[d] +=",
                             "row + 0 * head_dim;\n        for (int64_t d = 0; d < head_dim; ++d) o[d] +="),
 }
