@@ -91,20 +91,53 @@ def _stream(stream) -> Optional[int]:
 
 
 def _dev(t: torch.Tensor, dtype, name: str) -> int:
+    """Device pointer of a dense tensor of `dtype` on the current CUDA device
+    (the library launches on the current device)."""
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a tensor")
     if t.dtype != dtype:
         raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
     if not t.is_cuda:
         raise ValueError(f"{name} must be on a CUDA device")
+    if t.device.index != torch.cuda.current_device():
+        raise ValueError(f"{name} is on {t.device}, not on the current CUDA device "
+                         f"(cuda:{torch.cuda.current_device()}), where the library launches")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     return t.data_ptr()
 
 
+def _shape(t: torch.Tensor, shape, what: str) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{what} must be a tensor")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{what}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _attention_shapes(op: str, q, k_cache, v_cache, page_table, out, per_request) -> None:
+    """The sizes the library takes on trust: q [rows, Hq, D]; pools [slots, Hkv, D],
+    V like K; a 2-D page table; out like q; [batch] metadata per request."""
+    for name, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache), ("page_table", page_table)):
+        if not isinstance(t, torch.Tensor):
+            raise TypeError(f"{op}: {name} must be a tensor")
+    if q.dim() != 3:
+        raise ValueError(f"{op}: q must be [rows, num_q_heads, head_dim]")
+    if k_cache.dim() != 3 or k_cache.shape[2] != q.shape[2]:
+        raise ValueError(f"{op}: k_cache must be [num_slots, num_kv_heads, head_dim]")
+    _shape(v_cache, k_cache.shape, f"{op}: v_cache")
+    if page_table.dim() != 2:
+        raise ValueError(f"{op}: page_table must be [rows, stride]")
+    if out is not None:
+        _shape(out, q.shape, f"{op}: out")
+    for name, (t, shape) in per_request.items():
+        _shape(t, shape, f"{op}: {name}")
+
+
 def store_kv(k: torch.Tensor, v: torch.Tensor, out_loc: torch.Tensor, k_cache: torch.Tensor,
              v_cache: torch.Tensor, stream=None) -> None:
     """k_cache[out_loc[t]] = k[t]; v_cache[out_loc[t]] = v[t] (bf16 rows)."""
+    if k.dim() != 3 or k_cache.dim() != 3:
+        raise ValueError("store_kv: k must be [num_tokens, num_kv_heads, head_dim], k_cache [num_slots, ...]")
     t, hkv, d = k.shape
     if v.shape != k.shape or k_cache.shape[1:] != (hkv, d) or v_cache.shape != k_cache.shape:
         raise ValueError("store_kv: shape mismatch")
@@ -136,6 +169,9 @@ def decode_attn(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, p
                 num_partitions: int = 0, out: Optional[torch.Tensor] = None,
                 workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """Paged decode attention; returns out [B, Hq, D] bf16."""
+    b = q.shape[0] if isinstance(q, torch.Tensor) and q.dim() == 3 else -1
+    _attention_shapes("decode_attn", q, k_cache, v_cache, page_table, out,
+                      {"table_idx": (table_idx, (b,)), "seq_len": (seq_len, (b,))})
     b, hq, d = q.shape
     hkv = k_cache.shape[1]
     if out is None:
@@ -161,6 +197,9 @@ def store_decode_attn(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
                       num_partitions: int = 0, out: Optional[torch.Tensor] = None,
                       workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """store_kv(k_new, v_new, out_loc) then decode_attn, fused into one decode launch."""
+    b = q.shape[0] if isinstance(q, torch.Tensor) and q.dim() == 3 else -1
+    _attention_shapes("store_decode_attn", q, k_cache, v_cache, page_table, out,
+                      {"table_idx": (table_idx, (b,)), "seq_len": (seq_len, (b,))})
     b, hq, d = q.shape
     hkv = k_cache.shape[1]
     if k_new.shape != (b, hkv, d) or v_new.shape != k_new.shape or out_loc.shape != (b,):
@@ -189,11 +228,14 @@ def extend_attn(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, p
                 q_offset: torch.Tensor, max_q_len: int, max_seq_len: int, scale: float,
                 out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """Chunked-prefill extend attention; returns out [total_q, Hq, D] bf16."""
+    if not isinstance(seq_len, torch.Tensor) or seq_len.dim() != 1:
+        raise ValueError("extend_attn: seq_len must be [batch]")
+    b = seq_len.shape[0]
+    _attention_shapes("extend_attn", q, k_cache, v_cache, page_table, out,
+                      {"table_idx": (table_idx, (b,)), "cached_len": (cached_len, (b,)),
+                       "q_offset": (q_offset, (b + 1,))})
     total_q, hq, d = q.shape
     hkv = k_cache.shape[1]
-    b = seq_len.shape[0]
-    if q_offset.shape != (b + 1,):
-        raise ValueError("extend_attn: q_offset must be [batch + 1]")
     if out is None:
         out = torch.empty_like(q)
     _check(load().mg_extend_attn(_dev(q, torch.bfloat16, "q"), _dev(k_cache, torch.bfloat16, "k_cache"),
@@ -219,6 +261,9 @@ def decode_attn_static_workspace(q: torch.Tensor, k_cache: torch.Tensor, v_cache
     calls race).  Raises MgError(MG_ERR_WORKSPACE_TOO_SMALL) when the plan
     needs more than STATIC_WORKSPACE_BYTES.  Allocates nothing on the device
     except `out` when it is not given."""
+    b = q.shape[0] if isinstance(q, torch.Tensor) and q.dim() == 3 else -1
+    _attention_shapes("decode_attn_static_workspace", q, k_cache, v_cache, page_table, out,
+                      {"table_idx": (table_idx, (b,)), "seq_len": (seq_len, (b,))})
     b, hq, d = q.shape
     hkv = k_cache.shape[1]
     if out is None:

@@ -7,6 +7,7 @@ import re
 import subprocess
 
 import pytest
+import torch
 
 from paged_kv_attention_mg_b200 import build, mg
 
@@ -156,3 +157,76 @@ def test_decode_partial_slots_cover_every_segment(lib):
                 assert slot not in used and 0 <= slot < slots
                 used.add(slot)
                 u = end
+
+
+def test_binding_checks_the_sizes_the_library_takes_on_trust():
+    """The C ABI trusts the pool, output and metadata sizes it is given, so the
+    binding compares tensor shapes before any pointer is passed (host tensors
+    suffice: the shape checks come first)."""
+    bf, i32 = torch.bfloat16, torch.int32
+    b, hq, hkv, d, slots = 3, 8, 4, 128, 50
+    q = torch.zeros(b, hq, d, dtype=bf)
+    k = torch.zeros(slots, hkv, d, dtype=bf)
+    pt = torch.zeros(b + 1, 32, dtype=i32)
+    idx = torch.arange(b, dtype=i32)
+    seq = torch.ones(b, dtype=i32)
+    cases = [
+        (lambda: mg.decode_attn(q, k, k[:-1], pt, idx, seq, 16, 0.1), "v_cache"),
+        (lambda: mg.decode_attn(q, k, k, pt, idx, seq[:-1], 16, 0.1), "seq_len"),
+        (lambda: mg.decode_attn(q, k, k, pt, idx[:-1], seq, 16, 0.1), "table_idx"),
+        (lambda: mg.decode_attn(q, k, k, pt, idx, seq, 16, 0.1, out=q[:-1]), "out"),
+        (lambda: mg.decode_attn(q, k[..., :64], k[..., :64], pt, idx, seq, 16, 0.1), "k_cache"),
+        (lambda: mg.decode_attn(q, k, k, pt[0], idx, seq, 16, 0.1), "page_table"),
+        (lambda: mg.store_decode_attn(q, k[:b], k[:b], idx, k, k[:, :2], pt, idx, seq, 16, 0.1), "v_cache"),
+        (lambda: mg.decode_attn_static_workspace(q, k, k, pt, idx, seq, 16, 0.1, out=q[:, :4]), "out"),
+        (lambda: mg.extend_attn(q, k, k, pt, idx, seq - 1, seq, idx, 1, 16, 0.1), "q_offset"),
+        (lambda: mg.extend_attn(q, k, k, pt, idx, seq[:2] - 1, seq, torch.arange(b + 1, dtype=i32), 1, 16, 0.1),
+         "cached_len"),
+        (lambda: mg.store_kv(q[0], q[0], idx, k, k), "store_kv"),
+    ]
+    for call, what in cases:
+        with pytest.raises(ValueError, match=what):
+            call()
+    # right sizes on host memory: refused as not on a CUDA device
+    with pytest.raises(ValueError, match="CUDA device"):
+        mg.decode_attn(q, k, k, pt, idx, seq, 16, 0.1, num_partitions=4)
+
+
+def test_binding_shape_checks_accept_what_the_gpu_tests_pass():
+    """Every call pattern of the GPU tests, built on host memory, passes the
+    binding's shape checks and stops only at the device check."""
+    import sys
+    sys.path.insert(0, os.path.dirname(__file__))
+    from mg_testlib import GpuStep
+    from paged_kv_attention_mg_b200 import workload as wl
+    from paged_kv_attention_mg_b200.replicas import shard_kv_heads, take_heads
+
+    def refused_only_for_host_memory(call):
+        with pytest.raises(ValueError, match="must be on a CUDA device"):
+            call()
+
+    decode_cases = [([5, 9, 12], 16, 8), ([1], 16, 8), ([257, 190], 32, 2), ([130, 7, 400], 28, 4)]
+    for lengths, hq, hkv in decode_cases:
+        spec = wl.custom_spec("decode", [L - 1 for L in lengths], lengths, hq, hkv, sum(lengths) + 37, seed=1)
+        step = wl.make_step(spec)
+        g = GpuStep(step, wl.make_layer(step), device="cpu")
+        refused_only_for_host_memory(lambda: g.store())
+        refused_only_for_host_memory(lambda: g.decode(num_partitions=7))
+        refused_only_for_host_memory(lambda: g.store_decode(num_partitions=7))
+        refused_only_for_host_memory(lambda: mg.decode_attn_static_workspace(
+            g.q, g.k_cache, g.v_cache, g.page_table, g.table_idx, g.seq_len, step.max_seq_len, g.scale,
+            num_partitions=7))
+        for r in range(2):  # a tensor-parallel rank's slices
+            kv0, kv1, q0, q1 = shard_kv_heads(hq, hkv, r, 2)
+            refused_only_for_host_memory(lambda: mg.store_decode_attn(
+                take_heads(g.q, q0, q1), take_heads(g.k_new, kv0, kv1), take_heads(g.v_new, kv0, kv1), g.out_loc,
+                take_heads(g.k_cache, kv0, kv1), take_heads(g.v_cache, kv0, kv1), g.page_table, g.table_idx,
+                g.seq_len, step.max_seq_len, g.scale, num_partitions=7))
+    extend_cases = [([0], [1], 16, 8), ([130, 0], [300, 257], 16, 8), ([10, 20], [10, 50], 16, 8),
+                    ([0, 9], [100, 200], 12, 1)]
+    for cached, seq, hq, hkv in extend_cases:
+        spec = wl.custom_spec("extend", cached, seq, hq, hkv, sum(seq) + 37, seed=2)
+        step = wl.make_step(spec)
+        g = GpuStep(step, wl.make_layer(step), device="cpu")
+        refused_only_for_host_memory(lambda: g.extend())
+        refused_only_for_host_memory(lambda: g.extend(out=torch.empty_like(g.q)))
