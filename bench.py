@@ -577,6 +577,11 @@ def run_ours(args):
     step_ms = dist.max(step_ms_local)
     kernel_ms = dist.max(kernel_ms_local)
     events_ms = dist.max(events_ms_local)
+    # every rank draws its own lengths, so the job's work per step is the sum over ranks
+    step_work = dist.sum(float(bench.step_bytes if spec.kind == "decode" else bench.flops))
+    step_tokens = dist.sum(float(bench.tokens_per_step))
+    h2d_bytes = int(dist.sum(float(bench.h2d_bytes)))
+    d2h_bytes = int(dist.sum(float(bench.d2h_bytes)))
 
     # end to end through the public API with host buffers: this step's inputs
     # copied from pinned host memory into the fixed device buffers, the step,
@@ -603,7 +608,7 @@ def run_ours(args):
     hbm, tflops, tflops_sus, peak_src = measured_peaks()
     n = args.gpus
     if spec.kind == "decode":
-        value = n * bench.step_bytes / (step_ms * 1e-3) / 1e9
+        value = step_work / (step_ms * 1e-3) / 1e9
         unit = "GB/s"
         metric = METRIC
         achieved = bench.kernel_bytes / (kernel_ms * 1e-3) / 1e9
@@ -615,18 +620,18 @@ def run_ours(args):
                 "call_us": round(kernel_ms * 1e3, 3), "duration": "timed step / layer calls in it",
                 "call_us_events": round(events_ms * 1e3, 3),
                 "traffic": profiled_traffic(spec.name)}
-        extra = {"tokens_per_s": round(n * bench.tokens_per_step / (step_ms * 1e-3), 1),
+        extra = {"tokens_per_s": round(step_tokens / (step_ms * 1e-3), 1),
                  "frac_of_8tbs_nominal": round(value / n / 8000.0, 4),
                  "frac_of_measured_hbm": round(value / n / hbm, 4)}
     else:
-        value = n * bench.flops / (step_ms * 1e-3) / 1e12
+        value = step_work / (step_ms * 1e-3) / 1e12
         unit = "TFLOP/s"
         metric = EXTEND_METRIC
         achieved = bench.flops / (kernel_ms * 1e-3) / 1e12
         roof = {"bound": "tensor", "kernel": "extend_kernel", "achieved": round(achieved, 1), "peak": tflops,
                 "unit": "TFLOP/s", "frac": round(achieved / tflops, 4),
                 "peak_source": f"{peak_src} dense bf16 (burst)", "traffic": profiled_traffic(spec.name)}
-        extra = {"tokens_per_s": round(n * bench.tokens_per_step / (step_ms * 1e-3), 1),
+        extra = {"tokens_per_s": round(step_tokens / (step_ms * 1e-3), 1),
                  "frac_of_sustained_bf16": round(achieved / tflops_sus, 4) if tflops_sus else None}
 
     cpu = None
@@ -643,11 +648,10 @@ def run_ours(args):
                 "warmup": args.warmup, "ms_per_step": round(step_ms, 4), "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg,
                 **extra, **bench.details(), "roofline": roof, "cpu_baseline": cpu,
-                "e2e": ({"value": round(n * (bench.step_bytes / 1e9 if spec.kind == 'decode' else bench.flops / 1e12)
-                                       / (e2e * 1e-3), 2),
-                         "unit": unit, "ms_per_step": round(e2e, 4), "h2d_bytes_per_step": bench.h2d_bytes,
-                         "d2h_bytes_per_step": bench.d2h_bytes} if e2e else None),
-                "gpu_launches": bench.launches_per_step * args.steps, "clocks": clocks,
+                "e2e": ({"value": round(step_work / (1e9 if spec.kind == 'decode' else 1e12) / (e2e * 1e-3), 2),
+                         "unit": unit, "ms_per_step": round(e2e, 4), "h2d_bytes_per_step": h2d_bytes,
+                         "d2h_bytes_per_step": d2h_bytes} if e2e else None),
+                "gpu_launches": n * bench.launches_per_step * args.steps, "clocks": clocks,
                 "launch": "cuda graph per step" if use_graph else "eager",
                 "kernel_source_digest": source_digest()}
         print(json.dumps(line), flush=True)
