@@ -213,6 +213,7 @@ def test_binding_shape_checks_accept_what_the_gpu_tests_pass():
         refused_only_for_host_memory(lambda: g.store())
         refused_only_for_host_memory(lambda: g.decode(num_partitions=7))
         refused_only_for_host_memory(lambda: g.store_decode(num_partitions=7))
+        refused_only_for_host_memory(lambda: g.extend())  # a decode step as one-token chunks
         refused_only_for_host_memory(lambda: mg.decode_attn_static_workspace(
             g.q, g.k_cache, g.v_cache, g.page_table, g.table_idx, g.seq_len, step.max_seq_len, g.scale,
             num_partitions=7))
