@@ -45,3 +45,25 @@ def test_oracle_sampler_generates_inputs_once_and_fills_its_time_bound():
     es = bench.OracleSampler(ext, wl.make_step(ext), threads=1)
     work, secs, sample, unit = es.sample(0.0)
     assert unit == "TFLOP/s" and work > 0 and "1 requests" in sample and len(es._layers) == 1
+
+
+def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
+    """Under torchrun the oracle arm is rank 0's alone: other ranks print nothing and exit."""
+    import argparse
+    monkeypatch.setenv("RANK", "1")
+    args = argparse.Namespace(workload="tiny_decode", steps=1, warmup=0, gpus=2)
+    assert bench.run_reference(args) is None
+    assert capsys.readouterr().out == ""
+
+
+def test_reference_arm_line_on_a_small_workload(monkeypatch, capsys):
+    import argparse
+    import json
+    monkeypatch.setenv("RANK", "0")
+    args = argparse.Namespace(workload="tiny_decode", steps=2, warmup=1, gpus=1)
+    monkeypatch.setattr(bench, "cpu_threads", lambda: 1)
+    bench.run_reference(args)
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["unit"] == "GB/s" and line["value"] > 0
+    assert line["config"]["workload"] == "tiny_decode" and line["cpu_baseline"]["cores"] == 1
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["steps"] == 2 and line["warmup"] == 1
