@@ -33,11 +33,20 @@
  *     every bf16 tensor must start on a 16-byte boundary.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  All work is
  *     enqueued on it; no entry point synchronises the host, allocates device
- *     memory or keeps state between calls, so calls can be captured in a CUDA
- *     graph (mg_read_device_error excepted, which synchronises).
+ *     memory or keeps state between calls (save the wait limit of
+ *     mg_set_extend_wait_limit), so calls can be captured in a CUDA graph
+ *     (mg_read_device_error excepted, which synchronises).
  *   - The caller owns every buffer.  Inputs are read-only except the pools
  *     in mg_store_kv; outputs are written in full for every real (request,
  *     head) row.
+ *   - The softmax scale must be finite and > 0 (else MG_ERR_INVALID_ARGUMENT):
+ *     the kernels take row maxima of the unscaled scores and scale them after,
+ *     which needs a positive scale.  (scale = 0, whose result is the plain
+ *     mean of the V rows, is therefore not accepted.)
+ *   - page_table_rows is passed with the page table so that the kernels can
+ *     check table_idx against it; decode's num_partitions picks or forces the
+ *     number of workers of its plan (mg_decode_plan).  Extend needs no
+ *     workspace, so it takes none.
  *   - Errors found on the host (null pointer, bad size, unsupported shape,
  *     misalignment, workspace too small) return a status BEFORE anything is
  *     launched.  A failed launch returns MG_ERR_CUDA.  Metadata that can only
@@ -72,7 +81,10 @@ typedef enum mg_status {
 #define MG_DEVERR_SLOT_RANGE 0x1u    /* a slot (out_loc or page-table entry) outside [0, num_slots) */
 #define MG_DEVERR_ROW_RANGE 0x2u     /* table_idx outside [0, page_table_rows) */
 #define MG_DEVERR_LENGTH 0x4u        /* seq_len / cached_len / q_offset inconsistent or beyond hints */
-#define MG_DEVERR_WAIT_TIMEOUT 0x8u  /* a pipeline wait exceeded its iteration limit */
+#define MG_DEVERR_WAIT_TIMEOUT 0x8u  /* a pipeline wait ran past its time limit (mg_set_extend_wait_limit) */
+#define MG_DEVERR_INTERNAL 0x10u     /* a launch invariant failed on the device (a library fault, not
+                                        the caller's metadata): extend's shared memory not 1024-byte
+                                        aligned; the kernel refused to run */
 
 /* Human-readable name of a status. Never NULL. */
 const char *mg_status_string(mg_status status);
@@ -229,7 +241,9 @@ mg_status mg_extend_attn(const void *q, const void *k_cache, const void *v_cache
  *   - Nothing is allocated: no cudaMalloc, cudaFree or allocating library call.
  *   - The first call on each device looks up the array's device address (with
  *     that device current) and caches it; make that first call before any
- *     stream capture.
+ *     stream capture.  The cache is keyed on the CUDA context, so after
+ *     cudaDeviceReset the next call (again before any capture) looks the
+ *     address up anew in the new context.
  *   - All calls share the one array, which keeps the last call's contents.
  *     Nothing in it needs to start at zero (every value is written before it is
  *     read within a call), but calls that overlap on the GPU (e.g. on two
@@ -244,6 +258,32 @@ mg_status mg_decode_attn_static_workspace(const void *q, const void *k_cache, co
                                           int32_t max_seq_len, int32_t num_q_heads, int32_t num_kv_heads,
                                           int32_t head_dim, float scale, int32_t num_partitions, void *out,
                                           void *stream);
+
+/*
+ * mg_set_extend_wait_limit -- the time bound of mg_extend_attn's pipeline
+ * waits, and a fault-injection hook to test what happens when one runs out.
+ * (The pages have no counterpart; their engine bounds its distributed setup
+ * with a timeout, Stage 1 page §配置, distributed_timeout.)
+ *
+ * Inside the extend kernel the load warps, the MMA issuer and the softmax
+ * warps hand tiles to one another through shared-memory barriers.  Every wait
+ * on one gives up after limit_ns nanoseconds: the CTA then records
+ * MG_DEVERR_WAIT_TIMEOUT, raises an abort flag that releases every other
+ * wait, lets the copies and MMAs it already issued land, frees its tensor
+ * memory and returns, so the CUDA context stays usable and
+ * mg_read_device_error reports MG_ERR_DEVICE_TIMEOUT.  In normal operation
+ * every wait is satisfied within microseconds by the same CTA.
+ *
+ *   limit_ns      0 restores the default, 2 000 000 000 (2 s)
+ *   inject_stall  != 0: later extend launches withhold one hand-off (the
+ *                 first score tile of the first Q tile is computed but never
+ *                 signalled), so the waits on it run out -- a fault injected
+ *                 on purpose, for tests; 0 = normal operation (the default)
+ * Process-wide setting, read when mg_extend_attn launches (a launch captured
+ * in a CUDA graph keeps the values it was captured with).  The one piece of
+ * state the library keeps between calls.  Always MG_OK.
+ */
+mg_status mg_set_extend_wait_limit(uint64_t limit_ns, int32_t inject_stall);
 
 /*
  * mg_read_device_error -- synchronise `stream`, return the device error word

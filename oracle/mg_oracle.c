@@ -152,7 +152,7 @@ int oracle_decode(const uint16_t *q, const uint16_t *k_pool, const uint16_t *v_p
     int err = ORACLE_OK;
 #ifdef _OPENMP
     if (num_threads <= 0) num_threads = omp_get_max_threads();
-#pragma omp parallel for schedule(dynamic, 1) num_threads(num_threads)
+#pragma omp parallel for schedule(dynamic, 1) num_threads(num_threads) reduction(max : err)
 #endif
     for (int64_t u = 0; u < units; ++u) {
         const int64_t r = u / num_q_heads, h = u % num_q_heads;
@@ -203,7 +203,7 @@ int oracle_extend(const uint16_t *q, const uint16_t *k_pool, const uint16_t *v_p
     const int64_t units = batch * num_q_heads;
 #ifdef _OPENMP
     if (num_threads <= 0) num_threads = omp_get_max_threads();
-#pragma omp parallel for schedule(dynamic, 1) num_threads(num_threads)
+#pragma omp parallel for schedule(dynamic, 1) num_threads(num_threads) reduction(max : err)
 #endif
     for (int64_t u = 0; u < units; ++u) {
         const int64_t r = u / num_q_heads, h = u % num_q_heads;

@@ -363,8 +363,12 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
             const bool is_v = rr >= kKeys;
             const int sl = __shfl_sync(0xffffffffu, slot, key);
             const __nv_bfloat16 *src = (is_v ? p.v_cache : p.k_cache) + (int64_t)(sl < 0 ? 0 : sl) * head_stride + head_off;
-            if (key == new_key) src = (is_v ? p.v_new : p.k_new) + new_off;
-            cp_async_16(base + (is_v ? 2 * kHalfRows : 0) + swz(key, ch), src, sl < 0 ? 0u : 16u);
+            // the new token's row comes from k_new / v_new whatever its page-table
+            // entry holds, so the fused store writes it even when that entry was
+            // rejected (the key is then masked out of the attention, as a bad slot is)
+            const bool is_new = key == new_key;
+            if (is_new) src = (is_v ? p.v_new : p.k_new) + new_off;
+            cp_async_16(base + (is_v ? 2 * kHalfRows : 0) + swz(key, ch), src, (sl < 0 && !is_new) ? 0u : 16u);
         }
     };
 
@@ -496,9 +500,10 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
                 const float mu1 = mh[nt][1] == -INFINITY ? 0.f : mh[nt][1];
                 const float p0 = fast_exp2(sc[nt][0] - mu0), p1 = fast_exp2(sc[nt][1] - mu1);
                 const float p2 = fast_exp2(sc[nt][2] - mu0), p3 = fast_exp2(sc[nt][3] - mu1);
-                lh[nt][0] += p0 + p2;
-                lh[nt][1] += p1 + p3;
                 const uint32_t X = pack_bf16x2(p0, p1), Y = pack_bf16x2(p2, p3);
+                // the normaliser sums the same bf16-rounded weights the PV product uses
+                lh[nt][0] += bf16x2_lo(X) + bf16x2_lo(Y);
+                lh[nt][1] += bf16x2_hi(X) + bf16x2_hi(Y);
                 const uint32_t xa = __shfl_sync(0xffffffffu, X, s0), xb = __shfl_sync(0xffffffffu, X, s0 + 4);
                 const uint32_t ya = __shfl_sync(0xffffffffu, Y, s0), yb = __shfl_sync(0xffffffffu, Y, s0 + 4);
                 pb[nt][0] = __byte_perm(xa, xb, sel);

@@ -73,7 +73,7 @@ constexpr int kOffK = kOffQ + kQTiles * kTileBytes;
 constexpr int kOffV = kOffK + kKStages * kTileBytes;
 constexpr int kOffIdx = kOffV + kVStages * kTileBytes;
 constexpr int kOffBar = kOffIdx + kIdxRing * kN * 4;
-constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 3 * kQTiles;
+constexpr int kNumBars = 2 + 2 * kKStages + 2 * kVStages + 3 * kQTiles;  // + the abort drain
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffMisc + 16;
 static_assert(kSmemBytes <= 227 * 1024, "extend shared memory over the per-CTA limit");
@@ -94,6 +94,8 @@ struct Params {
     int32_t num_q_heads, num_kv_heads, group;
     int32_t tokens_per_qtile;  // floor(128 / group)
     float scale_log2;
+    uint64_t wait_limit_ns;    // bound of every pipeline wait
+    int32_t inject_stall;      // test hook: withhold the first score tile's hand-off
 };
 
 // UMMA shared-memory descriptor, 128-byte swizzle, sm_100 version bits.
@@ -118,24 +120,31 @@ __host__ __device__ constexpr uint32_t idesc_bf16(bool b_mn_major) {
 }
 
 struct Sync {
-    uint32_t q_full;
+    uint32_t q_full, drain;
     uint32_t k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
     uint32_t s_full[kQTiles], p_full[kQTiles], o_done[kQTiles];
 };
 
-// Waits with a time bound; on timeout records the error, raises the CTA abort
-// flag and returns false.  Once the flag is up every later wait returns false
-// at once, so all roles drain to the final barrier.
-__device__ __forceinline__ bool wait_or_abort_thread(uint32_t bar, uint32_t parity, volatile int *abort_flag) {
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t now;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(now));
+    return now;
+}
+
+// Waits with a time bound (limit_ns, timed from the wait's first check of the
+// clock); on timeout records the error, raises the CTA abort flag and returns
+// false.  Once the flag is up every later wait returns false at once, so all
+// roles drain to the final barrier.
+__device__ __forceinline__ bool wait_or_abort_thread(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                                     uint64_t limit_ns) {
     if (*abort_flag) return false;
     uint64_t t0 = 0;
     for (uint32_t it = 0;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((it & 1023u) == 1023u) {
-            uint64_t now;
-            asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(now));
+            const uint64_t now = global_ns();
             if (t0 == 0) t0 = now;
-            else if (now - t0 > 2000000000ull || *abort_flag) {  // 2 s
+            else if (now - t0 > limit_ns || *abort_flag) {
                 *abort_flag = 1;
                 atomicOr(&g_mg_device_error, MG_DEVERR_WAIT_TIMEOUT);
                 return false;
@@ -144,11 +153,27 @@ __device__ __forceinline__ bool wait_or_abort_thread(uint32_t bar, uint32_t pari
     }
 }
 
+// A bounded wait that ignores the abort flag: used after an abort to let work
+// already in flight (issued MMAs, a TMA load) land before the CTA frees TMEM
+// and exits.  Returns false if the bound ran out.
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+    uint64_t t0 = 0;
+    for (uint32_t it = 0;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 1023u) == 1023u) {
+            const uint64_t now = global_ns();
+            if (t0 == 0) t0 = now;
+            else if (now - t0 > limit_ns) return false;
+        }
+    }
+}
+
 // Warp-uniform form for roles where all 32 lanes wait together: the warp
 // proceeds only if every lane did (tcgen05.ld/st and __syncwarp need the whole
 // warp converged).  The single-thread MMA issuer uses wait_or_abort_thread.
-__device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, volatile int *abort_flag) {
-    const bool ok = wait_or_abort_thread(bar, parity, abort_flag);
+__device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                              uint64_t limit_ns) {
+    const bool ok = wait_or_abort_thread(bar, parity, abort_flag, limit_ns);
     return __all_sync(0xffffffffu, ok);
 }
 
@@ -157,10 +182,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     extern __shared__ __align__(1024) uint8_t smem[];
     const uint32_t sbase = smem_u32(smem);
     if (sbase & 1023u) {  // the swizzled layouts need 1024-byte alignment: refuse, never fault
-        if (threadIdx.x == 0) atomicOr(&g_mg_device_error, MG_DEVERR_WAIT_TIMEOUT);
+        if (threadIdx.x == 0) atomicOr(&g_mg_device_error, MG_DEVERR_INTERNAL);
         return;
     }
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffMisc);
+    const uint64_t lim = p.wait_limit_ns;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + kOffMisc + 4);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -199,6 +225,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     {
         uint32_t b = sbase + kOffBar;
         sy.q_full = b; b += 8;
+        sy.drain = b; b += 8;
         for (int s = 0; s < kKStages; ++s) { sy.k_full[s] = b; b += 8; }
         for (int s = 0; s < kKStages; ++s) { sy.k_empty[s] = b; b += 8; }
         for (int s = 0; s < kVStages; ++s) { sy.v_full[s] = b; b += 8; }
@@ -210,6 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         *abort_flag = 0;
         mbar_init(sy.q_full, 1);
+        mbar_init(sy.drain, 1);
         for (int s = 0; s < kKStages; ++s) {
             mbar_init(sy.k_full[s], kLoaders * 32);  // one arrival per lane of the load warps
             mbar_init(sy.k_empty[s], 1);
@@ -252,7 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float m_run = -INFINITY, l_run = 0.f;
         bool ok = active;
         for (int j = 0; ok && j < n_kv; ++j) {
-            if (!(ok = wait_or_abort(sy.s_full[t], j & 1, abort_flag))) break;
+            if (!(ok = wait_or_abort(sy.s_full[t], j & 1, abort_flag, lim))) break;
             tc_fence_after();
             uint32_t sv[128];
             tmem_ld_32x32b_x32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
@@ -307,16 +335,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const float2 x = ffma2(make_float2(__uint_as_float(sv[cb * 32 + 2 * e]),
                                                        __uint_as_float(sv[cb * 32 + 2 * e + 1])),
                                            sc2, nmu2);
-                    const float2 pp = make_float2(fast_exp2(x.x), fast_exp2(x.y));
-                    rs2 = fadd2(rs2, pp);
-                    pk[e] = pack_bf16x2(pp.x, pp.y);
+                    pk[e] = pack_bf16x2(fast_exp2(x.x), fast_exp2(x.y));
+                    // the row sum adds the same bf16-rounded P the PV product reads
+                    rs2 = fadd2(rs2, make_float2(bf16x2_lo(pk[e]), bf16x2_hi(pk[e])));
                 }
                 tmem_st_32x32b_x16(tS + cb * 16, pk);
             }
             l_run += rs2.x + rs2.y;
             if (warp_need && j > 0) {
                 // O holds the sum up to tile j-1; rescale it once that PV is done
-                if (!(ok = wait_or_abort(sy.o_done[t], (j - 1) & 1, abort_flag))) break;
+                if (!(ok = wait_or_abort(sy.o_done[t], (j - 1) & 1, abort_flag, lim))) break;
                 tc_fence_after();
 #pragma unroll
                 for (int cb = 0; cb < 4; ++cb) {
@@ -338,7 +366,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive(sy.p_full[t]);
         }
         // ---- epilogue: O / l -> bf16 -> out
-        if (ok && wait_or_abort(sy.o_done[t], (n_kv - 1) & 1, abort_flag)) {
+        if (ok && wait_or_abort(sy.o_done[t], (n_kv - 1) & 1, abort_flag, lim)) {
             tc_fence_after();
             const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
             __nv_bfloat16 *dst = p.out + ((int64_t)(qo + i) * p.num_q_heads + kvh * g + head_local) * kHeadDim;
@@ -368,7 +396,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) {
                 constexpr uint32_t idesc_qk = idesc_bf16(false);
                 constexpr uint32_t idesc_pv = idesc_bf16(true);
-                auto issue_s = [&](int t, int j) {
+                auto issue_s = [&](int t, int j, bool signal) {
                     const uint32_t qa = sbase + kOffQ + t * kTileBytes;
                     const uint32_t ka = sbase + kOffK + (j % kKStages) * kTileBytes;
 #pragma unroll
@@ -377,7 +405,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         umma_ss(tmem + col_s(t), sw128_desc(qa + off, 16, 1024), sw128_desc(ka + off, 16, 1024),
                                 idesc_qk, kk > 0);
                     }
-                    umma_commit(sy.s_full[t]);
+                    if (signal) umma_commit(sy.s_full[t]);
                 };
                 auto issue_pv = [&](int t, int j) {
                     const uint32_t va = sbase + kOffV + (j % kVStages) * kTileBytes;
@@ -387,40 +415,48 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 sw128_desc(va + kk * 2048, kHalfBytes, 1024), idesc_pv, (j > 0 || kk > 0));
                     umma_commit(sy.o_done[t]);
                 };
-                bool ok = wait_or_abort_thread(sy.q_full, 0, abort_flag) && wait_or_abort_thread(sy.k_full[0], 0, abort_flag);
+                bool ok = wait_or_abort_thread(sy.q_full, 0, abort_flag, lim) && wait_or_abort_thread(sy.k_full[0], 0, abort_flag, lim);
                 if (ok) {
                     fence_proxy_async_smem();
                     tc_fence_after();
-                    issue_s(0, 0);
-                    if (has_q1) issue_s(1, 0);
+                    // the fault-injection hook withholds Q tile 0's first hand-off, so its
+                    // softmax warps wait for a tile that is never signalled ready
+                    issue_s(0, 0, p.inject_stall == 0);
+                    if (has_q1) issue_s(1, 0, true);
                     umma_commit(sy.k_empty[0]);
                 }
                 for (int j = 0; ok && j < n_kv; ++j) {
                     const int sv = j % kVStages;
-                    if (!(ok = wait_or_abort_thread(sy.v_full[sv], (j / kVStages) & 1, abort_flag))) break;
+                    if (!(ok = wait_or_abort_thread(sy.v_full[sv], (j / kVStages) & 1, abort_flag, lim))) break;
                     fence_proxy_async_smem();  // cp.async (generic proxy) writes -> tensor core reads
-                    if (!(ok = wait_or_abort_thread(sy.p_full[0], j & 1, abort_flag))) break;
+                    if (!(ok = wait_or_abort_thread(sy.p_full[0], j & 1, abort_flag, lim))) break;
                     tc_fence_after();
                     issue_pv(0, j);
                     const bool more = j + 1 < n_kv;
                     if (more) {
                         const int sk = (j + 1) % kKStages;
-                        if (!(ok = wait_or_abort_thread(sy.k_full[sk], ((j + 1) / kKStages) & 1, abort_flag))) break;
+                        if (!(ok = wait_or_abort_thread(sy.k_full[sk], ((j + 1) / kKStages) & 1, abort_flag, lim))) break;
                         fence_proxy_async_smem();
                         tc_fence_after();
-                        issue_s(0, j + 1);
+                        issue_s(0, j + 1, true);
                     }
                     if (has_q1) {
-                        if (!(ok = wait_or_abort_thread(sy.p_full[1], j & 1, abort_flag))) break;
+                        if (!(ok = wait_or_abort_thread(sy.p_full[1], j & 1, abort_flag, lim))) break;
                         tc_fence_after();
                         issue_pv(1, j);
                     }
                     umma_commit(sy.v_empty[sv]);
                     if (more) {
-                        if (has_q1) issue_s(1, j + 1);
+                        if (has_q1) issue_s(1, j + 1, true);
                         umma_commit(sy.k_empty[(j + 1) % kKStages]);
                     }
                 }
+                // before TMEM is freed, every MMA this thread issued must have
+                // completed, also after an abort: one commit tracks them all, and
+                // its wait ignores the abort flag (after a normal run it returns
+                // at once: the softmax warps already waited for the last P V)
+                umma_commit(sy.drain);
+                wait_bounded(sy.drain, 0, lim);
             }
             __syncwarp();
         } else {
@@ -490,11 +526,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int j = 0; j <= n_kv; ++j) {
                 if (j < n_kv) {
                     const int s = j % kKStages;
-                    if (j >= kKStages && !wait_or_abort(sy.k_empty[s], ((j / kKStages) - 1) & 1, abort_flag)) break;
+                    if (j >= kKStages && !wait_or_abort(sy.k_empty[s], ((j / kKStages) - 1) & 1, abort_flag, lim)) break;
                 }
                 if (j >= 1) {
                     const int jv = j - 1, s = jv % kVStages;
-                    if (jv >= kVStages && !wait_or_abort(sy.v_empty[s], ((jv / kVStages) - 1) & 1, abort_flag)) break;
+                    if (jv >= kVStages && !wait_or_abort(sy.v_empty[s], ((jv / kVStages) - 1) & 1, abort_flag, lim)) break;
                 }
                 cp_async_wait<kIdxAhead - 1>();  // entries of tile j (kIdxAhead groups old) landed
                 __syncwarp();
@@ -514,6 +550,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 cp_async_commit();
             }
             cp_async_wait<0>();  // nothing in flight into shared memory at teardown
+            // the Q tiles' TMA load completes on q_full; after an abort nobody may
+            // have waited for it, and it must land before the CTA exits
+            if (li == 0 && lane == 0) wait_bounded(sy.q_full, 0, lim);
         }
     }
 

@@ -21,10 +21,47 @@ constexpr int kMaxDecodeWorkers = 1 << 22;
 
 // Per-device caches, filled on first use.  They are read without the lock,
 // so they are atomics: a thread that sees a value also sees what was done
-// before it was stored (the attributes set, the count read).
+// before it was stored (the attributes set, the count read).  What belongs to
+// a CUDA context (kernel attributes, a module global's address) is keyed on
+// the context's unique id, so a context created after cudaDeviceReset is set
+// up again instead of inheriting the old context's state.
 std::atomic<int> g_sm_count[kMaxDevices];
-std::atomic<bool> g_attr_done[kMaxDevices];
+std::atomic<unsigned long long> g_attr_ctx[kMaxDevices];  // context whose kernel attributes are set
 std::mutex g_attr_mutex;
+
+// mg_set_extend_wait_limit: process-wide, read at each extend launch.
+constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;
+std::atomic<uint64_t> g_extend_wait_limit_ns{kDefaultWaitLimitNs};
+std::atomic<int32_t> g_extend_inject_stall{0};
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long *);
+
+// Unique id of the calling thread's current CUDA context (0: none current, or
+// the driver cannot tell).  Ids are never reused within a process.
+unsigned long long current_context_id() {
+    static const CtxGetCurrentFn get_current = [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            return reinterpret_cast<CtxGetCurrentFn>(ptr);
+        return static_cast<CtxGetCurrentFn>(nullptr);
+    }();
+    static const CtxGetIdFn get_id = [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            return reinterpret_cast<CtxGetIdFn>(ptr);
+        return static_cast<CtxGetIdFn>(nullptr);
+    }();
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+    if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -50,9 +87,10 @@ mg_status sm_count(int &sms) {
 mg_status ensure_kernel_attributes() {
     int dev;
     if (current_device(dev) != MG_OK) return MG_ERR_CUDA;
-    if (g_attr_done[dev].load(std::memory_order_acquire)) return MG_OK;
+    const unsigned long long ctx = current_context_id();
+    if (ctx != 0 && g_attr_ctx[dev].load(std::memory_order_acquire) == ctx) return MG_OK;
     std::lock_guard<std::mutex> lock(g_attr_mutex);
-    if (g_attr_done[dev].load(std::memory_order_relaxed)) return MG_OK;
+    if (ctx != 0 && g_attr_ctx[dev].load(std::memory_order_relaxed) == ctx) return MG_OK;
     if (cudaFuncSetAttribute(decode::decode_kernel<1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              decode::kSmemBytes) != cudaSuccess ||
         cudaFuncSetAttribute(decode::decode_kernel<2, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -63,7 +101,9 @@ mg_status ensure_kernel_attributes() {
                              decode::kSmemBytes) != cudaSuccess)
         return MG_ERR_CUDA;
     if (extend::set_attributes() != cudaSuccess) return MG_ERR_CUDA;
-    g_attr_done[dev].store(true, std::memory_order_release);
+    // the calls above made the device's primary context current if none was
+    const unsigned long long now = current_context_id();
+    if (now != 0) g_attr_ctx[dev].store(now, std::memory_order_release);
     return MG_OK;
 }
 
@@ -328,7 +368,15 @@ mg_status mg_extend_attn(const void *q, const void *k_cache, const void *v_cache
     p.num_kv_heads = num_kv_heads;
     p.group = num_q_heads / num_kv_heads;
     p.scale_log2 = scale * kLog2e;
+    p.wait_limit_ns = g_extend_wait_limit_ns.load(std::memory_order_relaxed);
+    p.inject_stall = g_extend_inject_stall.load(std::memory_order_relaxed);
     return extend::launch(p, static_cast<cudaStream_t>(stream));
+}
+
+mg_status mg_set_extend_wait_limit(uint64_t limit_ns, int32_t inject_stall) {
+    g_extend_wait_limit_ns.store(limit_ns ? limit_ns : kDefaultWaitLimitNs, std::memory_order_relaxed);
+    g_extend_inject_stall.store(inject_stall ? 1 : 0, std::memory_order_relaxed);
+    return MG_OK;
 }
 
 mg_status mg_read_device_error(void *stream, uint32_t *bits_out) {
@@ -361,26 +409,35 @@ namespace {
 constexpr size_t kStaticDecodeWorkspaceBytes = MG_DECODE_STATIC_WORKSPACE_BYTES;
 static __device__ __align__(256) unsigned char g_decode_static_workspace[kStaticDecodeWorkspaceBytes];
 
-std::atomic<void *> g_static_ws_ptr[kMaxDevices];  // read without the lock, like the caches above
+// The array's device address, per device, with the context it belongs to.
+struct StaticWorkspaceAddress {
+    unsigned long long ctx = 0;
+    void *ptr = nullptr;
+};
+StaticWorkspaceAddress g_static_ws[kMaxDevices];  // guarded by g_static_ws_mutex
 std::mutex g_static_ws_mutex;
 
 // The array's device address on the current device.  In host code the
-// array's name is only a host-side stand-in, so the address is looked up once
-// per device, with that device current, and cached.
+// array's name is only a host-side stand-in, so the address is looked up with
+// the device current, once per device and context, and cached.  A module
+// global lives in a context: after cudaDeviceReset the next context holds it
+// at another address, so the cache is keyed on the context's unique id.
 mg_status static_workspace(void *&ptr) {
     int dev;
     if (current_device(dev) != MG_OK) return MG_ERR_CUDA;
-    void *p = g_static_ws_ptr[dev].load(std::memory_order_acquire);
-    if (!p) {
-        std::lock_guard<std::mutex> lock(g_static_ws_mutex);
-        p = g_static_ws_ptr[dev].load(std::memory_order_relaxed);
-        if (!p) {
-            if (cudaGetSymbolAddress(&p, g_decode_static_workspace) != cudaSuccess || p == nullptr)
-                return MG_ERR_CUDA;
-            g_static_ws_ptr[dev].store(p, std::memory_order_release);
-        }
+    std::lock_guard<std::mutex> lock(g_static_ws_mutex);
+    StaticWorkspaceAddress &c = g_static_ws[dev];
+    unsigned long long ctx = current_context_id();
+    if (ctx == 0 || ctx != c.ctx) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_decode_static_workspace) != cudaSuccess || p == nullptr)
+            return MG_ERR_CUDA;
+        ctx = current_context_id();  // the lookup makes the primary context current if none was
+        if (ctx == 0) return MG_ERR_CUDA;
+        c.ctx = ctx;
+        c.ptr = p;
     }
-    ptr = p;
+    ptr = c.ptr;
     return MG_OK;
 }
 

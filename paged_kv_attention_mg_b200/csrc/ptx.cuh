@@ -98,6 +98,9 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&v);
 }
+// the two halves of a packed bf16x2 as floats (exact: bf16 is the top half of an fp32)
+__device__ __forceinline__ float bf16x2_lo(uint32_t x) { return __uint_as_float(x << 16); }
+__device__ __forceinline__ float bf16x2_hi(uint32_t x) { return __uint_as_float(x & 0xFFFF0000u); }
 
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {

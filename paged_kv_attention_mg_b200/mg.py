@@ -31,6 +31,7 @@ DEVERR_SLOT_RANGE = 0x1
 DEVERR_ROW_RANGE = 0x2
 DEVERR_LENGTH = 0x4
 DEVERR_WAIT_TIMEOUT = 0x8
+DEVERR_INTERNAL = 0x10
 
 # name -> (restype, argtypes), the exact list of include/mg.h
 _P, _I32, _I64, _F32, _SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
@@ -48,6 +49,7 @@ SIGNATURES = {
                                       _I32, _I32, _I32, _I32, _F32, _P, _P]),
     "mg_decode_attn_static_workspace": (ctypes.c_int, [_P, _P, _P, _I64, _P, _I32, _I32, _P, _P, _I32, _I32,
                                                        _I32, _I32, _I32, _F32, _I32, _P, _P]),
+    "mg_set_extend_wait_limit": (ctypes.c_int, [ctypes.c_uint64, _I32]),
     "mg_read_device_error": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_uint32)]),
 }
 
@@ -275,6 +277,12 @@ def decode_attn_static_workspace(q: torch.Tensor, k_cache: torch.Tensor, v_cache
         _dev(seq_len, torch.int32, "seq_len"), b, max_seq_len, hq, hkv, d, float(scale), num_partitions,
         _dev(out, torch.bfloat16, "out"), _stream(stream)), "mg_decode_attn_static_workspace")
     return out
+
+
+def set_extend_wait_limit(limit_ns: int = 0, inject_stall: bool = False) -> None:
+    """Bound of extend's pipeline waits (0 = the default 2 s) and the
+    fault-injection hook that withholds one hand-off (tests only)."""
+    _check(load().mg_set_extend_wait_limit(int(limit_ns), 1 if inject_stall else 0), "mg_set_extend_wait_limit")
 
 
 def read_device_error(stream=None) -> int:

@@ -116,29 +116,48 @@ def bf16_ulp(x: np.ndarray) -> np.ndarray:
 
 
 def elementwise_bound(ref: np.ndarray) -> np.ndarray:
-    """The max-abs bound an output element is held to: 1e-2, or one bf16 ulp at
-    |ref| where that is larger.  A bf16 output cannot be closer to an fp64 value
-    than half an ulp in general, and that half ulp alone exceeds 1e-2 once
-    |ref| >= 4 (an attention output over few keys is about one V entry, and V
-    entries drawn from N(0, 1) reach 4 and more); below |ref| = 2 the bound is
-    exactly 1e-2."""
-    return np.maximum(MAX_ABS_TOL, bf16_ulp(ref))
+    """The max-abs bound an output element is held to.
+
+    Every element is held to 1e-2, except where the output's own resolution
+    makes that impossible: a bf16 value is in general half an ulp away from an
+    fp64 one, and half a bf16 ulp exceeds 1e-2 only from |ref| = 4 on (ulp
+    2^-5 there).  For those elements alone the bound is 1e-2 + half an ulp of
+    the reference, i.e. the kernel's result before its final rounding to bf16
+    must still lie within 1e-2.  (Attention over a few keys returns about one
+    V entry, and N(0, 1) V entries reach 4.5 in the larger cases.)"""
+    half = 0.5 * bf16_ulp(ref)
+    return np.where(half > MAX_ABS_TOL, MAX_ABS_TOL + half, MAX_ABS_TOL)
+
+
+# Elements that passed only through the |ref| >= 4 allowance, summed over the
+# session and printed in pytest's terminal summary (tests/conftest.py), so the
+# allowance is visible rather than silent.
+WIDENED = {"checked": 0, "over_plain_bound": 0, "worst_over": 0.0}
 
 
 def assert_matches_oracle(got: torch.Tensor, ref: np.ndarray, what: str = ""):
-    """got: bf16 kernel output (any device); ref: fp64 oracle, NaN rows = not computed."""
+    """got: bf16 kernel output (any device); ref: fp64 oracle, NaN rows = not computed.
+
+    Returns (max |err|, mean |err|, elements above a plain 1e-2)."""
     g = got.detach().to("cpu").to(torch.float64).numpy()
     sel = ~np.isnan(ref).any(axis=-1)
     assert sel.any(), "oracle computed no rows"
     gs, rs = g[sel], ref[sel]
     assert np.isfinite(gs).all(), f"{what}: non-finite kernel output"
     diff = np.abs(gs - rs)
-    excess = diff - elementwise_bound(rs)
+    bound = elementwise_bound(rs)
+    excess = diff - bound
     worst = np.unravel_index(np.argmax(excess), excess.shape)
+    over_plain = int((diff > MAX_ABS_TOL).sum())
     assert excess.max() <= 0, (f"{what}: |err| {diff[worst]:.3e} at |ref| {abs(rs[worst]):.3f} above its bound "
-                               f"{elementwise_bound(rs[worst]):.3e} (max abs err {diff.max():.3e}, mean {diff.mean():.3e})")
+                               f"{bound[worst]:.3e} (max abs err {diff.max():.3e}, mean {diff.mean():.3e}, "
+                               f"{over_plain} elements above a plain 1e-2)")
     assert diff.mean() <= MEAN_ABS_TOL, f"{what}: mean abs err {diff.mean():.3e}"
-    return float(diff.max()), float(diff.mean())
+    WIDENED["checked"] += int(diff.size)
+    WIDENED["over_plain_bound"] += over_plain
+    if over_plain:
+        WIDENED["worst_over"] = max(WIDENED["worst_over"], float(diff.max()))
+    return float(diff.max()), float(diff.mean()), over_plain
 
 
 class GpuStep:

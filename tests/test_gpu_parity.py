@@ -295,6 +295,26 @@ def test_store_decode_flags_out_loc_mismatch():
     assert mg.read_device_error() & mg.DEVERR_LENGTH
 
 
+def test_store_decode_stores_the_new_token_even_if_its_table_entry_is_bad():
+    """The new token's page-table entry (position L-1) outside the pool: the key
+    is flagged and left out of the attention, but out_loc is valid, so the pool
+    slot still receives the new K/V (as mg_store_kv would write it), never the
+    zero fill of a rejected row."""
+    step, data = _custom("decode", [9, 19], [10, 20], 16, 8, seed=43)
+    g = GpuStep(step, data)
+    mg.read_device_error()
+    row = int(step.table_idx[1])
+    g.page_table[row, 19] = g.k_cache.shape[0] + 7
+    out = mg.store_decode_attn(g.q, g.k_new, g.v_new, g.out_loc, g.k_cache, g.v_cache, g.page_table, g.table_idx,
+                               g.seq_len, 20, g.scale)
+    assert mg.read_device_error() & mg.DEVERR_SLOT_RANGE
+    loc = int(step.out_loc[1])
+    assert torch.equal(g.k_cache[loc].cpu().view(torch.int16), data.k_new[1].view(torch.int16))
+    assert torch.equal(g.v_cache[loc].cpu().view(torch.int16), data.v_new[1].view(torch.int16))
+    # request 0 is untouched by request 1's bad entry
+    assert_matches_oracle(out, oracle_decode(step, data, requests=[0]), "request 0 beside a bad entry")
+
+
 # ----------------------------------------------------------------------------- extend
 
 EXTEND_SMALL = [
