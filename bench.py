@@ -61,6 +61,7 @@ from paged_kv_attention_mg_b200 import workload as wl  # noqa: E402
 
 METRIC = "paged decode-attention KV GB/s (% of HBM peak) and decode tokens/s, 1 B200"
 EXTEND_METRIC = "chunked-prefill extend attention TFLOP/s (unmasked QK^T + PV flops), 1 B200"
+L2_BYTES = 126 * 1024 * 1024  # B200 L2; a decode step reading less than 4x this is timed with an L2 flush
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 KERNEL_SOURCES = ["include/mg.h", "paged_kv_attention_mg_b200/csrc/mg.cu",
@@ -84,6 +85,8 @@ def parse_args():
     ap.add_argument("--no-graph", action="store_true", help="launch every step eagerly instead of a CUDA graph")
     ap.add_argument("--unfused", action="store_true", help="separate KV-store launch before each decode")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="bound of the cpu_baseline sample")
+    ap.add_argument("--cpu-seconds-1thread", type=float, default=8.0,
+                    help="bound of the cpu_baseline's one-thread sample (0 skips it)")
     ap.add_argument("--soak-seconds", type=float, default=1.5,
                     help="extra untimed warm-up so the clock sampler sees the GPU under load")
     return ap.parse_args()
@@ -261,30 +264,56 @@ class DecodeBench:
         self.fused = fused
         self.spec, self.step, self.device = spec, step, device
         self.layers = make_layers(step, spec.num_layers, device)
-        self.meta = {n: getattr(step, n).to(device) for n in ("page_table", "table_idx", "seq_len", "out_loc")}
-        self.meta_host = {n: getattr(step, n).pin_memory() for n in ("page_table", "table_idx", "seq_len",
-                                                                      "out_loc")}
+        # shared-prefix workloads: groups of requests read their common prefix once
+        # (mg_decode_attn_shared_prefix after a separate store: the fused store
+        # runs without groups)
+        self.shared = step.group_first is not None
+        self.fused = fused and not self.shared
+        names = ("page_table", "table_idx", "seq_len", "out_loc") + (("group_first", "prefix_len") if self.shared
+                                                                      else ())
+        self.meta = {n: getattr(step, n).to(device) for n in names}
+        self.meta_host = {n: getattr(step, n).pin_memory() for n in names}
         self.max_seq_len = step.max_seq_len
         self.partitions = partitions
         B, hq, hkv = step.batch, spec.num_q_heads, spec.num_kv_heads
         self.workers, self.slots = mg.decode_plan(B, hkv, self.max_seq_len, partitions)
-        ws = mg.decode_workspace_bytes(B, hq, hkv, self.max_seq_len, partitions)
+        if self.shared:
+            ng = int(step.prefix_len.numel())
+            ws = mg.decode_shared_prefix_workspace_bytes(B, ng, hq, hkv, self.max_seq_len, partitions)
+        else:
+            ws = mg.decode_workspace_bytes(B, hq, hkv, self.max_seq_len, partitions)
         self.workspace = torch.empty(max(ws, 16), dtype=torch.uint8, device=device)
         pack_io(self, (B, hq, spec.head_dim))
         L = step.seq_len.tolist()
-        self.decode_bytes = rf.decode_bytes(L, hq, hkv, spec.head_dim)
+        if self.shared:
+            self.decode_bytes = rf.decode_bytes_shared_prefix(L, step.group_first.tolist(), step.prefix_len.tolist(),
+                                                              hq, hkv, spec.head_dim)
+        else:
+            self.decode_bytes = rf.decode_bytes(L, hq, hkv, spec.head_dim)
         self.store_bytes = rf.store_bytes(step.num_new_tokens, hkv, spec.head_dim)
         self.step_bytes = spec.num_layers * (self.decode_bytes + self.store_bytes)
         self.tokens_per_step = B
         # per layer: (store,) decode workers, merge
-        self.launches_per_step = spec.num_layers * (2 if fused else 3)
-        # what one timed call moves: the fused call also does the store
-        self.kernel_bytes = self.decode_bytes + (self.store_bytes if fused else 0)
+        self.launches_per_step = spec.num_layers * (2 if self.fused else 3)
+        # what one timed layer call moves: the store and the decode (fused or not;
+        # the call's duration is the step time over its layer calls)
+        self.kernel_bytes = self.decode_bytes + self.store_bytes
         self.h2d_bytes, self.d2h_bytes = io_bytes(self)
         self.ev = None
 
     def layer(self, lay, out, meta, events=None):
         mg = self.mg
+        if self.shared:
+            mg.store_kv(lay["k_new"], lay["v_new"], meta["out_loc"], lay["k_cache"], lay["v_cache"])
+            if events:
+                events[0].record()
+            mg.decode_attn_shared_prefix(lay["q"], lay["k_cache"], lay["v_cache"], meta["page_table"],
+                                         meta["table_idx"], meta["seq_len"], meta["group_first"],
+                                         meta["prefix_len"], self.max_seq_len, self.spec.scale,
+                                         num_partitions=self.partitions, out=out, workspace=self.workspace)
+            if events:
+                events[1].record()
+            return
         if self.fused:  # store + decode in one decode launch
             if events:
                 events[0].record()
@@ -323,7 +352,14 @@ class DecodeBench:
         return self.decode_bytes
 
     def details(self):
-        return {"decode_workers": self.workers, "store": "fused into decode" if self.fused else "separate launch"}
+        d = {"decode_workers": self.workers, "store": "fused into decode" if self.fused else "separate launch"}
+        if self.shared:
+            d["shared_prefix"] = {"groups": int(self.step.prefix_len.numel()),
+                                  "prefix_len": sorted(set(self.step.prefix_len.tolist())),
+                                  "bytes_if_unshared": rf.decode_bytes(self.step.seq_len.tolist(),
+                                                                       self.spec.num_q_heads, self.spec.num_kv_heads,
+                                                                       self.spec.head_dim)}
+        return d
 
 
 class ExtendBench:
@@ -364,17 +400,38 @@ class ExtendBench:
         return {}
 
 
+def decode_needs_flush(spec, step) -> bool:
+    """A decode step whose K/V reads are under 4x the L2 is timed with an L2
+    flush between steps (larger ones stream past the L2 by themselves)."""
+    if step.group_first is not None:
+        per_layer = rf.decode_bytes_shared_prefix(step.seq_len.tolist(), step.group_first.tolist(),
+                                                  step.prefix_len.tolist(), spec.num_q_heads, spec.num_kv_heads,
+                                                  spec.head_dim)
+    else:
+        per_layer = rf.decode_bytes(step.seq_len.tolist(), spec.num_q_heads, spec.num_kv_heads, spec.head_dim)
+    return spec.num_layers * per_layer < 4 * L2_BYTES
+
+
 def workload_config(spec, step, n_gpus: int) -> dict:
     """The `config` of the JSON line: the workload and how it is run, the same
     for this library's arm and the reference arm."""
     common = {"workload": spec.name, "batch": step.batch, "layers": spec.num_layers, "q_heads": spec.num_q_heads,
               "kv_heads": spec.num_kv_heads, "head_dim": spec.head_dim, "pool_slots": spec.num_slots}
     if spec.kind == "decode":
-        per_layer = rf.decode_bytes(step.seq_len.tolist(), spec.num_q_heads, spec.num_kv_heads, spec.head_dim)
+        if step.group_first is not None:
+            per_layer = rf.decode_bytes_shared_prefix(step.seq_len.tolist(), step.group_first.tolist(),
+                                                      step.prefix_len.tolist(), spec.num_q_heads,
+                                                      spec.num_kv_heads, spec.head_dim)
+        else:
+            per_layer = rf.decode_bytes(step.seq_len.tolist(), spec.num_q_heads, spec.num_kv_heads, spec.head_dim)
         common.update({"mean_seq_len": round(float(step.seq_len.double().mean()), 1),
-                       "max_seq_len": step.max_seq_len,
-                       "l2": f"inputs larger than L2: {spec.num_layers} per-layer pools, "
-                             f"{spec.num_layers * per_layer / 1e9:.2f} GB read per step"})
+                       "max_seq_len": step.max_seq_len})
+        if decode_needs_flush(spec, step):
+            common["l2"] = (f"L2 flushed between timed steps (256 MB write): {per_layer / 1e6:.0f} MB read per "
+                            f"step, under 4x the L2")
+        else:
+            common["l2"] = (f"inputs larger than L2: {spec.num_layers} per-layer pools, "
+                            f"{spec.num_layers * per_layer / 1e9:.2f} GB read per step")
     else:
         n = step.seq_len - step.cached_len
         common.update({"new_tokens": int(n.sum()), "mean_cached_len": round(float(step.cached_len.double().mean()), 1),
@@ -418,7 +475,13 @@ class OracleSampler:
         spec, step = self.spec, self.step
         work, total_t, calls = 0, 0.0, 0
         if spec.kind == "decode":
-            per_layer = rf.decode_bytes(step.seq_len.tolist(), spec.num_q_heads, spec.num_kv_heads, spec.head_dim)
+            if step.group_first is not None:  # the same algorithmic bytes as the GPU arm: a shared prefix once
+                per_layer = rf.decode_bytes_shared_prefix(step.seq_len.tolist(), step.group_first.tolist(),
+                                                          step.prefix_len.tolist(), spec.num_q_heads,
+                                                          spec.num_kv_heads, spec.head_dim)
+            else:
+                per_layer = rf.decode_bytes(step.seq_len.tolist(), spec.num_q_heads, spec.num_kv_heads,
+                                            spec.head_dim)
             while calls == 0 or total_t < seconds:
                 q, k, v = self._inputs(self._next)
                 self._next = (self._next + 1) % self.max_layers
@@ -443,6 +506,33 @@ class OracleSampler:
             work += rf.extend_flops([c[r]], [s[r]], spec.num_q_heads, spec.head_dim)
             calls += 1
         return work, total_t, f"{calls} requests of one layer (of {step.batch}, taken in turn)", "TFLOP/s"
+
+
+def cpu_model() -> str:
+    """The host CPU's model name (first processor in /proc/cpuinfo)."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def cpu_baseline(spec, step, seconds: float, seconds_1thread: float) -> dict:
+    """The oracle on this host: all cores (the reported value), then one thread."""
+    threads = cpu_threads()
+    w, secs, sample, unit = OracleSampler(spec, step, threads).sample(seconds)
+    scale = 1e9 if unit == "GB/s" else 1e12
+    line = {"value": round(w / secs / scale, 4), "unit": unit, "cores": threads, "kind": "oracle",
+            "sample": sample, "seconds": round(secs, 2), "cpu_model": cpu_model()}
+    if seconds_1thread > 0:
+        w1, s1, sample1, _ = OracleSampler(spec, step, 1).sample(seconds_1thread)
+        line.update({"value_1thread": round(w1 / s1 / scale, 4), "sample_1thread": sample1,
+                     "seconds_1thread": round(s1, 2)})
+    return line
 
 
 def cpu_threads():
@@ -495,7 +585,7 @@ def run_ours(args):
     bench = (DecodeBench if spec.kind == "decode" else ExtendBench)(spec, step, device, args.partitions,
                                                                      fused=not args.unfused)
     flush = None
-    if spec.kind == "extend":
+    if spec.kind == "extend" or decode_needs_flush(spec, step):
         flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
     torch.cuda.synchronize()
 
@@ -538,7 +628,7 @@ def run_ours(args):
     # the instrumented copy is replayed afterwards for the per-call events.
     # The extend step also holds the L2 flush, timed by its own events and
     # taken out, so that step runs instrumented.
-    run_step = run_plain if spec.kind == "decode" else run_timed
+    run_step = run_plain if flush is None else run_timed
     sampler = ClockSampler(dist.local)
     sampler.start()
     # warm-up (W steps) plus a short soak so clocks are sampled under load
@@ -577,6 +667,11 @@ def run_ours(args):
     step_ms = dist.max(step_ms_local)
     kernel_ms = dist.max(kernel_ms_local)
     events_ms = dist.max(events_ms_local)
+    # the roofline is per GPU: every rank's own work over its own call time (ranks
+    # draw their own lengths), and the line reports the lowest rank's figure
+    local_work = bench.kernel_bytes if spec.kind == "decode" else bench.flops
+    achieved_local = local_work / (kernel_ms_local * 1e-3) / (1e9 if spec.kind == "decode" else 1e12)
+    achieved_min = dist.min(achieved_local)
     # every rank draws its own lengths, so the job's work per step is the sum over ranks
     step_work = dist.sum(float(bench.step_bytes if spec.kind == "decode" else bench.flops))
     step_tokens = dist.sum(float(bench.tokens_per_step))
@@ -611,9 +706,11 @@ def run_ours(args):
         value = step_work / (step_ms * 1e-3) / 1e9
         unit = "GB/s"
         metric = METRIC
-        achieved = bench.kernel_bytes / (kernel_ms * 1e-3) / 1e9
+        achieved = achieved_min
         kname = ("decode_kernel<fused store> + decode_merge_kernel (one mg_store_decode_attn call)" if bench.fused
-                 else "decode_kernel + decode_merge_kernel (one mg_decode_attn call)")
+                 else "store_kv_kernel + decode_kernel<shared prefix> + decode_merge_kernel (mg_store_kv + "
+                      "mg_decode_attn_shared_prefix)" if bench.shared
+                 else "store_kv_kernel + decode_kernel + decode_merge_kernel (mg_store_kv + mg_decode_attn)")
         roof = {"bound": "hbm", "kernel": kname,
                 "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s", "frac": round(achieved / hbm, 4),
                 "peak_source": f"{peak_src} HBM copy bandwidth",
@@ -627,7 +724,7 @@ def run_ours(args):
         value = step_work / (step_ms * 1e-3) / 1e12
         unit = "TFLOP/s"
         metric = EXTEND_METRIC
-        achieved = bench.flops / (kernel_ms * 1e-3) / 1e12
+        achieved = achieved_min
         roof = {"bound": "tensor", "kernel": "extend_kernel", "achieved": round(achieved, 1), "peak": tflops,
                 "unit": "TFLOP/s", "frac": round(achieved / tflops, 4),
                 "peak_source": f"{peak_src} dense bf16 (burst)", "traffic": profiled_traffic(spec.name)}
@@ -636,11 +733,7 @@ def run_ours(args):
 
     cpu = None
     if dist.rank == 0 and n == 1 and not args.no_cpu_baseline:
-        threads = cpu_threads()
-        w, secs, sample, cunit = OracleSampler(spec, step, threads).sample(args.cpu_seconds)
-        cval = w / secs / (1e9 if cunit == "GB/s" else 1e12)
-        cpu = {"value": round(cval, 4), "unit": cunit, "cores": threads, "kind": "oracle",
-               "sample": sample, "seconds": round(secs, 2)}
+        cpu = cpu_baseline(spec, step, args.cpu_seconds, args.cpu_seconds_1thread)
 
     if dist.rank == 0:
         cfg = workload_config(spec, step, n)

@@ -11,6 +11,7 @@
  *   mg_decode_attn  one query token per request against its paged history
  *                   (balanced split-KV kernel + merge kernel);
  *   mg_store_decode_attn  the two above fused into one decode launch;
+ *   mg_decode_attn_shared_prefix  decode reading a shared prefix once per group;
  *   mg_extend_attn  a chunk of new tokens per request (chunked prefill),
  *                   causal over cached_len + i, on tcgen05 tensor cores.
  *
@@ -191,6 +192,46 @@ mg_status mg_store_decode_attn(const void *q, const void *k_new, const void *v_n
                                int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, float scale,
                                int32_t num_partitions, void *out, void *workspace, size_t workspace_bytes,
                                void *stream);
+
+/*
+ * mg_decode_attn_shared_prefix -- mg_decode_attn for a batch in which groups
+ * of requests share the beginning of their history, as a radix prefix cache
+ * hands out (Mini-SGLang tag page, KV Cache post: paged KV with prefix reuse,
+ * RadixPrefixCache): the shared tokens are stored once in the pool and every
+ * member's page-table row begins with the same slots.  The result is exactly
+ * mg_decode_attn's; the shared prefix's K/V rows are read from HBM once per
+ * group and KV head, for all the group's q heads, instead of once per request.
+ *
+ *   requests group_first[G] .. group_first[G+1]-1 form group G (consecutive
+ *   in the batch; group_first[0] = 0, group_first[num_groups] = batch, non-
+ *   decreasing), and share the first P = prefix_len[G] page-table entries:
+ *     page_table[table_idx[r]][j] == page_table[table_idx[group_first[G]]][j]
+ *     for every member r and j < P   (the caller's guarantee; not checked)
+ *   For each group and KV head, one pass over keys [0, P) of the first
+ *   member's row serves the q heads of all members; each request then
+ *   attends to its own keys [P, seq_len[r]); the merge kernel combines the
+ *   two log-sum-exp partials of every (request, q head).
+ *
+ *   group_first   [num_groups + 1] int32;  prefix_len [num_groups] int32
+ *   A group needs 0 <= P <= seq_len[r] - 1 for every member (the new token is
+ *   the request's own) and at most 16 / (num_q_heads / num_kv_heads) members;
+ *   P = 0 or a single member is allowed (no sharing).  A group that breaks
+ *   these rules sets MG_DEVERR_LENGTH and its members are served as plain
+ *   requests (the result stays exact).
+ *   workspace     >= mg_decode_shared_prefix_workspace_bytes(...) bytes
+ * Every other argument is mg_decode_attn's.  Two kernels on `stream`.
+ */
+size_t mg_decode_shared_prefix_workspace_bytes(int32_t batch, int32_t num_groups, int32_t num_q_heads,
+                                               int32_t num_kv_heads, int32_t head_dim, int32_t max_seq_len,
+                                               int32_t num_partitions);
+mg_status mg_decode_attn_shared_prefix(const void *q, const void *k_cache, const void *v_cache, int64_t num_slots,
+                                       const int32_t *page_table, int32_t page_table_rows,
+                                       int32_t page_table_stride, const int32_t *table_idx,
+                                       const int32_t *seq_len, int32_t batch, int32_t max_seq_len,
+                                       const int32_t *group_first, const int32_t *prefix_len,
+                                       int32_t num_groups, int32_t num_q_heads, int32_t num_kv_heads,
+                                       int32_t head_dim, float scale, int32_t num_partitions, void *out,
+                                       void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * mg_extend_attn -- chunked-prefill ("extend") attention over the paged pool

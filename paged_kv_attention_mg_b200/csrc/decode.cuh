@@ -93,8 +93,17 @@ struct Params {
     const int32_t *out_loc;
     __nv_bfloat16 *k_store;  // the pools, writable
     __nv_bfloat16 *v_store;
-    float *part_lse;  // [slots, group]
-    float *part_o;    // [slots, group, 128]
+    float *part_lse;  // [slots, rows_per_slot]
+    float *part_o;    // [slots, rows_per_slot, 128]
+    // shared-prefix (cascade) mode, else num_groups == 0: requests
+    // group_first[G] .. group_first[G+1]-1 share the first prefix_len[G]
+    // page-table entries, whose K/V rows are read once for all their q heads
+    const int32_t *group_first;  // [num_groups + 1]
+    const int32_t *prefix_len;   // [num_groups]
+    int32_t num_groups;
+    int32_t max_members;    // members one shared prefix serves (16 / group)
+    int32_t rows_per_slot;  // partial rows per workspace slot: group, or 16 in cascade mode
+    int32_t num_vreqs;      // virtual requests: batch (+ num_groups in cascade mode)
     int64_t num_slots;
     int32_t pt_rows, pt_stride;
     int32_t batch, num_q_heads, num_kv_heads, group;
@@ -115,6 +124,82 @@ __device__ __forceinline__ int64_t request_units(const Params &p, int r, int &L,
     if (row < 0 || row >= p.pt_rows) { bad |= MG_DEVERR_ROW_RANGE; return 0; }
     if (L < 1 || L > p.pt_stride || L > p.max_seq_len) { bad |= MG_DEVERR_LENGTH; return 0; }
     return (int64_t)((L + kKeys - 1) / kKeys) * p.num_kv_heads;
+}
+
+// ---- shared-prefix (cascade) mode: virtual requests.
+// A virtual request is a key range [k0, k1) of one page-table row attended by
+// the q heads of requests r0 .. r0 + m - 1.  Virtual requests 0 .. G-1 are the
+// groups' shared prefixes (keys [0, P) of the first member's row, all members'
+// q heads, m <= max_members); G .. G+B-1 are the requests, each over the keys
+// after its group's prefix.  A group that is malformed (members outside the
+// batch, too many members, or a prefix not shorter than every member's
+// length) is flagged and its members are served as plain requests.
+struct VReq {
+    int row, k0, k1, r0, m;
+    bool grouped;  // a request whose prefix is served by its group's virtual request
+};
+
+// The shared prefix length of group grp if the group is well formed and has
+// one (else 0).
+__device__ __forceinline__ int group_prefix(const Params &p, int grp, unsigned &bad) {
+    const int P = __ldg(p.prefix_len + grp);
+    if (P == 0) return 0;
+    const int f0 = __ldg(p.group_first + grp), f1 = __ldg(p.group_first + grp + 1);
+    bool ok = P > 0 && f0 >= 0 && f1 <= p.batch && f1 > f0 && f1 - f0 <= p.max_members;
+    if (ok) {
+        const int row0 = __ldg(p.table_idx + f0);
+        ok = row0 >= 0 && row0 < p.pt_rows;
+        for (int r = f0; ok && r < f1; ++r) {
+            const int L = __ldg(p.seq_len + r);
+            ok = L >= 1 && L <= p.pt_stride && L <= p.max_seq_len && P <= L - 1;
+        }
+    }
+    if (!ok) { bad |= MG_DEVERR_LENGTH; return 0; }
+    return P;
+}
+
+// The group whose member range holds request r, or -1 (group_first is
+// non-decreasing in a well-formed call; anything else leaves r ungrouped).
+__device__ __forceinline__ int group_of(const Params &p, int r) {
+    int lo = 0, hi = p.num_groups - 1;
+    while (lo < hi) {  // last group with group_first <= r
+        const int mid = (lo + hi + 1) >> 1;
+        if (__ldg(p.group_first + mid) <= r) lo = mid; else hi = mid - 1;
+    }
+    if (p.num_groups <= 0) return -1;
+    return (__ldg(p.group_first + lo) <= r && r < __ldg(p.group_first + lo + 1)) ? lo : -1;
+}
+
+// Units of virtual request v (cascade mode), and its description.
+__device__ __forceinline__ int64_t vreq_units(const Params &p, int v, VReq &vr, unsigned &bad) {
+    vr.m = 1;
+    vr.grouped = false;
+    vr.k0 = 0;
+    if (v < p.num_groups) {
+        const int P = group_prefix(p, v, bad);
+        if (P == 0) { vr.k1 = 0; return 0; }
+        vr.r0 = __ldg(p.group_first + v);
+        vr.m = __ldg(p.group_first + v + 1) - vr.r0;
+        vr.row = __ldg(p.table_idx + vr.r0);
+        vr.k1 = P;
+        return (int64_t)((P + kKeys - 1) / kKeys) * p.num_kv_heads;
+    }
+    const int r = v - p.num_groups;
+    int L;
+    const int64_t u = request_units(p, r, L, vr.row, bad);
+    vr.r0 = r;
+    vr.k1 = L;
+    if (u == 0) return 0;
+    const int grp = group_of(p, r);
+    if (grp >= 0) {
+        unsigned ignore = 0;  // flagged where the group's own virtual request is resolved
+        const int P = group_prefix(p, grp, ignore);
+        if (P > 0) {
+            vr.k0 = P;
+            vr.grouped = true;
+        }
+    }
+    return (int64_t)((L - vr.k0 + kKeys - 1) / kKeys) * p.num_kv_heads;
 }
 
 // First unit of worker w out of W over `total` units (the host guarantees
@@ -146,10 +231,14 @@ __device__ __forceinline__ int64_t block_scan_excl(int64_t v, int64_t &excl, int
     return total;
 }
 
-// The walk along a worker's units: pair (r, kvh), tile t of the pair.
+// The walk along a worker's units: pair (r, kvh), tile t of the pair.  In
+// cascade mode r is a virtual request, whose keys start at k0 and whose q
+// rows belong to requests r0 .. r0 + m - 1.
 struct Cursor {
     int r, kvh, t, tiles, L, row;
     int next_L, next_row;  // metadata of request r + 1, loaded ahead of the boundary
+    int k0, r0, m;         // cascade mode (else 0, r, 1)
+    bool grouped;
 };
 
 // What the pipeline stages need to know about one tile.
@@ -157,6 +246,8 @@ struct TileDesc {
     int r, kvh, t, tiles, L, row;
     unsigned valid;  // bit i: key i has an accepted slot (set when the tile is issued)
     int store_slot;  // fused store: out_loc[r] when this is the pair's last tile
+    int k0, r0, m;   // first key of the pair's range, first request and count of its q rows
+    int grouped;
 };
 
 __device__ __forceinline__ bool metadata_ok(const Params &p, int L, int row) {
@@ -171,42 +262,71 @@ __device__ __forceinline__ void cursor_prefetch_next(const Params &p, Cursor &c)
 }
 
 // Position the cursor on the first request >= c.r that owns units.
+template <bool CASCADE>
 __device__ __forceinline__ void cursor_load_request(const Params &p, Cursor &c) {
     for (;;) {
         unsigned bad = 0;
-        const int64_t u = request_units(p, c.r, c.L, c.row, bad);
+        int64_t u;
+        if constexpr (CASCADE) {
+            VReq vr;
+            u = vreq_units(p, c.r, vr, bad);
+            c.row = vr.row; c.L = vr.k1; c.k0 = vr.k0; c.r0 = vr.r0; c.m = vr.m; c.grouped = vr.grouped;
+        } else {
+            u = request_units(p, c.r, c.L, c.row, bad);
+            c.k0 = 0; c.r0 = c.r; c.m = 1; c.grouped = false;
+        }
         if (u > 0) {
-            c.tiles = (c.L + kKeys - 1) / kKeys;
-            cursor_prefetch_next(p, c);
+            c.tiles = (c.L - c.k0 + kKeys - 1) / kKeys;
+            if constexpr (!CASCADE) cursor_prefetch_next(p, c);
             return;
         }
         ++c.r;  // zero-unit (rejected) request: it owns no units, skip it
-        if (c.r >= p.batch) { c.tiles = 1; c.L = 0; return; }
+        if (c.r >= p.num_vreqs) { c.tiles = 1; c.L = 0; c.k0 = 0; return; }
     }
 }
 
+template <bool CASCADE>
 __device__ __forceinline__ void cursor_advance(const Params &p, Cursor &c) {
     if (++c.t < c.tiles) return;
     c.t = 0;
     if (++c.kvh < p.num_kv_heads) return;
     c.kvh = 0;
     ++c.r;
-    if (c.r >= p.batch) return;
+    if (c.r >= p.num_vreqs) return;
+    if constexpr (CASCADE) {
+        cursor_load_request<true>(p, c);
+        return;
+    }
     if (metadata_ok(p, c.next_L, c.next_row)) {  // the common case: no stall at the boundary
         c.L = c.next_L;
         c.row = c.next_row;
+        c.r0 = c.r;
         c.tiles = (c.L + kKeys - 1) / kKeys;
         cursor_prefetch_next(p, c);
     } else {
-        cursor_load_request(p, c);
+        cursor_load_request<false>(p, c);
     }
 }
 
-// NT: n-tiles of 8 GQA heads (1 for g <= 8, 2 for g <= 16).
+// Units of virtual request v (a request, outside cascade mode).
+template <bool CASCADE>
+__device__ __forceinline__ int64_t units_of(const Params &p, int v, unsigned &bad) {
+    if constexpr (CASCADE) {
+        VReq vr;
+        return vreq_units(p, v, vr, bad);
+    } else {
+        int L, row;
+        return request_units(p, v, L, row, bad);
+    }
+}
+
+// NT: n-tiles of 8 q rows (1 for g <= 8, 2 for g <= 16 or cascade mode).
 // FUSED: the KV store of the step's new tokens happens in the same launch.
-template <int NT, bool FUSED>
+// CASCADE: shared-prefix mode (virtual requests, partial outputs merged).
+template <int NT, bool FUSED, bool CASCADE = false>
 __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
     decode_kernel(const Params p) {
+    static_assert(!(FUSED && CASCADE), "the fused store runs without shared prefixes");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     __shared__ __align__(16) int idx_ring[kWarps][kDescRing][kKeys];
@@ -221,7 +341,7 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int W = p.num_workers;
     const int w = blockIdx.x * kWarps + warp;
-    const int nchunks = (p.batch + kScanChunk - 1) / kScanChunk;
+    const int nchunks = (p.num_vreqs + kScanChunk - 1) / kScanChunk;
     griddep_launch_dependents();  // the merge kernel may launch and wait on us
     griddep_wait();               // inputs written by the previous kernel (e.g. the KV store)
 
@@ -233,8 +353,7 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int r = ch * kScanChunk + tid * 4 + i;
-            int L, row;
-            if (r < p.batch) v += request_units(p, r, L, row, bad);
+            if (r < p.num_vreqs) v += units_of<CASCADE>(p, r, bad);
         }
         int64_t excl;
         const int64_t tot = block_scan_excl(v, excl, sh_scan);
@@ -260,9 +379,8 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
             const int r0 = ch * kScanChunk + tid * 4;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                int L, row;
                 unsigned dummy = 0;
-                u[i] = r0 + i < p.batch ? request_units(p, r0 + i, L, row, dummy) : 0;
+                u[i] = r0 + i < p.num_vreqs ? units_of<CASCADE>(p, r0 + i, dummy) : 0;
                 v += u[i];
             }
             int64_t excl;
@@ -271,7 +389,7 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int r = r0 + i;
-                if (r < p.batch) {
+                if (r < p.num_vreqs) {
                     if (blockIdx.x == 0) p.prefix[r] = pre;
 #pragma unroll
                     for (int k = 0; k < kWarps; ++k) {
@@ -285,7 +403,7 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
                 pre += u[i];
             }
         }
-        if (blockIdx.x == 0 && tid == 0) p.prefix[p.batch] = T;
+        if (blockIdx.x == 0 && tid == 0) p.prefix[p.num_vreqs] = T;
     }
     __syncthreads();
 
@@ -300,7 +418,7 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
 
     Cursor cur;  // position of the next tile whose page-table entries are fetched
     cur.r = sh_start_r[warp];
-    cursor_load_request(p, cur);
+    cursor_load_request<CASCADE>(p, cur);
     {
         const int64_t off = ub - sh_start_prefix[warp];
         cur.kvh = (int)(off / cur.tiles);
@@ -318,18 +436,19 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
                 TileDesc d;
                 d.r = cur.r; d.kvh = cur.kvh; d.t = cur.t; d.tiles = cur.tiles; d.L = cur.L; d.row = cur.row;
                 d.valid = 0; d.store_slot = -1;
+                d.k0 = cur.k0; d.r0 = cur.r0; d.m = cur.m; d.grouped = cur.grouped;
                 my_desc[e] = d;
                 if (FUSED && cur.t == cur.tiles - 1)  // the pair's last tile holds the new token
                     cp_async_4(smem_u32(&my_desc[e].store_slot), p.out_loc + cur.r);
             }
-            const int key = cur.t * kKeys + lane;
+            const int key = cur.k0 + cur.t * kKeys + lane;
             if (lane < kKeys) {
                 if (key < cur.L)
                     cp_async_4(smem_u32(&my_idx[e][lane]), p.page_table + (int64_t)cur.row * p.pt_stride + key);
                 else
                     my_idx[e][lane] = -1;
             }
-            cursor_advance(p, cur);
+            cursor_advance<CASCADE>(p, cur);
         }
     };
     // Issue stage: read tile j's entries, check them, gather its 16 K and 16 V
@@ -338,7 +457,7 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
         const int e = j % kDescRing, stage = j % kStages;
         const TileDesc d = my_desc[e];
         int slot = -1;
-        if (lane < kKeys && d.t * kKeys + lane < d.L) {
+        if (lane < kKeys && d.k0 + d.t * kKeys + lane < d.L) {
             slot = my_idx[e][lane];
             if (slot < 0 || (int64_t)slot >= p.num_slots) {
                 atomicOr(&g_mg_device_error, MG_DEVERR_SLOT_RANGE);
@@ -407,9 +526,17 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
                 const int hl = nt * 8 + (lane >> 2);
-                const bool hv = hl < g;
-                const __nv_bfloat16 *qh = p.q + ((int64_t)c.r * p.num_q_heads + (int64_t)c.kvh * g + hl) * kHeadDim +
-                                          quad * 2;
+                bool hv;
+                const __nv_bfloat16 *qh;
+                if constexpr (CASCADE) {  // row hl: head hl % g of member hl / g
+                    const int member = hl / g;
+                    hv = member < c.m;
+                    qh = p.q + ((int64_t)(c.r0 + member) * p.num_q_heads + (int64_t)c.kvh * g + (hl - member * g)) *
+                                   kHeadDim + quad * 2;
+                } else {
+                    hv = hl < g;
+                    qh = p.q + ((int64_t)c.r * p.num_q_heads + (int64_t)c.kvh * g + hl) * kHeadDim + quad * 2;
+                }
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     qb[nt][kk][0] = hv ? __ldg(reinterpret_cast<const uint32_t *>(qh + kk * 16)) : 0u;
@@ -576,10 +703,16 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
                 }
             }
             __syncwarp();
-            const bool whole = seg_first_t == 0 && c.t == c.tiles - 1;
-            const int64_t head0 = (int64_t)c.r * p.num_q_heads + (int64_t)c.kvh * g;
+            // a whole pair of a plain request writes the output; anything else
+            // (part of a pair, a shared prefix, a request whose prefix is
+            // shared) writes partials for the merge kernel
+            bool whole = seg_first_t == 0 && c.t == c.tiles - 1;
+            if constexpr (CASCADE) whole = whole && !c.grouped && c.r >= p.num_groups;
+            const int rows = CASCADE ? c.m * g : g;
+            const int64_t rs = CASCADE ? p.rows_per_slot : g;
+            const int64_t head0 = (int64_t)c.r0 * p.num_q_heads + (int64_t)c.kvh * g;
             const int64_t slot = (int64_t)c.r * p.num_kv_heads + c.kvh + w;
-            for (int h = 0; h < g; ++h) {
+            for (int h = 0; h < rows; ++h) {
                 const float4 v = *reinterpret_cast<const float4 *>(scr + h * kPitch + lane * 4);
                 if (whole) {
                     uint2 packed;
@@ -587,10 +720,10 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
                     packed.y = pack_bf16x2(v.z, v.w);
                     *reinterpret_cast<uint2 *>(p.out + (head0 + h) * kHeadDim + lane * 4) = packed;
                 } else {
-                    *reinterpret_cast<float4 *>(p.part_o + (slot * g + h) * kHeadDim + lane * 4) = v;
+                    *reinterpret_cast<float4 *>(p.part_o + (slot * rs + h) * kHeadDim + lane * 4) = v;
                 }
             }
-            if (!whole && lane < g) p.part_lse[slot * g + lane] = lse_scr[lane];
+            if (!whole && lane < rows) p.part_lse[slot * rs + lane] = lse_scr[lane];
             __syncwarp();  // scratch reads done before the stage is refilled
         }
     }
@@ -612,51 +745,70 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const Params p) {
     const int r = wg / p.num_q_heads, h = wg - r * p.num_q_heads;
     const int g = p.group;
     const int kvh = h / g, j = h - kvh * g;
-    const int64_t T = p.prefix[p.batch];
-    const int64_t pr = p.prefix[r], units_r = p.prefix[r + 1] - pr;
-    if (units_r <= 0 || T <= 0) return;  // rejected request (flagged by the decode kernel)
-    const int64_t tiles = units_r / p.num_kv_heads;
-    const int64_t u0 = pr + kvh * tiles, u1 = u0 + tiles;  // this pair's units
+    const int64_t T = p.prefix[p.num_vreqs];
     const int W = p.num_workers;
+    const int64_t rs = p.rows_per_slot;
     auto worker_of = [&](int64_t u) -> int {  // the worker whose share holds unit u
         const int64_t wv = ((u + 1) * (int64_t)W - 1) / T;
         return (int)(wv < W - 1 ? wv : W - 1);
     };
-    const int wf = worker_of(u0), wl = worker_of(u1 - 1);
-    if (wf == wl) return;  // one worker held the whole pair and wrote the output
-    const int64_t pair = (int64_t)r * p.num_kv_heads + kvh;
+    // the workers [wf, wl] that held pair (virtual request v, kvh)
+    auto pair_workers = [&](int v, int &wf, int &wl) -> bool {
+        const int64_t pr = p.prefix[v], units_v = p.prefix[v + 1] - pr;
+        if (units_v <= 0) return false;  // rejected (flagged by the decode kernel)
+        const int64_t tiles = units_v / p.num_kv_heads;
+        const int64_t u0 = pr + kvh * tiles;
+        wf = worker_of(u0);
+        wl = worker_of(u0 + tiles - 1);
+        return true;
+    };
+    const int vs = p.num_groups + r;  // the request's own virtual request
+    int wf, wl;
+    if (T <= 0 || !pair_workers(vs, wf, wl)) return;
+    int grp = -1, wfp = 0, wlp = -1;  // cascade: the group whose shared prefix this request reads
+    if (p.num_groups > 0) {
+        grp = group_of(p, r);
+        unsigned ignore = 0;
+        if (grp >= 0 && (group_prefix(p, grp, ignore) == 0 || !pair_workers(grp, wfp, wlp))) grp = -1;
+    }
+    if (grp < 0 && wf == wl) return;  // one worker held the whole pair and wrote the output
     // with at least as many units as workers every share is non-empty; else
     // skip the workers that got no units (and wrote no partial)
     const bool sparse = T < W;
     // online combine, kMergeBatch segments per round so their loads are in flight together
     float mx = -INFINITY, wsum = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int w0 = wf; w0 <= wl; w0 += kMergeBatch) {
-        float ls[kMergeBatch];
-        float4 v[kMergeBatch];
+    auto combine = [&](int64_t pair, int w_first, int w_last, int row) {
+        for (int w0 = w_first; w0 <= w_last; w0 += kMergeBatch) {
+            float ls[kMergeBatch];
+            float4 v[kMergeBatch];
 #pragma unroll
-        for (int i = 0; i < kMergeBatch; ++i) {
-            const int wk = w0 + i;
-            const bool use = wk <= wl && (!sparse || worker_begin(T, wk, W) != worker_begin(T, wk + 1, W));
-            const int64_t s = pair + wk;
-            ls[i] = use ? p.part_lse[s * g + j] : -INFINITY;
-            v[i] = use ? reinterpret_cast<const float4 *>(p.part_o + (s * g + j) * kHeadDim)[lane]
-                       : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
+            for (int i = 0; i < kMergeBatch; ++i) {
+                const int wk = w0 + i;
+                const bool use = wk <= w_last && (!sparse || worker_begin(T, wk, W) != worker_begin(T, wk + 1, W));
+                const int64_t s = pair + wk;
+                ls[i] = use ? p.part_lse[s * rs + row] : -INFINITY;
+                v[i] = use ? reinterpret_cast<const float4 *>(p.part_o + (s * rs + row) * kHeadDim)[lane]
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
 #pragma unroll
-        for (int i = 0; i < kMergeBatch; ++i) {
-            if (ls[i] == -INFINITY) continue;
-            const float mn = fmaxf(mx, ls[i]);
-            const float c = mx == -INFINITY ? 0.f : fast_exp2(mx - mn);
-            const float wt = fast_exp2(ls[i] - mn);
-            wsum = wsum * c + wt;
-            acc.x = acc.x * c + wt * v[i].x;
-            acc.y = acc.y * c + wt * v[i].y;
-            acc.z = acc.z * c + wt * v[i].z;
-            acc.w = acc.w * c + wt * v[i].w;
-            mx = mn;
+            for (int i = 0; i < kMergeBatch; ++i) {
+                if (ls[i] == -INFINITY) continue;
+                const float mn = fmaxf(mx, ls[i]);
+                const float c = mx == -INFINITY ? 0.f : fast_exp2(mx - mn);
+                const float wt = fast_exp2(ls[i] - mn);
+                wsum = wsum * c + wt;
+                acc.x = acc.x * c + wt * v[i].x;
+                acc.y = acc.y * c + wt * v[i].y;
+                acc.z = acc.z * c + wt * v[i].z;
+                acc.w = acc.w * c + wt * v[i].w;
+                mx = mn;
+            }
         }
-    }
+    };
+    combine((int64_t)vs * p.num_kv_heads + kvh, wf, wl, j);
+    if (grp >= 0)  // the shared prefix's partials: this request's row of its group's q rows
+        combine((int64_t)grp * p.num_kv_heads + kvh, wfp, wlp, (r - __ldg(p.group_first + grp)) * g + j);
     const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
     uint2 packed;
     packed.x = pack_bf16x2(acc.x * inv, acc.y * inv);

@@ -98,6 +98,8 @@ mg_status ensure_kernel_attributes() {
         cudaFuncSetAttribute(decode::decode_kernel<1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              decode::kSmemBytes) != cudaSuccess ||
         cudaFuncSetAttribute(decode::decode_kernel<2, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             decode::kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(decode::decode_kernel<2, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              decode::kSmemBytes) != cudaSuccess)
         return MG_ERR_CUDA;
     if (extend::set_attributes() != cudaSuccess) return MG_ERR_CUDA;
@@ -126,19 +128,22 @@ mg_status decode_plan(int batch, int hkv, int max_seq_len, int num_partitions, i
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
-// Workspace: per-request unit prefix (int64), then per-slot log-sum-exp and
-// partial outputs (fp32); slots = pairs + workers.
+// Workspace: per-(virtual) request unit prefix (int64), then per-slot
+// log-sum-exp and partial outputs (fp32) of `rows` q rows each; slots = pairs
+// + workers.  Plain decode: one virtual request per request, rows = group.
+// Shared-prefix decode: num_groups more virtual requests, rows = 16.
 struct DecodeWorkspace {
     size_t prefix, lse, o, total;
 };
-DecodeWorkspace decode_ws_layout(int batch, int hq, int hkv, int workers) {
-    const size_t slots = (size_t)batch * hkv + (size_t)workers;
-    const size_t g = (size_t)(hq / hkv);
+DecodeWorkspace decode_ws_layout(int batch, int hq, int hkv, int workers, int num_groups = 0) {
+    const size_t vreqs = (size_t)batch + (size_t)num_groups;
+    const size_t slots = vreqs * hkv + (size_t)workers;
+    const size_t rows = num_groups > 0 ? (size_t)decode::kRows : (size_t)(hq / hkv);
     DecodeWorkspace w;
     w.prefix = 0;
-    w.lse = align256((size_t)(batch + 1) * sizeof(int64_t));
-    w.o = w.lse + align256(slots * g * sizeof(float));
-    w.total = w.o + slots * g * kHeadDim * sizeof(float);
+    w.lse = align256((vreqs + 1) * sizeof(int64_t));
+    w.o = w.lse + align256(slots * rows * sizeof(float));
+    w.total = w.o + slots * rows * kHeadDim * sizeof(float);
     return w;
 }
 
@@ -159,13 +164,18 @@ namespace mg {
 namespace {
 // Decode attention; with k_new != nullptr the KV store of the step's new
 // tokens (one per request) is fused into the same launch.
+// With group_first != nullptr the shared-prefix (cascade) mode runs.
 mg_status decode_impl(const void *q, const void *k_new, const void *v_new, const int32_t *out_loc,
                       const void *k_cache, const void *v_cache, int64_t num_slots, const int32_t *page_table,
                       int32_t page_table_rows, int32_t page_table_stride, const int32_t *table_idx,
                       const int32_t *seq_len, int32_t batch, int32_t max_seq_len, int32_t num_q_heads,
                       int32_t num_kv_heads, int32_t head_dim, float scale, int32_t num_partitions, void *out,
-                      void *workspace, size_t workspace_bytes, void *stream) {
+                      void *workspace, size_t workspace_bytes, void *stream, const int32_t *group_first = nullptr,
+                      const int32_t *prefix_len = nullptr, int32_t num_groups = 0) {
     const bool fused = k_new != nullptr;
+    const bool cascade = group_first != nullptr;
+    if (cascade && (fused || !prefix_len || num_groups <= 0)) return MG_ERR_INVALID_ARGUMENT;
+    if (cascade && (int64_t)batch + num_groups > decode::kMaxBatch) return MG_ERR_UNSUPPORTED_SHAPE;
     mg_status st = check_attention_shape(num_q_heads, num_kv_heads, head_dim);
     if (st != MG_OK) return st;
     if (!valid_scale(scale)) return MG_ERR_INVALID_ARGUMENT;
@@ -184,7 +194,7 @@ mg_status decode_impl(const void *q, const void *k_new, const void *v_new, const
     // units <= batch * Hkv * ceil(max_seq_len / 16); the partition math multiplies by workers
     const double max_units = (double)batch * num_kv_heads * ((max_seq_len + 15) / 16);
     if (max_units * (double)(workers + 1) >= 4.0e18) return MG_ERR_UNSUPPORTED_SHAPE;
-    const DecodeWorkspace ws = decode_ws_layout(batch, num_q_heads, num_kv_heads, workers);
+    const DecodeWorkspace ws = decode_ws_layout(batch, num_q_heads, num_kv_heads, workers, cascade ? num_groups : 0);
     if (!workspace || workspace_bytes < ws.total) return MG_ERR_WORKSPACE_TOO_SMALL;
     if (!aligned16(workspace)) return MG_ERR_MISALIGNED;
     if (ensure_kernel_attributes() != MG_OK) return MG_ERR_CUDA;
@@ -216,12 +226,20 @@ mg_status decode_impl(const void *q, const void *k_new, const void *v_new, const
     p.num_workers = workers;
     p.max_seq_len = max_seq_len;
     p.scale_log2 = scale * kLog2e;
+    p.group_first = group_first;
+    p.prefix_len = prefix_len;
+    p.num_groups = cascade ? num_groups : 0;
+    p.max_members = decode::kRows / p.group;
+    p.rows_per_slot = cascade ? decode::kRows : p.group;
+    p.num_vreqs = batch + p.num_groups;
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int ctas = (workers + decode::kWarps - 1) / decode::kWarps;
     const dim3 grid(ctas), block(decode::kThreads);
     const size_t smem = decode::kSmemBytes;
-    if (p.group <= 8)
+    if (cascade)
+        st = launch_pdl(decode::decode_kernel<2, false, true>, grid, block, smem, s, p);
+    else if (p.group <= 8)
         st = fused ? launch_pdl(decode::decode_kernel<1, true>, grid, block, smem, s, p)
                    : launch_pdl(decode::decode_kernel<1, false>, grid, block, smem, s, p);
     else
@@ -324,6 +342,31 @@ mg_status mg_store_decode_attn(const void *q, const void *k_new, const void *v_n
     return decode_impl(q, k_new, v_new, out_loc, k_cache, v_cache, num_slots, page_table, page_table_rows,
                        page_table_stride, table_idx, seq_len, batch, max_seq_len, num_q_heads, num_kv_heads,
                        head_dim, scale, num_partitions, out, workspace, workspace_bytes, stream);
+}
+
+size_t mg_decode_shared_prefix_workspace_bytes(int32_t batch, int32_t num_groups, int32_t num_q_heads,
+                                               int32_t num_kv_heads, int32_t head_dim, int32_t max_seq_len,
+                                               int32_t num_partitions) {
+    int workers;
+    if (num_groups <= 0 || (int64_t)batch + num_groups > decode::kMaxBatch) return 0;
+    if (check_attention_shape(num_q_heads, num_kv_heads, head_dim) != MG_OK) return 0;
+    if (decode_plan(batch, num_kv_heads, max_seq_len, num_partitions, workers) != MG_OK) return 0;
+    return decode_ws_layout(batch, num_q_heads, num_kv_heads, workers, num_groups).total;
+}
+
+mg_status mg_decode_attn_shared_prefix(const void *q, const void *k_cache, const void *v_cache, int64_t num_slots,
+                                       const int32_t *page_table, int32_t page_table_rows,
+                                       int32_t page_table_stride, const int32_t *table_idx,
+                                       const int32_t *seq_len, int32_t batch, int32_t max_seq_len,
+                                       const int32_t *group_first, const int32_t *prefix_len,
+                                       int32_t num_groups, int32_t num_q_heads, int32_t num_kv_heads,
+                                       int32_t head_dim, float scale, int32_t num_partitions, void *out,
+                                       void *workspace, size_t workspace_bytes, void *stream) {
+    if (!group_first || !prefix_len || num_groups <= 0) return MG_ERR_INVALID_ARGUMENT;
+    return decode_impl(q, nullptr, nullptr, nullptr, k_cache, v_cache, num_slots, page_table, page_table_rows,
+                       page_table_stride, table_idx, seq_len, batch, max_seq_len, num_q_heads, num_kv_heads,
+                       head_dim, scale, num_partitions, out, workspace, workspace_bytes, stream, group_first,
+                       prefix_len, num_groups);
 }
 
 mg_status mg_extend_attn(const void *q, const void *k_cache, const void *v_cache, int64_t num_slots,

@@ -45,6 +45,9 @@ SIGNATURES = {
                                       _I32, _F32, _I32, _P, _P, _SZ, _P]),
     "mg_store_decode_attn": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _P, _I32, _I32, _P, _P, _I32, _I32,
                                             _I32, _I32, _I32, _F32, _I32, _P, _P, _SZ, _P]),
+    "mg_decode_shared_prefix_workspace_bytes": (_SZ, [_I32, _I32, _I32, _I32, _I32, _I32, _I32]),
+    "mg_decode_attn_shared_prefix": (ctypes.c_int, [_P, _P, _P, _I64, _P, _I32, _I32, _P, _P, _I32, _I32, _P, _P,
+                                                    _I32, _I32, _I32, _I32, _F32, _I32, _P, _P, _SZ, _P]),
     "mg_extend_attn": (ctypes.c_int, [_P, _P, _P, _I64, _P, _I32, _I32, _P, _P, _P, _P, _I32, _I32, _I32,
                                       _I32, _I32, _I32, _I32, _F32, _P, _P]),
     "mg_decode_attn_static_workspace": (ctypes.c_int, [_P, _P, _P, _I64, _P, _I32, _I32, _P, _P, _I32, _I32,
@@ -222,6 +225,46 @@ def store_decode_attn(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
                                        _dev(seq_len, torch.int32, "seq_len"), b, max_seq_len, hq, hkv, d,
                                        float(scale), num_partitions, _dev(out, torch.bfloat16, "out"), ws_ptr,
                                        ws_bytes, _stream(stream)), "mg_store_decode_attn")
+    return out
+
+
+def decode_shared_prefix_workspace_bytes(batch: int, num_groups: int, num_q_heads: int, num_kv_heads: int,
+                                         max_seq_len: int, num_partitions: int = 0, head_dim: int = 128) -> int:
+    return int(load().mg_decode_shared_prefix_workspace_bytes(batch, num_groups, num_q_heads, num_kv_heads,
+                                                               head_dim, max_seq_len, num_partitions))
+
+
+def decode_attn_shared_prefix(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                              page_table: torch.Tensor, table_idx: torch.Tensor, seq_len: torch.Tensor,
+                              group_first: torch.Tensor, prefix_len: torch.Tensor, max_seq_len: int,
+                              scale: float, num_partitions: int = 0, out: Optional[torch.Tensor] = None,
+                              workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """decode_attn where groups of consecutive requests share a prefix of their
+    page-table rows (group_first [G+1], prefix_len [G]); the shared K/V rows are
+    read once per group.  Returns out [B, Hq, D] bf16."""
+    b = q.shape[0] if isinstance(q, torch.Tensor) and q.dim() == 3 else -1
+    if not isinstance(prefix_len, torch.Tensor) or prefix_len.dim() != 1:
+        raise ValueError("decode_attn_shared_prefix: prefix_len must be [num_groups]")
+    ng = prefix_len.shape[0]
+    _attention_shapes("decode_attn_shared_prefix", q, k_cache, v_cache, page_table, out,
+                      {"table_idx": (table_idx, (b,)), "seq_len": (seq_len, (b,)),
+                       "group_first": (group_first, (ng + 1,))})
+    b, hq, d = q.shape
+    hkv = k_cache.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    need = decode_shared_prefix_workspace_bytes(b, ng, hq, hkv, max_seq_len, num_partitions, d)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = _dev(workspace, torch.uint8, "workspace") if workspace is not None else None
+    ws_bytes = workspace.numel() if workspace is not None else 0
+    _check(load().mg_decode_attn_shared_prefix(
+        _dev(q, torch.bfloat16, "q"), _dev(k_cache, torch.bfloat16, "k_cache"),
+        _dev(v_cache, torch.bfloat16, "v_cache"), k_cache.shape[0], _dev(page_table, torch.int32, "page_table"),
+        page_table.shape[0], page_table.shape[1], _dev(table_idx, torch.int32, "table_idx"),
+        _dev(seq_len, torch.int32, "seq_len"), b, max_seq_len, _dev(group_first, torch.int32, "group_first"),
+        _dev(prefix_len, torch.int32, "prefix_len"), ng, hq, hkv, d, float(scale), num_partitions,
+        _dev(out, torch.bfloat16, "out"), ws_ptr, ws_bytes, _stream(stream)), "mg_decode_attn_shared_prefix")
     return out
 
 

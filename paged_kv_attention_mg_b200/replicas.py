@@ -120,6 +120,9 @@ class Replicas:
     def sum(self, x: float) -> float:
         return self._reduce(x, self.pg.ReduceOp.SUM if self.pg else None)
 
+    def min(self, x: float) -> float:
+        return -self._reduce(-x, self.pg.ReduceOp.MAX if self.pg else None)
+
     def close(self):
         if self.pg:
             self.pg.barrier()

@@ -67,6 +67,20 @@ def decode_bytes(seq_lens: Iterable[int], num_q_heads: int, num_kv_heads: int, h
     return kv + qo + 4 * total
 
 
+def decode_bytes_shared_prefix(seq_lens: Sequence[int], group_first: Sequence[int], prefix_len: Sequence[int],
+                               num_q_heads: int, num_kv_heads: int, head_dim: int, dtype_bytes: int = 2) -> int:
+    """Decode where groups of requests share a prefix of their page-table rows:
+    the shared K/V rows (and their page-table entries) counted once per group,
+    each request's own keys after the prefix once, q read and out written once."""
+    seq_lens = [int(x) for x in seq_lens]
+    keys = sum(seq_lens)
+    for g0, g1, P in zip(group_first[:-1], group_first[1:], prefix_len):
+        keys -= (int(g1) - int(g0) - 1) * int(P)  # every member but the first reads the prefix through it
+    kv = keys * num_kv_heads * head_dim * dtype_bytes * 2
+    qo = 2 * len(seq_lens) * num_q_heads * head_dim * dtype_bytes
+    return kv + qo + 4 * keys
+
+
 def extend_bytes(cached: Sequence[int], seq: Sequence[int], num_q_heads: int, num_kv_heads: int,
                  head_dim: int, dtype_bytes: int = 2) -> int:
     """Extend: every context row of K and V once, q read and out written once."""

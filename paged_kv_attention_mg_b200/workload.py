@@ -35,6 +35,13 @@ Recipe (the same for every workload):
    and the slots the new tokens are about to be stored in, holds bf16 NaN
    (bit pattern 0xFFFF), so a read of a slot outside the history shows up as
    NaN in the output.
+3. shared-prefix workloads (a radix prefix cache hit, "Mini-SGLang" tag page,
+   KV Cache post): requests come in groups of consecutive requests; after
+   step 1, every member's first P page-table entries are overwritten with the
+   group's first member's, so the shared tokens sit in the pool once.  The
+   history (step 2) holds each slot the rows reference once, in the order of
+   first reference; the members' own slots of those positions are no longer
+   referenced and stay NaN.
 """
 from __future__ import annotations
 
@@ -65,6 +72,7 @@ class WorkloadSpec:
     max_len: int  # upper bound of seq_len by construction (page-table width before align)
     description: str
     lengths: Callable = field(repr=False, compare=False, default=None)
+    share: Optional[tuple] = None  # (members per group, shared prefix length P) or None
 
     @property
     def group(self) -> int:
@@ -115,6 +123,15 @@ def _uniform_extend(c_lo, c_hi, n_lo, n_hi):
     return draw
 
 
+def _prefix_decode(prefix, lo, hi):
+    """Decode lengths P + U[lo, hi]: every request has its own tokens after the
+    shared prefix (at least the new one)."""
+    def draw(gen, batch):
+        seq = prefix + torch.randint(lo, hi + 1, (batch,), generator=gen, dtype=torch.int64)
+        return seq - 1, seq
+    return draw
+
+
 WORKLOADS: List[WorkloadSpec] = [
     WorkloadSpec("tiny_decode", "decode", 3, 16, 8, 128, 512, 1, 1000, 12,
                  "3 requests, lengths 5/9/12 (new token included), Hq16/Hkv8, pool 512",
@@ -131,6 +148,10 @@ WORKLOADS: List[WorkloadSpec] = [
     WorkloadSpec("chunked_prefill_extend", "extend", 16, 16, 8, 128, 100_000, 1, 1004, 3072,
                  "16 requests, cached U[0,2048], chunk U[256,1024], Hq16/Hkv8, pool 100k",
                  _uniform_extend(0, 2048, 256, 1024)),
+    WorkloadSpec("shared_prefix_decode", "decode", 64, 16, 8, 128, 200_000, 1, 1005, 2560,
+                 "Qwen3-0.6B attention shape, batch 64 in 8 groups of 8 sharing a 2048-token prefix, "
+                 "own tokens U[16,512] after it, pool 200k",
+                 _prefix_decode(2048, 16, 512), share=(8, 2048)),
 ]
 
 BY_NAME = {w.name: w for w in WORKLOADS}
@@ -161,6 +182,8 @@ class Step:
     out_loc: torch.Tensor  # [T] int32, T = sum(seq_len - cached_len)
     q_offset: torch.Tensor  # [B+1] int32 prefix sums of new-token counts
     dummy_slot: int
+    group_first: Optional[torch.Tensor] = None  # shared-prefix workloads: [G+1] int32
+    prefix_len: Optional[torch.Tensor] = None   # [G] int32
 
     @property
     def batch(self) -> int:
@@ -180,14 +203,21 @@ class Step:
         return int(n.max()) if self.batch else 0
 
     def history_slots(self) -> torch.Tensor:
-        """Slots of positions [0, cached_len) of every request, request order."""
+        """Slots of positions [0, cached_len) of every request, request order,
+        each slot once (rows that share a prefix reference its slots again)."""
         rows = []
         for r in range(self.batch):
             row = self.page_table[int(self.table_idx[r])]
             rows.append(row[: int(self.cached_len[r])])
         if not rows:
             return torch.zeros(0, dtype=torch.int64)
-        return torch.cat(rows).to(torch.int64)
+        slots = torch.cat(rows).to(torch.int64)
+        uniq, inverse = torch.unique(slots, return_inverse=True)
+        if uniq.numel() == slots.numel():
+            return slots  # every slot once already (no shared prefix)
+        first = torch.full((uniq.numel(),), slots.numel(), dtype=torch.int64)
+        first.scatter_reduce_(0, inverse, torch.arange(slots.numel()), reduce="amin")
+        return slots[torch.sort(first).values]
 
 
 @dataclass
@@ -227,10 +257,30 @@ def make_step(spec: WorkloadSpec, page_table_stride: Optional[int] = None) -> St
     q_offset = torch.zeros(batch + 1, dtype=torch.int64)
     if batch:
         q_offset[1:] = torch.cumsum(n, 0)
-    return Step(spec=spec, cached_len=cached.to(torch.int32), seq_len=seq.to(torch.int32),
+    step = Step(spec=spec, cached_len=cached.to(torch.int32), seq_len=seq.to(torch.int32),
                 table_idx=table_idx.to(torch.int32), page_table=page_table,
                 out_loc=(torch.cat(out_loc) if out_loc else torch.zeros(0, dtype=torch.int32)),
                 q_offset=q_offset.to(torch.int32), dummy_slot=dummy_slot)
+    if spec.share:
+        share_prefixes(step, spec.share[0], spec.share[1])
+    return step
+
+
+def share_prefixes(step: Step, members: int, prefix: int) -> None:
+    """Groups of `members` consecutive requests share their first `prefix`
+    page-table entries (the first member's slots); sets group_first /
+    prefix_len.  The prefix must leave every member at least its new token."""
+    b = step.batch
+    firsts = list(range(0, b, members)) + [b]
+    plen = []
+    for g0, g1 in zip(firsts[:-1], firsts[1:]):
+        P = min(prefix, int(step.seq_len[g0:g1].min()) - 1, int(step.cached_len[g0:g1].min()))
+        lead = int(step.table_idx[g0])
+        for r in range(g0 + 1, g1):
+            step.page_table[int(step.table_idx[r]), :P] = step.page_table[lead, :P]
+        plen.append(P)
+    step.group_first = torch.tensor(firsts, dtype=torch.int32)
+    step.prefix_len = torch.tensor(plen, dtype=torch.int32)
 
 
 def _bf16_normal(gen, shape) -> torch.Tensor:

@@ -104,6 +104,22 @@ def test_decode_plan_with_forced_partitions_needs_no_device(lib):
     assert lib.mg_decode_workspace_bytes(8, 12, 8, 128, 32768, 1000) == 0  # unsupported shape
 
 
+def test_shared_prefix_workspace_and_host_validation(lib):
+    # 5 requests + 2 groups = 7 virtual requests; rows per slot = 16 (a group's q rows)
+    slots = 7 * 4 + 1000
+    a256 = lambda x: (x + 255) // 256 * 256
+    want = a256(8 * 8) + a256(slots * 16 * 4) + slots * 16 * 128 * 4
+    assert lib.mg_decode_shared_prefix_workspace_bytes(5, 2, 32, 4, 128, 4096, 1000) == want
+    assert lib.mg_decode_shared_prefix_workspace_bytes(5, 0, 32, 4, 128, 4096, 1000) == 0   # no groups
+    assert lib.mg_decode_shared_prefix_workspace_bytes(5, 2, 12, 8, 128, 4096, 1000) == 0   # unsupported shape
+    args = [4096, 4096, 4096, 100, 4096, 6, 32, 4096, 4096, 5, 32]
+    tail = [16, 8, 128, 0.1, 1000, 4096, 4096, 1 << 30, None]
+    assert lib.mg_decode_attn_shared_prefix(*args, None, 4096, 2, *tail) == 1      # no group_first
+    assert lib.mg_decode_attn_shared_prefix(*args, 4096, 4096, 0, *tail) == 1      # no groups
+    small = tail[:-2] + [16, None]
+    assert lib.mg_decode_attn_shared_prefix(*args, 4096, 4096, 2, *small) == 4     # workspace too small
+
+
 def test_extend_rejects_shapes_and_empty_is_noop(lib):
     assert lib.mg_extend_attn(4096, 4096, 4096, 100, 4096, 5, 32, 4096, 4096, 4096, 4096, 4, 10, 4, 32,
                               16, 8, 64, 0.1, 4096, None) == 2

@@ -40,6 +40,8 @@ def _rank_main(rank, world, port, queue):
         fake_ms = 10.0 + 5.0 * reps.rank
         t_max = reps.max(fake_ms)
         units = reps.sum(step.batch)
+        # the roofline line reports the lowest rank's own achieved rate
+        rate_min = reps.min(100.0 - 30.0 * reps.rank)
         # strong scaling: one global batch, contiguous request shards
         gspec = wl.custom_spec("decode", [4, 30, 7, 99, 12], [5, 31, 8, 100, 13], 8, 2, 400, seed=5)
         gstep = wl.make_step(gspec)
@@ -53,7 +55,7 @@ def _rank_main(rank, world, port, queue):
                              gstep.table_idx.numpy(), gstep.seq_len.numpy(), gspec.scale,
                              requests=range(b0, b1), threads=1)
         queue.put(dict(rank=reps.rank, seed=spec.seed, page_table=step.page_table.numpy(), out=out,
-                       t_max=t_max, units=units, shard=(b0, b1), part=part))
+                       t_max=t_max, units=units, rate_min=rate_min, shard=(b0, b1), part=part))
     finally:
         reps.close()
 
@@ -78,6 +80,7 @@ def test_two_gloo_ranks_replicas_and_shards():
     assert not np.array_equal(res[0]["page_table"], res[1]["page_table"])
     assert res[0]["t_max"] == res[1]["t_max"] == 15.0      # max over ranks
     assert res[0]["units"] == res[1]["units"] == 2 * canonical.batch
+    assert res[0]["rate_min"] == res[1]["rate_min"] == 70.0  # min over ranks
     assert np.isfinite(res[0]["out"]).all() and np.isfinite(res[1]["out"]).all()
     # shards cover the batch once, and the union equals the single-process result
     (a0, a1), (b0, b1) = res[0]["shard"], res[1]["shard"]

@@ -70,9 +70,20 @@ def test_workload_metadata_structure(spec):
     assert bool((cached >= 0).all()) and bool((cached < seq).all())
     if spec.kind == "decode":
         assert bool((cached == seq - 1).all())
-    # slots distinct across all requests, never the dummy slot
+    # slots distinct across all requests (a shared prefix counted once), never the dummy slot
     used = torch.cat([step.page_table[int(step.table_idx[r]), :int(seq[r])] for r in range(B)])
-    assert used.unique().numel() == used.numel() == int(seq.sum())
+    shared = 0
+    if spec.share:
+        gf, pl = step.group_first.tolist(), step.prefix_len.tolist()
+        assert gf[0] == 0 and gf[-1] == B and len(pl) == len(gf) - 1
+        for g0, g1, P in zip(gf[:-1], gf[1:], pl):
+            assert 0 < P <= int(cached[g0:g1].min())  # each member keeps at least its new token
+            lead = step.page_table[int(step.table_idx[g0]), :P]
+            for r in range(g0 + 1, g1):
+                assert torch.equal(step.page_table[int(step.table_idx[r]), :P], lead)
+            shared += (g1 - g0 - 1) * P
+        assert len(step.history_slots().unique()) == step.history_slots().numel()
+    assert used.unique().numel() == used.numel() - shared == int(seq.sum()) - shared
     assert int(used.max()) < step.dummy_slot == spec.num_slots - 1
     assert bool((step.page_table[B] == step.dummy_slot).all())
     # out_loc = page_table[table_idx, cached:seq], concatenated in request order
