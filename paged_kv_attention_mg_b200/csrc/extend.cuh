@@ -186,7 +186,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         return;
     }
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffMisc);
-    const uint64_t lim = p.wait_limit_ns;
+    const uint64_t lim = p.wait_limit_ns;  // nanoseconds
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + kOffMisc + 4);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -272,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int tok_local = qrow / g, head_local = qrow - tok_local * g;
         const int i = tok0 + t * tpq + tok_local;  // new-token index within the request
         const bool valid = tok_local < tpq && i < n;
-        const int lim = valid ? c + i : kv_len - 1;  // last visible key position
+        const int last_key = valid ? c + i : kv_len - 1;  // last visible key position
         const bool active = t == 0 || has_q1;
         const uint32_t lane_addr = (uint32_t)(wq * 32) << 16;
         const uint32_t tS = tmem + lane_addr + col_s(t);
@@ -289,7 +289,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_ld_32x32b_x32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
             tmem_ld_wait();
             const int key0 = j * kN;
-            const int nvis = min(max(lim - key0 + 1, 0), kN);  // visible keys in this tile
+            const int nvis = min(max(last_key - key0 + 1, 0), kN);  // visible keys in this tile
             // Row max of the raw scores (scale > 0, so scaling commutes with the
             // max); a tile every key of which is visible to the whole warp skips
             // the mask.
