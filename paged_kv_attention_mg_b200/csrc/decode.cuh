@@ -62,6 +62,12 @@ constexpr int kMaxBatch = 131072;                  // requests per call
 #ifndef MG_DECODE_MIN_BLOCKS
 #define MG_DECODE_MIN_BLOCKS 1  // resident CTAs per SM (the shared memory is sized for it)
 #endif
+#ifndef MG_DECODE_SPLIT_P
+// 1: P enters the PV product as bf16 hi + lo parts (two products), so the
+// weights carry ~2^-17 relative error instead of bf16's 2^-9; decode is bound
+// by HBM, not by its tensor-core products, so the second product is cheap
+#define MG_DECODE_SPLIT_P 1
+#endif
 #ifndef MG_DECODE_IDX_AHEAD
 #define MG_DECODE_IDX_AHEAD 12  // tiles of page-table entries fetched ahead of compute
 #endif
@@ -618,6 +624,9 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
         // ---- P^T (bf16) as B fragments: lane l needs keys 2(l%4), +1 (and +8)
         // of head l/4, which sit in lanes 8(l%4) + l/8 and that + 4
         uint32_t pb[NT][2];
+#if MG_DECODE_SPLIT_P
+        uint32_t pl[NT][2];  // the bf16 residuals p - hi
+#endif
         {
             const int s0 = 8 * quad + (lane >> 3);
             const uint32_t sel = ((lane >> 2) & 1) ? 0x7632u : 0x5410u;
@@ -628,16 +637,28 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
                 const float p0 = fast_exp2(sc[nt][0] - mu0), p1 = fast_exp2(sc[nt][1] - mu1);
                 const float p2 = fast_exp2(sc[nt][2] - mu0), p3 = fast_exp2(sc[nt][3] - mu1);
                 const uint32_t X = pack_bf16x2(p0, p1), Y = pack_bf16x2(p2, p3);
+#if MG_DECODE_SPLIT_P
+                // hi + lo carries P to ~2^-17 relative, so the fp32 weights are the normaliser
+                lh[nt][0] += p0 + p2;
+                lh[nt][1] += p1 + p3;
+                const uint32_t XL = pack_bf16x2(p0 - bf16x2_lo(X), p1 - bf16x2_hi(X));
+                const uint32_t YL = pack_bf16x2(p2 - bf16x2_lo(Y), p3 - bf16x2_hi(Y));
+                const uint32_t la = __shfl_sync(0xffffffffu, XL, s0), lb = __shfl_sync(0xffffffffu, XL, s0 + 4);
+                const uint32_t lc = __shfl_sync(0xffffffffu, YL, s0), ld = __shfl_sync(0xffffffffu, YL, s0 + 4);
+                pl[nt][0] = __byte_perm(la, lb, sel);
+                pl[nt][1] = __byte_perm(lc, ld, sel);
+#else
                 // the normaliser sums the same bf16-rounded weights the PV product uses
                 lh[nt][0] += bf16x2_lo(X) + bf16x2_lo(Y);
                 lh[nt][1] += bf16x2_hi(X) + bf16x2_hi(Y);
+#endif
                 const uint32_t xa = __shfl_sync(0xffffffffu, X, s0), xb = __shfl_sync(0xffffffffu, X, s0 + 4);
                 const uint32_t ya = __shfl_sync(0xffffffffu, Y, s0), yb = __shfl_sync(0xffffffffu, Y, s0 + 4);
                 pb[nt][0] = __byte_perm(xa, xb, sel);
                 pb[nt][1] = __byte_perm(ya, yb, sel);
             }
         }
-        // ---- O^T += V^T P^T
+        // ---- O^T += V^T P^T (hi, then lo parts of P)
         {
             const int mi = lane >> 3;
             const int key = (mi >> 1) * 8 + (lane & 7);
@@ -646,7 +667,12 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
                 uint32_t a[4];
                 ldmatrix_x4_trans(vt + swz(key, 2 * dt + (mi & 1)), a[0], a[1], a[2], a[3]);
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(o[nt][dt], a, pb[nt][0], pb[nt][1]);
+                for (int nt = 0; nt < NT; ++nt) {
+                    mma_bf16_16816(o[nt][dt], a, pb[nt][0], pb[nt][1]);
+#if MG_DECODE_SPLIT_P
+                    mma_bf16_16816(o[nt][dt], a, pl[nt][0], pl[nt][1]);
+#endif
+                }
             }
         }
         if (FUSED && c.t == c.tiles - 1) {

@@ -6,31 +6,42 @@
 // stored; new token i (query row q_offset[r] + i, position c + i) attends to the
 // keys at positions 0 .. c + i of its page-table row.
 //
-// Work decomposition (B200 design; 16 warps in four warpgroups with their
-// register budgets moved by setmaxnreg: warpgroups 0 and 3 load and issue
-// MMAs on 72 registers a thread, warpgroups 1 and 2 run the softmax on 184):
-//   * one CTA per (q block, kv head, request).  A q block is two 128-row Q
-//     tiles; a row is (token, head) with the g heads that share the KV head
-//     adjacent, so one K/V tile feeds 2 x 128 query rows (GQA packing).
-//   * seven load warps (0-3, 13-15): the Q tiles with 3-D TMA, the K and V
-//     tiles (128 keys each) with 16-byte cp.async straight from the paged pool
-//     into the 128-byte swizzled layout, behind mbarriers.  A warp keeps about
-//     one 512-byte cp.async in flight per 70 cycles whatever the SM does, so
-//     the copy rate grows with the number of issuing warps; every load warp
-//     owns every seventh pair of rows of each tile.
-//   * warp 12, one thread: issues tcgen05.mma (M=128, N=128, K=16, bf16 in,
-//     fp32 accumulate in TMEM).  S_t = Q_t K^T lands in TMEM; P_t (bf16) is
-//     written back over S_t and consumed straight from TMEM as the A operand
-//     of O_t += P_t V.  The MMAs of the two Q tiles interleave, each issued
-//     once its inputs are ready.  (Since P_t overwrites S_t, S_t of the next
-//     KV tile waits for P_t V; measured, both Q tiles' softmaxes then wait on
-//     the same KV tile, so the softmax and the tensor core mostly alternate
-//     instead of overlapping: the kernel's present bound.)
-//   * warpgroups 1 / 2: softmax for Q tile 0 / 1, one TMEM lane (= one query
-//     row) per thread: causal mask key <= c + i, online softmax in the exp2
-//     domain, O rescaled in TMEM only when the running max grows by more than
-//     2^8 (exact: the same stale max is used for P and for the row sum),
-//     epilogue O / l -> bf16 -> global.
+// Work decomposition (B200 design):
+//   * a work item is (request, kv head, q block); a q block is two 128-row Q
+//     tiles, a row being (token, head) with the g heads that share the KV head
+//     adjacent, so one K/V tile feeds 2 x 128 query rows (GQA packing).  An
+//     item costs one pass over its keys, ceil((c + last token + 1) / 128) KV
+//     tiles of 128 keys.
+//   * persistent CTAs, one per SM.  Every CTA computes the same work list
+//     (items sorted by cost, heaviest first, when there are at most
+//     kMaxSortItems) and takes its items in snake order (k, 2G-1-k, 2G+k, ...),
+//     so the heavy items start first and the loads even out.  Across a CTA's
+//     items the pipelines never drain: K/V rings, barrier phases and TMEM run
+//     on, the next item's Q tiles load while the current item finishes, and an
+//     item's epilogue overlaps the next item's first Q K^T.
+//   * 16 warps in four warpgroups, register budgets moved by setmaxnreg
+//     (warpgroups 0 and 3: 72 registers a thread; 1 and 2: 184):
+//       - warps 0-3 load K tiles, warps 13-15 load V tiles (decoupled rings, so
+//         K can run ahead of V): 16-byte cp.async straight from the paged pool
+//         into the 128-byte swizzled UMMA layout, each warp instruction moving
+//         two 256-byte rows; each lane holds the page-table entries of the keys
+//         it is responsible for in registers, fetched a tile ahead; the tile's
+//         full barrier is armed by cp.async.mbarrier.arrive.noinc, so it
+//         completes when the copies land and the loaders never wait for them.
+//       - warp 12, one thread: tcgen05.mma (M=128, N=128, K=16, bf16 in, fp32
+//         accumulate in TMEM).  S_t = Q_t K^T lands in TMEM; P_t (bf16) is
+//         written back over S_t and consumed straight from TMEM as the A
+//         operand of O_t += P_t V.  Issue order S0, S1, then per KV tile
+//         P0 V, S0', P1 V, S1': while one Q tile's softmax runs, the tensor
+//         core works on the other's.
+//       - warpgroups 1 / 2: softmax of Q tile 0 / 1, one TMEM lane (= query
+//         row) per thread: causal mask key <= c + i, online softmax in the
+//         exp2 domain (part of the exponentials on the FMA pipe, the rest on
+//         MUFU), O rescaled in TMEM only when the running max grows by more
+//         than 2^8 (exact: P and the row sum use the same stale max and the
+//         same bf16-rounded P), epilogue O / l -> bf16 -> global.  Each also
+//         loads its next item's Q tile by TMA as soon as its last score tile
+//         has landed (the tile's last reader is that Q K^T).
 // TMEM: S0 [0,128)  S1 [128,256)  O0 [256,384)  O1 [384,512) columns.
 #pragma once
 
@@ -44,39 +55,56 @@ namespace extend {
 constexpr int kM = 128;                     // query rows per Q tile
 constexpr int kN = 128;                     // keys per KV tile
 constexpr int kQTiles = 2;
-constexpr int kKStages = 3;                 // K ring: S of a tile needs K before P V needs V
+constexpr int kKStages = 3;                 // K ring
 constexpr int kVStages = 2;                 // V ring
-constexpr int kIdxAhead = 3;                // tiles of page-table entries in flight ahead of the K issue
-constexpr int kIdxRing = 4;                 // >= kIdxAhead + 1
-constexpr int kThreads = 512;               // 16 warps: 7 load, 1 MMA, 8 softmax
-constexpr int kLoaders = 7;                 // load warps 0-3 and 13-15
+constexpr int kThreads = 512;
+constexpr int kKLoadWarp0 = 0, kKLoaders = 4;    // K loaders: warps 0-3
 constexpr int kMmaWarp = 12;
+constexpr int kVLoadWarp0 = 13, kVLoaders = 3;   // V loaders: warps 13-15
 constexpr int kPairs = kN / 2;              // row pairs per tile (one warp instruction moves a pair)
-constexpr int kMaxPairsPerLoader = (kPairs + kLoaders - 1) / kLoaders;
 constexpr int kRegsLoad = 72;               // registers a thread in warpgroups 0 and 3
 constexpr int kRegsSoftmax = 184;           // registers a thread in warpgroups 1 and 2
 static_assert(2 * 128 * kRegsLoad + 2 * 128 * kRegsSoftmax == 65536 && 65536 / kThreads == 128,
               "the register split must add up to what the block is launched with");
-static_assert(2 * kMaxPairsPerLoader <= 32, "a load warp fetches one page-table entry per lane");
 constexpr int kHalfBytes = 128 * 128;       // 128 rows x 128 B (64 bf16): one swizzle column
 constexpr int kTileBytes = 2 * kHalfBytes;  // 128 rows x 256 B
 constexpr int kTmemCols = 512;
 __device__ __forceinline__ uint32_t col_s(int t) { return (uint32_t)t * 128u; }
 __device__ __forceinline__ uint32_t col_o(int t) { return 256u + (uint32_t)t * 128u; }
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
+constexpr int kMaxSortItems = 2048;         // work lists up to this size are sorted by cost
+constexpr int kMaxItemsPerCta = 32;         // sorted lists: items a CTA keeps (the host sizes the grid)
+constexpr int kMaxCost = 4095;              // cost key clamp (KV tiles)
+#ifndef MG_EXTEND_EMU_PAIRS
+#define MG_EXTEND_EMU_PAIRS 4  // of every 16 pairs of exponentials, this many on the FMA pipe
+#endif
+constexpr int kEmuPairs = MG_EXTEND_EMU_PAIRS;
+static_assert(kEmuPairs >= 0 && kEmuPairs <= 16, "pairs per chunk of 16");
 
 // shared memory map.  The kernel has no static shared memory, so its dynamic
 // shared memory starts on a 1024-byte boundary (checked at run time), as the
-// 128-byte swizzle atoms require; every region below keeps that alignment.
+// 128-byte swizzle atoms require; every tile region below keeps that alignment.
 constexpr int kOffQ = 0;
 constexpr int kOffK = kOffQ + kQTiles * kTileBytes;
 constexpr int kOffV = kOffK + kKStages * kTileBytes;
-constexpr int kOffIdx = kOffV + kVStages * kTileBytes;
-constexpr int kOffBar = kOffIdx + kIdxRing * kN * 4;
-constexpr int kNumBars = 2 + 2 * kKStages + 2 * kVStages + 3 * kQTiles;  // + the abort drain
-constexpr int kOffMisc = kOffBar + kNumBars * 8;
+constexpr int kOffBar = kOffV + kVStages * kTileBytes;
+// mbarriers, by index (8 bytes each from kOffBar)
+constexpr int kBarDrain = 0;
+constexpr int kBarQFull = kBarDrain + 1;          // + Q tile
+constexpr int kBarKFull = kBarQFull + kQTiles;    // + K stage
+constexpr int kBarKEmpty = kBarKFull + kKStages;
+constexpr int kBarVFull = kBarKEmpty + kKStages;  // + V stage
+constexpr int kBarVEmpty = kBarVFull + kVStages;
+constexpr int kBarSFull = kBarVEmpty + kVStages;  // + Q tile
+constexpr int kBarPFull = kBarSFull + kQTiles;
+constexpr int kBarODone = kBarPFull + kQTiles;
+constexpr int kBarOFree = kBarODone + kQTiles;
+constexpr int kNumBars = kBarOFree + kQTiles;
+constexpr int kOffItems = kOffBar + kNumBars * 8;
+constexpr int kOffMisc = kOffItems + kMaxItemsPerCta * 4;
 constexpr int kSmemBytes = kOffMisc + 16;
 static_assert(kSmemBytes <= 227 * 1024, "extend shared memory over the per-CTA limit");
+static_assert(kMaxSortItems * 4 <= kKStages * kTileBytes, "the sort runs in the K ring before any load");
 
 struct Params {
     const __nv_bfloat16 *q;
@@ -93,6 +121,8 @@ struct Params {
     int32_t batch, total_q, max_q_len, max_seq_len;
     int32_t num_q_heads, num_kv_heads, group;
     int32_t tokens_per_qtile;  // floor(128 / group)
+    int32_t num_qblocks;       // ceil(max_q_len / (2 * tokens_per_qtile))
+    int32_t num_items;         // num_qblocks * batch * num_kv_heads
     float scale_log2;
     uint64_t wait_limit_ns;    // bound of every pipeline wait
     int32_t inject_stall;      // test hook: withhold the first score tile's hand-off
@@ -119,11 +149,10 @@ __host__ __device__ constexpr uint32_t idesc_bf16(bool b_mn_major) {
            | ((uint32_t)(kM >> 4) << 24);    // M / 16
 }
 
-struct Sync {
-    uint32_t q_full, drain;
-    uint32_t k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
-    uint32_t s_full[kQTiles], p_full[kQTiles], o_done[kQTiles];
-};
+// shared-memory address of mbarrier `index`
+__device__ __forceinline__ uint32_t bar_at(uint32_t sbase, int index) {
+    return sbase + (uint32_t)(kOffBar + index * 8);
+}
 
 __device__ __forceinline__ uint64_t global_ns() {
     uint64_t now;
@@ -177,6 +206,184 @@ __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, vol
     return __all_sync(0xffffffffu, ok);
 }
 
+// ---------------------------------------------------------------- exp2 on the FMA pipe
+// 2^x for x <= 8 from fused multiply-adds and integer adds, for a share of the
+// softmax exponentials, so that the MUFU unit (16 results per clock per SM,
+// as many as the tensor core finishes (query, key) pairs at head_dim 128) is
+// not the only unit computing them.  Method: Cody-Waite range reduction
+// x = n + f with n = round(x) (by adding 1.5 * 2^23, which leaves round(x)
+// in the low mantissa bits) and f in [-1/2, 1/2]; 2^f by a degree-3
+// polynomial whose coefficients were fitted here to minimise the relative
+// error on that interval (7.5e-5, far below half a bf16 ulp, 2^-9); then n
+// added to the exponent field.  x is clamped at -126 first, so the exponent
+// never underflows past zero (such weights are below 2^-126 of the row max,
+// zero in bf16 after the sum).
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+    constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+    x.x = fmaxf(x.x, -126.0f);
+    x.y = fmaxf(x.y, -126.0f);
+    const float2 round2 = make_float2(kRound, kRound);
+    const float2 t = fadd2(x, round2);
+    const float2 f = fsub2(x, fsub2(t, round2));
+    float2 p = ffma2(make_float2(0.05517132208f, 0.05517132208f), f,
+                     make_float2(0.24261054396f, 0.24261054396f));
+    p = ffma2(p, f, make_float2(0.69326096773f, 0.69326096773f));
+    p = ffma2(p, f, make_float2(0.99992811680f, 0.99992811680f));
+    return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                       __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
+}
+
+// ---------------------------------------------------------------- work items
+// Item id enumeration (also the tie order of the sorted list): the q block
+// with the latest tokens first, then request, then kv head.
+struct Item {
+    int r, kvh, row, c, n, qo, tok0, kv_len, n_kv;
+    bool q1;  // the second Q tile holds tokens
+};
+
+// 1: the item has work; 0: its q block holds no token of the request;
+// -1: the request's metadata is inconsistent (no item of it runs).
+__device__ __forceinline__ int item_info(const Params &p, int id, Item &it) {
+    const int per_qb = p.batch * p.num_kv_heads;
+    const int qb = p.num_qblocks - 1 - id / per_qb;
+    const int rest = id - (id / per_qb) * per_qb;
+    it.r = rest / p.num_kv_heads;
+    it.kvh = rest - it.r * p.num_kv_heads;
+    it.row = __ldg(p.table_idx + it.r);
+    it.c = __ldg(p.cached_len + it.r);
+    const int L = __ldg(p.seq_len + it.r);
+    it.qo = __ldg(p.q_offset + it.r);
+    it.n = L - it.c;
+    if (it.row < 0 || it.row >= p.pt_rows || it.c < 0 || it.n < 0 || L > p.pt_stride || L > p.max_seq_len ||
+        it.n > p.max_q_len || it.qo < 0 || it.qo + it.n > p.total_q || __ldg(p.q_offset + it.r + 1) - it.qo != it.n)
+        return -1;
+    const int tpq = p.tokens_per_qtile;
+    it.tok0 = qb * kQTiles * tpq;
+    if (it.tok0 >= it.n) return 0;
+    const int last_tok = min(it.tok0 + kQTiles * tpq, it.n) - 1;
+    it.kv_len = it.c + last_tok + 1;
+    it.n_kv = (it.kv_len + kN - 1) / kN;
+    it.q1 = it.tok0 + tpq < it.n;
+    return 1;
+}
+
+// error bits of a request whose item_info returned -1
+__device__ __forceinline__ unsigned item_error(const Params &p, const Item &it) {
+    return (it.row < 0 || it.row >= p.pt_rows) ? (unsigned)MG_DEVERR_ROW_RANGE : (unsigned)MG_DEVERR_LENGTH;
+}
+
+// The position in the work list of this CTA's k-th item: snake order over the
+// G CTAs (k, 2G-1-k, 2G+k, ...).
+__device__ __forceinline__ int snake_position(int k) {
+    const int G = gridDim.x, c = blockIdx.x;
+    const int round = k >> 1;
+    return round * 2 * G + ((k & 1) ? 2 * G - 1 - c : c);
+}
+
+// Walks this CTA's items: sorted mode reads the CTA's list, otherwise the
+// item ids at the snake positions of the enumeration (skipping empty ones).
+struct ItemCursor {
+    int k;  // next index into the CTA's sequence
+};
+// With `flag` set, an item whose request metadata is inconsistent is flagged
+// (unsorted mode: each CTA flags the items at its own positions; sorted mode
+// flags them while the list is built).
+__device__ __forceinline__ bool next_item(const Params &p, ItemCursor &cur, const int *list, int list_len,
+                                          bool sorted, Item &it, bool flag = false) {
+    for (;;) {
+        int id;
+        if (sorted) {
+            if (cur.k >= list_len) return false;
+            id = list[cur.k++];
+        } else {
+            id = snake_position(cur.k++);
+            if (id >= p.num_items) return false;
+        }
+        const int st = item_info(p, id, it);
+        if (st == 1) return true;
+        if (st < 0 && flag && !sorted) atomicOr(&g_mg_device_error, item_error(p, it));
+    }
+}
+
+// ---------------------------------------------------------------- loaders
+// One loader group (NW warps) copies the K (or V) rows of every tile of the
+// CTA's items into its ring.  Warp u of the group owns the row pairs
+// p = u, u + NW, ... of a tile (keys 2p, 2p+1); its key list index i is pair
+// i / 2, key 2p + (i & 1), and lane l holds the page-table entries (slots) of
+// list indices l and l + 32, fetched one tile ahead.
+template <int NW, int STAGES>
+__device__ __forceinline__ void load_rows(const Params &p, uint32_t ring_base, uint32_t full0, uint32_t empty0,
+                                          const __nv_bfloat16 *pool, int u, int lane, const int *list, int list_len,
+                                          bool sorted, volatile int *abort_flag, uint64_t lim, bool flag_errors) {
+    constexpr int kMaxPairs = (kPairs + NW - 1) / NW;
+    const int npairs = (kPairs - u + NW - 1) / NW;
+    const int64_t head_stride = (int64_t)p.num_kv_heads * kHeadDim;
+    auto key_of = [&](int i) { return 2 * (u + NW * (i >> 1)) + (i & 1); };
+    // slots of (item, tile j) for list indices lane and lane + 32 (-1: none)
+    auto fetch = [&](int row, int kv_len, int j, int &sa, int &sb) {
+        const int32_t *pt = p.page_table + (int64_t)row * p.pt_stride;
+        sa = sb = -1;
+        const int ka = j * kN + key_of(lane), kb = j * kN + key_of(lane + 32);
+        if (lane < 2 * npairs && ka < kv_len) sa = __ldg(pt + ka);
+        if (lane + 32 < 2 * npairs && kb < kv_len) sb = __ldg(pt + kb);
+    };
+    // a slot outside the pool: flagged, and its row zero-filled (and masked by
+    // the causal limit or never read: a rejected key of a visible position
+    // reads as zeros, as in the other kernels' bounds checks)
+    auto check = [&](int &s, bool present) {
+        if (present && (s < 0 || (int64_t)s >= p.num_slots)) {
+            if (flag_errors) atomicOr(&g_mg_device_error, MG_DEVERR_SLOT_RANGE);
+            s = -1;
+        }
+    };
+    ItemCursor cur{0};
+    const bool flag_items = flag_errors && u == 0 && lane == 0;
+    int row, kvh, kv_len, n_kv;  // the current item, as the copies need it
+    {
+        Item it;
+        if (!next_item(p, cur, list, list_len, sorted, it, flag_items)) return;
+        row = it.row; kvh = it.kvh; kv_len = it.kv_len; n_kv = it.n_kv;
+    }
+    int j = 0;
+    int sa, sb;
+    fetch(row, kv_len, 0, sa, sb);
+    const int c = lane & 15, half = c >> 3, cc = c & 7;
+    for (int seq = 0;; ++seq) {
+        // tile (it, j): wait for its ring stage
+        const int stage = seq % STAGES;
+        if (seq >= STAGES && !wait_or_abort(empty0 + stage * 8, ((seq / STAGES) - 1) & 1, abort_flag, lim)) break;
+        check(sa, lane < 2 * npairs && j * kN + key_of(lane) < kv_len);
+        check(sb, lane + 32 < 2 * npairs && j * kN + key_of(lane + 32) < kv_len);
+        const uint32_t tile = ring_base + (uint32_t)(stage * kTileBytes);
+#pragma unroll
+        for (int m = 0; m < kMaxPairs; ++m) {
+            if (m < npairs) {
+                const int i = 2 * m + (lane >> 4);  // list index this half-warp copies
+                const int key = key_of(i);
+                const int slot = m < 16 ? __shfl_sync(0xffffffffu, sa, i & 31) : __shfl_sync(0xffffffffu, sb, i & 31);
+                const __nv_bfloat16 *src = pool + (int64_t)(slot < 0 ? 0 : slot) * head_stride +
+                                           (int64_t)kvh * kHeadDim + c * 8;
+                const uint32_t dst = tile + half * kHalfBytes + key * 128 + ((cc ^ (key & 7)) << 4);
+                cp_async_16(dst, src, slot < 0 ? 0u : 16u);
+            }
+        }
+        cp_async_arrive_noinc(full0 + stage * 8);
+        // advance to the next tile and fetch its page-table entries now, so they
+        // arrive while this warp waits for the next stage
+        if (++j == n_kv) {
+            Item it;
+            if (!next_item(p, cur, list, list_len, sorted, it, flag_items)) break;
+            row = it.row; kvh = it.kvh; kv_len = it.kv_len; n_kv = it.n_kv;
+            j = 0;
+        }
+        fetch(row, kv_len, j, sa, sb);
+    }
+    cp_async_commit();
+    cp_async_wait<0>();  // nothing in flight into shared memory at teardown
+}
+
+// ---------------------------------------------------------------- the kernel
+
 __global__ void __launch_bounds__(kThreads, 1)
     extend_kernel(const __grid_constant__ CUtensorMap tm_q, const Params p) {
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -186,70 +393,80 @@ __global__ void __launch_bounds__(kThreads, 1)
         return;
     }
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffMisc);
-    const uint64_t lim = p.wait_limit_ns;  // nanoseconds
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + kOffMisc + 4);
-
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int r = blockIdx.z, kvh = blockIdx.y;
+    int *sh_count = reinterpret_cast<int *>(smem + kOffMisc + 8);
+    int *items = reinterpret_cast<int *>(smem + kOffItems);
+    const uint64_t lim = p.wait_limit_ns;  // nanoseconds
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     griddep_launch_dependents();
     griddep_wait();  // inputs written by the previous kernel (e.g. the KV store)
-    const int qb = gridDim.x - 1 - blockIdx.x;  // heaviest (latest) q blocks first
 
-    // ---- request metadata (uniform across the CTA; exit before any barrier)
-    const int row = __ldg(p.table_idx + r);
-    const int c = __ldg(p.cached_len + r);
-    const int L = __ldg(p.seq_len + r);
-    const int qo = __ldg(p.q_offset + r);
-    const int n = L - c;
-    {
+    // ---- the work list.  Sorted mode: every CTA sorts the same keys (cost
+    // descending, enumeration order for ties) in the K ring, which no load has
+    // touched yet, and keeps the ids at its snake positions.
+    const bool sorted = p.num_items <= kMaxSortItems;
+    if (sorted) {
+        uint32_t *keys = reinterpret_cast<uint32_t *>(smem + kOffK);
+        int m = 1;
+        while (m < p.num_items) m <<= 1;
         unsigned bad = 0;
-        if (row < 0 || row >= p.pt_rows) bad |= MG_DEVERR_ROW_RANGE;
-        if (c < 0 || n < 0 || L > p.pt_stride || L > p.max_seq_len || n > p.max_q_len || qo < 0 ||
-            qo + n > p.total_q || __ldg(p.q_offset + r + 1) - qo != n)
-            bad |= MG_DEVERR_LENGTH;
-        if (bad) {
-            if (threadIdx.x == 0 && blockIdx.x == 0 && kvh == 0) atomicOr(&g_mg_device_error, bad);
-            return;
+        for (int i = tid; i < m; i += kThreads) {
+            uint32_t key = 0;
+            if (i < p.num_items) {
+                Item it;
+                const int st = item_info(p, i, it);
+                if (st == 1) key = ((uint32_t)min(it.n_kv, kMaxCost) << 20) | (uint32_t)(0xFFFFF - i);
+                if (st < 0) bad |= item_error(p, it);
+            }
+            keys[i] = key;
         }
+        if (bad && blockIdx.x == 0) atomicOr(&g_mg_device_error, bad);
+        __syncthreads();
+        for (int k = 2; k <= m; k <<= 1) {  // bitonic sort, descending
+            for (int jj = k >> 1; jj > 0; jj >>= 1) {
+                for (int i = tid; i < m; i += kThreads) {
+                    const int ixj = i ^ jj;
+                    if (ixj > i) {
+                        const uint32_t a = keys[i], b = keys[ixj];
+                        if ((i & k) == 0 ? a < b : a > b) {
+                            keys[i] = b;
+                            keys[ixj] = a;
+                        }
+                    }
+                }
+                __syncthreads();
+            }
+        }
+        if (tid == 0) {
+            int cnt = 0;
+            for (int k = 0; cnt < kMaxItemsPerCta; ++k) {
+                const int pos = snake_position(k);
+                if (pos >= m || keys[pos] == 0) break;
+                items[cnt++] = 0xFFFFF - (int)(keys[pos] & 0xFFFFFu);
+            }
+            *sh_count = cnt;
+        }
+    } else if (tid == 0) {
+        *sh_count = 0;
     }
-    const int tpq = p.tokens_per_qtile;
-    const int g = p.group;
-    const int tok0 = qb * kQTiles * tpq;
-    if (tok0 >= n) return;
-    const int last_tok = min(tok0 + kQTiles * tpq, n) - 1;
-    const int kv_len = c + last_tok + 1;  // keys this CTA needs: positions [0, kv_len)
-    const int n_kv = (kv_len + kN - 1) / kN;
-    const bool has_q1 = tok0 + tpq < n;
 
-    Sync sy;
-    {
-        uint32_t b = sbase + kOffBar;
-        sy.q_full = b; b += 8;
-        sy.drain = b; b += 8;
-        for (int s = 0; s < kKStages; ++s) { sy.k_full[s] = b; b += 8; }
-        for (int s = 0; s < kKStages; ++s) { sy.k_empty[s] = b; b += 8; }
-        for (int s = 0; s < kVStages; ++s) { sy.v_full[s] = b; b += 8; }
-        for (int s = 0; s < kVStages; ++s) { sy.v_empty[s] = b; b += 8; }
-        for (int t = 0; t < kQTiles; ++t) { sy.s_full[t] = b; b += 8; }
-        for (int t = 0; t < kQTiles; ++t) { sy.p_full[t] = b; b += 8; }
-        for (int t = 0; t < kQTiles; ++t) { sy.o_done[t] = b; b += 8; }
-    }
-    if (threadIdx.x == 0) {
+    if (tid == 0) {
         *abort_flag = 0;
-        mbar_init(sy.q_full, 1);
-        mbar_init(sy.drain, 1);
+        mbar_init(bar_at(sbase, kBarDrain), 1);
+        for (int t = 0; t < kQTiles; ++t) {
+            mbar_init(bar_at(sbase, kBarQFull + t), 1);
+            mbar_init(bar_at(sbase, kBarSFull + t), 1);
+            mbar_init(bar_at(sbase, kBarPFull + t), 128);
+            mbar_init(bar_at(sbase, kBarODone + t), 1);
+            mbar_init(bar_at(sbase, kBarOFree + t), 128);
+        }
         for (int s = 0; s < kKStages; ++s) {
-            mbar_init(sy.k_full[s], kLoaders * 32);  // one arrival per lane of the load warps
-            mbar_init(sy.k_empty[s], 1);
+            mbar_init(bar_at(sbase, kBarKFull + s), kKLoaders * 32);  // one arrival per lane of the K loaders
+            mbar_init(bar_at(sbase, kBarKEmpty + s), 1);
         }
         for (int s = 0; s < kVStages; ++s) {
-            mbar_init(sy.v_full[s], kLoaders * 32);
-            mbar_init(sy.v_empty[s], 1);
-        }
-        for (int t = 0; t < kQTiles; ++t) {
-            mbar_init(sy.s_full[t], 1);
-            mbar_init(sy.p_full[t], 128);
-            mbar_init(sy.o_done[t], 1);
+            mbar_init(bar_at(sbase, kBarVFull + s), kVLoaders * 32);
+            mbar_init(bar_at(sbase, kBarVEmpty + s), 1);
         }
         fence_mbarrier_init();
     }
@@ -258,9 +475,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_relinquish();
     }
     tc_fence_before();
-    __syncthreads();
+    __syncthreads();  // also: the sort scratch in the K ring is dead from here on
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
+    const int list_len = *sh_count;
+    const int g = p.group, tpq = p.tokens_per_qtile;
 
     // setmaxnreg is issued once per warpgroup role, at the top of its branch
     if (warp >= 4 && warp < 12) {
@@ -270,106 +489,152 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int wq = warp & 3;        // TMEM lane quarter this warp may access
         const int qrow = wq * 32 + lane;
         const int tok_local = qrow / g, head_local = qrow - tok_local * g;
-        const int i = tok0 + t * tpq + tok_local;  // new-token index within the request
-        const bool valid = tok_local < tpq && i < n;
-        const int last_key = valid ? c + i : kv_len - 1;  // last visible key position
-        const bool active = t == 0 || has_q1;
         const uint32_t lane_addr = (uint32_t)(wq * 32) << 16;
         const uint32_t tS = tmem + lane_addr + col_s(t);
         const uint32_t tO = tmem + lane_addr + col_o(t);
-        float m_run = -INFINITY, l_run = 0.f;
-        bool ok = active;
-        for (int j = 0; ok && j < n_kv; ++j) {
-            if (!(ok = wait_or_abort(sy.s_full[t], j & 1, abort_flag, lim))) break;
-            tc_fence_after();
-            uint32_t sv[128];
-            tmem_ld_32x32b_x32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-            tmem_ld_32x32b_x32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-            tmem_ld_32x32b_x32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[64]));
-            tmem_ld_32x32b_x32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
-            tmem_ld_wait();
-            const int key0 = j * kN;
-            const int nvis = min(max(last_key - key0 + 1, 0), kN);  // visible keys in this tile
-            // Row max of the raw scores (scale > 0, so scaling commutes with the
-            // max); a tile every key of which is visible to the whole warp skips
-            // the mask.
-            const bool full = __all_sync(0xffffffffu, nvis == kN);
-            float mx;
-            if (full) {
-                float m0 = -INFINITY, m1 = -INFINITY;
-#pragma unroll
-                for (int e = 0; e < 128; e += 4) {
-                    m0 = fmax3(m0, __uint_as_float(sv[e]), __uint_as_float(sv[e + 1]));
-                    m1 = fmax3(m1, __uint_as_float(sv[e + 2]), __uint_as_float(sv[e + 3]));
-                }
-                mx = fmaxf(m0, m1);
-            } else {
-                mx = -INFINITY;
-#pragma unroll
-                for (int e = 0; e < 128; ++e) {
-                    const float x = e < nvis ? __uint_as_float(sv[e]) : -INFINITY;
-                    sv[e] = __float_as_uint(x);
-                    mx = fmaxf(mx, x);
-                }
+        const bool elected = (warp & 3) == 0 && lane == 0;  // issues this Q tile's TMA loads
+        const uint32_t qbytes = (uint32_t)(2 * 128 * g * tpq);
+        const uint32_t b_q = bar_at(sbase, kBarQFull + t), b_s = bar_at(sbase, kBarSFull + t);
+        const uint32_t b_p = bar_at(sbase, kBarPFull + t), b_o = bar_at(sbase, kBarODone + t);
+        const uint32_t b_free = bar_at(sbase, kBarOFree + t);
+        auto load_q = [&](const Item &it) {
+            mbar_arrive_expect_tx(b_q, qbytes);
+            for (int h = 0; h < 2; ++h)
+                tma_load_3d(sbase + kOffQ + t * kTileBytes + h * kHalfBytes, &tm_q, b_q, h * 64, it.kvh * g,
+                            it.qo + it.tok0 + t * tpq);
+        };
+        // the items that use this Q tile: all of them for tile 0, those whose
+        // second tile holds tokens for tile 1
+        auto next_active = [&](ItemCursor &c, Item &out) {
+            while (next_item(p, c, items, list_len, sorted, out))
+                if (t == 0 || out.q1) return true;
+            return false;
+        };
+        ItemCursor cur{0}, ahead{0};
+        Item it, nx;
+        int cnt = 0;       // KV tiles this Q tile has processed (phase of s_full / p_full / o_done)
+        int q_issued = 0;  // Q loads issued for this Q tile (phase of q_full)
+        bool ok = true;
+        if (elected) {  // the first item's Q tile
+            prefetch_tmap(&tm_q);
+            if (next_active(ahead, nx)) {
+                load_q(nx);
+                ++q_issued;
             }
-            const float m_new = fmaxf(m_run, mx * p.scale_log2);
-            const bool need = m_new > m_run + kRescaleThreshold;  // also true for the first tile
-            const bool warp_need = __any_sync(0xffffffffu, need);
-            float corr = 1.f;
-            if (warp_need) {
-                const float m_tgt = need ? m_new : m_run;
-                corr = m_run == -INFINITY ? 0.f : fast_exp2(m_run - m_tgt);
-                m_run = m_tgt;
-                l_run *= corr;
-            }
-            // P = 2^(s * scale_log2 - m), one fused multiply-add per pair of keys
-            const float mu = m_run == -INFINITY ? 0.f : m_run;
-            const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
-            const float2 nmu2 = make_float2(-mu, -mu);
-            float2 rs2 = make_float2(0.f, 0.f);
-#pragma unroll
-            for (int cb = 0; cb < 4; ++cb) {  // masked keys hold -inf and give exactly 0
-                uint32_t pk[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const float2 x = ffma2(make_float2(__uint_as_float(sv[cb * 32 + 2 * e]),
-                                                       __uint_as_float(sv[cb * 32 + 2 * e + 1])),
-                                           sc2, nmu2);
-                    pk[e] = pack_bf16x2(fast_exp2(x.x), fast_exp2(x.y));
-                    // the row sum adds the same bf16-rounded P the PV product reads
-                    rs2 = fadd2(rs2, make_float2(bf16x2_lo(pk[e]), bf16x2_hi(pk[e])));
-                }
-                tmem_st_32x32b_x16(tS + cb * 16, pk);
-            }
-            l_run += rs2.x + rs2.y;
-            if (warp_need && j > 0) {
-                // O holds the sum up to tile j-1; rescale it once that PV is done
-                if (!(ok = wait_or_abort(sy.o_done[t], (j - 1) & 1, abort_flag, lim))) break;
+        }
+        __syncwarp();
+        while (ok && next_active(cur, it)) {
+            const int i = it.tok0 + t * tpq + tok_local;  // new-token index within the request
+            const bool valid = tok_local < tpq && i < it.n;
+            const int last_key = valid ? it.c + i : it.kv_len - 1;  // last visible key position
+            const int n_kv = it.n_kv;
+            const int64_t out_row = (int64_t)(it.qo + i) * p.num_q_heads + it.kvh * g + head_local;
+            float m_run = -INFINITY, l_run = 0.f;
+            for (int j = 0; j < n_kv; ++j) {
+                if (!(ok = wait_or_abort(b_s, (cnt + j) & 1, abort_flag, lim))) break;
                 tc_fence_after();
+                if (j == n_kv - 1 && elected && next_active(ahead, nx)) {
+                    // the last Q K^T of this item has completed: Q tile t is free for
+                    // the next item that uses it
+                    load_q(nx);
+                    ++q_issued;
+                }
+                __syncwarp();  // the TMEM loads below are warp-collective
+                uint32_t sv[128];
+                tmem_ld_32x32b_x32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+                tmem_ld_32x32b_x32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+                tmem_ld_32x32b_x32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[64]));
+                tmem_ld_32x32b_x32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
+                tmem_ld_wait();
+                const int key0 = j * kN;
+                const int nvis = min(max(last_key - key0 + 1, 0), kN);  // visible keys in this tile
+                // Row max of the raw scores (scale > 0, so scaling commutes with the
+                // max); a tile every key of which is visible to the whole warp skips
+                // the mask.
+                const bool full = __all_sync(0xffffffffu, nvis == kN);
+                float mx;
+                if (full) {
+                    float m0 = -INFINITY, m1 = -INFINITY;
 #pragma unroll
-                for (int cb = 0; cb < 4; ++cb) {
-                    uint32_t ov[32];
-                    tmem_ld_32x32b_x32(tO + cb * 32, ov);
-                    tmem_ld_wait();
-                    uint32_t lo[16], hi[16];
+                    for (int e = 0; e < 128; e += 4) {
+                        m0 = fmax3(m0, __uint_as_float(sv[e]), __uint_as_float(sv[e + 1]));
+                        m1 = fmax3(m1, __uint_as_float(sv[e + 2]), __uint_as_float(sv[e + 3]));
+                    }
+                    mx = fmaxf(m0, m1);
+                } else {
+                    mx = -INFINITY;
+#pragma unroll
+                    for (int e = 0; e < 128; ++e) {
+                        const float x = e < nvis ? __uint_as_float(sv[e]) : -INFINITY;
+                        sv[e] = __float_as_uint(x);
+                        mx = fmaxf(mx, x);
+                    }
+                }
+                const float m_new = fmaxf(m_run, mx * p.scale_log2);
+                const bool need = m_new > m_run + kRescaleThreshold;  // also true for the first tile
+                const bool warp_need = __any_sync(0xffffffffu, need);
+                float corr = 1.f;
+                if (warp_need) {
+                    const float m_tgt = need ? m_new : m_run;
+                    corr = m_run == -INFINITY ? 0.f : fast_exp2(m_run - m_tgt);
+                    m_run = m_tgt;
+                    l_run *= corr;
+                }
+                // P = 2^(s * scale_log2 - m), one fused multiply-add per pair of keys;
+                // the first kEmuPairs pairs of every 16 on the FMA pipe, the rest on MUFU
+                const float mu = m_run == -INFINITY ? 0.f : m_run;
+                const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+                const float2 nmu2 = make_float2(-mu, -mu);
+                float2 rs2 = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int cb = 0; cb < 4; ++cb) {  // masked keys hold -inf and give exactly 0
+                    uint32_t pk[16];
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
-                        lo[e] = __float_as_uint(__uint_as_float(ov[e]) * corr);
-                        hi[e] = __float_as_uint(__uint_as_float(ov[16 + e]) * corr);
+                        const float2 x = ffma2(make_float2(__uint_as_float(sv[cb * 32 + 2 * e]),
+                                                           __uint_as_float(sv[cb * 32 + 2 * e + 1])),
+                                               sc2, nmu2);
+                        if (e < kEmuPairs) {
+                            const float2 ex = exp2_fma2(x);
+                            pk[e] = pack_bf16x2(ex.x, ex.y);
+                        } else {
+                            pk[e] = pack_bf16x2(fast_exp2(x.x), fast_exp2(x.y));
+                        }
+                        // the row sum adds the same bf16-rounded P the PV product reads
+                        rs2 = fadd2(rs2, make_float2(bf16x2_lo(pk[e]), bf16x2_hi(pk[e])));
                     }
-                    tmem_st_32x32b_x16(tO + cb * 32, lo);
-                    tmem_st_32x32b_x16(tO + cb * 32 + 16, hi);
+                    tmem_st_32x32b_x16(tS + cb * 16, pk);
                 }
+                l_run += rs2.x + rs2.y;
+                if (warp_need && j > 0) {
+                    // O holds the sum up to tile j-1; rescale it once that PV is done
+                    if (!(ok = wait_or_abort(b_o, (cnt + j - 1) & 1, abort_flag, lim))) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int cb = 0; cb < 4; ++cb) {
+                        uint32_t ov[32];
+                        tmem_ld_32x32b_x32(tO + cb * 32, ov);
+                        tmem_ld_wait();
+                        uint32_t lo[16], hi[16];
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) {
+                            lo[e] = __float_as_uint(__uint_as_float(ov[e]) * corr);
+                            hi[e] = __float_as_uint(__uint_as_float(ov[16 + e]) * corr);
+                        }
+                        tmem_st_32x32b_x16(tO + cb * 32, lo);
+                        tmem_st_32x32b_x16(tO + cb * 32 + 16, hi);
+                    }
+                }
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(b_p);
             }
-            tmem_st_wait();
-            tc_fence_before();
-            mbar_arrive(sy.p_full[t]);
-        }
-        // ---- epilogue: O / l -> bf16 -> out
-        if (ok && wait_or_abort(sy.o_done[t], (n_kv - 1) & 1, abort_flag, lim)) {
+            if (!ok) break;
+            // ---- epilogue: O / l -> bf16 -> out, then O is free for the next item
+            if (!(ok = wait_or_abort(b_o, (cnt + n_kv - 1) & 1, abort_flag, lim))) break;
             tc_fence_after();
             const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-            __nv_bfloat16 *dst = p.out + ((int64_t)(qo + i) * p.num_q_heads + kvh * g + head_local) * kHeadDim;
+            __nv_bfloat16 *dst = p.out + out_row * kHeadDim;
 #pragma unroll
             for (int cb = 0; cb < 4; ++cb) {
                 uint32_t ov[32];
@@ -388,7 +653,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             }
+            tc_fence_before();
+            mbar_arrive(b_free);
+            cnt += n_kv;
         }
+        // a Q load issued for an item that never ran (after an abort) must land
+        // before the CTA exits; after a normal run it has long completed
+        if (elected && q_issued > 0) wait_bounded(b_q, (q_issued - 1) & 1, lim);
     } else {
         setmaxnreg_dec<kRegsLoad>();
         if (warp == kMmaWarp) {
@@ -396,163 +667,122 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) {
                 constexpr uint32_t idesc_qk = idesc_bf16(false);
                 constexpr uint32_t idesc_pv = idesc_bf16(true);
-                auto issue_s = [&](int t, int j, bool signal) {
+                auto issue_s = [&](int t, int stage, bool signal) {
                     const uint32_t qa = sbase + kOffQ + t * kTileBytes;
-                    const uint32_t ka = sbase + kOffK + (j % kKStages) * kTileBytes;
-#pragma unroll
+                    const uint32_t ka = sbase + kOffK + stage * kTileBytes;
+                    // unrolled by two only: fully unrolled, the descriptors of every
+                    // stage and k step are hoisted out of the item loop and spill
+#pragma unroll 2
                     for (int kk = 0; kk < 8; ++kk) {
                         const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
                         umma_ss(tmem + col_s(t), sw128_desc(qa + off, 16, 1024), sw128_desc(ka + off, 16, 1024),
                                 idesc_qk, kk > 0);
                     }
-                    if (signal) umma_commit(sy.s_full[t]);
+                    if (signal) umma_commit(bar_at(sbase, kBarSFull + t));
                 };
-                auto issue_pv = [&](int t, int j) {
-                    const uint32_t va = sbase + kOffV + (j % kVStages) * kTileBytes;
-#pragma unroll
+                auto issue_pv = [&](int t, int stage, bool accumulate) {
+                    const uint32_t va = sbase + kOffV + stage * kTileBytes;
+#pragma unroll 2
                     for (int kk = 0; kk < 8; ++kk)
                         umma_ts(tmem + col_o(t), tmem + col_s(t) + kk * 8,
-                                sw128_desc(va + kk * 2048, kHalfBytes, 1024), idesc_pv, (j > 0 || kk > 0));
-                    umma_commit(sy.o_done[t]);
+                                sw128_desc(va + kk * 2048, kHalfBytes, 1024), idesc_pv, (accumulate || kk > 0));
+                    umma_commit(bar_at(sbase, kBarODone + t));
                 };
-                bool ok = wait_or_abort_thread(sy.q_full, 0, abort_flag, lim) && wait_or_abort_thread(sy.k_full[0], 0, abort_flag, lim);
-                if (ok) {
+                ItemCursor cur{0};
+                Item it;
+                int cnt[kQTiles] = {0, 0};      // KV tiles processed per Q tile
+                int items_t[kQTiles] = {0, 0};  // items processed per Q tile (phase of q_full / o_free)
+                int kseq = 0, vseq = 0;
+                bool ok = true, first = true;
+                while (ok && next_item(p, cur, items, list_len, sorted, it)) {
+                    const bool q1 = it.q1;
+                    ok = wait_or_abort_thread(bar_at(sbase, kBarQFull), items_t[0] & 1, abort_flag, lim) &&
+                         (!q1 || wait_or_abort_thread(bar_at(sbase, kBarQFull + 1), items_t[1] & 1, abort_flag, lim)) &&
+                         wait_or_abort_thread(bar_at(sbase, kBarKFull + kseq % kKStages), (kseq / kKStages) & 1,
+                                              abort_flag, lim);
+                    if (!ok) break;
                     fence_proxy_async_smem();
                     tc_fence_after();
-                    // the fault-injection hook withholds Q tile 0's first hand-off, so its
-                    // softmax warps wait for a tile that is never signalled ready
-                    issue_s(0, 0, p.inject_stall == 0);
-                    if (has_q1) issue_s(1, 0, true);
-                    umma_commit(sy.k_empty[0]);
-                }
-                for (int j = 0; ok && j < n_kv; ++j) {
-                    const int sv = j % kVStages;
-                    if (!(ok = wait_or_abort_thread(sy.v_full[sv], (j / kVStages) & 1, abort_flag, lim))) break;
-                    fence_proxy_async_smem();  // cp.async (generic proxy) writes -> tensor core reads
-                    if (!(ok = wait_or_abort_thread(sy.p_full[0], j & 1, abort_flag, lim))) break;
-                    tc_fence_after();
-                    issue_pv(0, j);
-                    const bool more = j + 1 < n_kv;
-                    if (more) {
-                        const int sk = (j + 1) % kKStages;
-                        if (!(ok = wait_or_abort_thread(sy.k_full[sk], ((j + 1) / kKStages) & 1, abort_flag, lim))) break;
-                        fence_proxy_async_smem();
-                        tc_fence_after();
-                        issue_s(0, j + 1, true);
+                    {
+                        const int ks = kseq % kKStages;
+                        // the fault-injection hook withholds the first item's first
+                        // hand-off to Q tile 0's softmax, which then waits for a tile
+                        // that is never signalled ready
+                        issue_s(0, ks, !(first && p.inject_stall));
+                        if (q1) issue_s(1, ks, true);
+                        umma_commit(bar_at(sbase, kBarKEmpty + ks));
+                        ++kseq;
                     }
-                    if (has_q1) {
-                        if (!(ok = wait_or_abort_thread(sy.p_full[1], j & 1, abort_flag, lim))) break;
+                    first = false;
+                    for (int j = 0; j < it.n_kv; ++j) {
+                        const int vs = vseq % kVStages;
+                        if (!(ok = wait_or_abort_thread(bar_at(sbase, kBarVFull + vs), (vseq / kVStages) & 1,
+                                                        abort_flag, lim)))
+                            break;
+                        fence_proxy_async_smem();  // cp.async (generic proxy) writes -> tensor core reads
+                        if (!(ok = wait_or_abort_thread(bar_at(sbase, kBarPFull), (cnt[0] + j) & 1, abort_flag, lim)))
+                            break;
+                        // O_0 holds the previous item's result until its epilogue has read it
+                        if (j == 0 && items_t[0] > 0 &&
+                            !(ok = wait_or_abort_thread(bar_at(sbase, kBarOFree), (items_t[0] - 1) & 1, abort_flag,
+                                                        lim)))
+                            break;
                         tc_fence_after();
-                        issue_pv(1, j);
+                        issue_pv(0, vs, j > 0);
+                        const bool more = j + 1 < it.n_kv;
+                        const int ks = kseq % kKStages;
+                        if (more) {
+                            if (!(ok = wait_or_abort_thread(bar_at(sbase, kBarKFull + ks), (kseq / kKStages) & 1,
+                                                            abort_flag, lim)))
+                                break;
+                            fence_proxy_async_smem();
+                            tc_fence_after();
+                            issue_s(0, ks, true);
+                        }
+                        if (q1) {
+                            if (!(ok = wait_or_abort_thread(bar_at(sbase, kBarPFull + 1), (cnt[1] + j) & 1, abort_flag,
+                                                            lim)))
+                                break;
+                            if (j == 0 && items_t[1] > 0 &&
+                                !(ok = wait_or_abort_thread(bar_at(sbase, kBarOFree + 1), (items_t[1] - 1) & 1,
+                                                            abort_flag, lim)))
+                                break;
+                            tc_fence_after();
+                            issue_pv(1, vs, j > 0);
+                        }
+                        umma_commit(bar_at(sbase, kBarVEmpty + vs));
+                        ++vseq;
+                        if (more) {
+                            if (q1) issue_s(1, ks, true);
+                            umma_commit(bar_at(sbase, kBarKEmpty + ks));
+                            ++kseq;
+                        }
                     }
-                    umma_commit(sy.v_empty[sv]);
-                    if (more) {
-                        if (has_q1) issue_s(1, j + 1, true);
-                        umma_commit(sy.k_empty[(j + 1) % kKStages]);
+                    cnt[0] += it.n_kv;
+                    ++items_t[0];
+                    if (q1) {
+                        cnt[1] += it.n_kv;
+                        ++items_t[1];
                     }
                 }
                 // before TMEM is freed, every MMA this thread issued must have
                 // completed, also after an abort: one commit tracks them all, and
                 // its wait ignores the abort flag (after a normal run it returns
                 // at once: the softmax warps already waited for the last P V)
-                umma_commit(sy.drain);
-                wait_bounded(sy.drain, 0, lim);
+                umma_commit(bar_at(sbase, kBarDrain));
+                wait_bounded(bar_at(sbase, kBarDrain), 0, lim);
             }
             __syncwarp();
+        } else if (warp < kKLoadWarp0 + kKLoaders) {
+            // =============================================================== K loads
+            load_rows<kKLoaders, kKStages>(p, sbase + kOffK, bar_at(sbase, kBarKFull), bar_at(sbase, kBarKEmpty),
+                                           p.k_cache, warp - kKLoadWarp0, lane, items, list_len, sorted, abort_flag,
+                                           lim, true);
         } else {
-            // =============================================================== loads
-            const int li = warp < 4 ? warp : warp - 9;  // load warp index 0 .. kLoaders - 1
-            if (li == 0 && lane == 0) {
-                prefetch_tmap(&tm_q);
-                const uint32_t qbytes = (uint32_t)(kQTiles * 2 * 128 * g * tpq);
-                mbar_arrive_expect_tx(sy.q_full, qbytes);
-                for (int t = 0; t < kQTiles; ++t)
-                    for (int h = 0; h < 2; ++h)
-                        tma_load_3d(sbase + kOffQ + t * kTileBytes + h * kHalfBytes, &tm_q, sy.q_full, h * 64,
-                                    kvh * g, qo + tok0 + t * tpq);
-            }
-            const int32_t *pt = p.page_table + (int64_t)row * p.pt_stride;
-            const int64_t head_stride = (int64_t)p.num_kv_heads * kHeadDim;
-            int *idx_ring = reinterpret_cast<int *>(smem + kOffIdx);
-            // this warp's row pairs of every tile: li, li + kLoaders, ... (< kPairs)
-            const int npairs = (kPairs - li + kLoaders - 1) / kLoaders;
-            // lane l < 2 * npairs owns the page-table entry of key 2 (li + kLoaders (l / 2)) + l % 2
-            const bool has_key = lane < 2 * npairs;
-            const int my_key = 2 * (li + kLoaders * (lane >> 1)) + (lane & 1);
-            // Iteration j copies this warp's K rows of tile j and V rows of tile
-            // j - 1 (K leads V by one tile); each lane then arms the tile's full
-            // barrier with cp.async.mbarrier.arrive.noinc, so the barrier
-            // completes when every load lane's copies have landed, without the
-            // load warps waiting for them.  The page-table entries of tile
-            // j + kIdxAhead ride in the iteration's commit group, the only group
-            // the warp waits for.
-            auto fetch_idx = [&](int j) {
-                if (j < n_kv && has_key) {
-                    const int key = j * kN + my_key;
-                    int *dst = idx_ring + (j % kIdxRing) * kN + my_key;
-                    if (key < kv_len) cp_async_4(smem_u32(dst), pt + key);
-                    else *dst = -1;
-                }
-            };
-            // This warp's row pairs of K or V into a tile stored as two 64-column
-            // halves with the 128-byte swizzle; each warp instruction moves one pair.
-            auto copy_rows = [&](int j, const __nv_bfloat16 *pool, uint32_t tile_base) {
-                const int *ids = idx_ring + (j % kIdxRing) * kN;
-                const int c = lane & 15, half = c >> 3, cc = c & 7;
-#pragma unroll
-                for (int m = 0; m < kMaxPairsPerLoader; ++m) {
-                    if (m < npairs) {
-                        const int key = 2 * (li + kLoaders * m) + (lane >> 4);
-                        int slot = j * kN + key < kv_len ? ids[key] : -1;
-                        if (slot >= 0 && (int64_t)slot >= p.num_slots) slot = -1;  // flagged by check_rows
-                        const __nv_bfloat16 *src = pool + (int64_t)(slot < 0 ? 0 : slot) * head_stride +
-                                                   (int64_t)kvh * kHeadDim + c * 8;
-                        const uint32_t dst = tile_base + half * kHalfBytes + key * 128 + ((cc ^ (key & 7)) << 4);
-                        cp_async_16(dst, src, slot < 0 ? 0u : 16u);
-                    }
-                }
-            };
-            auto check_rows = [&](int j) {  // record rejected page-table entries (they were zero-filled)
-                if (has_key && j * kN + my_key < kv_len) {
-                    const int slot = idx_ring[(j % kIdxRing) * kN + my_key];
-                    if (slot < 0 || (int64_t)slot >= p.num_slots) atomicOr(&g_mg_device_error, MG_DEVERR_SLOT_RANGE);
-                }
-            };
-#pragma unroll
-            for (int j = 0; j < kIdxAhead; ++j) {
-                fetch_idx(j);
-                cp_async_commit();
-            }
-            for (int j = 0; j <= n_kv; ++j) {
-                if (j < n_kv) {
-                    const int s = j % kKStages;
-                    if (j >= kKStages && !wait_or_abort(sy.k_empty[s], ((j / kKStages) - 1) & 1, abort_flag, lim)) break;
-                }
-                if (j >= 1) {
-                    const int jv = j - 1, s = jv % kVStages;
-                    if (jv >= kVStages && !wait_or_abort(sy.v_empty[s], ((jv / kVStages) - 1) & 1, abort_flag, lim)) break;
-                }
-                cp_async_wait<kIdxAhead - 1>();  // entries of tile j (kIdxAhead groups old) landed
-                __syncwarp();
-                if (j < n_kv) {
-                    check_rows(j);
-                    copy_rows(j, p.k_cache, sbase + kOffK + (j % kKStages) * kTileBytes);
-                    cp_async_arrive_noinc(sy.k_full[j % kKStages]);
-                }
-                if (j >= 1) {
-                    copy_rows(j - 1, p.v_cache, sbase + kOffV + ((j - 1) % kVStages) * kTileBytes);
-                    cp_async_arrive_noinc(sy.v_full[(j - 1) % kVStages]);
-                }
-                // only now reuse the ring slot of tile j - 1 (every lane has read its
-                // entries for the V rows just issued)
-                __syncwarp();
-                fetch_idx(j + kIdxAhead);
-                cp_async_commit();
-            }
-            cp_async_wait<0>();  // nothing in flight into shared memory at teardown
-            // the Q tiles' TMA load completes on q_full; after an abort nobody may
-            // have waited for it, and it must land before the CTA exits
-            if (li == 0 && lane == 0) wait_bounded(sy.q_full, 0, lim);
+            // =============================================================== V loads
+            load_rows<kVLoaders, kVStages>(p, sbase + kOffV, bar_at(sbase, kBarVFull), bar_at(sbase, kBarVEmpty),
+                                           p.v_cache, warp - kVLoadWarp0, lane, items, list_len, sorted, abort_flag,
+                                           lim, false);
         }
     }
 
@@ -571,7 +801,7 @@ inline cudaError_t set_attributes() {
     return cudaFuncSetAttribute(extend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
 }
 
-inline mg_status launch(Params &p, cudaStream_t stream) {
+inline mg_status launch(Params &p, int sms, cudaStream_t stream) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return MG_ERR_CUDA;
     const int g = p.group;
@@ -587,11 +817,21 @@ inline mg_status launch(Params &p, cudaStream_t stream) {
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return MG_ERR_CUDA;
     }
-    const int tokens_per_cta = kQTiles * p.tokens_per_qtile;
-    const int nqb = (p.max_q_len + tokens_per_cta - 1) / tokens_per_cta;
-    if (nqb > 0x7fffffff || p.batch > 65535 || p.num_kv_heads > 65535) return MG_ERR_INVALID_ARGUMENT;
-    dim3 grid((unsigned)nqb, (unsigned)p.num_kv_heads, (unsigned)p.batch);
-    return launch_pdl(extend_kernel, grid, dim3(kThreads), kSmemBytes, stream, tq, p);
+    const int64_t tokens_per_item = kQTiles * p.tokens_per_qtile;
+    const int64_t nqb = (p.max_q_len + tokens_per_item - 1) / tokens_per_item;
+    const int64_t items = nqb * p.batch * p.num_kv_heads;
+    if (items <= 0) return MG_OK;
+    if (items >= (int64_t)1 << 30) return MG_ERR_UNSUPPORTED_SHAPE;
+    p.num_qblocks = (int32_t)nqb;
+    p.num_items = (int32_t)items;
+    // one CTA per SM; with a sorted list no CTA may need more than
+    // kMaxItemsPerCta items
+    int64_t grid = items < sms ? items : sms;
+    if (items <= kMaxSortItems) {
+        const int64_t min_grid = (items + kMaxItemsPerCta - 1) / kMaxItemsPerCta;
+        if (grid < min_grid) grid = min_grid;
+    }
+    return launch_pdl(extend_kernel, dim3((unsigned)grid), dim3(kThreads), kSmemBytes, stream, tq, p);
 }
 
 }  // namespace extend

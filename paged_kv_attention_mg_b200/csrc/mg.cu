@@ -413,7 +413,9 @@ mg_status mg_extend_attn(const void *q, const void *k_cache, const void *v_cache
     p.scale_log2 = scale * kLog2e;
     p.wait_limit_ns = g_extend_wait_limit_ns.load(std::memory_order_relaxed);
     p.inject_stall = g_extend_inject_stall.load(std::memory_order_relaxed);
-    return extend::launch(p, static_cast<cudaStream_t>(stream));
+    int sms;
+    if (sm_count(sms) != MG_OK) return MG_ERR_CUDA;
+    return extend::launch(p, sms, static_cast<cudaStream_t>(stream));
 }
 
 mg_status mg_set_extend_wait_limit(uint64_t limit_ns, int32_t inject_stall) {
