@@ -306,7 +306,6 @@ __device__ __forceinline__ void cursor_advance(const Params &p, Cursor &c) {
     if (metadata_ok(p, c.next_L, c.next_row)) {  // the common case: no stall at the boundary
         c.L = c.next_L;
         c.row = c.next_row;
-        c.r0 = c.r;
         c.tiles = (c.L + kKeys - 1) / kKeys;
         cursor_prefetch_next(p, c);
     } else {
@@ -442,7 +441,7 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
                 TileDesc d;
                 d.r = cur.r; d.kvh = cur.kvh; d.t = cur.t; d.tiles = cur.tiles; d.L = cur.L; d.row = cur.row;
                 d.valid = 0; d.store_slot = -1;
-                d.k0 = cur.k0; d.r0 = cur.r0; d.m = cur.m; d.grouped = cur.grouped;
+                if constexpr (CASCADE) { d.k0 = cur.k0; d.r0 = cur.r0; d.m = cur.m; d.grouped = cur.grouped; }
                 my_desc[e] = d;
                 if (FUSED && cur.t == cur.tiles - 1)  // the pair's last tile holds the new token
                     cp_async_4(smem_u32(&my_desc[e].store_slot), p.out_loc + cur.r);
@@ -463,7 +462,7 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
         const int e = j % kDescRing, stage = j % kStages;
         const TileDesc d = my_desc[e];
         int slot = -1;
-        if (lane < kKeys && d.k0 + d.t * kKeys + lane < d.L) {
+        if (lane < kKeys && (CASCADE ? d.k0 : 0) + d.t * kKeys + lane < d.L) {
             slot = my_idx[e][lane];
             if (slot < 0 || (int64_t)slot >= p.num_slots) {
                 atomicOr(&g_mg_device_error, MG_DEVERR_SLOT_RANGE);
@@ -472,14 +471,19 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
         }
         const unsigned valid = __ballot_sync(0xffffffffu, slot >= 0) & 0xFFFFu;
         if (lane == 0) my_desc[e].valid = valid;
+        // fused store: the new token (position L-1) is read from k_new / v_new,
+        // the pool slot is written only after this tile lands.  Its row comes
+        // from k_new / v_new whatever its page-table entry holds, so the store
+        // writes it even when that entry was rejected (the key is then masked
+        // out of the attention, as any rejected key is): its copy is given a
+        // non-negative stand-in slot here, once, rather than a test per row below
+        const int new_key = (FUSED && d.t == d.tiles - 1) ? d.L - 1 - (CASCADE ? d.k0 : 0) - d.t * kKeys : -1;
+        if (FUSED && lane == new_key && slot < 0) slot = 0;
         // 16-byte cp.async: each warp instruction moves two whole 256-byte rows
         // (lanes 0-15 and 16-31); 32 rows per tile (16 K then 16 V)
         const uint32_t base = ring + (uint32_t)(stage * kTileBytes);
         const int ch = lane & 15;
         const int64_t head_off = (int64_t)d.kvh * kHeadDim + ch * 8;
-        // fused store: the new token (position L-1) is read from k_new / v_new,
-        // the pool slot is written only after this tile lands
-        const int new_key = (FUSED && d.t == d.tiles - 1) ? d.L - 1 - d.t * kKeys : -1;
         const int64_t new_off = ((int64_t)d.r * p.num_kv_heads + d.kvh) * kHeadDim + ch * 8;
 #pragma unroll
         for (int it = 0; it < 16; ++it) {
@@ -488,12 +492,8 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
             const bool is_v = rr >= kKeys;
             const int sl = __shfl_sync(0xffffffffu, slot, key);
             const __nv_bfloat16 *src = (is_v ? p.v_cache : p.k_cache) + (int64_t)(sl < 0 ? 0 : sl) * head_stride + head_off;
-            // the new token's row comes from k_new / v_new whatever its page-table
-            // entry holds, so the fused store writes it even when that entry was
-            // rejected (the key is then masked out of the attention, as a bad slot is)
-            const bool is_new = key == new_key;
-            if (is_new) src = (is_v ? p.v_new : p.k_new) + new_off;
-            cp_async_16(base + (is_v ? 2 * kHalfRows : 0) + swz(key, ch), src, (sl < 0 && !is_new) ? 0u : 16u);
+            if (key == new_key) src = (is_v ? p.v_new : p.k_new) + new_off;
+            cp_async_16(base + (is_v ? 2 * kHalfRows : 0) + swz(key, ch), src, sl < 0 ? 0u : 16u);
         }
     };
 
@@ -736,7 +736,7 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
             if constexpr (CASCADE) whole = whole && !c.grouped && c.r >= p.num_groups;
             const int rows = CASCADE ? c.m * g : g;
             const int64_t rs = CASCADE ? p.rows_per_slot : g;
-            const int64_t head0 = (int64_t)c.r0 * p.num_q_heads + (int64_t)c.kvh * g;
+            const int64_t head0 = (int64_t)(CASCADE ? c.r0 : c.r) * p.num_q_heads + (int64_t)c.kvh * g;
             const int64_t slot = (int64_t)c.r * p.num_kv_heads + c.kvh + w;
             for (int h = 0; h < rows; ++h) {
                 const float4 v = *reinterpret_cast<const float4 *>(scr + h * kPitch + lane * 4);

@@ -55,12 +55,16 @@ namespace extend {
 constexpr int kM = 128;                     // query rows per Q tile
 constexpr int kN = 128;                     // keys per KV tile
 constexpr int kQTiles = 2;
-constexpr int kKStages = 3;                 // K ring
-constexpr int kVStages = 2;                 // V ring
+// Ring depths and loader warps: V gets the deeper ring and the larger loader
+// group because a V tile is needed only ~one softmax after its K tile but its
+// slot frees later (after both Q tiles' P V); measured with K 3 / V 2, the MMA
+// issuer waited for V tiles while K tiles sat ready for over 10k cycles.
+constexpr int kKStages = 2;                 // K ring
+constexpr int kVStages = 3;                 // V ring
 constexpr int kThreads = 512;
-constexpr int kKLoadWarp0 = 0, kKLoaders = 4;    // K loaders: warps 0-3
+constexpr int kKLoadWarp0 = 13, kKLoaders = 3;   // K loaders: warps 13-15
 constexpr int kMmaWarp = 12;
-constexpr int kVLoadWarp0 = 13, kVLoaders = 3;   // V loaders: warps 13-15
+constexpr int kVLoadWarp0 = 0, kVLoaders = 4;    // V loaders: warps 0-3
 constexpr int kPairs = kN / 2;              // row pairs per tile (one warp instruction moves a pair)
 constexpr int kRegsLoad = 72;               // registers a thread in warpgroups 0 and 3
 constexpr int kRegsSoftmax = 184;           // registers a thread in warpgroups 1 and 2
@@ -529,6 +533,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int last_key = valid ? it.c + i : it.kv_len - 1;  // last visible key position
             const int n_kv = it.n_kv;
             const int64_t out_row = (int64_t)(it.qo + i) * p.num_q_heads + it.kvh * g + head_local;
+            // a warp whose 32 rows are all padding (a ragged last Q tile, a
+            // one-token request) computes nothing: its rows of P and O are never
+            // read back, it only passes the hand-offs on
+            const bool live = __any_sync(0xffffffffu, valid);
             float m_run = -INFINITY, l_run = 0.f;
             for (int j = 0; j < n_kv; ++j) {
                 if (!(ok = wait_or_abort(b_s, (cnt + j) & 1, abort_flag, lim))) break;
@@ -540,6 +548,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ++q_issued;
                 }
                 __syncwarp();  // the TMEM loads below are warp-collective
+                if (!live) {
+                    tc_fence_before();
+                    mbar_arrive(b_p);
+                    continue;
+                }
                 uint32_t sv[128];
                 tmem_ld_32x32b_x32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
                 tmem_ld_32x32b_x32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
@@ -636,7 +649,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
             __nv_bfloat16 *dst = p.out + out_row * kHeadDim;
 #pragma unroll
-            for (int cb = 0; cb < 4; ++cb) {
+            for (int cb = 0; cb < 4 && live; ++cb) {
                 uint32_t ov[32];
                 tmem_ld_32x32b_x32(tO + cb * 32, ov);
                 tmem_ld_wait();
@@ -773,7 +786,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 wait_bounded(bar_at(sbase, kBarDrain), 0, lim);
             }
             __syncwarp();
-        } else if (warp < kKLoadWarp0 + kKLoaders) {
+        } else if (warp >= kKLoadWarp0 && warp < kKLoadWarp0 + kKLoaders) {
             // =============================================================== K loads
             load_rows<kKLoaders, kKStages>(p, sbase + kOffK, bar_at(sbase, kBarKFull), bar_at(sbase, kBarKEmpty),
                                            p.k_cache, warp - kKLoadWarp0, lane, items, list_len, sorted, abort_flag,

@@ -132,6 +132,19 @@ def _prefix_decode(prefix, lo, hi):
     return draw
 
 
+def _mixed(prefills, c_lo, c_hi, n_lo, n_hi, d_lo, d_hi):
+    """A chunked-prefill scheduler's mixed batch: `prefills` prompt chunks
+    (cached U[c_lo, c_hi], chunk U[n_lo, n_hi]) first, then decode requests (one
+    new token after U[d_lo, d_hi] cached ones)."""
+    def draw(gen, batch):
+        pc = torch.randint(c_lo, c_hi + 1, (prefills,), generator=gen, dtype=torch.int64)
+        pn = torch.randint(n_lo, n_hi + 1, (prefills,), generator=gen, dtype=torch.int64)
+        dc = torch.randint(d_lo, d_hi + 1, (batch - prefills,), generator=gen, dtype=torch.int64)
+        cached = torch.cat([pc, dc])
+        return cached, cached + torch.cat([pn, torch.ones(batch - prefills, dtype=torch.int64)])
+    return draw
+
+
 WORKLOADS: List[WorkloadSpec] = [
     WorkloadSpec("tiny_decode", "decode", 3, 16, 8, 128, 512, 1, 1000, 12,
                  "3 requests, lengths 5/9/12 (new token included), Hq16/Hkv8, pool 512",
@@ -152,6 +165,10 @@ WORKLOADS: List[WorkloadSpec] = [
                  "Qwen3-0.6B attention shape, batch 64 in 8 groups of 8 sharing a 2048-token prefix, "
                  "own tokens U[16,512] after it, pool 200k",
                  _prefix_decode(2048, 16, 512), share=(8, 2048)),
+    WorkloadSpec("mixed_prefill_decode", "extend", 204, 16, 8, 128, 300_000, 1, 1006, 3072,
+                 "one launch over a mixed batch: 4 prompt chunks (cached U[0,1024], chunk U[256,1024]) and "
+                 "200 decode requests (one new token after U[128,2047] cached), Hq16/Hkv8, pool 300k",
+                 _mixed(4, 0, 1024, 256, 1024, 128, 2047)),
 ]
 
 BY_NAME = {w.name: w for w in WORKLOADS}

@@ -29,4 +29,5 @@ def pytest_terminal_summary(terminalreporter):
         terminalreporter.write_line(
             f"parity bound: {WIDENED['checked']} output elements compared with the oracle; "
             f"{WIDENED['over_plain_bound']} above a plain 1e-2 (allowed only where |ref| >= 4, "
-            f"worst |err| {WIDENED['worst_over']:.4e})")
+            f"worst |err| {WIDENED['worst_over']:.4e}); smallest slack to the bound {WIDENED['min_slack']:.4e} "
+            f"at {WIDENED['min_slack_at']}")

@@ -444,6 +444,31 @@ def test_extend_serves_a_mixed_batch():
     assert_matches_oracle(out, oracle_extend(step, data), "mixed decode / prefill batch")
 
 
+def test_extend_serves_the_mixed_workload():
+    """The mixed_prefill_decode workload in one mg_extend_attn launch: 200
+    one-token decode requests and 4 prompt chunks, each decode request an item
+    of its own in the persistent kernel's work list (its padding rows skipped).
+    Sampled rows against the oracle; every decode row also against the decode
+    kernel on the same pool."""
+    spec = wl.BY_NAME["mixed_prefill_decode"]
+    step = wl.make_step(spec)
+    data = wl.make_layer(step)
+    g = GpuStep(step, data)
+    g.store()
+    out = g.extend()
+    assert mg.read_device_error() == 0
+    assert torch.isfinite(out.float()).all()
+    req = [0, 1, 2, 3] + list(range(4, 204, 13))
+    assert_matches_oracle(out, oracle_extend(step, data, requests=req), "mixed_prefill_decode")
+    # decode requests (rows q_offset[r] of out) equal the decode kernel's rows
+    dec_rows = step.q_offset[4:204].long()
+    dq = g.q[dec_rows.cuda()].contiguous()
+    ti, sl = g.table_idx[4:].contiguous(), g.seq_len[4:].contiguous()
+    dec = mg.decode_attn(dq, g.k_cache, g.v_cache, g.page_table, ti, sl, step.max_seq_len, g.scale).float()
+    ext = out[dec_rows.cuda()].float()
+    assert bool(((dec - ext).abs() <= dec.abs() * 2.0 ** -7 + 2e-3).all())
+
+
 # --------------------------------------------------------------------------- shared prefix
 
 def test_decode_and_extend_over_a_shared_prefix():
