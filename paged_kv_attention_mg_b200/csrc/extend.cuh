@@ -14,7 +14,8 @@
 //     tiles of 128 keys.
 //   * persistent CTAs, one per SM.  Every CTA computes the same work list
 //     (items sorted by cost, heaviest first, when there are at most
-//     kMaxSortItems) and takes its items in snake order (k, 2G-1-k, 2G+k, ...),
+//     kMaxSortGroups (request, q block) groups; one warp sorts them in
+//     registers) and takes its items in snake order (k, 2G-1-k, 2G+k, ...),
 //     so the heavy items start first and the loads even out.  Across a CTA's
 //     items the pipelines never drain: K/V rings, barrier phases and TMEM run
 //     on, the next item's Q tiles load while the current item finishes, and an
@@ -47,6 +48,8 @@
 
 #include <cuda.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace mg {
@@ -76,9 +79,14 @@ constexpr int kTmemCols = 512;
 __device__ __forceinline__ uint32_t col_s(int t) { return (uint32_t)t * 128u; }
 __device__ __forceinline__ uint32_t col_o(int t) { return 256u + (uint32_t)t * 128u; }
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
-constexpr int kMaxSortItems = 2048;         // work lists up to this size are sorted by cost
-constexpr int kMaxItemsPerCta = 32;         // sorted lists: items a CTA keeps (the host sizes the grid)
-constexpr int kMaxCost = 4095;              // cost key clamp (KV tiles)
+// The work list is sorted by cost when it has at most kMaxSortGroups groups
+// (a group: the Hkv items of one (request, q block), which cost the same); one
+// warp sorts the group keys in registers.  A CTA keeps at most
+// kMaxItemsPerCta items of a sorted list (the host sizes the grid for that).
+constexpr int kSortPerLane = 8;
+constexpr int kMaxSortGroups = 32 * kSortPerLane;
+constexpr int kMaxItemsPerCta = 32;
+constexpr int kMaxCost = 0xFFFF;            // cost key clamp (KV tiles)
 #ifndef MG_EXTEND_EMU_PAIRS
 #define MG_EXTEND_EMU_PAIRS 4  // of every 16 pairs of exponentials, this many on the FMA pipe
 #endif
@@ -108,7 +116,7 @@ constexpr int kOffItems = kOffBar + kNumBars * 8;
 constexpr int kOffMisc = kOffItems + kMaxItemsPerCta * 4;
 constexpr int kSmemBytes = kOffMisc + 16;
 static_assert(kSmemBytes <= 227 * 1024, "extend shared memory over the per-CTA limit");
-static_assert(kMaxSortItems * 4 <= kKStages * kTileBytes, "the sort runs in the K ring before any load");
+static_assert(kMaxSortGroups * 4 <= kKStages * kTileBytes, "the sort runs in the K ring before any load");
 
 struct Params {
     const __nv_bfloat16 *q;
@@ -127,6 +135,7 @@ struct Params {
     int32_t tokens_per_qtile;  // floor(128 / group)
     int32_t num_qblocks;       // ceil(max_q_len / (2 * tokens_per_qtile))
     int32_t num_items;         // num_qblocks * batch * num_kv_heads
+    int32_t sorted;            // num_qblocks * batch <= kMaxSortGroups: the list is sorted by cost
     float scale_log2;
     uint64_t wait_limit_ns;    // bound of every pipeline wait
     int32_t inject_stall;      // test hook: withhold the first score tile's hand-off
@@ -405,50 +414,76 @@ __global__ void __launch_bounds__(kThreads, 1)
     griddep_launch_dependents();
     griddep_wait();  // inputs written by the previous kernel (e.g. the KV store)
 
-    // ---- the work list.  Sorted mode: every CTA sorts the same keys (cost
-    // descending, enumeration order for ties) in the K ring, which no load has
-    // touched yet, and keeps the ids at its snake positions.
-    const bool sorted = p.num_items <= kMaxSortItems;
+    // ---- the work list.  Sorted mode: every CTA sorts the same group keys
+    // (cost descending, enumeration order for ties; a group is the Hkv items of
+    // one (request, q block), which cost the same) and keeps the item ids at its
+    // snake positions of the expanded list.  The keys live in the K ring, which
+    // no load has touched yet.
+    const bool sorted = p.sorted != 0;
     if (sorted) {
         uint32_t *keys = reinterpret_cast<uint32_t *>(smem + kOffK);
-        int m = 1;
-        while (m < p.num_items) m <<= 1;
-        unsigned bad = 0;
-        for (int i = tid; i < m; i += kThreads) {
+        const int groups = p.num_qblocks * p.batch;
+        if (tid < kMaxSortGroups) {
             uint32_t key = 0;
-            if (i < p.num_items) {
+            if (tid < groups) {
                 Item it;
-                const int st = item_info(p, i, it);
-                if (st == 1) key = ((uint32_t)min(it.n_kv, kMaxCost) << 20) | (uint32_t)(0xFFFFF - i);
-                if (st < 0) bad |= item_error(p, it);
+                const int st = item_info(p, tid * p.num_kv_heads, it);
+                if (st == 1) key = ((uint32_t)min(it.n_kv, kMaxCost) << 16) | (uint32_t)(0xFFFF - tid);
+                if (st < 0 && blockIdx.x == 0) atomicOr(&g_mg_device_error, item_error(p, it));
             }
-            keys[i] = key;
+            keys[tid] = key;
         }
-        if (bad && blockIdx.x == 0) atomicOr(&g_mg_device_error, bad);
         __syncthreads();
-        for (int k = 2; k <= m; k <<= 1) {  // bitonic sort, descending
-            for (int jj = k >> 1; jj > 0; jj >>= 1) {
-                for (int i = tid; i < m; i += kThreads) {
-                    const int ixj = i ^ jj;
-                    if (ixj > i) {
-                        const uint32_t a = keys[i], b = keys[ixj];
-                        if ((i & k) == 0 ? a < b : a > b) {
-                            keys[i] = b;
-                            keys[ixj] = a;
-                        }
+        if (warp == 0) {
+            // bitonic sort, descending, of 256 keys held 8 per lane (element
+            // e = lane * 8 + r): partners within a lane by register, across lanes
+            // by shuffle
+            uint32_t kr[kSortPerLane];
+#pragma unroll
+            for (int r = 0; r < kSortPerLane; ++r) kr[r] = keys[lane * kSortPerLane + r];
+            auto local_stage = [&](int k, auto jc) {
+                constexpr int J = decltype(jc)::value;
+#pragma unroll
+                for (int r = 0; r < kSortPerLane; ++r) {
+                    if ((r & J) == 0) {
+                        const int e = lane * kSortPerLane + r;
+                        const bool desc = (e & k) == 0;
+                        const uint32_t a = kr[r], b = kr[r | J];
+                        const bool swap = desc ? a < b : a > b;
+                        kr[r] = swap ? b : a;
+                        kr[r | J] = swap ? a : b;
                     }
                 }
-                __syncthreads();
+            };
+            for (int k = 2; k <= kMaxSortGroups; k <<= 1) {
+                for (int j = k >> 1; j >= kSortPerLane; j >>= 1) {
+                    const int lane_mask = j / kSortPerLane;
+#pragma unroll
+                    for (int r = 0; r < kSortPerLane; ++r) {
+                        const int e = lane * kSortPerLane + r;
+                        const uint32_t other = __shfl_xor_sync(0xffffffffu, kr[r], lane_mask);
+                        const bool lower = (e & j) == 0, desc = (e & k) == 0;
+                        kr[r] = lower == desc ? max(kr[r], other) : min(kr[r], other);
+                    }
+                }
+                if (k >= 8) local_stage(k, std::integral_constant<int, 4>{});
+                if (k >= 4) local_stage(k, std::integral_constant<int, 2>{});
+                local_stage(k, std::integral_constant<int, 1>{});
             }
-        }
-        if (tid == 0) {
-            int cnt = 0;
-            for (int k = 0; cnt < kMaxItemsPerCta; ++k) {
-                const int pos = snake_position(k);
-                if (pos >= m || keys[pos] == 0) break;
-                items[cnt++] = 0xFFFFF - (int)(keys[pos] & 0xFFFFFu);
+            __syncwarp();
+#pragma unroll
+            for (int r = 0; r < kSortPerLane; ++r) keys[lane * kSortPerLane + r] = kr[r];
+            __syncwarp();
+            if (lane == 0) {
+                int cnt = 0;
+                for (int k = 0; cnt < kMaxItemsPerCta; ++k) {
+                    const int pos = snake_position(k);
+                    const int grp = pos / p.num_kv_heads;
+                    if (grp >= kMaxSortGroups || keys[grp] == 0) break;
+                    items[cnt++] = (0xFFFF - (int)(keys[grp] & 0xFFFFu)) * p.num_kv_heads + (pos - grp * p.num_kv_heads);
+                }
+                *sh_count = cnt;
             }
-            *sh_count = cnt;
         }
     } else if (tid == 0) {
         *sh_count = 0;
@@ -837,10 +872,11 @@ inline mg_status launch(Params &p, int sms, cudaStream_t stream) {
     if (items >= (int64_t)1 << 30) return MG_ERR_UNSUPPORTED_SHAPE;
     p.num_qblocks = (int32_t)nqb;
     p.num_items = (int32_t)items;
+    p.sorted = nqb * p.batch <= kMaxSortGroups ? 1 : 0;
     // one CTA per SM; with a sorted list no CTA may need more than
     // kMaxItemsPerCta items
     int64_t grid = items < sms ? items : sms;
-    if (items <= kMaxSortItems) {
+    if (p.sorted) {
         const int64_t min_grid = (items + kMaxItemsPerCta - 1) / kMaxItemsPerCta;
         if (grid < min_grid) grid = min_grid;
     }
