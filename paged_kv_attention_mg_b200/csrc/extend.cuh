@@ -88,7 +88,7 @@ constexpr int kMaxSortGroups = 32 * kSortPerLane;
 constexpr int kMaxItemsPerCta = 32;
 constexpr int kMaxCost = 0xFFFF;            // cost key clamp (KV tiles)
 #ifndef MG_EXTEND_EMU_PAIRS
-#define MG_EXTEND_EMU_PAIRS 4  // of every 16 pairs of exponentials, this many on the FMA pipe
+#define MG_EXTEND_EMU_PAIRS 2  // of every 16 pairs of exponentials, this many on the FMA pipe
 #endif
 constexpr int kEmuPairs = MG_EXTEND_EMU_PAIRS;
 static_assert(kEmuPairs >= 0 && kEmuPairs <= 16, "pairs per chunk of 16");
@@ -589,27 +589,46 @@ __global__ void __launch_bounds__(kThreads, 1)
                     continue;
                 }
                 uint32_t sv[128];
-                tmem_ld_32x32b_x32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-                tmem_ld_32x32b_x32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-                tmem_ld_32x32b_x32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[64]));
-                tmem_ld_32x32b_x32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
-                tmem_ld_wait();
                 const int key0 = j * kN;
                 const int nvis = min(max(last_key - key0 + 1, 0), kN);  // visible keys in this tile
                 // Row max of the raw scores (scale > 0, so scaling commutes with the
                 // max); a tile every key of which is visible to the whole warp skips
-                // the mask.
+                // the mask, and takes the max of its first 64 columns while the other
+                // 64 are still being read from TMEM.
                 const bool full = __all_sync(0xffffffffu, nvis == kN);
                 float mx;
                 if (full) {
-                    float m0 = -INFINITY, m1 = -INFINITY;
+                    tmem_ld_32x32b_x32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+                    tmem_ld_32x32b_x32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+                    tmem_ld_wait();
+                    reg_barrier<64>(&sv[0]);
+                    tmem_ld_32x32b_x32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[64]));
+                    tmem_ld_32x32b_x32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
+                    // eight independent chains: the max is a latency chain otherwise
+                    float mc[8];
 #pragma unroll
-                    for (int e = 0; e < 128; e += 4) {
-                        m0 = fmax3(m0, __uint_as_float(sv[e]), __uint_as_float(sv[e + 1]));
-                        m1 = fmax3(m1, __uint_as_float(sv[e + 2]), __uint_as_float(sv[e + 3]));
-                    }
-                    mx = fmaxf(m0, m1);
+                    for (int c = 0; c < 8; ++c) mc[c] = fmaxf(__uint_as_float(sv[8 * c]), __uint_as_float(sv[8 * c + 1]));
+#pragma unroll
+                    for (int e = 2; e < 8; e += 2)
+#pragma unroll
+                        for (int c = 0; c < 8; ++c)
+                            mc[c] = fmax3(mc[c], __uint_as_float(sv[8 * c + e]), __uint_as_float(sv[8 * c + e + 1]));
+                    tmem_ld_wait();
+                    reg_barrier<64>(&sv[64]);
+#pragma unroll
+                    for (int e = 0; e < 8; e += 2)
+#pragma unroll
+                        for (int c = 0; c < 8; ++c)
+                            mc[c] = fmax3(mc[c], __uint_as_float(sv[64 + 8 * c + e]), __uint_as_float(sv[64 + 8 * c + e + 1]));
+                    mx = fmaxf(fmaxf(fmaxf(mc[0], mc[1]), fmaxf(mc[2], mc[3])),
+                               fmaxf(fmaxf(mc[4], mc[5]), fmaxf(mc[6], mc[7])));
                 } else {
+                    tmem_ld_32x32b_x32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+                    tmem_ld_32x32b_x32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+                    tmem_ld_32x32b_x32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[64]));
+                    tmem_ld_32x32b_x32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
+                    tmem_ld_wait();
+                    reg_barrier<128>(&sv[0]);
                     mx = -INFINITY;
 #pragma unroll
                     for (int e = 0; e < 128; ++e) {
@@ -633,7 +652,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float mu = m_run == -INFINITY ? 0.f : m_run;
                 const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
                 const float2 nmu2 = make_float2(-mu, -mu);
-                float2 rs2 = make_float2(0.f, 0.f);
+                float2 rs2[4];  // four row-sum chains, one per column block
+#pragma unroll
+                for (int cb = 0; cb < 4; ++cb) rs2[cb] = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int cb = 0; cb < 4; ++cb) {  // masked keys hold -inf and give exactly 0
                     uint32_t pk[16];
@@ -649,11 +670,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                             pk[e] = pack_bf16x2(fast_exp2(x.x), fast_exp2(x.y));
                         }
                         // the row sum adds the same bf16-rounded P the PV product reads
-                        rs2 = fadd2(rs2, make_float2(bf16x2_lo(pk[e]), bf16x2_hi(pk[e])));
+                        rs2[cb] = fadd2(rs2[cb], make_float2(bf16x2_lo(pk[e]), bf16x2_hi(pk[e])));
                     }
                     tmem_st_32x32b_x16(tS + cb * 16, pk);
                 }
-                l_run += rs2.x + rs2.y;
+                {
+                    const float2 a = fadd2(rs2[0], rs2[1]), b = fadd2(rs2[2], rs2[3]);
+                    const float2 t2 = fadd2(a, b);
+                    l_run += t2.x + t2.y;
+                }
                 if (warp_need && j > 0) {
                     // O holds the sum up to tile j-1; rescale it once that PV is done
                     if (!(ok = wait_or_abort(b_o, (cnt + j - 1) & 1, abort_flag, lim))) break;

@@ -216,6 +216,13 @@ __device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_
         : "memory");
 }
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
+// After tcgen05.wait::ld: an empty volatile statement that "rewrites" the
+// loaded registers, so the compiler cannot move any use of them above the wait
+// (the loads' outputs are otherwise ordinary register results to it).
+template <int N> __device__ __forceinline__ void reg_barrier(uint32_t *r) {
+#pragma unroll
+    for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
+}
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
