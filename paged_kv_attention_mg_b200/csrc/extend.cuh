@@ -88,7 +88,7 @@ constexpr int kMaxSortGroups = 32 * kSortPerLane;
 constexpr int kMaxItemsPerCta = 32;
 constexpr int kMaxCost = 0xFFFF;            // cost key clamp (KV tiles)
 #ifndef MG_EXTEND_EMU_PAIRS
-#define MG_EXTEND_EMU_PAIRS 2  // of every 16 pairs of exponentials, this many on the FMA pipe
+#define MG_EXTEND_EMU_PAIRS 0  // of every 16 pairs of exponentials, this many on the FMA pipe
 #endif
 constexpr int kEmuPairs = MG_EXTEND_EMU_PAIRS;
 static_assert(kEmuPairs >= 0 && kEmuPairs <= 16, "pairs per chunk of 16");
