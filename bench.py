@@ -377,18 +377,30 @@ class ExtendBench:
         self.extend_bytes = rf.extend_bytes(c, s, spec.num_q_heads, spec.num_kv_heads, spec.head_dim)
         self.store_bytes = rf.store_bytes(step.num_new_tokens, spec.num_kv_heads, spec.head_dim)
         self.tokens_per_step = step.num_new_tokens
-        self.launches_per_step = spec.num_layers * 2
+        # a mixed batch runs through mg_mixed_attn: store, decode workers, merge, extend
+        self.mixed = spec.mixed
+        self.launches_per_step = spec.num_layers * (4 if self.mixed else 2)
         self.h2d_bytes, self.d2h_bytes = io_bytes(self)
         self.workers = None
+        if self.mixed:
+            ws = mg.mixed_workspace_bytes(step.batch, spec.num_q_heads, spec.num_kv_heads, step.max_seq_len, partitions)
+            self.workspace = torch.empty(max(ws, 16), dtype=torch.uint8, device=device)
+            self.workers, _ = mg.decode_plan(step.batch, spec.num_kv_heads, step.max_seq_len, partitions)
+        self.partitions = partitions
 
     def layer(self, lay, out, meta, events=None):
         mg, st = self.mg, self.step
         mg.store_kv(lay["k_new"], lay["v_new"], meta["out_loc"], lay["k_cache"], lay["v_cache"])
         if events:
             events[0].record()
-        mg.extend_attn(lay["q"], lay["k_cache"], lay["v_cache"], meta["page_table"], meta["table_idx"],
-                       meta["cached_len"], meta["seq_len"], meta["q_offset"], st.max_q_len, st.max_seq_len,
-                       self.spec.scale, out=out)
+        if self.mixed:
+            mg.mixed_attn(lay["q"], lay["k_cache"], lay["v_cache"], meta["page_table"], meta["table_idx"],
+                          meta["cached_len"], meta["seq_len"], meta["q_offset"], st.max_q_len, st.max_seq_len,
+                          self.spec.scale, num_partitions=self.partitions, out=out, workspace=self.workspace)
+        else:
+            mg.extend_attn(lay["q"], lay["k_cache"], lay["v_cache"], meta["page_table"], meta["table_idx"],
+                           meta["cached_len"], meta["seq_len"], meta["q_offset"], st.max_q_len, st.max_seq_len,
+                           self.spec.scale, out=out)
         if events:
             events[1].record()
 
@@ -397,7 +409,11 @@ class ExtendBench:
     copy_out = DecodeBench.copy_out
 
     def details(self):
-        return {"kv_bytes_per_step": self.extend_bytes}
+        d = {"kv_bytes_per_step": self.extend_bytes}
+        if self.mixed:
+            d.update({"entry_point": "mg_mixed_attn (one-token requests: decode kernel + merge; chunks: extend kernel)",
+                      "decode_workers": self.workers})
+        return d
 
 
 def decode_needs_flush(spec, step) -> bool:
@@ -729,7 +745,9 @@ def run_ours(args):
         # bytes (a batch of mostly decode requests), whichever takes longer at peak
         kv_gbs = bench.extend_bytes / (kernel_ms_local * 1e-3) / 1e9
         if bench.extend_bytes / (hbm * 1e9) > bench.flops / (tflops * 1e12):
-            roof = {"bound": "hbm", "kernel": "extend_kernel", "achieved": round(kv_gbs, 1), "peak": hbm,
+            kname = ("decode_kernel + decode_merge_kernel + extend_kernel (one mg_mixed_attn call)" if bench.mixed
+                     else "extend_kernel")
+            roof = {"bound": "hbm", "kernel": kname, "achieved": round(kv_gbs, 1), "peak": hbm,
                     "unit": "GB/s", "frac": round(kv_gbs / hbm, 4), "peak_source": f"{peak_src} HBM copy bandwidth",
                     "tflops": round(achieved, 1), "traffic": profiled_traffic(spec.name)}
         else:

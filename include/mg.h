@@ -12,6 +12,8 @@
  *                   (balanced split-KV kernel + merge kernel);
  *   mg_store_decode_attn  the two above fused into one decode launch;
  *   mg_decode_attn_shared_prefix  decode reading a shared prefix once per group;
+ *   mg_mixed_attn   extend semantics for mixed batches: one-token requests by
+ *                   the decode kernel, prompt chunks by the extend kernel;
  *   mg_extend_attn  a chunk of new tokens per request (chunked prefill),
  *                   causal over cached_len + i, on tcgen05 tensor cores.
  *
@@ -260,6 +262,31 @@ mg_status mg_extend_attn(const void *q, const void *k_cache, const void *v_cache
                          int32_t max_q_len, int32_t max_seq_len, int32_t num_q_heads,
                          int32_t num_kv_heads, int32_t head_dim, float scale, void *out,
                          void *stream);
+
+/*
+ * mg_mixed_attn -- mg_extend_attn for the mixed batches a chunked-prefill
+ * scheduler forms (Mini-SGLang tag page, Scheduler post: continuous batching
+ * with chunked prefill), where most requests are decoding (one new token) and
+ * a few carry a prompt chunk.  Same arguments, metadata and result as
+ * mg_extend_attn, plus a workspace.  Requests with exactly one new token go
+ * through the split-KV decode kernel and its merge (query and output row
+ * q_offset[r]; all keys 0 .. seq_len-1, the causal limit of a token at
+ * position seq_len-1), every other request through the extend kernel, which
+ * leaves the one-token requests alone: one call, three kernels on `stream`,
+ * each request served by the kernel built for its shape.
+ *   num_partitions  the decode kernel's plan (mg_decode_plan)
+ *   workspace       >= mg_mixed_workspace_bytes(...) bytes (the decode plan's)
+ * Metadata errors are flagged as in mg_decode_attn / mg_extend_attn.
+ */
+size_t mg_mixed_workspace_bytes(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                int32_t max_seq_len, int32_t num_partitions);
+mg_status mg_mixed_attn(const void *q, const void *k_cache, const void *v_cache, int64_t num_slots,
+                        const int32_t *page_table, int32_t page_table_rows, int32_t page_table_stride,
+                        const int32_t *table_idx, const int32_t *cached_len, const int32_t *seq_len,
+                        const int32_t *q_offset, int32_t batch, int32_t total_q, int32_t max_q_len,
+                        int32_t max_seq_len, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                        float scale, int32_t num_partitions, void *out, void *workspace, size_t workspace_bytes,
+                        void *stream);
 
 /*
  * mg_decode_attn_static_workspace -- mg_decode_attn for callers that cannot

@@ -110,6 +110,11 @@ struct Params {
     int32_t max_members;    // members one shared prefix serves (16 / group)
     int32_t rows_per_slot;  // partial rows per workspace slot: group, or 16 in cascade mode
     int32_t num_vreqs;      // virtual requests: batch (+ num_groups in cascade mode)
+    // mixed-batch mode, else null: q and out rows of request r are row row_map[r]
+    // ([batch + 1] prefix sums of new tokens, the extend layout) and only
+    // requests with exactly one new token are served
+    const int32_t *row_map;
+    int32_t total_rows;
     int64_t num_slots;
     int32_t pt_rows, pt_stride;
     int32_t batch, num_q_heads, num_kv_heads, group;
@@ -127,9 +132,19 @@ __device__ __forceinline__ uint32_t swz(int row, int c) {
 __device__ __forceinline__ int64_t request_units(const Params &p, int r, int &L, int &row, unsigned &bad) {
     row = __ldg(p.table_idx + r);
     L = __ldg(p.seq_len + r);
+    if (p.row_map) {  // mixed batch: requests with other than one new token are not ours
+        const int q0 = __ldg(p.row_map + r), q1 = __ldg(p.row_map + r + 1);
+        if (q1 - q0 != 1) return 0;
+        if (q0 < 0 || q0 >= p.total_rows) { bad |= MG_DEVERR_LENGTH; return 0; }
+    }
     if (row < 0 || row >= p.pt_rows) { bad |= MG_DEVERR_ROW_RANGE; return 0; }
     if (L < 1 || L > p.pt_stride || L > p.max_seq_len) { bad |= MG_DEVERR_LENGTH; return 0; }
     return (int64_t)((L + kKeys - 1) / kKeys) * p.num_kv_heads;
+}
+
+// q / out row of request r (its own index, or its row of a mixed batch)
+__device__ __forceinline__ int64_t row_of(const Params &p, int r) {
+    return p.row_map ? (int64_t)__ldg(p.row_map + r) : (int64_t)r;
 }
 
 // ---- shared-prefix (cascade) mode: virtual requests.
@@ -303,7 +318,7 @@ __device__ __forceinline__ void cursor_advance(const Params &p, Cursor &c) {
         cursor_load_request<true>(p, c);
         return;
     }
-    if (metadata_ok(p, c.next_L, c.next_row)) {  // the common case: no stall at the boundary
+    if (!p.row_map && metadata_ok(p, c.next_L, c.next_row)) {  // the common case: no stall at the boundary
         c.L = c.next_L;
         c.row = c.next_row;
         c.tiles = (c.L + kKeys - 1) / kKeys;
@@ -541,7 +556,7 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
                                    kHeadDim + quad * 2;
                 } else {
                     hv = hl < g;
-                    qh = p.q + ((int64_t)c.r * p.num_q_heads + (int64_t)c.kvh * g + hl) * kHeadDim + quad * 2;
+                    qh = p.q + (row_of(p, c.r) * p.num_q_heads + (int64_t)c.kvh * g + hl) * kHeadDim + quad * 2;
                 }
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
@@ -736,7 +751,7 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
             if constexpr (CASCADE) whole = whole && !c.grouped && c.r >= p.num_groups;
             const int rows = CASCADE ? c.m * g : g;
             const int64_t rs = CASCADE ? p.rows_per_slot : g;
-            const int64_t head0 = (int64_t)(CASCADE ? c.r0 : c.r) * p.num_q_heads + (int64_t)c.kvh * g;
+            const int64_t head0 = (CASCADE ? (int64_t)c.r0 : row_of(p, c.r)) * p.num_q_heads + (int64_t)c.kvh * g;
             const int64_t slot = (int64_t)c.r * p.num_kv_heads + c.kvh + w;
             for (int h = 0; h < rows; ++h) {
                 const float4 v = *reinterpret_cast<const float4 *>(scr + h * kPitch + lane * 4);
@@ -839,7 +854,7 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const Params p) {
     uint2 packed;
     packed.x = pack_bf16x2(acc.x * inv, acc.y * inv);
     packed.y = pack_bf16x2(acc.z * inv, acc.w * inv);
-    *reinterpret_cast<uint2 *>(p.out + ((int64_t)r * p.num_q_heads + h) * kHeadDim + lane * 4) = packed;
+    *reinterpret_cast<uint2 *>(p.out + (row_of(p, r) * p.num_q_heads + h) * kHeadDim + lane * 4) = packed;
 }
 
 }  // namespace decode

@@ -137,6 +137,7 @@ struct Params {
     int32_t num_items;         // num_qblocks * batch * num_kv_heads
     int32_t sorted;            // num_qblocks * batch <= kMaxSortGroups: the list is sorted by cost
     float scale_log2;
+    int32_t skip_single;       // mixed batches: requests with one new token are served by decode
     uint64_t wait_limit_ns;    // bound of every pipeline wait
     int32_t inject_stall;      // test hook: withhold the first score tile's hand-off
 };
@@ -272,7 +273,7 @@ __device__ __forceinline__ int item_info(const Params &p, int id, Item &it) {
         return -1;
     const int tpq = p.tokens_per_qtile;
     it.tok0 = qb * kQTiles * tpq;
-    if (it.tok0 >= it.n) return 0;
+    if (it.tok0 >= it.n || (p.skip_single && it.n == 1)) return 0;
     const int last_tok = min(it.tok0 + kQTiles * tpq, it.n) - 1;
     it.kv_len = it.c + last_tok + 1;
     it.n_kv = (it.kv_len + kN - 1) / kN;

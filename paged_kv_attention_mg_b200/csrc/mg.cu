@@ -171,7 +171,8 @@ mg_status decode_impl(const void *q, const void *k_new, const void *v_new, const
                       const int32_t *seq_len, int32_t batch, int32_t max_seq_len, int32_t num_q_heads,
                       int32_t num_kv_heads, int32_t head_dim, float scale, int32_t num_partitions, void *out,
                       void *workspace, size_t workspace_bytes, void *stream, const int32_t *group_first = nullptr,
-                      const int32_t *prefix_len = nullptr, int32_t num_groups = 0) {
+                      const int32_t *prefix_len = nullptr, int32_t num_groups = 0, const int32_t *row_map = nullptr,
+                      int32_t total_rows = 0) {
     const bool fused = k_new != nullptr;
     const bool cascade = group_first != nullptr;
     if (cascade && (fused || !prefix_len || num_groups <= 0)) return MG_ERR_INVALID_ARGUMENT;
@@ -232,6 +233,8 @@ mg_status decode_impl(const void *q, const void *k_new, const void *v_new, const
     p.max_members = decode::kRows / p.group;
     p.rows_per_slot = cascade ? decode::kRows : p.group;
     p.num_vreqs = batch + p.num_groups;
+    p.row_map = row_map;
+    p.total_rows = total_rows;
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int ctas = (workers + decode::kWarps - 1) / decode::kWarps;
@@ -248,6 +251,60 @@ mg_status decode_impl(const void *q, const void *k_new, const void *v_new, const
     if (st != MG_OK) return st;
     const int warps = batch * num_q_heads;
     return launch_pdl(decode::decode_merge_kernel, dim3((warps + 3) / 4), dim3(128), 0, s, p);
+}
+}  // namespace
+}  // namespace mg
+
+namespace mg {
+namespace {
+// Extend attention; with skip_single the requests with exactly one new token
+// are left to the decode kernel (mixed batches).
+mg_status extend_impl(const void *q, const void *k_cache, const void *v_cache, int64_t num_slots,
+                      const int32_t *page_table, int32_t page_table_rows, int32_t page_table_stride,
+                      const int32_t *table_idx, const int32_t *cached_len, const int32_t *seq_len,
+                      const int32_t *q_offset, int32_t batch, int32_t total_q, int32_t max_q_len,
+                      int32_t max_seq_len, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, float scale,
+                      void *out, void *stream, bool skip_single) {
+    mg_status st = check_attention_shape(num_q_heads, num_kv_heads, head_dim);
+    if (st != MG_OK) return st;
+    if (!valid_scale(scale)) return MG_ERR_INVALID_ARGUMENT;
+    if (batch <= 0 || total_q < 0 || max_q_len < 0 || num_slots <= 0 || page_table_rows <= 0 ||
+        page_table_stride <= 0 || max_seq_len <= 0 || max_seq_len > page_table_stride)
+        return MG_ERR_INVALID_ARGUMENT;
+    if (total_q == 0 || max_q_len == 0) return MG_OK;
+    if (!q || !k_cache || !v_cache || !page_table || !table_idx || !cached_len || !seq_len ||
+        !q_offset || !out)
+        return MG_ERR_INVALID_ARGUMENT;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
+        return MG_ERR_MISALIGNED;
+    if (ensure_kernel_attributes() != MG_OK) return MG_ERR_CUDA;
+    extend::Params p;
+    p.q = static_cast<const __nv_bfloat16 *>(q);
+    p.k_cache = static_cast<const __nv_bfloat16 *>(k_cache);
+    p.v_cache = static_cast<const __nv_bfloat16 *>(v_cache);
+    p.page_table = page_table;
+    p.table_idx = table_idx;
+    p.cached_len = cached_len;
+    p.seq_len = seq_len;
+    p.q_offset = q_offset;
+    p.out = static_cast<__nv_bfloat16 *>(out);
+    p.num_slots = num_slots;
+    p.pt_rows = page_table_rows;
+    p.pt_stride = page_table_stride;
+    p.batch = batch;
+    p.total_q = total_q;
+    p.max_q_len = max_q_len;
+    p.max_seq_len = max_seq_len;
+    p.num_q_heads = num_q_heads;
+    p.num_kv_heads = num_kv_heads;
+    p.group = num_q_heads / num_kv_heads;
+    p.scale_log2 = scale * kLog2e;
+    p.wait_limit_ns = g_extend_wait_limit_ns.load(std::memory_order_relaxed);
+    p.inject_stall = g_extend_inject_stall.load(std::memory_order_relaxed);
+    p.skip_single = skip_single ? 1 : 0;
+    int sms;
+    if (sm_count(sms) != MG_OK) return MG_ERR_CUDA;
+    return extend::launch(p, sms, static_cast<cudaStream_t>(stream));
 }
 }  // namespace
 }  // namespace mg
@@ -377,6 +434,24 @@ mg_status mg_extend_attn(const void *q, const void *k_cache, const void *v_cache
                          int32_t max_q_len, int32_t max_seq_len, int32_t num_q_heads,
                          int32_t num_kv_heads, int32_t head_dim, float scale, void *out,
                          void *stream) {
+    return extend_impl(q, k_cache, v_cache, num_slots, page_table, page_table_rows, page_table_stride, table_idx,
+                       cached_len, seq_len, q_offset, batch, total_q, max_q_len, max_seq_len, num_q_heads,
+                       num_kv_heads, head_dim, scale, out, stream, false);
+}
+
+size_t mg_mixed_workspace_bytes(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                int32_t max_seq_len, int32_t num_partitions) {
+    return mg_decode_workspace_bytes(batch, num_q_heads, num_kv_heads, head_dim, max_seq_len, num_partitions);
+}
+
+mg_status mg_mixed_attn(const void *q, const void *k_cache, const void *v_cache, int64_t num_slots,
+                        const int32_t *page_table, int32_t page_table_rows, int32_t page_table_stride,
+                        const int32_t *table_idx, const int32_t *cached_len, const int32_t *seq_len,
+                        const int32_t *q_offset, int32_t batch, int32_t total_q, int32_t max_q_len,
+                        int32_t max_seq_len, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                        float scale, int32_t num_partitions, void *out, void *workspace, size_t workspace_bytes,
+                        void *stream) {
+    // the same checks as mg_extend_attn, before anything is launched
     mg_status st = check_attention_shape(num_q_heads, num_kv_heads, head_dim);
     if (st != MG_OK) return st;
     if (!valid_scale(scale)) return MG_ERR_INVALID_ARGUMENT;
@@ -384,38 +459,17 @@ mg_status mg_extend_attn(const void *q, const void *k_cache, const void *v_cache
         page_table_stride <= 0 || max_seq_len <= 0 || max_seq_len > page_table_stride)
         return MG_ERR_INVALID_ARGUMENT;
     if (total_q == 0 || max_q_len == 0) return MG_OK;
-    if (!q || !k_cache || !v_cache || !page_table || !table_idx || !cached_len || !seq_len ||
-        !q_offset || !out)
-        return MG_ERR_INVALID_ARGUMENT;
-    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
-        return MG_ERR_MISALIGNED;
-    if (ensure_kernel_attributes() != MG_OK) return MG_ERR_CUDA;
-    extend::Params p;
-    p.q = static_cast<const __nv_bfloat16 *>(q);
-    p.k_cache = static_cast<const __nv_bfloat16 *>(k_cache);
-    p.v_cache = static_cast<const __nv_bfloat16 *>(v_cache);
-    p.page_table = page_table;
-    p.table_idx = table_idx;
-    p.cached_len = cached_len;
-    p.seq_len = seq_len;
-    p.q_offset = q_offset;
-    p.out = static_cast<__nv_bfloat16 *>(out);
-    p.num_slots = num_slots;
-    p.pt_rows = page_table_rows;
-    p.pt_stride = page_table_stride;
-    p.batch = batch;
-    p.total_q = total_q;
-    p.max_q_len = max_q_len;
-    p.max_seq_len = max_seq_len;
-    p.num_q_heads = num_q_heads;
-    p.num_kv_heads = num_kv_heads;
-    p.group = num_q_heads / num_kv_heads;
-    p.scale_log2 = scale * kLog2e;
-    p.wait_limit_ns = g_extend_wait_limit_ns.load(std::memory_order_relaxed);
-    p.inject_stall = g_extend_inject_stall.load(std::memory_order_relaxed);
-    int sms;
-    if (sm_count(sms) != MG_OK) return MG_ERR_CUDA;
-    return extend::launch(p, sms, static_cast<cudaStream_t>(stream));
+    if (!q_offset) return MG_ERR_INVALID_ARGUMENT;
+    // one-token requests: the split-KV decode kernel and its merge, rows by q_offset
+    st = decode_impl(q, nullptr, nullptr, nullptr, k_cache, v_cache, num_slots, page_table, page_table_rows,
+                     page_table_stride, table_idx, seq_len, batch, max_seq_len, num_q_heads, num_kv_heads, head_dim,
+                     scale, num_partitions, out, workspace, workspace_bytes, stream, nullptr, nullptr, 0, q_offset,
+                     total_q);
+    if (st != MG_OK || max_q_len <= 1) return st;
+    // every other request: the extend kernel, which leaves the one-token ones alone
+    return extend_impl(q, k_cache, v_cache, num_slots, page_table, page_table_rows, page_table_stride, table_idx,
+                       cached_len, seq_len, q_offset, batch, total_q, max_q_len, max_seq_len, num_q_heads,
+                       num_kv_heads, head_dim, scale, out, stream, true);
 }
 
 mg_status mg_set_extend_wait_limit(uint64_t limit_ns, int32_t inject_stall) {

@@ -50,6 +50,9 @@ SIGNATURES = {
                                                     _I32, _I32, _I32, _I32, _F32, _I32, _P, _P, _SZ, _P]),
     "mg_extend_attn": (ctypes.c_int, [_P, _P, _P, _I64, _P, _I32, _I32, _P, _P, _P, _P, _I32, _I32, _I32,
                                       _I32, _I32, _I32, _I32, _F32, _P, _P]),
+    "mg_mixed_workspace_bytes": (_SZ, [_I32, _I32, _I32, _I32, _I32, _I32]),
+    "mg_mixed_attn": (ctypes.c_int, [_P, _P, _P, _I64, _P, _I32, _I32, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32,
+                                     _I32, _I32, _F32, _I32, _P, _P, _SZ, _P]),
     "mg_decode_attn_static_workspace": (ctypes.c_int, [_P, _P, _P, _I64, _P, _I32, _I32, _P, _P, _I32, _I32,
                                                        _I32, _I32, _I32, _F32, _I32, _P, _P]),
     "mg_set_extend_wait_limit": (ctypes.c_int, [ctypes.c_uint64, _I32]),
@@ -291,6 +294,44 @@ def extend_attn(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, p
                                  _dev(seq_len, torch.int32, "seq_len"), _dev(q_offset, torch.int32, "q_offset"),
                                  b, total_q, max_q_len, max_seq_len, hq, hkv, d, float(scale),
                                  _dev(out, torch.bfloat16, "out"), _stream(stream)), "mg_extend_attn")
+    return out
+
+
+def mixed_workspace_bytes(batch: int, num_q_heads: int, num_kv_heads: int, max_seq_len: int,
+                          num_partitions: int = 0, head_dim: int = 128) -> int:
+    return int(load().mg_mixed_workspace_bytes(batch, num_q_heads, num_kv_heads, head_dim, max_seq_len,
+                                               num_partitions))
+
+
+def mixed_attn(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, page_table: torch.Tensor,
+               table_idx: torch.Tensor, cached_len: torch.Tensor, seq_len: torch.Tensor, q_offset: torch.Tensor,
+               max_q_len: int, max_seq_len: int, scale: float, num_partitions: int = 0,
+               out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+               stream=None) -> torch.Tensor:
+    """extend_attn for a mixed batch: one-token requests through the decode
+    kernel, the others through the extend kernel; returns out [total_q, Hq, D]."""
+    if not isinstance(seq_len, torch.Tensor) or seq_len.dim() != 1:
+        raise ValueError("mixed_attn: seq_len must be [batch]")
+    b = seq_len.shape[0]
+    _attention_shapes("mixed_attn", q, k_cache, v_cache, page_table, out,
+                      {"table_idx": (table_idx, (b,)), "cached_len": (cached_len, (b,)),
+                       "q_offset": (q_offset, (b + 1,))})
+    total_q, hq, d = q.shape
+    hkv = k_cache.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    need = mixed_workspace_bytes(b, hq, hkv, max_seq_len, num_partitions, d)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = _dev(workspace, torch.uint8, "workspace") if workspace is not None else None
+    ws_bytes = workspace.numel() if workspace is not None else 0
+    _check(load().mg_mixed_attn(_dev(q, torch.bfloat16, "q"), _dev(k_cache, torch.bfloat16, "k_cache"),
+                                _dev(v_cache, torch.bfloat16, "v_cache"), k_cache.shape[0],
+                                _dev(page_table, torch.int32, "page_table"), page_table.shape[0], page_table.shape[1],
+                                _dev(table_idx, torch.int32, "table_idx"), _dev(cached_len, torch.int32, "cached_len"),
+                                _dev(seq_len, torch.int32, "seq_len"), _dev(q_offset, torch.int32, "q_offset"),
+                                b, total_q, max_q_len, max_seq_len, hq, hkv, d, float(scale), num_partitions,
+                                _dev(out, torch.bfloat16, "out"), ws_ptr, ws_bytes, _stream(stream)), "mg_mixed_attn")
     return out
 
 

@@ -73,6 +73,7 @@ class WorkloadSpec:
     description: str
     lengths: Callable = field(repr=False, compare=False, default=None)
     share: Optional[tuple] = None  # (members per group, shared prefix length P) or None
+    mixed: bool = False  # a chunked-prefill scheduler's mixed batch (served by mg_mixed_attn)
 
     @property
     def group(self) -> int:
@@ -168,7 +169,7 @@ WORKLOADS: List[WorkloadSpec] = [
     WorkloadSpec("mixed_prefill_decode", "extend", 204, 16, 8, 128, 300_000, 1, 1006, 3072,
                  "one launch over a mixed batch: 4 prompt chunks (cached U[0,1024], chunk U[256,1024]) and "
                  "200 decode requests (one new token after U[128,2047] cached), Hq16/Hkv8, pool 300k",
-                 _mixed(4, 0, 1024, 256, 1024, 128, 2047)),
+                 _mixed(4, 0, 1024, 256, 1024, 128, 2047), mixed=True),
 ]
 
 BY_NAME = {w.name: w for w in WORKLOADS}

@@ -469,6 +469,44 @@ def test_extend_serves_the_mixed_workload():
     assert bool(((dec - ext).abs() <= dec.abs() * 2.0 ** -7 + 2e-3).all())
 
 
+MIXED_SMALL = [
+    # cached, seq: one-token requests beside chunks, a request with no new tokens, a fresh prompt
+    ([1999, 0, 512, 3000, 77, 40], [2000, 700, 1024, 3001, 78, 40]),
+    ([5, 0, 130], [6, 1, 131]),                 # every request one token (decode only)
+    ([0, 300], [260, 500]),                     # no one-token request (extend only)
+]
+
+
+@pytest.mark.parametrize("cached,seq", MIXED_SMALL)
+@pytest.mark.parametrize("parts", [0, 7])
+def test_mixed_attn_matches_oracle(cached, seq, parts):
+    step, data = _custom("extend", cached, seq, 16, 8, seed=sum(seq) + parts)
+    g = GpuStep(step, data)
+    g.store()
+    out = mg.mixed_attn(g.q, g.k_cache, g.v_cache, g.page_table, g.table_idx, g.cached_len, g.seq_len, g.q_offset,
+                        max(step.max_q_len, 1), step.max_seq_len, g.scale, num_partitions=parts)
+    assert mg.read_device_error() == 0
+    assert_matches_oracle(out, oracle_extend(step, data), f"mixed {cached}->{seq} partitions {parts}")
+
+
+def test_mixed_attn_on_the_mixed_workload():
+    """The mixed workload through mg_mixed_attn (decode kernel for its 200
+    one-token requests, extend kernel for its 4 chunks) matches the oracle on
+    sampled requests and the single extend launch row for row."""
+    spec = wl.BY_NAME["mixed_prefill_decode"]
+    step = wl.make_step(spec)
+    data = wl.make_layer(step)
+    g = GpuStep(step, data)
+    g.store()
+    out = mg.mixed_attn(g.q, g.k_cache, g.v_cache, g.page_table, g.table_idx, g.cached_len, g.seq_len, g.q_offset,
+                        step.max_q_len, step.max_seq_len, g.scale)
+    assert mg.read_device_error() == 0
+    req = [0, 1, 2, 3] + list(range(4, 204, 11))
+    assert_matches_oracle(out, oracle_extend(step, data, requests=req), "mixed_attn, mixed_prefill_decode")
+    ext = g.extend().float()
+    assert bool(((out.float() - ext).abs() <= ext.abs() * 2.0 ** -7 + 2e-3).all())
+
+
 # --------------------------------------------------------------------------- shared prefix
 
 def test_decode_and_extend_over_a_shared_prefix():
