@@ -48,8 +48,6 @@
 
 #include <cuda.h>
 
-#include <type_traits>
-
 #include "common.cuh"
 
 namespace mg {
@@ -396,6 +394,51 @@ __device__ __forceinline__ void load_rows(const Params &p, uint32_t ring_base, u
     cp_async_wait<0>();  // nothing in flight into shared memory at teardown
 }
 
+// ---------------------------------------------------------------- the sort
+// One warp sorts the 32 * R keys at `keys` (shared memory) in descending order:
+// a bitonic network over elements e = lane * R + r, partners within a lane
+// compared by register, partners across lanes by shuffle.
+template <int R, int J>
+__device__ __forceinline__ void sort_local_stage(uint32_t (&kr)[R], int lane, int k) {
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        if ((r & J) == 0) {
+            const int e = lane * R + r;
+            const bool desc = (e & k) == 0;
+            const uint32_t a = kr[r], b = kr[r | J];
+            const bool swap = desc ? a < b : a > b;
+            kr[r] = swap ? b : a;
+            kr[r | J] = swap ? a : b;
+        }
+    }
+}
+template <int R>
+__device__ __forceinline__ void warp_sort_desc(uint32_t *keys, int lane) {
+    uint32_t kr[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) kr[r] = keys[lane * R + r];
+    for (int k = 2; k <= 32 * R; k <<= 1) {
+        for (int j = k >> 1; j >= R; j >>= 1) {
+            const int lane_mask = j / R;
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                const int e = lane * R + r;
+                const uint32_t other = __shfl_xor_sync(0xffffffffu, kr[r], lane_mask);
+                const bool lower = (e & j) == 0, desc = (e & k) == 0;
+                kr[r] = lower == desc ? max(kr[r], other) : min(kr[r], other);
+            }
+        }
+        if constexpr (R >= 8) {
+            if (k >= 8) sort_local_stage<R, 4>(kr, lane, k);
+        }
+        if (k >= 4) sort_local_stage<R, 2>(kr, lane, k);
+        sort_local_stage<R, 1>(kr, lane, k);
+    }
+    __syncwarp();
+#pragma unroll
+    for (int r = 0; r < R; ++r) keys[lane * R + r] = kr[r];
+}
+
 // ---------------------------------------------------------------- the kernel
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -436,44 +479,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncthreads();
         if (warp == 0) {
-            // bitonic sort, descending, of 256 keys held 8 per lane (element
-            // e = lane * 8 + r): partners within a lane by register, across lanes
-            // by shuffle
-            uint32_t kr[kSortPerLane];
-#pragma unroll
-            for (int r = 0; r < kSortPerLane; ++r) kr[r] = keys[lane * kSortPerLane + r];
-            auto local_stage = [&](int k, auto jc) {
-                constexpr int J = decltype(jc)::value;
-#pragma unroll
-                for (int r = 0; r < kSortPerLane; ++r) {
-                    if ((r & J) == 0) {
-                        const int e = lane * kSortPerLane + r;
-                        const bool desc = (e & k) == 0;
-                        const uint32_t a = kr[r], b = kr[r | J];
-                        const bool swap = desc ? a < b : a > b;
-                        kr[r] = swap ? b : a;
-                        kr[r | J] = swap ? a : b;
-                    }
-                }
-            };
-            for (int k = 2; k <= kMaxSortGroups; k <<= 1) {
-                for (int j = k >> 1; j >= kSortPerLane; j >>= 1) {
-                    const int lane_mask = j / kSortPerLane;
-#pragma unroll
-                    for (int r = 0; r < kSortPerLane; ++r) {
-                        const int e = lane * kSortPerLane + r;
-                        const uint32_t other = __shfl_xor_sync(0xffffffffu, kr[r], lane_mask);
-                        const bool lower = (e & j) == 0, desc = (e & k) == 0;
-                        kr[r] = lower == desc ? max(kr[r], other) : min(kr[r], other);
-                    }
-                }
-                if (k >= 8) local_stage(k, std::integral_constant<int, 4>{});
-                if (k >= 4) local_stage(k, std::integral_constant<int, 2>{});
-                local_stage(k, std::integral_constant<int, 1>{});
-            }
-            __syncwarp();
-#pragma unroll
-            for (int r = 0; r < kSortPerLane; ++r) keys[lane * kSortPerLane + r] = kr[r];
+            if (groups <= 32 * 4) warp_sort_desc<4>(keys, lane);
+            else warp_sort_desc<kSortPerLane>(keys, lane);
             __syncwarp();
             if (lane == 0) {
                 int cnt = 0;
@@ -599,28 +606,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const bool full = __all_sync(0xffffffffu, nvis == kN);
                 float mx;
                 if (full) {
-                    tmem_ld_32x32b_x32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-                    tmem_ld_32x32b_x32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-                    tmem_ld_wait();
-                    reg_barrier<64>(&sv[0]);
-                    tmem_ld_32x32b_x32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[64]));
-                    tmem_ld_32x32b_x32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
-                    // eight independent chains: the max is a latency chain otherwise
+                    // the four 32-column chunks of S come from TMEM one behind the
+                    // other, each chunk's max taken while the next one loads, in
+                    // eight independent chains (the max is a latency chain otherwise)
                     float mc[8];
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) mc[c] = fmaxf(__uint_as_float(sv[8 * c]), __uint_as_float(sv[8 * c + 1]));
-#pragma unroll
-                    for (int e = 2; e < 8; e += 2)
-#pragma unroll
-                        for (int c = 0; c < 8; ++c)
-                            mc[c] = fmax3(mc[c], __uint_as_float(sv[8 * c + e]), __uint_as_float(sv[8 * c + e + 1]));
+                    for (int c = 0; c < 8; ++c) mc[c] = -INFINITY;
+                    tmem_ld_32x32b_x32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
                     tmem_ld_wait();
-                    reg_barrier<64>(&sv[64]);
+                    reg_barrier<32>(&sv[0]);
 #pragma unroll
-                    for (int e = 0; e < 8; e += 2)
+                    for (int cb = 0; cb < 4; ++cb) {
+                        if (cb < 3)
+                            tmem_ld_32x32b_x32(tS + 32 * (cb + 1), *reinterpret_cast<uint32_t(*)[32]>(&sv[32 * (cb + 1)]));
 #pragma unroll
                         for (int c = 0; c < 8; ++c)
-                            mc[c] = fmax3(mc[c], __uint_as_float(sv[64 + 8 * c + e]), __uint_as_float(sv[64 + 8 * c + e + 1]));
+                            mc[c] = fmax3(mc[c], fmaxf(__uint_as_float(sv[32 * cb + 4 * c]), __uint_as_float(sv[32 * cb + 4 * c + 1])),
+                                          fmaxf(__uint_as_float(sv[32 * cb + 4 * c + 2]), __uint_as_float(sv[32 * cb + 4 * c + 3])));
+                        if (cb < 3) {
+                            tmem_ld_wait();
+                            reg_barrier<32>(&sv[32 * (cb + 1)]);
+                        }
+                    }
                     mx = fmaxf(fmaxf(fmaxf(mc[0], mc[1]), fmaxf(mc[2], mc[3])),
                                fmaxf(fmaxf(mc[4], mc[5]), fmaxf(mc[6], mc[7])));
                 } else {
@@ -653,9 +660,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float mu = m_run == -INFINITY ? 0.f : m_run;
                 const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
                 const float2 nmu2 = make_float2(-mu, -mu);
-                float2 rs2[4];  // four row-sum chains, one per column block
+                float rs[8];  // eight row-sum chains: two per column block
 #pragma unroll
-                for (int cb = 0; cb < 4; ++cb) rs2[cb] = make_float2(0.f, 0.f);
+                for (int c = 0; c < 8; ++c) rs[c] = 0.f;
 #pragma unroll
                 for (int cb = 0; cb < 4; ++cb) {  // masked keys hold -inf and give exactly 0
                     uint32_t pk[16];
@@ -671,15 +678,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                             pk[e] = pack_bf16x2(fast_exp2(x.x), fast_exp2(x.y));
                         }
                         // the row sum adds the same bf16-rounded P the PV product reads
-                        rs2[cb] = fadd2(rs2[cb], make_float2(bf16x2_lo(pk[e]), bf16x2_hi(pk[e])));
+                        add_bf16x2_f32(rs[2 * cb], rs[2 * cb + 1], pk[e]);
                     }
                     tmem_st_32x32b_x16(tS + cb * 16, pk);
                 }
-                {
-                    const float2 a = fadd2(rs2[0], rs2[1]), b = fadd2(rs2[2], rs2[3]);
-                    const float2 t2 = fadd2(a, b);
-                    l_run += t2.x + t2.y;
-                }
+                l_run += ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
                 if (warp_need && j > 0) {
                     // O holds the sum up to tile j-1; rescale it once that PV is done
                     if (!(ok = wait_or_abort(b_o, (cnt + j - 1) & 1, abort_flag, lim))) break;

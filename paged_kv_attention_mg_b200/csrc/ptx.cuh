@@ -106,6 +106,13 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&v);
 }
+// lo_acc += low bf16 half of x, hi_acc += high half, each widened exactly and
+// added in fp32 (mixed-precision add, sm_100)
+__device__ __forceinline__ void add_bf16x2_f32(float &lo_acc, float &hi_acc, uint32_t x) {
+    asm("{\n.reg .b16 l, h;\nmov.b32 {l, h}, %2;\nadd.rn.f32.bf16 %0, l, %0;\nadd.rn.f32.bf16 %1, h, %1;\n}"
+        : "+f"(lo_acc), "+f"(hi_acc)
+        : "r"(x));
+}
 // the two halves of a packed bf16x2 as floats (exact: bf16 is the top half of an fp32)
 __device__ __forceinline__ float bf16x2_lo(uint32_t x) { return __uint_as_float(x << 16); }
 __device__ __forceinline__ float bf16x2_hi(uint32_t x) { return __uint_as_float(x & 0xFFFF0000u); }
