@@ -84,6 +84,9 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch every step eagerly instead of a CUDA graph")
     ap.add_argument("--unfused", action="store_true", help="separate KV-store launch before each decode")
+    ap.add_argument("--plain", action="store_true",
+                    help="shared-prefix workloads: plain mg_decode_attn over the same shared page tables "
+                         "(every request reads the prefix), for comparison with the shared-prefix decode")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="bound of the cpu_baseline sample")
     ap.add_argument("--cpu-seconds-1thread", type=float, default=8.0,
                     help="bound of the cpu_baseline's one-thread sample (0 skips it)")
@@ -258,7 +261,7 @@ def io_bytes(bench):
 
 
 class DecodeBench:
-    def __init__(self, spec, step, device, partitions, fused=True):
+    def __init__(self, spec, step, device, partitions, fused=True, plain=False):
         from paged_kv_attention_mg_b200 import mg
         self.mg = mg
         self.fused = fused
@@ -267,8 +270,8 @@ class DecodeBench:
         # shared-prefix workloads: groups of requests read their common prefix once
         # (mg_decode_attn_shared_prefix after a separate store: the fused store
         # runs without groups)
-        self.shared = step.group_first is not None
-        self.fused = fused and not self.shared
+        self.shared = step.group_first is not None and not plain
+        self.fused = fused and step.group_first is None
         names = ("page_table", "table_idx", "seq_len", "out_loc") + (("group_first", "prefix_len") if self.shared
                                                                       else ())
         self.meta = {n: getattr(step, n).to(device) for n in names}
@@ -285,7 +288,7 @@ class DecodeBench:
         self.workspace = torch.empty(max(ws, 16), dtype=torch.uint8, device=device)
         pack_io(self, (B, hq, spec.head_dim))
         L = step.seq_len.tolist()
-        if self.shared:
+        if step.group_first is not None:  # the prefix counted once, whichever kernel reads it
             self.decode_bytes = rf.decode_bytes_shared_prefix(L, step.group_first.tolist(), step.prefix_len.tolist(),
                                                               hq, hkv, spec.head_dim)
         else:
@@ -353,8 +356,10 @@ class DecodeBench:
 
     def details(self):
         d = {"decode_workers": self.workers, "store": "fused into decode" if self.fused else "separate launch"}
-        if self.shared:
-            d["shared_prefix"] = {"groups": int(self.step.prefix_len.numel()),
+        if self.step.group_first is not None:
+            d["shared_prefix"] = {"read": "once per group (mg_decode_attn_shared_prefix)" if self.shared
+                                  else "by every request (mg_decode_attn over the same page tables)",
+                                  "groups": int(self.step.prefix_len.numel()),
                                   "prefix_len": sorted(set(self.step.prefix_len.tolist())),
                                   "bytes_if_unshared": rf.decode_bytes(self.step.seq_len.tolist(),
                                                                        self.spec.num_q_heads, self.spec.num_kv_heads,
@@ -363,7 +368,7 @@ class DecodeBench:
 
 
 class ExtendBench:
-    def __init__(self, spec, step, device, partitions, fused=True):
+    def __init__(self, spec, step, device, partitions, fused=True, plain=False):
         from paged_kv_attention_mg_b200 import mg
         self.mg = mg
         self.spec, self.step, self.device = spec, step, device
@@ -599,7 +604,7 @@ def run_ours(args):
         spec = dataclasses.replace(spec, num_layers=min(args.layers, spec.num_layers))
     step = wl.make_step(spec)
     bench = (DecodeBench if spec.kind == "decode" else ExtendBench)(spec, step, device, args.partitions,
-                                                                     fused=not args.unfused)
+                                                                     fused=not args.unfused, plain=args.plain)
     flush = None
     if spec.kind == "extend" or decode_needs_flush(spec, step):
         flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
