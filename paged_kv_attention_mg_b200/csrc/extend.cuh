@@ -140,15 +140,18 @@ struct Params {
     int32_t inject_stall;      // test hook: withhold the first score tile's hand-off
 };
 
-// UMMA shared-memory descriptor, 128-byte swizzle, sm_100 version bits.
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-    uint64_t d = 0;
-    d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
-    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
-    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
-    d |= (uint64_t)1 << 46;  // descriptor version (Blackwell)
-    d |= (uint64_t)2 << 61;  // SWIZZLE_128B
-    return d;
+// UMMA shared-memory descriptor, 128-byte swizzle, sm_100 version bits, as
+// its two 32-bit words.  The low word holds the start address (bits 0-13, in
+// 16-byte units) and the leading byte offset; the high word the stride byte
+// offset, the version bit (46) and the swizzle mode (61-63), fixed per operand
+// kind.  A k step or a stage moves only the address field, by a constant: the
+// issuer adds it to the low word (the field cannot carry: shared addresses
+// stay below 2^18 bytes).
+__device__ __forceinline__ uint32_t sw128_lo(uint32_t saddr, uint32_t lbo) {
+    return ((saddr & 0x3FFFFu) >> 4) | (((lbo >> 4) & 0x3FFFu) << 16);
+}
+__host__ __device__ constexpr uint32_t sw128_hi(uint32_t sbo) {
+    return ((sbo >> 4) & 0x3FFFu) | (1u << 14) | (2u << 29);
 }
 
 // Instruction descriptor, kind::f16: bf16 x bf16 -> f32, M = 128, N = 128.
@@ -744,25 +747,32 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) {
                 constexpr uint32_t idesc_qk = idesc_bf16(false);
                 constexpr uint32_t idesc_pv = idesc_bf16(true);
+                constexpr uint32_t kHiK = sw128_hi(1024), kHiV = sw128_hi(1024);
+                // Fully unrolled: per MMA, the two address words are the stage's
+                // base plus a constant.  The bases pass through an empty asm so
+                // the compiler cannot precompute every stage's and step's words
+                // outside the item loop (they would not fit in 72 registers).
                 auto issue_s = [&](int t, int stage, bool signal) {
-                    const uint32_t qa = sbase + kOffQ + t * kTileBytes;
-                    const uint32_t ka = sbase + kOffK + stage * kTileBytes;
-                    // unrolled by two only: fully unrolled, the descriptors of every
-                    // stage and k step are hoisted out of the item loop and spill
-#pragma unroll 2
+                    uint32_t qa = sw128_lo(sbase + kOffQ + t * kTileBytes, 16);
+                    uint32_t ka = sw128_lo(sbase + kOffK + stage * kTileBytes, 16);
+                    opaque_u32(qa);
+                    opaque_u32(ka);
+                    const uint32_t d = tmem + col_s(t);
+#pragma unroll
                     for (int kk = 0; kk < 8; ++kk) {
-                        const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-                        umma_ss(tmem + col_s(t), sw128_desc(qa + off, 16, 1024), sw128_desc(ka + off, 16, 1024),
-                                idesc_qk, kk > 0);
+                        const uint32_t off = (uint32_t)((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
+                        umma_ss_words(d, qa + off, kHiK, ka + off, kHiK, idesc_qk, kk > 0 ? 1u : 0u);
                     }
                     if (signal) umma_commit(bar_at(sbase, kBarSFull + t));
                 };
                 auto issue_pv = [&](int t, int stage, bool accumulate) {
-                    const uint32_t va = sbase + kOffV + stage * kTileBytes;
-#pragma unroll 2
-                    for (int kk = 0; kk < 8; ++kk)
-                        umma_ts(tmem + col_o(t), tmem + col_s(t) + kk * 8,
-                                sw128_desc(va + kk * 2048, kHalfBytes, 1024), idesc_pv, (accumulate || kk > 0));
+                    uint32_t vb = sw128_lo(sbase + kOffV + stage * kTileBytes, kHalfBytes);
+                    opaque_u32(vb);
+                    const uint32_t d = tmem + col_o(t), a = tmem + col_s(t);
+                    umma_ts_words(d, a, vb, kHiV, idesc_pv, accumulate ? 1u : 0u);
+#pragma unroll
+                    for (int kk = 1; kk < 8; ++kk)
+                        umma_ts_words(d, a + kk * 8, vb + (uint32_t)(kk * 2048 >> 4), kHiV, idesc_pv, 1u);
                     umma_commit(bar_at(sbase, kBarODone + t));
                 };
                 ItemCursor cur{0};
