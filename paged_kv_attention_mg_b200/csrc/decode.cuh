@@ -540,233 +540,251 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
         cp_async_commit();
         if (k < 0) continue;
         const TileDesc c = my_desc[k % kDescRing];
-        const bool first = k == 0 || c.t == 0;
-        const bool last = k == n_units - 1 || c.t == c.tiles - 1;
-        if (first) {
-            // new segment: this pair's q as B fragments (head l/4 of each n-tile), reset the state
+        // n-tiles this tile's query rows need: a grouped shared prefix can fill
+        // two, a request's own keys (g <= 8 rows) one
+        const int ntu = NT == 1 ? 1 : ((CASCADE ? c.m * g : g) > 8 ? 2 : 1);
+        // the tile's work, compiled once per n-tile count so each path keeps
+        // its two n-tiles' products interleaved (or has no second one at all)
+        auto tile = [&](auto ntu_c) {
+            constexpr int NTU = decltype(ntu_c)::value;
+            const bool first = k == 0 || c.t == 0;
+            const bool last = k == n_units - 1 || c.t == c.tiles - 1;
+            if (first) {
+                // new segment: this pair's q as B fragments (head l/4 of each n-tile), reset the state
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                const int hl = nt * 8 + (lane >> 2);
-                bool hv;
-                const __nv_bfloat16 *qh;
-                if constexpr (CASCADE) {  // row hl: head hl % g of member hl / g
-                    const int member = hl / g;
-                    hv = member < c.m;
-                    qh = p.q + ((int64_t)(c.r0 + member) * p.num_q_heads + (int64_t)c.kvh * g + (hl - member * g)) *
-                                   kHeadDim + quad * 2;
-                } else {
-                    hv = hl < g;
-                    qh = p.q + (row_of(p, c.r) * p.num_q_heads + (int64_t)c.kvh * g + hl) * kHeadDim + quad * 2;
+                for (int nt = 0; nt < NT; ++nt) {
+                    const int hl = nt * 8 + (lane >> 2);
+                    bool hv;
+                    const __nv_bfloat16 *qh;
+                    if constexpr (CASCADE) {  // row hl: head hl % g of member hl / g
+                        const int member = hl / g;
+                        hv = member < c.m;
+                        qh = p.q + ((int64_t)(c.r0 + member) * p.num_q_heads + (int64_t)c.kvh * g + (hl - member * g)) *
+                                       kHeadDim + quad * 2;
+                    } else {
+                        hv = hl < g;
+                        qh = p.q + (row_of(p, c.r) * p.num_q_heads + (int64_t)c.kvh * g + hl) * kHeadDim + quad * 2;
+                    }
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        if (nt >= NTU) break;
+                        qb[nt][kk][0] = hv ? __ldg(reinterpret_cast<const uint32_t *>(qh + kk * 16)) : 0u;
+                        qb[nt][kk][1] = hv ? __ldg(reinterpret_cast<const uint32_t *>(qh + kk * 16 + 8)) : 0u;
+                    }
+#pragma unroll
+                    for (int dt = 0; dt < 8; ++dt) o[nt][dt][0] = o[nt][dt][1] = o[nt][dt][2] = o[nt][dt][3] = 0.f;
+                    mh[nt][0] = mh[nt][1] = -INFINITY;
+                    lh[nt][0] = lh[nt][1] = 0.f;
                 }
+                seg_first_t = c.t;
+            }
+            cp_async_wait<kStages - 1>();  // tile k landed
+            __syncwarp();
+
+            const uint32_t kt = ring + (uint32_t)((k % kStages) * kTileBytes);
+            const uint32_t vt = kt + 2 * kHalfRows;
+
+            // ---- S^T = K Q^T: two accumulators (even / odd k-steps) halve the MMA chain
+            float sa[NT][4], sb[NT][4];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) sa[nt][e] = sb[nt][e] = 0.f;
+            {
+                const int mi = lane >> 3;
+                const int key = (mi & 1) * 8 + (lane & 7);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
-                    qb[nt][kk][0] = hv ? __ldg(reinterpret_cast<const uint32_t *>(qh + kk * 16)) : 0u;
-                    qb[nt][kk][1] = hv ? __ldg(reinterpret_cast<const uint32_t *>(qh + kk * 16 + 8)) : 0u;
-                }
+                    uint32_t a[4];
+                    ldmatrix_x4(kt + swz(key, 2 * kk + (mi >> 1)), a[0], a[1], a[2], a[3]);
 #pragma unroll
-                for (int dt = 0; dt < 8; ++dt) o[nt][dt][0] = o[nt][dt][1] = o[nt][dt][2] = o[nt][dt][3] = 0.f;
-                mh[nt][0] = mh[nt][1] = -INFINITY;
-                lh[nt][0] = lh[nt][1] = 0.f;
-            }
-            seg_first_t = c.t;
-        }
-        cp_async_wait<kStages - 1>();  // tile k landed
-        __syncwarp();
-
-        const uint32_t kt = ring + (uint32_t)((k % kStages) * kTileBytes);
-        const uint32_t vt = kt + 2 * kHalfRows;
-
-        // ---- S^T = K Q^T: two accumulators (even / odd k-steps) halve the MMA chain
-        float sa[NT][4], sb[NT][4];
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) sa[nt][e] = sb[nt][e] = 0.f;
-        {
-            const int mi = lane >> 3;
-            const int key = (mi & 1) * 8 + (lane & 7);
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                uint32_t a[4];
-                ldmatrix_x4(kt + swz(key, 2 * kk + (mi >> 1)), a[0], a[1], a[2], a[3]);
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    if (kk & 1) mma_bf16_16816(sb[nt], a, qb[nt][kk][0], qb[nt][kk][1]);
-                    else mma_bf16_16816(sa[nt], a, qb[nt][kk][0], qb[nt][kk][1]);
+                    for (int nt = 0; nt < NT; ++nt) {
+                        if (nt >= NTU) break;
+                        if (kk & 1) mma_bf16_16816(sb[nt], a, qb[nt][kk][0], qb[nt][kk][1]);
+                        else mma_bf16_16816(sa[nt], a, qb[nt][kk][0], qb[nt][kk][1]);
+                    }
                 }
             }
-        }
-        // keys past the end, or whose slot was rejected (zero-filled), are masked
-        const bool v0 = (c.valid >> (lane >> 2)) & 1u, v1 = (c.valid >> ((lane >> 2) + 8)) & 1u;
-        bool changed = false;
-        float sc[NT][4];
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            sc[nt][0] = v0 ? (sa[nt][0] + sb[nt][0]) * p.scale_log2 : -INFINITY;  // key l/4,   head even
-            sc[nt][1] = v0 ? (sa[nt][1] + sb[nt][1]) * p.scale_log2 : -INFINITY;  // key l/4,   head odd
-            sc[nt][2] = v1 ? (sa[nt][2] + sb[nt][2]) * p.scale_log2 : -INFINITY;  // key l/4+8, head even
-            sc[nt][3] = v1 ? (sa[nt][3] + sb[nt][3]) * p.scale_log2 : -INFINITY;  // key l/4+8, head odd
-            float x0 = fmaxf(sc[nt][0], sc[nt][2]), x1 = fmaxf(sc[nt][1], sc[nt][3]);
-#pragma unroll
-            for (int off = 4; off < 32; off <<= 1) {
-                x0 = fmaxf(x0, __shfl_xor_sync(0xffffffffu, x0, off));
-                x1 = fmaxf(x1, __shfl_xor_sync(0xffffffffu, x1, off));
-            }
-            const float n0 = fmaxf(mh[nt][0], x0), n1 = fmaxf(mh[nt][1], x1);
-            changed |= (n0 != mh[nt][0]) || (n1 != mh[nt][1]);
-            sa[nt][0] = n0;  // reuse: new maxima
-            sa[nt][1] = n1;
-        }
-        if (__any_sync(0xffffffffu, changed)) {
+            // keys past the end, or whose slot was rejected (zero-filled), are masked
+            const bool v0 = (c.valid >> (lane >> 2)) & 1u, v1 = (c.valid >> ((lane >> 2) + 8)) & 1u;
+            bool changed = false;
+            float sc[NT][4];
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
-                const float n0 = sa[nt][0], n1 = sa[nt][1];
-                const float c0 = mh[nt][0] == -INFINITY ? 0.f : fast_exp2(mh[nt][0] - (n0 == -INFINITY ? 0.f : n0));
-                const float c1 = mh[nt][1] == -INFINITY ? 0.f : fast_exp2(mh[nt][1] - (n1 == -INFINITY ? 0.f : n1));
-                lh[nt][0] *= c0;
-                lh[nt][1] *= c1;
-#pragma unroll
-                for (int dt = 0; dt < 8; ++dt) {
-                    o[nt][dt][0] *= c0;
-                    o[nt][dt][1] *= c1;
-                    o[nt][dt][2] *= c0;
-                    o[nt][dt][3] *= c1;
-                }
-                mh[nt][0] = n0;
-                mh[nt][1] = n1;
-            }
-        }
-        // ---- P^T (bf16) as B fragments: lane l needs keys 2(l%4), +1 (and +8)
-        // of head l/4, which sit in lanes 8(l%4) + l/8 and that + 4
-        uint32_t pb[NT][2];
-#if MG_DECODE_SPLIT_P
-        uint32_t pl[NT][2];  // the bf16 residuals p - hi
-#endif
-        {
-            const int s0 = 8 * quad + (lane >> 3);
-            const uint32_t sel = ((lane >> 2) & 1) ? 0x7632u : 0x5410u;
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                const float mu0 = mh[nt][0] == -INFINITY ? 0.f : mh[nt][0];
-                const float mu1 = mh[nt][1] == -INFINITY ? 0.f : mh[nt][1];
-                const float p0 = fast_exp2(sc[nt][0] - mu0), p1 = fast_exp2(sc[nt][1] - mu1);
-                const float p2 = fast_exp2(sc[nt][2] - mu0), p3 = fast_exp2(sc[nt][3] - mu1);
-                const uint32_t X = pack_bf16x2(p0, p1), Y = pack_bf16x2(p2, p3);
-#if MG_DECODE_SPLIT_P
-                // hi + lo carries P to ~2^-17 relative, so the fp32 weights are the normaliser
-                lh[nt][0] += p0 + p2;
-                lh[nt][1] += p1 + p3;
-                const uint32_t XL = pack_bf16x2(p0 - bf16x2_lo(X), p1 - bf16x2_hi(X));
-                const uint32_t YL = pack_bf16x2(p2 - bf16x2_lo(Y), p3 - bf16x2_hi(Y));
-                const uint32_t la = __shfl_sync(0xffffffffu, XL, s0), lb = __shfl_sync(0xffffffffu, XL, s0 + 4);
-                const uint32_t lc = __shfl_sync(0xffffffffu, YL, s0), ld = __shfl_sync(0xffffffffu, YL, s0 + 4);
-                pl[nt][0] = __byte_perm(la, lb, sel);
-                pl[nt][1] = __byte_perm(lc, ld, sel);
-#else
-                // the normaliser sums the same bf16-rounded weights the PV product uses
-                lh[nt][0] += bf16x2_lo(X) + bf16x2_lo(Y);
-                lh[nt][1] += bf16x2_hi(X) + bf16x2_hi(Y);
-#endif
-                const uint32_t xa = __shfl_sync(0xffffffffu, X, s0), xb = __shfl_sync(0xffffffffu, X, s0 + 4);
-                const uint32_t ya = __shfl_sync(0xffffffffu, Y, s0), yb = __shfl_sync(0xffffffffu, Y, s0 + 4);
-                pb[nt][0] = __byte_perm(xa, xb, sel);
-                pb[nt][1] = __byte_perm(ya, yb, sel);
-            }
-        }
-        // ---- O^T += V^T P^T (hi, then lo parts of P)
-        {
-            const int mi = lane >> 3;
-            const int key = (mi >> 1) * 8 + (lane & 7);
-#pragma unroll
-            for (int dt = 0; dt < 8; ++dt) {
-                uint32_t a[4];
-                ldmatrix_x4_trans(vt + swz(key, 2 * dt + (mi & 1)), a[0], a[1], a[2], a[3]);
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    mma_bf16_16816(o[nt][dt], a, pb[nt][0], pb[nt][1]);
-#if MG_DECODE_SPLIT_P
-                    mma_bf16_16816(o[nt][dt], a, pl[nt][0], pl[nt][1]);
-#endif
-                }
-            }
-        }
-        if (FUSED && c.t == c.tiles - 1) {
-            // fused store: lanes 0-15 copy the new token's K row, lanes 16-31 its V row,
-            // 16 bytes each, from the landed stage into pool slot out_loc[r]
-            const int nk = c.L - 1 - c.t * kKeys;
-            const int ss = c.store_slot;
-            const int pt_slot = my_idx[k % kDescRing][nk];
-            if (ss < 0 || (int64_t)ss >= p.num_slots) {
-                if (lane == 0) atomicOr(&g_mg_device_error, MG_DEVERR_SLOT_RANGE);
-            } else {
-                if (lane == 0 && ss != pt_slot) atomicOr(&g_mg_device_error, MG_DEVERR_LENGTH);
-                const int ch = lane & 15;
-                const bool is_v = lane >= 16;
-                uint4 v;
-                asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];\n"
-                             : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                             : "r"(kt + (is_v ? 2 * kHalfRows : 0) + swz(nk, ch)));
-                __nv_bfloat16 *dst = (is_v ? p.v_store : p.k_store) + (int64_t)ss * head_stride +
-                                     (int64_t)c.kvh * kHeadDim + ch * 8;
-                *reinterpret_cast<uint4 *>(dst) = v;
-            }
-        }
-        __syncwarp();  // every lane is done reading this stage
-
-        if (last) {
-            // ---- finish the segment through the (now idle) stage as fp32 scratch
-            // [heads][dims + 4]: whole pair -> bf16 out, else a partial
-            float *scr = reinterpret_cast<float *>(smem + (size_t)(warp * kStages + k % kStages) * kTileBytes);
-            constexpr int kPitch = NT == 1 ? kHeadDim + 4 : kHeadDim;  // pad when there is room
-            static_assert(NT * 8 * kPitch * 4 <= kTileBytes, "scratch must fit in one stage");
-            float *lse_scr = sh_lse[warp];
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                float l0 = lh[nt][0], l1 = lh[nt][1];
+                if (nt >= NTU) break;
+                sc[nt][0] = v0 ? (sa[nt][0] + sb[nt][0]) * p.scale_log2 : -INFINITY;  // key l/4,   head even
+                sc[nt][1] = v0 ? (sa[nt][1] + sb[nt][1]) * p.scale_log2 : -INFINITY;  // key l/4,   head odd
+                sc[nt][2] = v1 ? (sa[nt][2] + sb[nt][2]) * p.scale_log2 : -INFINITY;  // key l/4+8, head even
+                sc[nt][3] = v1 ? (sa[nt][3] + sb[nt][3]) * p.scale_log2 : -INFINITY;  // key l/4+8, head odd
+                float x0 = fmaxf(sc[nt][0], sc[nt][2]), x1 = fmaxf(sc[nt][1], sc[nt][3]);
 #pragma unroll
                 for (int off = 4; off < 32; off <<= 1) {
-                    l0 += __shfl_xor_sync(0xffffffffu, l0, off);
-                    l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+                    x0 = fmaxf(x0, __shfl_xor_sync(0xffffffffu, x0, off));
+                    x1 = fmaxf(x1, __shfl_xor_sync(0xffffffffu, x1, off));
                 }
-                const float i0 = l0 > 0.f ? 1.f / l0 : 0.f, i1 = l1 > 0.f ? 1.f / l1 : 0.f;
-                const int h0 = nt * 8 + 2 * quad;
+                const float n0 = fmaxf(mh[nt][0], x0), n1 = fmaxf(mh[nt][1], x1);
+                changed |= (n0 != mh[nt][0]) || (n1 != mh[nt][1]);
+                sa[nt][0] = n0;  // reuse: new maxima
+                sa[nt][1] = n1;
+            }
+            if (__any_sync(0xffffffffu, changed)) {
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    if (nt >= NTU) break;
+                    const float n0 = sa[nt][0], n1 = sa[nt][1];
+                    const float c0 = mh[nt][0] == -INFINITY ? 0.f : fast_exp2(mh[nt][0] - (n0 == -INFINITY ? 0.f : n0));
+                    const float c1 = mh[nt][1] == -INFINITY ? 0.f : fast_exp2(mh[nt][1] - (n1 == -INFINITY ? 0.f : n1));
+                    lh[nt][0] *= c0;
+                    lh[nt][1] *= c1;
+#pragma unroll
+                    for (int dt = 0; dt < 8; ++dt) {
+                        o[nt][dt][0] *= c0;
+                        o[nt][dt][1] *= c1;
+                        o[nt][dt][2] *= c0;
+                        o[nt][dt][3] *= c1;
+                    }
+                    mh[nt][0] = n0;
+                    mh[nt][1] = n1;
+                }
+            }
+            // ---- P^T (bf16) as B fragments: lane l needs keys 2(l%4), +1 (and +8)
+            // of head l/4, which sit in lanes 8(l%4) + l/8 and that + 4
+            uint32_t pb[NT][2];
+    #if MG_DECODE_SPLIT_P
+            uint32_t pl[NT][2];  // the bf16 residuals p - hi
+    #endif
+            {
+                const int s0 = 8 * quad + (lane >> 3);
+                const uint32_t sel = ((lane >> 2) & 1) ? 0x7632u : 0x5410u;
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    if (nt >= NTU) break;
+                    const float mu0 = mh[nt][0] == -INFINITY ? 0.f : mh[nt][0];
+                    const float mu1 = mh[nt][1] == -INFINITY ? 0.f : mh[nt][1];
+                    const float p0 = fast_exp2(sc[nt][0] - mu0), p1 = fast_exp2(sc[nt][1] - mu1);
+                    const float p2 = fast_exp2(sc[nt][2] - mu0), p3 = fast_exp2(sc[nt][3] - mu1);
+                    const uint32_t X = pack_bf16x2(p0, p1), Y = pack_bf16x2(p2, p3);
+    #if MG_DECODE_SPLIT_P
+                    // hi + lo carries P to ~2^-17 relative, so the fp32 weights are the normaliser
+                    lh[nt][0] += p0 + p2;
+                    lh[nt][1] += p1 + p3;
+                    const uint32_t XL = pack_bf16x2(p0 - bf16x2_lo(X), p1 - bf16x2_hi(X));
+                    const uint32_t YL = pack_bf16x2(p2 - bf16x2_lo(Y), p3 - bf16x2_hi(Y));
+                    const uint32_t la = __shfl_sync(0xffffffffu, XL, s0), lb = __shfl_sync(0xffffffffu, XL, s0 + 4);
+                    const uint32_t lc = __shfl_sync(0xffffffffu, YL, s0), ld = __shfl_sync(0xffffffffu, YL, s0 + 4);
+                    pl[nt][0] = __byte_perm(la, lb, sel);
+                    pl[nt][1] = __byte_perm(lc, ld, sel);
+    #else
+                    // the normaliser sums the same bf16-rounded weights the PV product uses
+                    lh[nt][0] += bf16x2_lo(X) + bf16x2_lo(Y);
+                    lh[nt][1] += bf16x2_hi(X) + bf16x2_hi(Y);
+    #endif
+                    const uint32_t xa = __shfl_sync(0xffffffffu, X, s0), xb = __shfl_sync(0xffffffffu, X, s0 + 4);
+                    const uint32_t ya = __shfl_sync(0xffffffffu, Y, s0), yb = __shfl_sync(0xffffffffu, Y, s0 + 4);
+                    pb[nt][0] = __byte_perm(xa, xb, sel);
+                    pb[nt][1] = __byte_perm(ya, yb, sel);
+                }
+            }
+            // ---- O^T += V^T P^T (hi, then lo parts of P)
+            {
+                const int mi = lane >> 3;
+                const int key = (mi >> 1) * 8 + (lane & 7);
 #pragma unroll
                 for (int dt = 0; dt < 8; ++dt) {
-                    const int d0 = dt * 16 + (lane >> 2);
-                    scr[h0 * kPitch + d0] = o[nt][dt][0] * i0;
-                    scr[(h0 + 1) * kPitch + d0] = o[nt][dt][1] * i1;
-                    scr[h0 * kPitch + d0 + 8] = o[nt][dt][2] * i0;
-                    scr[(h0 + 1) * kPitch + d0 + 8] = o[nt][dt][3] * i1;
-                }
-                if (lane < 4) {  // log2-sum-exp of heads h0, h0 + 1
-                    lse_scr[h0] = l0 > 0.f ? mh[nt][0] + __log2f(l0) : -INFINITY;
-                    lse_scr[h0 + 1] = l1 > 0.f ? mh[nt][1] + __log2f(l1) : -INFINITY;
+                    uint32_t a[4];
+                    ldmatrix_x4_trans(vt + swz(key, 2 * dt + (mi & 1)), a[0], a[1], a[2], a[3]);
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        if (nt >= NTU) break;
+                        mma_bf16_16816(o[nt][dt], a, pb[nt][0], pb[nt][1]);
+    #if MG_DECODE_SPLIT_P
+                        mma_bf16_16816(o[nt][dt], a, pl[nt][0], pl[nt][1]);
+    #endif
+                    }
                 }
             }
-            __syncwarp();
-            // a whole pair of a plain request writes the output; anything else
-            // (part of a pair, a shared prefix, a request whose prefix is
-            // shared) writes partials for the merge kernel
-            bool whole = seg_first_t == 0 && c.t == c.tiles - 1;
-            if constexpr (CASCADE) whole = whole && !c.grouped && c.r >= p.num_groups;
-            const int rows = CASCADE ? c.m * g : g;
-            const int64_t rs = CASCADE ? p.rows_per_slot : g;
-            const int64_t head0 = (CASCADE ? (int64_t)c.r0 : row_of(p, c.r)) * p.num_q_heads + (int64_t)c.kvh * g;
-            const int64_t slot = (int64_t)c.r * p.num_kv_heads + c.kvh + w;
-            for (int h = 0; h < rows; ++h) {
-                const float4 v = *reinterpret_cast<const float4 *>(scr + h * kPitch + lane * 4);
-                if (whole) {
-                    uint2 packed;
-                    packed.x = pack_bf16x2(v.x, v.y);
-                    packed.y = pack_bf16x2(v.z, v.w);
-                    *reinterpret_cast<uint2 *>(p.out + (head0 + h) * kHeadDim + lane * 4) = packed;
+            if (FUSED && c.t == c.tiles - 1) {
+                // fused store: lanes 0-15 copy the new token's K row, lanes 16-31 its V row,
+                // 16 bytes each, from the landed stage into pool slot out_loc[r]
+                const int nk = c.L - 1 - c.t * kKeys;
+                const int ss = c.store_slot;
+                const int pt_slot = my_idx[k % kDescRing][nk];
+                if (ss < 0 || (int64_t)ss >= p.num_slots) {
+                    if (lane == 0) atomicOr(&g_mg_device_error, MG_DEVERR_SLOT_RANGE);
                 } else {
-                    *reinterpret_cast<float4 *>(p.part_o + (slot * rs + h) * kHeadDim + lane * 4) = v;
+                    if (lane == 0 && ss != pt_slot) atomicOr(&g_mg_device_error, MG_DEVERR_LENGTH);
+                    const int ch = lane & 15;
+                    const bool is_v = lane >= 16;
+                    uint4 v;
+                    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];\n"
+                                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                                 : "r"(kt + (is_v ? 2 * kHalfRows : 0) + swz(nk, ch)));
+                    __nv_bfloat16 *dst = (is_v ? p.v_store : p.k_store) + (int64_t)ss * head_stride +
+                                         (int64_t)c.kvh * kHeadDim + ch * 8;
+                    *reinterpret_cast<uint4 *>(dst) = v;
                 }
             }
-            if (!whole && lane < rows) p.part_lse[slot * rs + lane] = lse_scr[lane];
-            __syncwarp();  // scratch reads done before the stage is refilled
-        }
+            __syncwarp();  // every lane is done reading this stage
+
+            if (last) {
+                // ---- finish the segment through the (now idle) stage as fp32 scratch
+                // [heads][dims + 4]: whole pair -> bf16 out, else a partial
+                float *scr = reinterpret_cast<float *>(smem + (size_t)(warp * kStages + k % kStages) * kTileBytes);
+                constexpr int kPitch = NT == 1 ? kHeadDim + 4 : kHeadDim;  // pad when there is room
+                static_assert(NT * 8 * kPitch * 4 <= kTileBytes, "scratch must fit in one stage");
+                float *lse_scr = sh_lse[warp];
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    if (nt >= NTU) break;
+                    float l0 = lh[nt][0], l1 = lh[nt][1];
+#pragma unroll
+                    for (int off = 4; off < 32; off <<= 1) {
+                        l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+                        l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+                    }
+                    const float i0 = l0 > 0.f ? 1.f / l0 : 0.f, i1 = l1 > 0.f ? 1.f / l1 : 0.f;
+                    const int h0 = nt * 8 + 2 * quad;
+#pragma unroll
+                    for (int dt = 0; dt < 8; ++dt) {
+                        const int d0 = dt * 16 + (lane >> 2);
+                        scr[h0 * kPitch + d0] = o[nt][dt][0] * i0;
+                        scr[(h0 + 1) * kPitch + d0] = o[nt][dt][1] * i1;
+                        scr[h0 * kPitch + d0 + 8] = o[nt][dt][2] * i0;
+                        scr[(h0 + 1) * kPitch + d0 + 8] = o[nt][dt][3] * i1;
+                    }
+                    if (lane < 4) {  // log2-sum-exp of heads h0, h0 + 1
+                        lse_scr[h0] = l0 > 0.f ? mh[nt][0] + __log2f(l0) : -INFINITY;
+                        lse_scr[h0 + 1] = l1 > 0.f ? mh[nt][1] + __log2f(l1) : -INFINITY;
+                    }
+                }
+                __syncwarp();
+                // a whole pair of a plain request writes the output; anything else
+                // (part of a pair, a shared prefix, a request whose prefix is
+                // shared) writes partials for the merge kernel
+                bool whole = seg_first_t == 0 && c.t == c.tiles - 1;
+                if constexpr (CASCADE) whole = whole && !c.grouped && c.r >= p.num_groups;
+                const int rows = CASCADE ? c.m * g : g;
+                const int64_t rs = CASCADE ? p.rows_per_slot : g;
+                const int64_t head0 = (CASCADE ? (int64_t)c.r0 : row_of(p, c.r)) * p.num_q_heads + (int64_t)c.kvh * g;
+                const int64_t slot = (int64_t)c.r * p.num_kv_heads + c.kvh + w;
+                for (int h = 0; h < rows; ++h) {
+                    const float4 v = *reinterpret_cast<const float4 *>(scr + h * kPitch + lane * 4);
+                    if (whole) {
+                        uint2 packed;
+                        packed.x = pack_bf16x2(v.x, v.y);
+                        packed.y = pack_bf16x2(v.z, v.w);
+                        *reinterpret_cast<uint2 *>(p.out + (head0 + h) * kHeadDim + lane * 4) = packed;
+                    } else {
+                        *reinterpret_cast<float4 *>(p.part_o + (slot * rs + h) * kHeadDim + lane * 4) = v;
+                    }
+                }
+                if (!whole && lane < rows) p.part_lse[slot * rs + lane] = lse_scr[lane];
+                __syncwarp();  // scratch reads done before the stage is refilled
+            }
+        };
+        if constexpr (NT == 1 || !CASCADE) tile(std::integral_constant<int, NT>{});
+        else if (ntu == 1) tile(std::integral_constant<int, 1>{});
+        else tile(std::integral_constant<int, 2>{});
     }
     cp_async_wait<0>();  // page-table copies still in flight
 }
