@@ -13,16 +13,17 @@
 //     item costs one pass over its keys, ceil((c + last token + 1) / 128) KV
 //     tiles of 128 keys.
 //   * persistent CTAs, one per SM.  Every CTA computes the same work list
-//     (items sorted by cost, heaviest first, when there are at most
-//     kMaxSortGroups (request, q block) groups; one warp sorts them in
-//     registers) and takes its items in snake order (k, 2G-1-k, 2G+k, ...),
+//     (items sorted by cost, heaviest first, when at most kMaxSortGroups
+//     (request, q block) groups hold tokens: a block-wide scan over the
+//     requests compacts them, one warp sorts them in registers) and takes its
+//     items in snake order (k, 2G-1-k, 2G+k, ...),
 //     so the heavy items start first and the loads even out.  Across a CTA's
 //     items the pipelines never drain: K/V rings, barrier phases and TMEM run
 //     on, the next item's Q tiles load while the current item finishes, and an
 //     item's epilogue overlaps the next item's first Q K^T.
 //   * 16 warps in four warpgroups, register budgets moved by setmaxnreg
 //     (warpgroups 0 and 3: 72 registers a thread; 1 and 2: 184):
-//       - warps 0-3 load K tiles, warps 13-15 load V tiles (decoupled rings, so
+//       - warps 0-3 load V tiles, warps 13-15 load K tiles (decoupled rings, so
 //         K can run ahead of V): 16-byte cp.async straight from the paged pool
 //         into the 128-byte swizzled UMMA layout, each warp instruction moving
 //         two 256-byte rows; each lane holds the page-table entries of the keys
@@ -37,8 +38,8 @@
 //         core works on the other's.
 //       - warpgroups 1 / 2: softmax of Q tile 0 / 1, one TMEM lane (= query
 //         row) per thread: causal mask key <= c + i, online softmax in the
-//         exp2 domain (part of the exponentials on the FMA pipe, the rest on
-//         MUFU), O rescaled in TMEM only when the running max grows by more
+//         exp2 domain (exponentials on MUFU), O rescaled in TMEM only when the
+//         running max grows by more
 //         than 2^8 (exact: P and the row sum use the same stale max and the
 //         same bf16-rounded P), epilogue O / l -> bf16 -> global.  Each also
 //         loads its next item's Q tile by TMA as soon as its last score tile
@@ -77,10 +78,12 @@ constexpr int kTmemCols = 512;
 __device__ __forceinline__ uint32_t col_s(int t) { return (uint32_t)t * 128u; }
 __device__ __forceinline__ uint32_t col_o(int t) { return 256u + (uint32_t)t * 128u; }
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
-// The work list is sorted by cost when it has at most kMaxSortGroups groups
-// (a group: the Hkv items of one (request, q block), which cost the same); one
-// warp sorts the group keys in registers.  A CTA keeps at most
-// kMaxItemsPerCta items of a sorted list (the host sizes the grid for that).
+// The work list is sorted by cost when at most kMaxSortGroups groups hold
+// tokens (a group: the Hkv items of one (request, q block), which cost the
+// same); one warp sorts the group keys in registers.  A CTA keeps at most
+// kMaxItemsPerCta items of a sorted list: the host sizes the grid for that
+// when every group may hold tokens, otherwise the kernel checks it and walks
+// the unsorted enumeration instead.
 constexpr int kSortPerLane = 8;
 constexpr int kMaxSortGroups = 32 * kSortPerLane;
 constexpr int kMaxItemsPerCta = 32;
@@ -114,7 +117,8 @@ constexpr int kOffItems = kOffBar + kNumBars * 8;
 constexpr int kOffMisc = kOffItems + kMaxItemsPerCta * 4;
 constexpr int kSmemBytes = kOffMisc + 16;
 static_assert(kSmemBytes <= 227 * 1024, "extend shared memory over the per-CTA limit");
-static_assert(kMaxSortGroups * 4 <= kKStages * kTileBytes, "the sort runs in the K ring before any load");
+static_assert(kMaxSortGroups * 4 + (kThreads / 32 + 1) * 4 <= kKStages * kTileBytes,
+              "the group scan and the sort run in the K ring before any load");
 
 struct Params {
     const __nv_bfloat16 *q;
@@ -133,7 +137,7 @@ struct Params {
     int32_t tokens_per_qtile;  // floor(128 / group)
     int32_t num_qblocks;       // ceil(max_q_len / (2 * tokens_per_qtile))
     int32_t num_items;         // num_qblocks * batch * num_kv_heads
-    int32_t sorted;            // num_qblocks * batch <= kMaxSortGroups: the list is sorted by cost
+    int32_t sorted;            // num_qblocks * batch < 2^16: try the sorted list (group ids fit a key)
     float scale_log2;
     int32_t skip_single;       // mixed batches: requests with one new token are served by decode
     uint64_t wait_limit_ns;    // bound of every pipeline wait
@@ -178,9 +182,12 @@ __device__ __forceinline__ uint64_t global_ns() {
 // Waits with a time bound (limit_ns, timed from the wait's first check of the
 // clock); on timeout records the error, raises the CTA abort flag and returns
 // false.  Once the flag is up every later wait returns false at once, so all
-// roles drain to the final barrier.
+// roles drain to the final barrier.  A phase that has already completed (the
+// common case for the issuer's K and V waits) returns at the first,
+// non-blocking test.
 __device__ __forceinline__ bool wait_or_abort_thread(uint32_t bar, uint32_t parity, volatile int *abort_flag,
                                                      uint64_t limit_ns) {
+    if (mbar_test_wait(bar, parity)) return true;
     if (*abort_flag) return false;
     uint64_t t0 = 0;
     for (uint32_t it = 0;; ++it) {
@@ -256,14 +263,10 @@ struct Item {
     bool q1;  // the second Q tile holds tokens
 };
 
-// 1: the item has work; 0: its q block holds no token of the request;
-// -1: the request's metadata is inconsistent (no item of it runs).
-__device__ __forceinline__ int item_info(const Params &p, int id, Item &it) {
-    const int per_qb = p.batch * p.num_kv_heads;
-    const int qb = p.num_qblocks - 1 - id / per_qb;
-    const int rest = id - (id / per_qb) * per_qb;
-    it.r = rest / p.num_kv_heads;
-    it.kvh = rest - it.r * p.num_kv_heads;
+// Request r's metadata into it (row, c, n, qo): 1, or -1 when it is
+// inconsistent (no item of the request runs).
+__device__ __forceinline__ int request_info(const Params &p, int r, Item &it) {
+    it.r = r;
     it.row = __ldg(p.table_idx + it.r);
     it.c = __ldg(p.cached_len + it.r);
     const int L = __ldg(p.seq_len + it.r);
@@ -272,6 +275,17 @@ __device__ __forceinline__ int item_info(const Params &p, int id, Item &it) {
     if (it.row < 0 || it.row >= p.pt_rows || it.c < 0 || it.n < 0 || L > p.pt_stride || L > p.max_seq_len ||
         it.n > p.max_q_len || it.qo < 0 || it.qo + it.n > p.total_q || __ldg(p.q_offset + it.r + 1) - it.qo != it.n)
         return -1;
+    return 1;
+}
+
+// 1: the item has work; 0: its q block holds no token of the request;
+// -1: the request's metadata is inconsistent (no item of it runs).
+__device__ __forceinline__ int item_info(const Params &p, int id, Item &it) {
+    const int per_qb = p.batch * p.num_kv_heads;
+    const int qb = p.num_qblocks - 1 - id / per_qb;
+    const int rest = id - (id / per_qb) * per_qb;
+    if (request_info(p, rest / p.num_kv_heads, it) < 0) return -1;
+    it.kvh = rest - it.r * p.num_kv_heads;
     const int tpq = p.tokens_per_qtile;
     it.tok0 = qb * kQTiles * tpq;
     if (it.tok0 >= it.n || (p.skip_single && it.n == 1)) return 0;
@@ -466,22 +480,61 @@ __global__ void __launch_bounds__(kThreads, 1)
     // one (request, q block), which cost the same) and keeps the item ids at its
     // snake positions of the expanded list.  The keys live in the K ring, which
     // no load has touched yet.
-    const bool sorted = p.sorted != 0;
-    if (sorted) {
+    bool sorted = false;
+    int groups = 0;  // groups that hold tokens
+    if (p.sorted) {
         uint32_t *keys = reinterpret_cast<uint32_t *>(smem + kOffK);
-        const int groups = p.num_qblocks * p.batch;
-        if (tid < kMaxSortGroups) {
-            uint32_t key = 0;
-            if (tid < groups) {
-                Item it;
-                const int st = item_info(p, tid * p.num_kv_heads, it);
-                if (st == 1) key = ((uint32_t)min(it.n_kv, kMaxCost) << 16) | (uint32_t)(0xFFFF - tid);
-                if (st < 0 && blockIdx.x == 0) atomicOr(&g_mg_device_error, item_error(p, it));
+        int *scan = reinterpret_cast<int *>(smem + kOffK + kMaxSortGroups * 4);  // kThreads / 32 + 1 ints
+        if (tid < kMaxSortGroups) keys[tid] = 0;
+        // each thread counts the groups of its requests that hold tokens ...
+        int mine = 0;
+        for (int r = tid; r < p.batch; r += kThreads) {
+            Item it;
+            const int st = request_info(p, r, it);
+            if (st < 0 && blockIdx.x == 0) atomicOr(&g_mg_device_error, item_error(p, it));
+            if (st >= 0 && !(p.skip_single && it.n == 1)) mine += (it.n + kQTiles * p.tokens_per_qtile - 1) /
+                                                                 (kQTiles * p.tokens_per_qtile);
+        }
+        // ... a block-wide exclusive scan places them ...
+        int incl = mine;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (lane == 31) scan[warp] = incl;
+        __syncthreads();
+        if (tid == 0) {
+            int run = 0;
+            for (int w = 0; w < kThreads / 32; ++w) {
+                const int x = scan[w];
+                scan[w] = run;
+                run += x;
             }
-            keys[tid] = key;
+            scan[kThreads / 32] = run;
         }
         __syncthreads();
-        if (warp == 0) {
+        groups = scan[kThreads / 32];
+        // ... and, if the sorted list fits, writes their keys (cost descending,
+        // enumeration order for ties; the key's low half is 0xFFFF - group id)
+        sorted = groups <= kMaxSortGroups &&
+                 (int64_t)groups * p.num_kv_heads <= (int64_t)kMaxItemsPerCta * gridDim.x;
+        if (sorted && mine > 0) {
+            int at = scan[warp] + incl - mine;
+            for (int r = tid; r < p.batch; r += kThreads) {
+                Item it;
+                if (request_info(p, r, it) < 0 || (p.skip_single && it.n == 1)) continue;
+                const int span = kQTiles * p.tokens_per_qtile;
+                for (int qb = 0; qb * span < it.n; ++qb) {
+                    const int kv_len = it.c + min((qb + 1) * span, it.n);
+                    const int n_kv = (kv_len + kN - 1) / kN;
+                    const int gid = (p.num_qblocks - 1 - qb) * p.batch + r;
+                    keys[at++] = ((uint32_t)min(n_kv, kMaxCost) << 16) | (uint32_t)(0xFFFF - gid);
+                }
+            }
+        }
+        __syncthreads();
+        if (sorted && warp == 0) {
             if (groups <= 32 * 4) warp_sort_desc<4>(keys, lane);
             else warp_sort_desc<kSortPerLane>(keys, lane);
             __syncwarp();
@@ -496,9 +549,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 *sh_count = cnt;
             }
         }
-    } else if (tid == 0) {
-        *sh_count = 0;
     }
+    if (!sorted && tid == 0) *sh_count = 0;
 
     if (tid == 0) {
         *abort_flag = 0;
@@ -911,11 +963,13 @@ inline mg_status launch(Params &p, int sms, cudaStream_t stream) {
     if (items >= (int64_t)1 << 30) return MG_ERR_UNSUPPORTED_SHAPE;
     p.num_qblocks = (int32_t)nqb;
     p.num_items = (int32_t)items;
-    p.sorted = nqb * p.batch <= kMaxSortGroups ? 1 : 0;
-    // one CTA per SM; with a sorted list no CTA may need more than
-    // kMaxItemsPerCta items
+    // the kernel sorts the groups that hold tokens when there are at most
+    // kMaxSortGroups of them; group ids must fit the key's low 16 bits
+    p.sorted = nqb * p.batch < 0xFFFF ? 1 : 0;
+    // one CTA per SM; when every group may hold tokens and the list is sure to
+    // be sorted, no CTA may need more than kMaxItemsPerCta items
     int64_t grid = items < sms ? items : sms;
-    if (p.sorted) {
+    if (nqb * p.batch <= kMaxSortGroups) {
         const int64_t min_grid = (items + kMaxItemsPerCta - 1) / kMaxItemsPerCta;
         if (grid < min_grid) grid = min_grid;
     }

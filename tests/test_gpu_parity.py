@@ -394,6 +394,26 @@ def test_extend_deterministic():
     assert torch.equal(a, b)
 
 
+@pytest.mark.parametrize("batch", [250, 300])
+def test_extend_work_list_sorted_or_walked(batch):
+    """The kernel sorts the (request, q block) groups that hold tokens when
+    there are at most 256 of them, and walks the plain enumeration otherwise:
+    250 and 300 short prompts (one group each) take the two paths, with
+    requests that have nothing new in between."""
+    rng = np.random.default_rng(batch)
+    cached = [int(x) for x in rng.integers(0, 200, size=batch)]
+    seq = [c + int(rng.integers(1, 40)) for c in cached]
+    for r in range(0, batch, 17):
+        seq[r] = cached[r]  # no new token: no group
+    step, data = _custom("extend", cached, seq, 16, 8, seed=900 + batch)
+    g = GpuStep(step, data)
+    g.store()
+    out = g.extend()
+    assert mg.read_device_error() == 0
+    req = sorted(set(range(0, batch, 23)) | {1, batch - 1})
+    assert_matches_oracle(out, oracle_extend(step, data, requests=req), f"extend, {batch} short prompts")
+
+
 # --------------------------------------------------------------------------- tensor-parallel head shards
 
 @pytest.mark.parametrize("world", [2, 16])
