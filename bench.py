@@ -19,7 +19,9 @@ The JSON line: `value` = algorithmic bytes (K/V rows once per GQA group, q,
 out, page-table entries, plus the store's reads and writes) per step summed
 over ranks / step time, in GB/s; `e2e` = the same through the public API with
 the step's inputs copied from pinned host memory into the fixed buffers and
-the outputs copied back inside the timed region; `roofline` = one layer's
+the outputs copied back inside the timed region (layer l+1's rows travel on a
+copy stream while layer l computes, and each layer's output goes back as soon
+as it is done, all captured in the step's graph); `roofline` = one layer's
 mg_store_decode_attn call (decode kernel with the store fused, then the merge
 kernel; --unfused: mg_decode_attn after a separate mg_store_kv) against the
 measured HBM copy bandwidth, its duration the timed step's device time over
@@ -260,6 +262,36 @@ def io_bytes(bench):
     return h2d, bench.out_host.numel() * bench.out_host.element_size()
 
 
+def overlapped_io_step(bench, side_in, side_out, ev_in, ev_out):
+    """One end-to-end step with its host copies overlapped with the layers:
+    the metadata first, then every layer's q / k / v rows on a copy stream
+    (layer l's rows are waited for just before layer l runs), and each layer's
+    output copied back on a second copy stream as soon as that layer is done.
+    The step ends when the last copy has landed, as an engine's would."""
+    main = torch.cuda.current_stream()
+    for n, t in bench.meta_host.items():
+        bench.meta[n].copy_(t, non_blocking=True)
+    L = len(bench.layers)
+    per_in, per_out = bench.in_dev.numel() // L, bench.out_dev.numel() // L
+    side_in.wait_stream(main)
+    side_out.wait_stream(main)
+    with torch.cuda.stream(side_in):
+        for i in range(L):
+            bench.in_dev[i * per_in:(i + 1) * per_in].copy_(bench.in_host[i * per_in:(i + 1) * per_in],
+                                                            non_blocking=True)
+            ev_in[i].record(side_in)
+    for i, lay in enumerate(bench.layers):
+        main.wait_event(ev_in[i])
+        bench.layer(lay, bench.outs[i], bench.meta)
+        ev_out[i].record(main)
+        side_out.wait_event(ev_out[i])
+        with torch.cuda.stream(side_out):
+            bench.out_host[i * per_out:(i + 1) * per_out].copy_(bench.out_dev[i * per_out:(i + 1) * per_out],
+                                                                non_blocking=True)
+    main.wait_stream(side_out)
+    main.wait_stream(side_in)
+
+
 class DecodeBench:
     def __init__(self, spec, step, device, partitions, fused=True, plain=False):
         from paged_kv_attention_mg_b200 import mg
@@ -340,17 +372,6 @@ class DecodeBench:
         for i, lay in enumerate(self.layers):
             self.layer(lay, self.outs[i], self.meta, events[i] if events else None)
 
-    def copy_in(self):
-        """This step's inputs from pinned host memory into the fixed device buffers:
-        the metadata, then every layer's q / k / v rows in one copy."""
-        for n, t in self.meta_host.items():
-            self.meta[n].copy_(t, non_blocking=True)
-        self.in_dev.copy_(self.in_host, non_blocking=True)
-
-    def copy_out(self):
-        """Every layer's attention output back to pinned host memory in one copy."""
-        self.out_host.copy_(self.out_dev, non_blocking=True)
-
     def kernel_bytes(self):
         return self.decode_bytes
 
@@ -410,8 +431,6 @@ class ExtendBench:
             events[1].record()
 
     run_step = DecodeBench.run_step
-    copy_in = DecodeBench.copy_in
-    copy_out = DecodeBench.copy_out
 
     def details(self):
         d = {"kv_bytes_per_step": self.extend_bytes}
@@ -704,10 +723,22 @@ def run_ours(args):
     # the outputs copied back to pinned host memory
     e2e = None
     if not args.no_e2e:
-        def e2e_step():
-            bench.copy_in()
-            run_plain()
-            bench.copy_out()
+        side_in, side_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
+        ev_in = [torch.cuda.Event() for _ in range(spec.num_layers)]
+        ev_out = [torch.cuda.Event() for _ in range(spec.num_layers)]
+
+        def e2e_enqueue():
+            overlapped_io_step(bench, side_in, side_out, ev_in, ev_out)
+        e2e_enqueue()  # eager once: the copy streams warm up
+        torch.cuda.synchronize()
+        if use_graph:
+            g_e2e = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g_e2e):
+                e2e_enqueue()
+            graphs.append(g_e2e)
+            e2e_step = g_e2e.replay
+        else:
+            e2e_step = e2e_enqueue
         for _ in range(2):
             e2e_step()
         torch.cuda.synchronize()
