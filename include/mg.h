@@ -42,6 +42,15 @@
  *   - The caller owns every buffer.  Inputs are read-only except the pools
  *     in mg_store_kv; outputs are written in full for every real (request,
  *     head) row.
+ *   - The kernels are launched with programmatic dependent launch, so one
+ *     may start while the previous kernel on the stream finishes.  Before it
+ *     waits for that kernel, a kernel of this library reads only the request
+ *     metadata (page_table, table_idx, seq_len, cached_len, q_offset,
+ *     group_first, prefix_len), which none of its kernels writes: the pools,
+ *     q, the new K/V rows, the workspace and the outputs are touched only
+ *     after the wait.  A kernel of the caller's that ends with a programmatic
+ *     launch trigger must therefore have written that metadata before its
+ *     trigger (a kernel without a trigger completes before ours start).
  *   - The softmax scale must be finite and > 0 (else MG_ERR_INVALID_ARGUMENT):
  *     the kernels take row maxima of the unscaled scores and scale them after,
  *     which needs a positive scale.  (scale = 0, whose result is the plain

@@ -363,9 +363,11 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
     const int w = blockIdx.x * kWarps + warp;
     const int nchunks = (p.num_vreqs + kScanChunk - 1) / kScanChunk;
     griddep_launch_dependents();  // the merge kernel may launch and wait on us
-    griddep_wait();               // inputs written by the previous kernel (e.g. the KV store)
 
-    // ---- pass 1: units per scan chunk (and the total T)
+    // ---- pass 1: units per scan chunk (and the total T).  It reads request
+    // metadata only, which no kernel of this library writes, so it runs before
+    // the wait on the previous kernel (e.g. the KV store, or the previous
+    // layer's merge) and overlaps that kernel's tail.
     unsigned bad = 0;
     int64_t running = 0;
     for (int ch = 0; ch < nchunks; ++ch) {
@@ -386,7 +388,11 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
     __syncthreads();
 
     // ---- pass 2: locate the request holding each worker's first unit (CTA 0
-    // scans every chunk and also publishes the per-request prefix for the merge)
+    // scans every chunk and also publishes the per-request prefix for the
+    // merge, so it waits first: the workspace may still be read by the
+    // previous call's merge; every other CTA waits after this pass, before
+    // its first pool, workspace or output access)
+    if (blockIdx.x == 0) griddep_wait();
     if (tid <= kWarps) sh_bound[tid] = worker_begin(T, blockIdx.x * kWarps + tid, W);
     __syncthreads();
     {
@@ -426,6 +432,8 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
         if (blockIdx.x == 0 && tid == 0) p.prefix[p.num_vreqs] = T;
     }
     __syncthreads();
+
+    if (blockIdx.x != 0) griddep_wait();
 
     // ---- this warp's share
     const int64_t ub = sh_bound[warp], ue = sh_bound[warp + 1];

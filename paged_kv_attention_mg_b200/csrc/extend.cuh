@@ -473,7 +473,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t lim = p.wait_limit_ns;  // nanoseconds
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     griddep_launch_dependents();
-    griddep_wait();  // inputs written by the previous kernel (e.g. the KV store)
 
     // ---- the work list.  Sorted mode: every CTA sorts the same group keys
     // (cost descending, enumeration order for ties; a group is the Hkv items of
@@ -579,6 +578,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
     __syncthreads();  // also: the sort scratch in the K ring is dead from here on
     tc_fence_after();
+    // The work list above reads request metadata only, which no kernel of this
+    // library writes, so it was built while the previous kernel (e.g. the KV
+    // store) may still run; the pool, q and out are touched only from here on.
+    griddep_wait();
     const uint32_t tmem = *tmem_holder;
     const int list_len = *sh_count;
     const int g = p.group, tpq = p.tokens_per_qtile;
