@@ -390,7 +390,7 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
     // ---- pass 2: locate the request holding each worker's first unit (CTA 0
     // scans every chunk and also publishes the per-request prefix for the
     // merge, so it waits first: the workspace may still be read by the
-    // previous call's merge; every other CTA waits after this pass, before
+    // previous call's merge; every other warp waits in its main loop, before
     // its first pool, workspace or output access)
     if (blockIdx.x == 0) griddep_wait();
     if (tid <= kWarps) sh_bound[tid] = worker_begin(T, blockIdx.x * kWarps + tid, W);
@@ -432,8 +432,6 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
         if (blockIdx.x == 0 && tid == 0) p.prefix[p.num_vreqs] = T;
     }
     __syncthreads();
-
-    if (blockIdx.x != 0) griddep_wait();
 
     // ---- this warp's share
     const int64_t ub = sh_bound[warp], ue = sh_bound[warp + 1];
@@ -544,6 +542,9 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
         const int j = k + kStages - 1;
         cp_async_wait<kIdxAhead - kStages>();
         __syncwarp();
+        // the page-table fetches before the first K/V gather read metadata
+        // only, so they run ahead of the wait on the previous kernel
+        if (k == 1 - kStages && blockIdx.x != 0) griddep_wait();
         if (j >= 0 && j < n_units) issue(j);
         cp_async_commit();
         if (k < 0) continue;
