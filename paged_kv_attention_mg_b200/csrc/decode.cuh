@@ -804,25 +804,64 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
 #define MG_DECODE_MERGE_BATCH 8
 #endif
 constexpr int kMergeBatch = MG_DECODE_MERGE_BATCH;  // partial segments loaded per round
+constexpr int kMergeScanMax = 1024;  // requests a merge warp counts units over itself
 __global__ void __launch_bounds__(128) decode_merge_kernel(const Params p) {
     const int wg = blockIdx.x * 4 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     griddep_launch_dependents();
-    griddep_wait();  // the decode kernel's partials
     if (wg >= p.batch * p.num_q_heads) return;
     const int r = wg / p.num_q_heads, h = wg - r * p.num_q_heads;
     const int g = p.group;
     const int kvh = h / g, j = h - kvh * g;
-    const int64_t T = p.prefix[p.num_vreqs];
+    const int vs = p.num_groups + r;  // the request's own virtual request
+    // Before the wait, from request metadata only (which no kernel of this
+    // library writes), so it overlaps the decode kernel: with few requests and
+    // no shared prefixes, the unit offsets of this request's pair are counted
+    // here exactly as the decode kernel counts them; otherwise they come from
+    // the table the decode kernel publishes.
+    const bool own_scan = p.num_groups == 0 && p.num_vreqs <= kMergeScanMax;
+    int64_t T = 0, pr0 = 0, pr1 = 0;
+    if (own_scan) {
+        int64_t tot = 0, before = 0, mine = 0;
+        for (int v = lane; v < p.num_vreqs; v += 32) {
+            int L, row;
+            unsigned bad = 0;
+            const int64_t u = request_units(p, v, L, row, bad);
+            tot += u;
+            before += v < vs ? u : 0;
+            mine += v == vs ? u : 0;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            tot += __shfl_xor_sync(0xffffffffu, tot, o);
+            before += __shfl_xor_sync(0xffffffffu, before, o);
+            mine += __shfl_xor_sync(0xffffffffu, mine, o);
+        }
+        T = tot;
+        pr0 = before;
+        pr1 = before + mine;
+    }
+    int grp = -1;  // cascade: the group whose shared prefix this request reads
+    if (p.num_groups > 0) {
+        grp = group_of(p, r);
+        unsigned ignore = 0;
+        if (grp >= 0 && group_prefix(p, grp, ignore) == 0) grp = -1;
+    }
+    griddep_wait();  // the decode kernel's partials (and its unit table)
+    if (!own_scan) {
+        T = p.prefix[p.num_vreqs];
+        pr0 = p.prefix[vs];
+        pr1 = p.prefix[vs + 1];
+    }
     const int W = p.num_workers;
     const int64_t rs = p.rows_per_slot;
     auto worker_of = [&](int64_t u) -> int {  // the worker whose share holds unit u
         const int64_t wv = ((u + 1) * (int64_t)W - 1) / T;
         return (int)(wv < W - 1 ? wv : W - 1);
     };
-    // the workers [wf, wl] that held pair (virtual request v, kvh)
-    auto pair_workers = [&](int v, int &wf, int &wl) -> bool {
-        const int64_t pr = p.prefix[v], units_v = p.prefix[v + 1] - pr;
+    // the workers [wf, wl] that held the pair of kv head kvh of a virtual
+    // request whose units start at unit pr (units_v of them)
+    auto pair_workers = [&](int64_t pr, int64_t units_v, int &wf, int &wl) -> bool {
         if (units_v <= 0) return false;  // rejected (flagged by the decode kernel)
         const int64_t tiles = units_v / p.num_kv_heads;
         const int64_t u0 = pr + kvh * tiles;
@@ -830,15 +869,10 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const Params p) {
         wl = worker_of(u0 + tiles - 1);
         return true;
     };
-    const int vs = p.num_groups + r;  // the request's own virtual request
     int wf, wl;
-    if (T <= 0 || !pair_workers(vs, wf, wl)) return;
-    int grp = -1, wfp = 0, wlp = -1;  // cascade: the group whose shared prefix this request reads
-    if (p.num_groups > 0) {
-        grp = group_of(p, r);
-        unsigned ignore = 0;
-        if (grp >= 0 && (group_prefix(p, grp, ignore) == 0 || !pair_workers(grp, wfp, wlp))) grp = -1;
-    }
+    if (T <= 0 || !pair_workers(pr0, pr1 - pr0, wf, wl)) return;
+    int wfp = 0, wlp = -1;
+    if (grp >= 0 && !pair_workers(p.prefix[grp], p.prefix[grp + 1] - p.prefix[grp], wfp, wlp)) grp = -1;
     if (grp < 0 && wf == wl) return;  // one worker held the whole pair and wrote the output
     // with at least as many units as workers every share is non-empty; else
     // skip the workers that got no units (and wrote no partial)
