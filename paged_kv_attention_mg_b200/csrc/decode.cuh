@@ -804,7 +804,7 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
 #define MG_DECODE_MERGE_BATCH 8
 #endif
 constexpr int kMergeBatch = MG_DECODE_MERGE_BATCH;  // partial segments loaded per round
-constexpr int kMergeScanMax = 1024;  // requests a merge warp counts units over itself
+constexpr int kMergeScanMax = 64;  // requests a merge warp counts units over itself (two per lane)
 __global__ void __launch_bounds__(128) decode_merge_kernel(const Params p) {
     const int wg = blockIdx.x * 4 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
