@@ -721,9 +721,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 float rs[8];  // eight row-sum chains: two per column block
 #pragma unroll
                 for (int c = 0; c < 8; ++c) rs[c] = 0.f;
+                // 32-key chunks past every row's last visible key (the causal edge of a
+                // diagonal tile) hold no weight for any row of the warp: their P is
+                // stored as zeros without computing it
+                const int live_chunks = full ? 4 : (int)__reduce_max_sync(0xffffffffu, (unsigned)(nvis + 31) / 32u);
 #pragma unroll
                 for (int cb = 0; cb < 4; ++cb) {  // masked keys hold -inf and give exactly 0
                     uint32_t pk[16];
+                    if (cb >= live_chunks) {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) pk[e] = 0u;
+                        tmem_st_32x32b_x16(tS + cb * 16, pk);
+                        continue;
+                    }
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
                         const float2 x = ffma2(make_float2(__uint_as_float(sv[cb * 32 + 2 * e]),
