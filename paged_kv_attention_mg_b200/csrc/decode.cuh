@@ -362,7 +362,6 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
     const int W = p.num_workers;
     const int w = blockIdx.x * kWarps + warp;
     const int nchunks = (p.num_vreqs + kScanChunk - 1) / kScanChunk;
-    griddep_launch_dependents();  // the merge kernel may launch and wait on us
 
     // ---- pass 1: units per scan chunk (and the total T).  It reads request
     // metadata only, which no kernel of this library writes, so it runs before
@@ -432,6 +431,11 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
         if (blockIdx.x == 0 && tid == 0) p.prefix[p.num_vreqs] = T;
     }
     __syncthreads();
+
+    // the merge kernel may launch now and wait on us (triggered after the scans
+    // rather than at the start: merge CTAs resident beside the scans measured
+    // slower on the shared-prefix workload)
+    griddep_launch_dependents();
 
     // ---- this warp's share
     const int64_t ub = sh_bound[warp], ue = sh_bound[warp + 1];
