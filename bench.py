@@ -768,7 +768,7 @@ def run_ours(args):
                 "peak_source": f"{peak_src} HBM copy bandwidth",
                 "call_us": round(kernel_ms * 1e3, 3), "duration": "timed step / layer calls in it",
                 "call_us_events": round(events_ms * 1e3, 3),
-                "traffic": profiled_traffic(spec.name)}
+                "traffic": profiled_traffic(spec.name + (":plain" if args.plain else ""))}
         extra = {"tokens_per_s": round(step_tokens / (step_ms * 1e-3), 1),
                  "frac_of_8tbs_nominal": round(value / n / 8000.0, 4),
                  "frac_of_measured_hbm": round(value / n / hbm, 4)}
