@@ -19,9 +19,9 @@ The JSON line: `value` = algorithmic bytes (K/V rows once per GQA group, q,
 out, page-table entries, plus the store's reads and writes) per step summed
 over ranks / step time, in GB/s; `e2e` = the same through the public API with
 the step's inputs copied from pinned host memory into the fixed buffers and
-the outputs copied back inside the timed region (layer l+1's rows travel on a
-copy stream while layer l computes, and each layer's output goes back as soon
-as it is done, all captured in the step's graph); `roofline` = one layer's
+the outputs copied back inside the timed region (two buffer sets in turn, so
+a step's host copies, on two copy streams, overlap the neighbouring steps'
+layer calls, as a serving loop's would); `roofline` = one layer's
 mg_store_decode_attn call (decode kernel with the store fused, then the merge
 kernel; --unfused: mg_decode_attn after a separate mg_store_kv) against the
 measured HBM copy bandwidth, its duration the timed step's device time over
@@ -262,34 +262,60 @@ def io_bytes(bench):
     return h2d, bench.out_host.numel() * bench.out_host.element_size()
 
 
-def overlapped_io_step(bench, side_in, side_out, ev_in, ev_out):
-    """One end-to-end step with its host copies overlapped with the layers:
-    the metadata first, then every layer's q / k / v rows on a copy stream
-    (layer l's rows are waited for just before layer l runs), and each layer's
-    output copied back on a second copy stream as soon as that layer is done.
-    The step ends when the last copy has landed, as an engine's would."""
+class IoSet:
+    """One of the two buffer sets an end-to-end step alternates between: device
+    copies of the step's inputs (metadata, every layer's q / k / v rows) and
+    outputs, a pinned host buffer for the outputs, the layers' views into them,
+    and the events that order its copies and its layer calls."""
+
+    def __init__(self, bench, first: bool):
+        if first:  # the buffers the bench already holds
+            self.in_dev, self.out_dev, self.meta = bench.in_dev, bench.out_dev, bench.meta
+            self.layers, self.outs = bench.layers, bench.outs
+            self.out_host = bench.out_host
+        else:
+            self.in_dev = bench.in_dev.clone()
+            self.out_dev = torch.empty_like(bench.out_dev)
+            self.out_host = torch.empty_like(bench.out_host).pin_memory()
+            self.meta = {n: t.clone() for n, t in bench.meta.items()}
+            base, es = bench.in_dev.data_ptr(), bench.in_dev.element_size()
+
+            def view(t):  # the same view of this set's input buffer
+                off = (t.data_ptr() - base) // es
+                return self.in_dev[off:off + t.numel()].view(t.shape)
+            self.layers = [dict(lay, q=view(lay["q"]), k_new=view(lay["k_new"]), v_new=view(lay["v_new"]))
+                           for lay in bench.layers]
+            per = bench.out_dev.numel() // len(bench.layers)
+            self.outs = [self.out_dev[i * per:(i + 1) * per].view(o.shape) for i, o in enumerate(bench.outs)]
+        self.in_done, self.compute_done, self.out_done = torch.cuda.Event(), torch.cuda.Event(), torch.cuda.Event()
+        self.run = None
+
+    def compute(self, bench):
+        for i, lay in enumerate(self.layers):
+            bench.layer(lay, self.outs[i], self.meta)
+
+
+def pipelined_io_step(bench, io, side_in, side_out):
+    """One end-to-end step on buffer set `io`: its inputs copied from pinned host
+    memory on a copy stream, its layer calls, its outputs copied back on a
+    second copy stream.  Consecutive steps use the two sets in turn, so a
+    step's copies overlap its neighbours' layers, as a serving loop's would;
+    each set's copies wait for the last use of the buffers they overwrite."""
     main = torch.cuda.current_stream()
-    for n, t in bench.meta_host.items():
-        bench.meta[n].copy_(t, non_blocking=True)
-    L = len(bench.layers)
-    per_in, per_out = bench.in_dev.numel() // L, bench.out_dev.numel() // L
-    side_in.wait_stream(main)
-    side_out.wait_stream(main)
+    side_in.wait_event(io.compute_done)  # the previous step on this set has read its inputs
     with torch.cuda.stream(side_in):
-        for i in range(L):
-            bench.in_dev[i * per_in:(i + 1) * per_in].copy_(bench.in_host[i * per_in:(i + 1) * per_in],
-                                                            non_blocking=True)
-            ev_in[i].record(side_in)
-    for i, lay in enumerate(bench.layers):
-        main.wait_event(ev_in[i])
-        bench.layer(lay, bench.outs[i], bench.meta)
-        ev_out[i].record(main)
-        side_out.wait_event(ev_out[i])
-        with torch.cuda.stream(side_out):
-            bench.out_host[i * per_out:(i + 1) * per_out].copy_(bench.out_dev[i * per_out:(i + 1) * per_out],
-                                                                non_blocking=True)
-    main.wait_stream(side_out)
-    main.wait_stream(side_in)
+        for n, t in bench.meta_host.items():
+            io.meta[n].copy_(t, non_blocking=True)
+        io.in_dev.copy_(bench.in_host, non_blocking=True)
+        io.in_done.record(side_in)
+    main.wait_event(io.in_done)
+    main.wait_event(io.out_done)  # ... and its outputs have left the device
+    io.run()
+    io.compute_done.record(main)
+    side_out.wait_event(io.compute_done)
+    with torch.cuda.stream(side_out):
+        io.out_host.copy_(io.out_dev, non_blocking=True)
+        io.out_done.record(side_out)
 
 
 class DecodeBench:
@@ -724,30 +750,31 @@ def run_ours(args):
     e2e = None
     if not args.no_e2e:
         side_in, side_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
-        ev_in = [torch.cuda.Event() for _ in range(spec.num_layers)]
-        ev_out = [torch.cuda.Event() for _ in range(spec.num_layers)]
-
-        def e2e_enqueue():
-            overlapped_io_step(bench, side_in, side_out, ev_in, ev_out)
-        e2e_enqueue()  # eager once: the copy streams warm up
+        sets = [IoSet(bench, True), IoSet(bench, False)]
+        for io in sets:
+            if use_graph:  # each set's layer calls as one graph, like the timed step
+                io.compute(bench)
+                torch.cuda.synchronize()
+                g_io = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g_io):
+                    io.compute(bench)
+                graphs.append(g_io)
+                io.run = g_io.replay
+            else:
+                io.run = (lambda io=io: io.compute(bench))
         torch.cuda.synchronize()
-        if use_graph:
-            g_e2e = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g_e2e):
-                e2e_enqueue()
-            graphs.append(g_e2e)
-            e2e_step = g_e2e.replay
-        else:
-            e2e_step = e2e_enqueue
-        for _ in range(2):
-            e2e_step()
+        for k in range(4):
+            pipelined_io_step(bench, sets[k & 1], side_in, side_out)
         torch.cuda.synchronize()
         dist.barrier()
+        main = torch.cuda.current_stream()
         ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e2e_steps = max(3, args.steps)
         ea.record()
-        for _ in range(e2e_steps):
-            e2e_step()
+        for k in range(e2e_steps):
+            pipelined_io_step(bench, sets[k & 1], side_in, side_out)
+        main.wait_stream(side_out)
+        main.wait_stream(side_in)
         eb.record()
         torch.cuda.synchronize()
         e2e = dist.max(ea.elapsed_time(eb) / e2e_steps)
