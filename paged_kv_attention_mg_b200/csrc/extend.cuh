@@ -346,7 +346,7 @@ __device__ __forceinline__ void load_rows(const Params &p, uint32_t ring_base, u
                                           bool sorted, volatile int *abort_flag, uint64_t lim, bool flag_errors) {
     constexpr int kMaxPairs = (kPairs + NW - 1) / NW;
     const int npairs = (kPairs - u + NW - 1) / NW;
-    const int64_t head_stride = (int64_t)p.num_kv_heads * kHeadDim;
+    const uint32_t row_bytes = (uint32_t)p.num_kv_heads * kHeadDim * 2;  // one slot's K (or V) row
     auto key_of = [&](int i) { return 2 * (u + NW * (i >> 1)) + (i & 1); };
     // slots of (item, tile j) for list indices lane and lane + 32 (-1: none)
     auto fetch = [&](int row, int kv_len, int j, int &sa, int &sb) {
@@ -377,6 +377,14 @@ __device__ __forceinline__ void load_rows(const Params &p, uint32_t ring_base, u
     int sa, sb;
     fetch(row, kv_len, 0, sa, sb);
     const int c = lane & 15, half = c >> 3, cc = c & 7;
+    // the shared-memory offset of each of this lane's copies within a stage: the
+    // same for every tile, so it is computed once
+    uint32_t doff[kMaxPairs];
+#pragma unroll
+    for (int m = 0; m < kMaxPairs; ++m) {
+        const int key = key_of(2 * m + (lane >> 4));
+        doff[m] = (uint32_t)(half * kHalfBytes + key * 128 + ((cc ^ (key & 7)) << 4));
+    }
     for (int seq = 0;; ++seq) {
         // tile (it, j): wait for its ring stage
         const int stage = seq % STAGES;
@@ -384,16 +392,15 @@ __device__ __forceinline__ void load_rows(const Params &p, uint32_t ring_base, u
         check(sa, lane < 2 * npairs && j * kN + key_of(lane) < kv_len);
         check(sb, lane + 32 < 2 * npairs && j * kN + key_of(lane + 32) < kv_len);
         const uint32_t tile = ring_base + (uint32_t)(stage * kTileBytes);
+        const char *base = reinterpret_cast<const char *>(pool + (int64_t)kvh * kHeadDim + c * 8);
 #pragma unroll
         for (int m = 0; m < kMaxPairs; ++m) {
             if (m < npairs) {
                 const int i = 2 * m + (lane >> 4);  // list index this half-warp copies
-                const int key = key_of(i);
                 const int slot = m < 16 ? __shfl_sync(0xffffffffu, sa, i & 31) : __shfl_sync(0xffffffffu, sb, i & 31);
-                const __nv_bfloat16 *src = pool + (int64_t)(slot < 0 ? 0 : slot) * head_stride +
-                                           (int64_t)kvh * kHeadDim + c * 8;
-                const uint32_t dst = tile + half * kHalfBytes + key * 128 + ((cc ^ (key & 7)) << 4);
-                cp_async_16(dst, src, slot < 0 ? 0u : 16u);
+                // one wide multiply-add: base + slot * row bytes (a slot row is at most 4 KB)
+                const char *src = base + (uint64_t)(uint32_t)max(slot, 0) * row_bytes;
+                cp_async_16(tile + doff[m], src, slot < 0 ? 0u : 16u);
             }
         }
         cp_async_arrive_noinc(full0 + stage * 8);
