@@ -481,6 +481,16 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
             cursor_advance<CASCADE>(p, cur);
         }
     };
+    // this lane's shared-memory offsets within a stage for its 16 copies of a
+    // tile (lanes 0-15 and 16-31 move one row each per copy: K rows first, then
+    // V): the same for every tile, so computed once
+    uint32_t soff[16];
+#pragma unroll
+    for (int it = 0; it < 16; ++it) {
+        const int rr = it * 2 + (lane >> 4);
+        soff[it] = (rr >= kKeys ? 2 * kHalfRows : 0) + swz(rr & (kKeys - 1), lane & 15);
+    }
+    const uint32_t row_bytes = (uint32_t)(head_stride * (int64_t)sizeof(__nv_bfloat16));  // one slot's K (or V) row
     // Issue stage: read tile j's entries, check them, gather its 16 K and 16 V
     // rows into the tile's shared-memory stage.
     auto issue = [&](int j) {
@@ -508,17 +518,28 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
         // (lanes 0-15 and 16-31); 32 rows per tile (16 K then 16 V)
         const uint32_t base = ring + (uint32_t)(stage * kTileBytes);
         const int ch = lane & 15;
-        const int64_t head_off = (int64_t)d.kvh * kHeadDim + ch * 8;
-        const int64_t new_off = ((int64_t)d.r * p.num_kv_heads + d.kvh) * kHeadDim + ch * 8;
+        const size_t head_off = ((size_t)d.kvh * kHeadDim + ch * 8) * sizeof(__nv_bfloat16);
+        const char *kb = reinterpret_cast<const char *>(p.k_cache) + head_off;
+        const char *vb = reinterpret_cast<const char *>(p.v_cache) + head_off;
+        if (FUSED && new_key >= 0) {  // the pair's last tile, which holds the new token
+            const int64_t new_off = ((int64_t)d.r * p.num_kv_heads + d.kvh) * kHeadDim + ch * 8;
 #pragma unroll
-        for (int it = 0; it < 16; ++it) {
-            const int rr = it * 2 + (lane >> 4);
-            const int key = rr & (kKeys - 1);
-            const bool is_v = rr >= kKeys;
-            const int sl = __shfl_sync(0xffffffffu, slot, key);
-            const __nv_bfloat16 *src = (is_v ? p.v_cache : p.k_cache) + (int64_t)(sl < 0 ? 0 : sl) * head_stride + head_off;
-            if (key == new_key) src = (is_v ? p.v_new : p.k_new) + new_off;
-            cp_async_16(base + (is_v ? 2 * kHalfRows : 0) + swz(key, ch), src, sl < 0 ? 0u : 16u);
+            for (int it = 0; it < 16; ++it) {
+                const int key = (it * 2 + (lane >> 4)) & (kKeys - 1);
+                const bool is_v = it >= kKeys / 2;
+                const int sl = __shfl_sync(0xffffffffu, slot, key);
+                const void *src = (is_v ? vb : kb) + (uint64_t)(uint32_t)max(sl, 0) * row_bytes;
+                if (key == new_key) src = (is_v ? p.v_new : p.k_new) + new_off;
+                cp_async_16(base + soff[it], src, sl < 0 ? 0u : 16u);
+            }
+        } else {
+#pragma unroll
+            for (int it = 0; it < 16; ++it) {
+                const int key = (it * 2 + (lane >> 4)) & (kKeys - 1);
+                const int sl = __shfl_sync(0xffffffffu, slot, key);
+                cp_async_16(base + soff[it], (it >= kKeys / 2 ? vb : kb) + (uint64_t)(uint32_t)max(sl, 0) * row_bytes,
+                            sl < 0 ? 0u : 16u);
+            }
         }
     };
 
