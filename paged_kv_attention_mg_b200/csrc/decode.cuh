@@ -24,8 +24,16 @@
 //   * transposed warp-level bf16 tensor-core products (m16n8k16, fp32
 //     accumulate): S^T = K Q^T and O^T += V^T P^T with keys / head dims in M and
 //     the GQA heads in N, so each K/V row is read from HBM once for all g heads
-//     and a g <= 8 group takes 16 MMAs per 16-key tile; online softmax in the
-//     exp2 domain with quad shuffles, O kept in registers.
+//     and a g <= 8 group takes 8 QK^T MMAs per 16-key tile, plus 16 for P V,
+//     whose P enters as a bf16 high part and a bf16 residual (P to ~2^-17, so
+//     the fp32 row sum of the weights is the normaliser); online softmax in
+//     the exp2 domain with quad shuffles, O kept in registers.
+//   * shared-prefix mode (CASCADE): the units run over virtual requests, first
+//     one per group (the group's common prefix keys, its members' q rows
+//     stacked, up to 16 rows = two n-tiles), then one per request (its keys
+//     after the prefix); the merge combines a request's own partials with its
+//     group's.  Mixed-batch mode (row_map): only the one-token requests count
+//     units, each writing the output row q_offset[r].
 //   * fused store (mg_store_decode_attn): the new token (position L-1) is read
 //     from k_new / v_new instead of the pool, and the worker that owns that tile
 //     writes it to its pool slot from shared memory once the tile has landed.

@@ -38,10 +38,11 @@
 //         core works on the other's.
 //       - warpgroups 1 / 2: softmax of Q tile 0 / 1, one TMEM lane (= query
 //         row) per thread: causal mask key <= c + i, online softmax in the
-//         exp2 domain (exponentials on MUFU), O rescaled in TMEM only when the
-//         running max grows by more
-//         than 2^8 (exact: P and the row sum use the same stale max and the
-//         same bf16-rounded P), epilogue O / l -> bf16 -> global.  Each also
+//         exp2 domain (exponentials on MUFU; 32-key chunks past every row's
+//         causal edge skipped), O rescaled in TMEM only when the running max
+//         grows by more than 2^8 (exact: P and the row sum use the same stale
+//         max and the same bf16-rounded P), epilogue O / l -> bf16 -> global.
+//         Each also
 //         loads its next item's Q tile by TMA as soon as its last score tile
 //         has landed (the tile's last reader is that Q K^T).
 // TMEM: S0 [0,128)  S1 [128,256)  O0 [256,384)  O1 [384,512) columns.
