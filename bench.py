@@ -80,6 +80,9 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="qwen3_0.6b_decode_28l", choices=sorted(wl.BY_NAME))
     ap.add_argument("--partitions", type=int, default=0, help="decode workers (0 = automatic plan)")
+    ap.add_argument("--extend-ctas", type=int, default=-1,
+                    help="mixed batches: SMs for the extend kernel beside the decode kernel "
+                         "(-1 = mg.mixed_extend_ctas's estimate, 0 = one kernel after the other)")
     ap.add_argument("--layers", type=int, default=0,
                     help="run only the first N layers (small cases for profiling; 0 = the workload's own)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -319,7 +322,7 @@ def pipelined_io_step(bench, io, side_in, side_out):
 
 
 class DecodeBench:
-    def __init__(self, spec, step, device, partitions, fused=True, plain=False):
+    def __init__(self, spec, step, device, partitions, fused=True, plain=False, extend_ctas=-1):
         from paged_kv_attention_mg_b200 import mg
         self.mg = mg
         self.fused = fused
@@ -415,7 +418,7 @@ class DecodeBench:
 
 
 class ExtendBench:
-    def __init__(self, spec, step, device, partitions, fused=True, plain=False):
+    def __init__(self, spec, step, device, partitions, fused=True, plain=False, extend_ctas=-1):
         from paged_kv_attention_mg_b200 import mg
         self.mg = mg
         self.spec, self.step, self.device = spec, step, device
@@ -434,10 +437,18 @@ class ExtendBench:
         self.launches_per_step = spec.num_layers * (4 if self.mixed else 2)
         self.h2d_bytes, self.d2h_bytes = io_bytes(self)
         self.workers = None
+        self.extend_ctas = 0
         if self.mixed:
             ws = mg.mixed_workspace_bytes(step.batch, spec.num_q_heads, spec.num_kv_heads, step.max_seq_len, partitions)
             self.workspace = torch.empty(max(ws, 16), dtype=torch.uint8, device=device)
             self.workers, _ = mg.decode_plan(step.batch, spec.num_kv_heads, step.max_seq_len, partitions)
+            sms = torch.cuda.get_device_properties(device).multi_processor_count
+            self.extend_ctas = (mg.mixed_extend_ctas(c, s, spec.num_q_heads, spec.num_kv_heads, sms)
+                                if extend_ctas < 0 else extend_ctas)
+            if self.extend_ctas > 0:  # the decode kernel's workers: 7 a CTA on the SMs left to it
+                w = 7 * (sms - min(self.extend_ctas, sms - 1))
+                self.workers, _ = mg.decode_plan(step.batch, spec.num_kv_heads, step.max_seq_len,
+                                                 partitions if 0 < partitions < w else w)
         self.partitions = partitions
 
     def layer(self, lay, out, meta, events=None):
@@ -448,7 +459,8 @@ class ExtendBench:
         if self.mixed:
             mg.mixed_attn(lay["q"], lay["k_cache"], lay["v_cache"], meta["page_table"], meta["table_idx"],
                           meta["cached_len"], meta["seq_len"], meta["q_offset"], st.max_q_len, st.max_seq_len,
-                          self.spec.scale, num_partitions=self.partitions, out=out, workspace=self.workspace)
+                          self.spec.scale, num_partitions=self.partitions, extend_ctas=self.extend_ctas, out=out,
+                          workspace=self.workspace)
         else:
             mg.extend_attn(lay["q"], lay["k_cache"], lay["v_cache"], meta["page_table"], meta["table_idx"],
                            meta["cached_len"], meta["seq_len"], meta["q_offset"], st.max_q_len, st.max_seq_len,
@@ -462,7 +474,7 @@ class ExtendBench:
         d = {"kv_bytes_per_step": self.extend_bytes}
         if self.mixed:
             d.update({"entry_point": "mg_mixed_attn (one-token requests: decode kernel + merge; chunks: extend kernel)",
-                      "decode_workers": self.workers})
+                      "decode_workers": self.workers, "extend_ctas": self.extend_ctas})
         return d
 
 
@@ -649,7 +661,8 @@ def run_ours(args):
         spec = dataclasses.replace(spec, num_layers=min(args.layers, spec.num_layers))
     step = wl.make_step(spec)
     bench = (DecodeBench if spec.kind == "decode" else ExtendBench)(spec, step, device, args.partitions,
-                                                                     fused=not args.unfused, plain=args.plain)
+                                                                     fused=not args.unfused, plain=args.plain,
+                                                                     extend_ctas=args.extend_ctas)
     flush = None
     if spec.kind == "extend" or decode_needs_flush(spec, step):
         flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)

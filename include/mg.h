@@ -35,10 +35,12 @@
  *     bf16 data is passed as void*.  Every tensor is dense and row-major, and
  *     every bf16 tensor must start on a 16-byte boundary.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  All work is
- *     enqueued on it; no entry point synchronises the host, allocates device
- *     memory or keeps state between calls (save the wait limit of
- *     mg_set_extend_wait_limit), so calls can be captured in a CUDA graph
- *     (mg_read_device_error excepted, which synchronises).
+ *     enqueued on it (mg_mixed_attn's split also forks onto a stream of the
+ *     library's and joins back); no entry point synchronises the host,
+ *     allocates device memory or keeps state between calls (save the wait
+ *     limit of mg_set_extend_wait_limit and that one stream per device), so
+ *     calls can be captured in a CUDA graph (mg_read_device_error excepted,
+ *     which synchronises).
  *   - The caller owns every buffer.  Inputs are read-only except the pools
  *     in mg_store_kv; outputs are written in full for every real (request,
  *     head) row.
@@ -281,9 +283,23 @@ mg_status mg_extend_attn(const void *q, const void *k_cache, const void *v_cache
  * through the split-KV decode kernel and its merge (query and output row
  * q_offset[r]; all keys 0 .. seq_len-1, the causal limit of a token at
  * position seq_len-1), every other request through the extend kernel, which
- * leaves the one-token requests alone: one call, three kernels on `stream`,
- * each request served by the kernel built for its shape.
+ * leaves the one-token requests alone: one call, three kernels, each request
+ * served by the kernel built for its shape.
  *   num_partitions  the decode kernel's plan (mg_decode_plan)
+ *   extend_ctas     0: the kernels run one after the other on `stream`.  > 0:
+ *                   the extend kernel runs on that many SMs at the same time
+ *                   as the decode kernel runs on the rest (capped at the SM
+ *                   count - 1; the decode plan then has 7 workers per
+ *                   remaining SM, or num_partitions if fewer): the decode
+ *                   kernel is bound by HBM and the extend kernel by its
+ *                   softmax and tensor cores, so they overlap.  The extend
+ *                   kernel then runs on a stream the library creates once per
+ *                   device and context, forked from and joined back to
+ *                   `stream` with two events created and released by the
+ *                   call (graph capture follows the fork and the join).  A
+ *                   good split gives each kernel the SMs that make them finish
+ *                   together; `mixed_extend_ctas` in the Python binding
+ *                   estimates it from the batch's lengths.  < 0: invalid.
  *   workspace       >= mg_mixed_workspace_bytes(...) bytes (the decode plan's)
  * Metadata errors are flagged as in mg_decode_attn / mg_extend_attn.
  */
@@ -294,8 +310,8 @@ mg_status mg_mixed_attn(const void *q, const void *k_cache, const void *v_cache,
                         const int32_t *table_idx, const int32_t *cached_len, const int32_t *seq_len,
                         const int32_t *q_offset, int32_t batch, int32_t total_q, int32_t max_q_len,
                         int32_t max_seq_len, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
-                        float scale, int32_t num_partitions, void *out, void *workspace, size_t workspace_bytes,
-                        void *stream);
+                        float scale, int32_t num_partitions, int32_t extend_ctas, void *out, void *workspace,
+                        size_t workspace_bytes, void *stream);
 
 /*
  * mg_decode_attn_static_workspace -- mg_decode_attn for callers that cannot

@@ -34,6 +34,16 @@ constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;
 std::atomic<uint64_t> g_extend_wait_limit_ns{kDefaultWaitLimitNs};
 std::atomic<int32_t> g_extend_inject_stall{0};
 
+// mg_mixed_attn with a split: the extend half runs on a library stream of the
+// device (non-blocking, created once per context), forked from and joined back
+// to the caller's stream by events.
+struct SideStream {
+    unsigned long long ctx;
+    cudaStream_t stream;
+};
+SideStream g_side[kMaxDevices];
+std::mutex g_side_mutex;
+
 using CtxGetCurrentFn = CUresult (*)(CUcontext *);
 using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long *);
 
@@ -80,6 +90,21 @@ mg_status sm_count(int &sms) {
         g_sm_count[dev].store(v, std::memory_order_release);
     }
     sms = v;
+    return MG_OK;
+}
+
+mg_status side_stream(cudaStream_t &out) {
+    int dev;
+    if (current_device(dev) != MG_OK) return MG_ERR_CUDA;
+    const unsigned long long ctx = current_context_id();
+    std::lock_guard<std::mutex> lock(g_side_mutex);
+    if (g_side[dev].stream == nullptr || g_side[dev].ctx != ctx) {
+        cudaStream_t st = nullptr;
+        if (cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking) != cudaSuccess) return MG_ERR_CUDA;
+        g_side[dev].stream = st;
+        g_side[dev].ctx = ctx;
+    }
+    out = g_side[dev].stream;
     return MG_OK;
 }
 
@@ -172,7 +197,7 @@ mg_status decode_impl(const void *q, const void *k_new, const void *v_new, const
                       int32_t num_kv_heads, int32_t head_dim, float scale, int32_t num_partitions, void *out,
                       void *workspace, size_t workspace_bytes, void *stream, const int32_t *group_first = nullptr,
                       const int32_t *prefix_len = nullptr, int32_t num_groups = 0, const int32_t *row_map = nullptr,
-                      int32_t total_rows = 0) {
+                      int32_t total_rows = 0, bool check_only = false) {
     const bool fused = k_new != nullptr;
     const bool cascade = group_first != nullptr;
     if (cascade && (fused || !prefix_len || num_groups <= 0)) return MG_ERR_INVALID_ARGUMENT;
@@ -198,6 +223,7 @@ mg_status decode_impl(const void *q, const void *k_new, const void *v_new, const
     const DecodeWorkspace ws = decode_ws_layout(batch, num_q_heads, num_kv_heads, workers, cascade ? num_groups : 0);
     if (!workspace || workspace_bytes < ws.total) return MG_ERR_WORKSPACE_TOO_SMALL;
     if (!aligned16(workspace)) return MG_ERR_MISALIGNED;
+    if (check_only) return MG_OK;  // the host checks alone (a caller about to launch other work first)
     if (ensure_kernel_attributes() != MG_OK) return MG_ERR_CUDA;
 
     decode::Params p;
@@ -264,7 +290,7 @@ mg_status extend_impl(const void *q, const void *k_cache, const void *v_cache, i
                       const int32_t *table_idx, const int32_t *cached_len, const int32_t *seq_len,
                       const int32_t *q_offset, int32_t batch, int32_t total_q, int32_t max_q_len,
                       int32_t max_seq_len, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, float scale,
-                      void *out, void *stream, bool skip_single) {
+                      void *out, void *stream, bool skip_single, int max_ctas = 0) {
     mg_status st = check_attention_shape(num_q_heads, num_kv_heads, head_dim);
     if (st != MG_OK) return st;
     if (!valid_scale(scale)) return MG_ERR_INVALID_ARGUMENT;
@@ -304,7 +330,7 @@ mg_status extend_impl(const void *q, const void *k_cache, const void *v_cache, i
     p.skip_single = skip_single ? 1 : 0;
     int sms;
     if (sm_count(sms) != MG_OK) return MG_ERR_CUDA;
-    return extend::launch(p, sms, static_cast<cudaStream_t>(stream));
+    return extend::launch(p, max_ctas > 0 && max_ctas < sms ? max_ctas : sms, static_cast<cudaStream_t>(stream));
 }
 }  // namespace
 }  // namespace mg
@@ -327,7 +353,7 @@ const char *mg_status_string(mg_status s) {
     return "MG_ERR_UNKNOWN";
 }
 
-int32_t mg_abi_version(void) { return 1; }
+int32_t mg_abi_version(void) { return 2; }
 
 mg_status mg_store_kv(const void *k, const void *v, const int32_t *out_loc, int32_t num_tokens,
                       void *k_cache, void *v_cache, int64_t num_slots, int32_t num_kv_heads,
@@ -449,17 +475,62 @@ mg_status mg_mixed_attn(const void *q, const void *k_cache, const void *v_cache,
                         const int32_t *table_idx, const int32_t *cached_len, const int32_t *seq_len,
                         const int32_t *q_offset, int32_t batch, int32_t total_q, int32_t max_q_len,
                         int32_t max_seq_len, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
-                        float scale, int32_t num_partitions, void *out, void *workspace, size_t workspace_bytes,
-                        void *stream) {
+                        float scale, int32_t num_partitions, int32_t extend_ctas, void *out, void *workspace,
+                        size_t workspace_bytes, void *stream) {
     // the same checks as mg_extend_attn, before anything is launched
     mg_status st = check_attention_shape(num_q_heads, num_kv_heads, head_dim);
     if (st != MG_OK) return st;
     if (!valid_scale(scale)) return MG_ERR_INVALID_ARGUMENT;
     if (batch <= 0 || total_q < 0 || max_q_len < 0 || num_slots <= 0 || page_table_rows <= 0 ||
-        page_table_stride <= 0 || max_seq_len <= 0 || max_seq_len > page_table_stride)
+        page_table_stride <= 0 || max_seq_len <= 0 || max_seq_len > page_table_stride || extend_ctas < 0)
         return MG_ERR_INVALID_ARGUMENT;
     if (total_q == 0 || max_q_len == 0) return MG_OK;
     if (!q_offset) return MG_ERR_INVALID_ARGUMENT;
+    int sms = 1;  // the device is asked only when a split is requested
+    if (extend_ctas > 0 && max_q_len > 1 && sm_count(sms) != MG_OK) return MG_ERR_CUDA;
+    if (extend_ctas > 0 && max_q_len > 1 && sms > 1) {
+        // The split: the extend kernel on extend_ctas SMs, on a side stream,
+        // while the decode kernel's workers fill the other SMs (the decode
+        // kernel is bound by HBM, the extend kernel by its softmax and tensor
+        // cores, so the two overlap instead of following each other).
+        const int e = extend_ctas < sms ? extend_ctas : sms - 1;
+        int32_t workers = decode::kWarps * (sms - e);
+        if (num_partitions > 0 && num_partitions < workers) workers = num_partitions;
+        // every host check of both halves before anything is enqueued
+        if (!cached_len) return MG_ERR_INVALID_ARGUMENT;
+        st = decode_impl(q, nullptr, nullptr, nullptr, k_cache, v_cache, num_slots, page_table, page_table_rows,
+                         page_table_stride, table_idx, seq_len, batch, max_seq_len, num_q_heads, num_kv_heads,
+                         head_dim, scale, workers, out, workspace, workspace_bytes, stream, nullptr, nullptr, 0,
+                         q_offset, total_q, true);
+        if (st != MG_OK) return st;
+        cudaStream_t side, s = static_cast<cudaStream_t>(stream);
+        if (side_stream(side) != MG_OK) return MG_ERR_CUDA;
+        cudaEvent_t fork = nullptr, join = nullptr;
+        if (cudaEventCreateWithFlags(&fork, cudaEventDisableTiming) != cudaSuccess) return MG_ERR_CUDA;
+        if (cudaEventCreateWithFlags(&join, cudaEventDisableTiming) != cudaSuccess) {
+            cudaEventDestroy(fork);
+            return MG_ERR_CUDA;
+        }
+        st = MG_OK;
+        if (cudaEventRecord(fork, s) != cudaSuccess || cudaStreamWaitEvent(side, fork, 0) != cudaSuccess)
+            st = MG_ERR_CUDA;
+        if (st == MG_OK)
+            st = extend_impl(q, k_cache, v_cache, num_slots, page_table, page_table_rows, page_table_stride,
+                             table_idx, cached_len, seq_len, q_offset, batch, total_q, max_q_len, max_seq_len,
+                             num_q_heads, num_kv_heads, head_dim, scale, out, side, true, e);
+        if (st == MG_OK)
+            st = decode_impl(q, nullptr, nullptr, nullptr, k_cache, v_cache, num_slots, page_table, page_table_rows,
+                             page_table_stride, table_idx, seq_len, batch, max_seq_len, num_q_heads, num_kv_heads,
+                             head_dim, scale, workers, out, workspace, workspace_bytes, stream, nullptr, nullptr, 0,
+                             q_offset, total_q);
+        // the join is recorded whatever happened above, so the caller's stream
+        // never runs ahead of work already enqueued on the side stream
+        const bool joined = cudaEventRecord(join, side) == cudaSuccess && cudaStreamWaitEvent(s, join, 0) == cudaSuccess;
+        cudaEventDestroy(fork);
+        cudaEventDestroy(join);
+        if (st == MG_OK && !joined) st = MG_ERR_CUDA;
+        return st;
+    }
     // one-token requests: the split-KV decode kernel and its merge, rows by q_offset
     st = decode_impl(q, nullptr, nullptr, nullptr, k_cache, v_cache, num_slots, page_table, page_table_rows,
                      page_table_stride, table_idx, seq_len, batch, max_seq_len, num_q_heads, num_kv_heads, head_dim,

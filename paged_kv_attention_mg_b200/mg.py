@@ -52,7 +52,7 @@ SIGNATURES = {
                                       _I32, _I32, _I32, _I32, _F32, _P, _P]),
     "mg_mixed_workspace_bytes": (_SZ, [_I32, _I32, _I32, _I32, _I32, _I32]),
     "mg_mixed_attn": (ctypes.c_int, [_P, _P, _P, _I64, _P, _I32, _I32, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32,
-                                     _I32, _I32, _F32, _I32, _P, _P, _SZ, _P]),
+                                     _I32, _I32, _F32, _I32, _I32, _P, _P, _SZ, _P]),
     "mg_decode_attn_static_workspace": (ctypes.c_int, [_P, _P, _P, _I64, _P, _I32, _I32, _P, _P, _I32, _I32,
                                                        _I32, _I32, _I32, _F32, _I32, _P, _P]),
     "mg_set_extend_wait_limit": (ctypes.c_int, [ctypes.c_uint64, _I32]),
@@ -306,10 +306,12 @@ def mixed_workspace_bytes(batch: int, num_q_heads: int, num_kv_heads: int, max_s
 def mixed_attn(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, page_table: torch.Tensor,
                table_idx: torch.Tensor, cached_len: torch.Tensor, seq_len: torch.Tensor, q_offset: torch.Tensor,
                max_q_len: int, max_seq_len: int, scale: float, num_partitions: int = 0,
-               out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
-               stream=None) -> torch.Tensor:
+               extend_ctas: int = 0, out: Optional[torch.Tensor] = None,
+               workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """extend_attn for a mixed batch: one-token requests through the decode
-    kernel, the others through the extend kernel; returns out [total_q, Hq, D]."""
+    kernel, the others through the extend kernel; returns out [total_q, Hq, D].
+    extend_ctas > 0 runs the extend kernel on that many SMs at the same time as
+    the decode kernel on the rest (see mixed_extend_ctas)."""
     if not isinstance(seq_len, torch.Tensor) or seq_len.dim() != 1:
         raise ValueError("mixed_attn: seq_len must be [batch]")
     b = seq_len.shape[0]
@@ -331,8 +333,42 @@ def mixed_attn(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, pa
                                 _dev(table_idx, torch.int32, "table_idx"), _dev(cached_len, torch.int32, "cached_len"),
                                 _dev(seq_len, torch.int32, "seq_len"), _dev(q_offset, torch.int32, "q_offset"),
                                 b, total_q, max_q_len, max_seq_len, hq, hkv, d, float(scale), num_partitions,
-                                _dev(out, torch.bfloat16, "out"), ws_ptr, ws_bytes, _stream(stream)), "mg_mixed_attn")
+                                extend_ctas, _dev(out, torch.bfloat16, "out"), ws_ptr, ws_bytes, _stream(stream)),
+           "mg_mixed_attn")
     return out
+
+
+# Per-SM rates the split estimate works with, measured on B200 with this
+# library's kernels: a 128-key tile of an extend item (two Q tiles, causal
+# edge tiles counted whole) every ~3.6 us per SM, and ~39 GB/s of K/V per SM
+# for the decode kernel (5.8 TB/s over 148 SMs).
+_EXTEND_TILE_S = 3.6e-6
+_DECODE_SM_BYTES_PER_S = 39e9
+
+
+def mixed_extend_ctas(cached_len, seq_len, num_q_heads: int, num_kv_heads: int, sms: int,
+                      head_dim: int = 128) -> int:
+    """How many SMs mg_mixed_attn should give the extend kernel so that it and
+    the decode kernel finish together, from the batch's host-side lengths (the
+    scheduler that formed the batch has them): the extend items' KV tiles
+    against the one-token requests' K/V bytes, at the per-SM rates above.
+    0 when the batch has no prompt chunk or no one-token request."""
+    g = num_q_heads // num_kv_heads
+    span = 2 * (128 // g)  # tokens of a q block
+    tiles, dec_bytes = 0, 0
+    for c, L in zip(cached_len, seq_len):
+        c, L = int(c), int(L)
+        n = L - c
+        if n == 1:
+            dec_bytes += L * num_kv_heads * head_dim * 2 * 2
+        elif n > 1:
+            for t0 in range(0, n, span):
+                tiles += -(-(c + min(t0 + span, n)) // 128) * num_kv_heads
+    if tiles == 0 or dec_bytes == 0:
+        return 0
+    ext_s = tiles * _EXTEND_TILE_S
+    dec_s = dec_bytes / _DECODE_SM_BYTES_PER_S
+    return max(1, min(sms - 1, round(sms * ext_s / (ext_s + dec_s))))
 
 
 STATIC_WORKSPACE_BYTES = 16 << 20  # MG_DECODE_STATIC_WORKSPACE_BYTES in include/mg.h

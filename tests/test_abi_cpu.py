@@ -48,7 +48,7 @@ def test_build_targets_sm100a_only():
 def test_status_strings(lib):
     for code, name in mg.STATUS.items():
         assert lib.mg_status_string(code).decode() == name
-    assert lib.mg_abi_version() == 1
+    assert lib.mg_abi_version() == 2
 
 
 def test_store_zero_tokens_is_noop(lib):
@@ -124,11 +124,12 @@ def test_mixed_attn_host_validation(lib):
     assert lib.mg_mixed_workspace_bytes(8, 32, 4, 128, 32768, 1000) == lib.mg_decode_workspace_bytes(8, 32, 4, 128,
                                                                                                        32768, 1000)
     args = [4096, 4096, 4096, 100, 4096, 5, 32, 4096, 4096, 4096, 4096, 4, 10, 4, 32, 16, 8]
-    assert lib.mg_mixed_attn(*args, 64, 0.1, 0, 4096, 4096, 1 << 30, None) == 2            # head_dim 64
-    assert lib.mg_mixed_attn(*args, 128, -1.0, 0, 4096, 4096, 1 << 30, None) == 1          # scale
+    assert lib.mg_mixed_attn(*args, 64, 0.1, 0, 0, 4096, 4096, 1 << 30, None) == 2            # head_dim 64
+    assert lib.mg_mixed_attn(*args, 128, -1.0, 0, 0, 4096, 4096, 1 << 30, None) == 1          # scale
+    assert lib.mg_mixed_attn(*args, 128, 0.1, 0, -1, 4096, 4096, 1 << 30, None) == 1          # extend_ctas < 0
     no_tokens = [4096, 4096, 4096, 100, 4096, 5, 32, 4096, 4096, 4096, 4096, 4, 0, 0, 32, 16, 8]
-    assert lib.mg_mixed_attn(*no_tokens, 128, 0.1, 0, 4096, None, 0, None) == 0            # nothing to do
-    assert lib.mg_mixed_attn(*args, 128, 0.1, 1000, 4096, 4096, 16, None) == 4             # workspace too small
+    assert lib.mg_mixed_attn(*no_tokens, 128, 0.1, 0, 0, 4096, None, 0, None) == 0            # nothing to do
+    assert lib.mg_mixed_attn(*args, 128, 0.1, 1000, 0, 4096, 4096, 16, None) == 4             # workspace too small
 
 
 def test_extend_rejects_shapes_and_empty_is_noop(lib):

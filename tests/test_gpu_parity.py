@@ -498,15 +498,18 @@ MIXED_SMALL = [
 
 
 @pytest.mark.parametrize("cached,seq", MIXED_SMALL)
-@pytest.mark.parametrize("parts", [0, 7])
-def test_mixed_attn_matches_oracle(cached, seq, parts):
+@pytest.mark.parametrize("parts,ectas", [(0, 0), (7, 0), (0, 20), (7, 1), (0, 400)])
+def test_mixed_attn_matches_oracle(cached, seq, parts, ectas):
+    """Both halves one after the other (extend_ctas 0) and side by side on
+    split SMs (a few, one, more than the GPU has)."""
     step, data = _custom("extend", cached, seq, 16, 8, seed=sum(seq) + parts)
     g = GpuStep(step, data)
     g.store()
     out = mg.mixed_attn(g.q, g.k_cache, g.v_cache, g.page_table, g.table_idx, g.cached_len, g.seq_len, g.q_offset,
-                        max(step.max_q_len, 1), step.max_seq_len, g.scale, num_partitions=parts)
+                        max(step.max_q_len, 1), step.max_seq_len, g.scale, num_partitions=parts, extend_ctas=ectas)
+    torch.cuda.synchronize()
     assert mg.read_device_error() == 0
-    assert_matches_oracle(out, oracle_extend(step, data), f"mixed {cached}->{seq} partitions {parts}")
+    assert_matches_oracle(out, oracle_extend(step, data), f"mixed {cached}->{seq} partitions {parts} ectas {ectas}")
 
 
 def test_mixed_attn_on_the_mixed_workload():
@@ -525,6 +528,22 @@ def test_mixed_attn_on_the_mixed_workload():
     assert_matches_oracle(out, oracle_extend(step, data, requests=req), "mixed_attn, mixed_prefill_decode")
     ext = g.extend().float()
     assert bool(((out.float() - ext).abs() <= ext.abs() * 2.0 ** -7 + 2e-3).all())
+    # the same call with the two kernels side by side on split SMs, at the split
+    # the bench times: the same rows as the sequential call, bit for bit (each
+    # row is computed by the same kernel either way)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    ectas = mg.mixed_extend_ctas(step.cached_len.tolist(), step.seq_len.tolist(), spec.num_q_heads,
+                                 spec.num_kv_heads, sms)
+    assert 0 < ectas < sms
+    split = mg.mixed_attn(g.q, g.k_cache, g.v_cache, g.page_table, g.table_idx, g.cached_len, g.seq_len,
+                          g.q_offset, step.max_q_len, step.max_seq_len, g.scale, extend_ctas=ectas)
+    torch.cuda.synchronize()
+    assert mg.read_device_error() == 0
+    ext_rows = torch.zeros(out.shape[0], dtype=torch.bool)
+    for r in range(4):
+        ext_rows[int(step.q_offset[r]):int(step.q_offset[r + 1])] = True
+    assert torch.equal(split[ext_rows.cuda()], out[ext_rows.cuda()])
+    assert_matches_oracle(split, oracle_extend(step, data, requests=req), "mixed_attn split, mixed_prefill_decode")
 
 
 # --------------------------------------------------------------------------- shared prefix
