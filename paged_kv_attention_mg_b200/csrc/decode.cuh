@@ -377,15 +377,18 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
     // layer's merge) and overlaps that kernel's tail.
     unsigned bad = 0;
     int64_t running = 0;
+    int64_t u1[4], excl1 = 0;  // the first chunk's units and prefix, reused by pass 2 when it is the only one
     for (int ch = 0; ch < nchunks; ++ch) {
         int64_t v = 0;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int r = ch * kScanChunk + tid * 4 + i;
-            if (r < p.num_vreqs) v += units_of<CASCADE>(p, r, bad);
+            u1[i] = r < p.num_vreqs ? units_of<CASCADE>(p, r, bad) : 0;
+            v += u1[i];
         }
         int64_t excl;
         const int64_t tot = block_scan_excl(v, excl, sh_scan);
+        if (ch == 0) excl1 = excl;
         if (tid == 0) sh_chunk_excl[ch] = running;
         running += tot;
     }
@@ -410,14 +413,20 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
             if (!needed) continue;  // uniform across the CTA
             int64_t u[4], v = 0;
             const int r0 = ch * kScanChunk + tid * 4;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                unsigned dummy = 0;
-                u[i] = r0 + i < p.num_vreqs ? units_of<CASCADE>(p, r0 + i, dummy) : 0;
-                v += u[i];
-            }
             int64_t excl;
-            block_scan_excl(v, excl, sh_scan);
+            if (nchunks == 1) {  // (uniform) pass 1 scanned this chunk already
+#pragma unroll
+                for (int i = 0; i < 4; ++i) u[i] = u1[i];
+                excl = excl1;
+            } else {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    unsigned dummy = 0;
+                    u[i] = r0 + i < p.num_vreqs ? units_of<CASCADE>(p, r0 + i, dummy) : 0;
+                    v += u[i];
+                }
+                block_scan_excl(v, excl, sh_scan);
+            }
             int64_t pre = lo + excl;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
