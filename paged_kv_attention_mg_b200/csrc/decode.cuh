@@ -199,16 +199,39 @@ __device__ __forceinline__ int group_of(const Params &p, int r) {
     return (__ldg(p.group_first + lo) <= r && r < __ldg(p.group_first + lo + 1)) ? lo : -1;
 }
 
-// Units of virtual request v (cascade mode), and its description.
-__device__ __forceinline__ int64_t vreq_units(const Params &p, int v, VReq &vr, unsigned &bad) {
+// Every group's member range and checked prefix length (0 when it has none
+// or is malformed), copied to shared memory once per CTA when there are at
+// most kGroupCache groups, so that a virtual request's description costs one
+// round of metadata loads instead of a chain of them.
+constexpr int kGroupCache = kThreads;
+struct GroupCache {
+    int first[kGroupCache + 1];
+    int prefix[kGroupCache];
+};
+
+// group_of over the cached group_first
+__device__ __forceinline__ int group_of_cached(const GroupCache &gc, int num_groups, int r) {
+    if (num_groups <= 0) return -1;
+    int lo = 0, hi = num_groups - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (gc.first[mid] <= r) lo = mid; else hi = mid - 1;
+    }
+    return (gc.first[lo] <= r && r < gc.first[lo + 1]) ? lo : -1;
+}
+
+// Units of virtual request v (cascade mode), and its description; gc, when
+// given, holds the groups' ranges and prefixes.
+__device__ __forceinline__ int64_t vreq_units(const Params &p, int v, VReq &vr, unsigned &bad,
+                                              const GroupCache *gc = nullptr) {
     vr.m = 1;
     vr.grouped = false;
     vr.k0 = 0;
     if (v < p.num_groups) {
-        const int P = group_prefix(p, v, bad);
+        const int P = gc ? gc->prefix[v] : group_prefix(p, v, bad);
         if (P == 0) { vr.k1 = 0; return 0; }
-        vr.r0 = __ldg(p.group_first + v);
-        vr.m = __ldg(p.group_first + v + 1) - vr.r0;
+        vr.r0 = gc ? gc->first[v] : __ldg(p.group_first + v);
+        vr.m = (gc ? gc->first[v + 1] : __ldg(p.group_first + v + 1)) - vr.r0;
         vr.row = __ldg(p.table_idx + vr.r0);
         vr.k1 = P;
         return (int64_t)((P + kKeys - 1) / kKeys) * p.num_kv_heads;
@@ -219,10 +242,10 @@ __device__ __forceinline__ int64_t vreq_units(const Params &p, int v, VReq &vr, 
     vr.r0 = r;
     vr.k1 = L;
     if (u == 0) return 0;
-    const int grp = group_of(p, r);
+    const int grp = gc ? group_of_cached(*gc, p.num_groups, r) : group_of(p, r);
     if (grp >= 0) {
         unsigned ignore = 0;  // flagged where the group's own virtual request is resolved
-        const int P = group_prefix(p, grp, ignore);
+        const int P = gc ? gc->prefix[grp] : group_prefix(p, grp, ignore);
         if (P > 0) {
             vr.k0 = P;
             vr.grouped = true;
@@ -292,13 +315,13 @@ __device__ __forceinline__ void cursor_prefetch_next(const Params &p, Cursor &c)
 
 // Position the cursor on the first request >= c.r that owns units.
 template <bool CASCADE>
-__device__ __forceinline__ void cursor_load_request(const Params &p, Cursor &c) {
+__device__ __forceinline__ void cursor_load_request(const Params &p, Cursor &c, const GroupCache *gc = nullptr) {
     for (;;) {
         unsigned bad = 0;
         int64_t u;
         if constexpr (CASCADE) {
             VReq vr;
-            u = vreq_units(p, c.r, vr, bad);
+            u = vreq_units(p, c.r, vr, bad, gc);
             c.row = vr.row; c.L = vr.k1; c.k0 = vr.k0; c.r0 = vr.r0; c.m = vr.m; c.grouped = vr.grouped;
         } else {
             u = request_units(p, c.r, c.L, c.row, bad);
@@ -315,7 +338,7 @@ __device__ __forceinline__ void cursor_load_request(const Params &p, Cursor &c) 
 }
 
 template <bool CASCADE>
-__device__ __forceinline__ void cursor_advance(const Params &p, Cursor &c) {
+__device__ __forceinline__ void cursor_advance(const Params &p, Cursor &c, const GroupCache *gc = nullptr) {
     if (++c.t < c.tiles) return;
     c.t = 0;
     if (++c.kvh < p.num_kv_heads) return;
@@ -323,7 +346,7 @@ __device__ __forceinline__ void cursor_advance(const Params &p, Cursor &c) {
     ++c.r;
     if (c.r >= p.num_vreqs) return;
     if constexpr (CASCADE) {
-        cursor_load_request<true>(p, c);
+        cursor_load_request<true>(p, c, gc);
         return;
     }
     if (!p.row_map && metadata_ok(p, c.next_L, c.next_row)) {  // the common case: no stall at the boundary
@@ -338,10 +361,10 @@ __device__ __forceinline__ void cursor_advance(const Params &p, Cursor &c) {
 
 // Units of virtual request v (a request, outside cascade mode).
 template <bool CASCADE>
-__device__ __forceinline__ int64_t units_of(const Params &p, int v, unsigned &bad) {
+__device__ __forceinline__ int64_t units_of(const Params &p, int v, unsigned &bad, const GroupCache *gc = nullptr) {
     if constexpr (CASCADE) {
         VReq vr;
-        return vreq_units(p, v, vr, bad);
+        return vreq_units(p, v, vr, bad, gc);
     } else {
         int L, row;
         return request_units(p, v, L, row, bad);
@@ -376,6 +399,19 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
     // the wait on the previous kernel (e.g. the KV store, or the previous
     // layer's merge) and overlaps that kernel's tail.
     unsigned bad = 0;
+    // shared-prefix mode: the groups' ranges and prefixes, checked once
+    __shared__ GroupCache sh_gc;
+    const GroupCache *gc = nullptr;
+    if constexpr (CASCADE) {
+        if (p.num_groups <= kGroupCache) {  // uniform
+            for (int gi = tid; gi <= p.num_groups; gi += kThreads) {
+                sh_gc.first[gi] = __ldg(p.group_first + gi);
+                if (gi < p.num_groups) sh_gc.prefix[gi] = group_prefix(p, gi, bad);
+            }
+            __syncthreads();
+            gc = &sh_gc;
+        }
+    }
     int64_t running = 0;
     int64_t u1[4], excl1 = 0;  // the first chunk's units and prefix, reused by pass 2 when it is the only one
     for (int ch = 0; ch < nchunks; ++ch) {
@@ -383,7 +419,7 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int r = ch * kScanChunk + tid * 4 + i;
-            u1[i] = r < p.num_vreqs ? units_of<CASCADE>(p, r, bad) : 0;
+            u1[i] = r < p.num_vreqs ? units_of<CASCADE>(p, r, bad, gc) : 0;
             v += u1[i];
         }
         int64_t excl;
@@ -422,7 +458,7 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     unsigned dummy = 0;
-                    u[i] = r0 + i < p.num_vreqs ? units_of<CASCADE>(p, r0 + i, dummy) : 0;
+                    u[i] = r0 + i < p.num_vreqs ? units_of<CASCADE>(p, r0 + i, dummy, gc) : 0;
                     v += u[i];
                 }
                 block_scan_excl(v, excl, sh_scan);
@@ -465,7 +501,7 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
 
     Cursor cur;  // position of the next tile whose page-table entries are fetched
     cur.r = sh_start_r[warp];
-    cursor_load_request<CASCADE>(p, cur);
+    cursor_load_request<CASCADE>(p, cur, gc);
     {
         const int64_t off = ub - sh_start_prefix[warp];
         cur.kvh = (int)(off / cur.tiles);
@@ -495,7 +531,7 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
                 else
                     my_idx[e][lane] = -1;
             }
-            cursor_advance<CASCADE>(p, cur);
+            cursor_advance<CASCADE>(p, cur, gc);
         }
     };
     // this lane's shared-memory offsets within a stage for its 16 copies of a
