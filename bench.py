@@ -445,8 +445,9 @@ class ExtendBench:
             sms = torch.cuda.get_device_properties(device).multi_processor_count
             self.extend_ctas = (mg.mixed_extend_ctas(c, s, spec.num_q_heads, spec.num_kv_heads, sms)
                                 if extend_ctas < 0 else extend_ctas)
-            if self.extend_ctas > 0:  # the decode kernel's workers: 7 a CTA on the SMs left to it
-                w = 7 * (sms - min(self.extend_ctas, sms - 1))
+            if self.extend_ctas > 0:  # the decode kernel's workers on the SMs left to it
+                per_sm = mg.decode_plan(step.batch, spec.num_kv_heads, step.max_seq_len, 0)[0] // sms
+                w = per_sm * (sms - min(self.extend_ctas, sms - 1))
                 self.workers, _ = mg.decode_plan(step.batch, spec.num_kv_heads, step.max_seq_len,
                                                  partitions if 0 < partitions < w else w)
         self.partitions = partitions

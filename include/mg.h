@@ -134,8 +134,8 @@ mg_status mg_store_kv(const void *k, const void *v, const int32_t *out_loc, int3
  * units of 16 keys of one (request, kv head) pair; `workers` warps share the
  * units equally and in order, so a pair may be split across workers, whose
  * partial results a merge kernel combines.  num_partitions == 0 picks one
- * worker per warp of the decode grid on the current device (SMs x 7 warps,
- * one CTA per SM); > 0 forces that many workers.
+ * worker per warp of the decode grid on the current device (SMs x 2 CTAs x
+ * 4 warps); > 0 forces that many workers.
  * slots_out = batch * num_kv_heads + workers partial slots.
  * The plan depends only on these arguments (never on the lengths), so a
  * captured launch stays valid for any batch with lengths <= max_seq_len.
@@ -289,7 +289,7 @@ mg_status mg_extend_attn(const void *q, const void *k_cache, const void *v_cache
  *   extend_ctas     0: the kernels run one after the other on `stream`.  > 0:
  *                   the extend kernel runs on that many SMs at the same time
  *                   as the decode kernel runs on the rest (capped at the SM
- *                   count - 1; the decode plan then has 7 workers per
+ *                   count - 1; the decode plan then has 8 workers per
  *                   remaining SM, or num_partitions if fewer): the decode
  *                   kernel is bound by HBM and the extend kernel by its
  *                   softmax and tensor cores, so they overlap.  The extend

@@ -55,7 +55,7 @@ namespace decode {
 
 constexpr int kKeys = 16;          // keys per unit / pipeline tile
 #ifndef MG_DECODE_WARPS
-#define MG_DECODE_WARPS 7  // workers per CTA (build-time tunable)
+#define MG_DECODE_WARPS 4  // workers per CTA (build-time tunable)
 #endif
 constexpr int kWarps = MG_DECODE_WARPS;
 constexpr int kThreads = kWarps * 32;
@@ -68,7 +68,7 @@ constexpr int kMaxBatch = 131072;                  // requests per call
 #define MG_DECODE_STAGES 3  // per-worker ring depth (build-time tunable)
 #endif
 #ifndef MG_DECODE_MIN_BLOCKS
-#define MG_DECODE_MIN_BLOCKS 1  // resident CTAs per SM (the shared memory is sized for it)
+#define MG_DECODE_MIN_BLOCKS 2  // resident CTAs per SM (the shared memory is sized for it)
 #endif
 #ifndef MG_DECODE_SPLIT_P
 // 1: P enters the PV product as bf16 hi + lo parts (two products), so the

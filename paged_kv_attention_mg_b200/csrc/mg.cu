@@ -494,7 +494,7 @@ mg_status mg_mixed_attn(const void *q, const void *k_cache, const void *v_cache,
         // kernel is bound by HBM, the extend kernel by its softmax and tensor
         // cores, so the two overlap instead of following each other).
         const int e = extend_ctas < sms ? extend_ctas : sms - 1;
-        int32_t workers = decode::kWarps * (sms - e);
+        int32_t workers = MG_DECODE_MIN_BLOCKS * decode::kWarps * (sms - e);
         if (num_partitions > 0 && num_partitions < workers) workers = num_partitions;
         // every host check of both halves before anything is enqueued
         if (!cached_len) return MG_ERR_INVALID_ARGUMENT;
