@@ -329,10 +329,10 @@ class DecodeBench:
         self.spec, self.step, self.device = spec, step, device
         self.layers = make_layers(step, spec.num_layers, device)
         # shared-prefix workloads: groups of requests read their common prefix once
-        # (mg_decode_attn_shared_prefix after a separate store: the fused store
-        # runs without groups)
+        # (mg_store_decode_attn_shared_prefix; --unfused: mg_store_kv, then
+        # mg_decode_attn_shared_prefix; --plain: the plain decode over the same tables)
         self.shared = step.group_first is not None and not plain
-        self.fused = fused and step.group_first is None
+        self.fused = fused
         names = ("page_table", "table_idx", "seq_len", "out_loc") + (("group_first", "prefix_len") if self.shared
                                                                       else ())
         self.meta = {n: getattr(step, n).to(device) for n in names}
@@ -367,6 +367,17 @@ class DecodeBench:
 
     def layer(self, lay, out, meta, events=None):
         mg = self.mg
+        if self.shared and self.fused:
+            if events:
+                events[0].record()
+            mg.store_decode_attn_shared_prefix(lay["q"], lay["k_new"], lay["v_new"], meta["out_loc"],
+                                               lay["k_cache"], lay["v_cache"], meta["page_table"],
+                                               meta["table_idx"], meta["seq_len"], meta["group_first"],
+                                               meta["prefix_len"], self.max_seq_len, self.spec.scale,
+                                               num_partitions=self.partitions, out=out, workspace=self.workspace)
+            if events:
+                events[1].record()
+            return
         if self.shared:
             mg.store_kv(lay["k_new"], lay["v_new"], meta["out_loc"], lay["k_cache"], lay["v_cache"])
             if events:
@@ -800,9 +811,11 @@ def run_ours(args):
         unit = "GB/s"
         metric = METRIC
         achieved = achieved_min
-        kname = ("decode_kernel<fused store> + decode_merge_kernel (one mg_store_decode_attn call)" if bench.fused
+        kname = ("decode_kernel<shared prefix, fused store> + decode_merge_kernel (one "
+                 "mg_store_decode_attn_shared_prefix call)" if bench.shared and bench.fused
                  else "store_kv_kernel + decode_kernel<shared prefix> + decode_merge_kernel (mg_store_kv + "
                       "mg_decode_attn_shared_prefix)" if bench.shared
+                 else "decode_kernel<fused store> + decode_merge_kernel (one mg_store_decode_attn call)" if bench.fused
                  else "store_kv_kernel + decode_kernel + decode_merge_kernel (mg_store_kv + mg_decode_attn)")
         roof = {"bound": "hbm", "kernel": kname,
                 "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s", "frac": round(achieved / hbm, 4),

@@ -12,6 +12,7 @@
  *                   (balanced split-KV kernel + merge kernel);
  *   mg_store_decode_attn  the two above fused into one decode launch;
  *   mg_decode_attn_shared_prefix  decode reading a shared prefix once per group;
+ *   mg_store_decode_attn_shared_prefix  the store fused into that decode;
  *   mg_mixed_attn   extend semantics for mixed batches: one-token requests by
  *                   the decode kernel, prompt chunks by the extend kernel;
  *   mg_extend_attn  a chunk of new tokens per request (chunked prefill),
@@ -245,6 +246,27 @@ mg_status mg_decode_attn_shared_prefix(const void *q, const void *k_cache, const
                                        int32_t num_groups, int32_t num_q_heads, int32_t num_kv_heads,
                                        int32_t head_dim, float scale, int32_t num_partitions, void *out,
                                        void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * mg_store_decode_attn_shared_prefix -- mg_store_kv of the step's new tokens
+ * followed by mg_decode_attn_shared_prefix, in one launch of the decode kernel
+ * (plus the merge kernel), as mg_store_decode_attn does for mg_decode_attn.
+ * k_new, v_new and out_loc are mg_store_decode_attn's; every other argument
+ * and the output are mg_decode_attn_shared_prefix's.  A request's new token
+ * (position seq_len-1) lies after its group's prefix, so it is always read
+ * and stored by the worker that owns the last tile of the request's own keys.
+ * The same checks of out_loc set the same error bits.
+ */
+mg_status mg_store_decode_attn_shared_prefix(const void *q, const void *k_new, const void *v_new,
+                                             const int32_t *out_loc, void *k_cache, void *v_cache,
+                                             int64_t num_slots, const int32_t *page_table,
+                                             int32_t page_table_rows, int32_t page_table_stride,
+                                             const int32_t *table_idx, const int32_t *seq_len, int32_t batch,
+                                             int32_t max_seq_len, const int32_t *group_first,
+                                             const int32_t *prefix_len, int32_t num_groups,
+                                             int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                             float scale, int32_t num_partitions, void *out, void *workspace,
+                                             size_t workspace_bytes, void *stream);
 
 /*
  * mg_extend_attn -- chunked-prefill ("extend") attention over the paged pool

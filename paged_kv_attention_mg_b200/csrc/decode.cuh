@@ -377,7 +377,6 @@ __device__ __forceinline__ int64_t units_of(const Params &p, int v, unsigned &ba
 template <int NT, bool FUSED, bool CASCADE = false>
 __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
     decode_kernel(const Params p) {
-    static_assert(!(FUSED && CASCADE), "the fused store runs without shared prefixes");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     __shared__ __align__(16) int idx_ring[kWarps][kDescRing][kKeys];
@@ -521,8 +520,10 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
                 d.valid = 0; d.store_slot = -1;
                 if constexpr (CASCADE) { d.k0 = cur.k0; d.r0 = cur.r0; d.m = cur.m; d.grouped = cur.grouped; }
                 my_desc[e] = d;
-                if (FUSED && cur.t == cur.tiles - 1)  // the pair's last tile holds the new token
-                    cp_async_4(smem_u32(&my_desc[e].store_slot), p.out_loc + cur.r);
+                // the pair's last tile holds the new token (in shared-prefix mode: of
+                // a request's own keys; a group's prefix holds none)
+                if (FUSED && cur.t == cur.tiles - 1 && (!CASCADE || cur.r >= p.num_groups))
+                    cp_async_4(smem_u32(&my_desc[e].store_slot), p.out_loc + (CASCADE ? cur.r0 : cur.r));
             }
             const int key = cur.k0 + cur.t * kKeys + lane;
             if (lane < kKeys) {
@@ -565,7 +566,9 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
         // writes it even when that entry was rejected (the key is then masked
         // out of the attention, as any rejected key is): its copy is given a
         // non-negative stand-in slot here, once, rather than a test per row below
-        const int new_key = (FUSED && d.t == d.tiles - 1) ? d.L - 1 - (CASCADE ? d.k0 : 0) - d.t * kKeys : -1;
+        const int new_key = (FUSED && d.t == d.tiles - 1 && (!CASCADE || d.r >= p.num_groups))
+                                ? d.L - 1 - (CASCADE ? d.k0 : 0) - d.t * kKeys
+                                : -1;
         if (FUSED && lane == new_key && slot < 0) slot = 0;
         // 16-byte cp.async: each warp instruction moves two whole 256-byte rows
         // (lanes 0-15 and 16-31); 32 rows per tile (16 K then 16 V)
@@ -575,7 +578,7 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
         const char *kb = reinterpret_cast<const char *>(p.k_cache) + head_off;
         const char *vb = reinterpret_cast<const char *>(p.v_cache) + head_off;
         if (FUSED && new_key >= 0) {  // the pair's last tile, which holds the new token
-            const int64_t new_off = ((int64_t)d.r * p.num_kv_heads + d.kvh) * kHeadDim + ch * 8;
+            const int64_t new_off = ((int64_t)(CASCADE ? d.r0 : d.r) * p.num_kv_heads + d.kvh) * kHeadDim + ch * 8;
 #pragma unroll
             for (int it = 0; it < 16; ++it) {
                 const int key = (it * 2 + (lane >> 4)) & (kKeys - 1);
@@ -790,10 +793,10 @@ __global__ void __launch_bounds__(kThreads, MG_DECODE_MIN_BLOCKS)
                     }
                 }
             }
-            if (FUSED && c.t == c.tiles - 1) {
+            if (FUSED && c.t == c.tiles - 1 && (!CASCADE || c.r >= p.num_groups)) {
                 // fused store: lanes 0-15 copy the new token's K row, lanes 16-31 its V row,
                 // 16 bytes each, from the landed stage into pool slot out_loc[r]
-                const int nk = c.L - 1 - c.t * kKeys;
+                const int nk = c.L - 1 - (CASCADE ? c.k0 : 0) - c.t * kKeys;
                 const int ss = c.store_slot;
                 const int pt_slot = my_idx[k % kDescRing][nk];
                 if (ss < 0 || (int64_t)ss >= p.num_slots) {

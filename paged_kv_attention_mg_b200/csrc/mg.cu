@@ -125,6 +125,8 @@ mg_status ensure_kernel_attributes() {
         cudaFuncSetAttribute(decode::decode_kernel<2, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              decode::kSmemBytes) != cudaSuccess ||
         cudaFuncSetAttribute(decode::decode_kernel<2, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             decode::kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(decode::decode_kernel<2, true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              decode::kSmemBytes) != cudaSuccess)
         return MG_ERR_CUDA;
     if (extend::set_attributes() != cudaSuccess) return MG_ERR_CUDA;
@@ -200,7 +202,7 @@ mg_status decode_impl(const void *q, const void *k_new, const void *v_new, const
                       int32_t total_rows = 0, bool check_only = false) {
     const bool fused = k_new != nullptr;
     const bool cascade = group_first != nullptr;
-    if (cascade && (fused || !prefix_len || num_groups <= 0)) return MG_ERR_INVALID_ARGUMENT;
+    if (cascade && (!prefix_len || num_groups <= 0)) return MG_ERR_INVALID_ARGUMENT;
     if (cascade && (int64_t)batch + num_groups > decode::kMaxBatch) return MG_ERR_UNSUPPORTED_SHAPE;
     mg_status st = check_attention_shape(num_q_heads, num_kv_heads, head_dim);
     if (st != MG_OK) return st;
@@ -267,7 +269,8 @@ mg_status decode_impl(const void *q, const void *k_new, const void *v_new, const
     const dim3 grid(ctas), block(decode::kThreads);
     const size_t smem = decode::kSmemBytes;
     if (cascade)
-        st = launch_pdl(decode::decode_kernel<2, false, true>, grid, block, smem, s, p);
+        st = fused ? launch_pdl(decode::decode_kernel<2, true, true>, grid, block, smem, s, p)
+                   : launch_pdl(decode::decode_kernel<2, false, true>, grid, block, smem, s, p);
     else if (p.group <= 8)
         st = fused ? launch_pdl(decode::decode_kernel<1, true>, grid, block, smem, s, p)
                    : launch_pdl(decode::decode_kernel<1, false>, grid, block, smem, s, p);
@@ -447,6 +450,23 @@ mg_status mg_decode_attn_shared_prefix(const void *q, const void *k_cache, const
                                        void *workspace, size_t workspace_bytes, void *stream) {
     if (!group_first || !prefix_len || num_groups <= 0) return MG_ERR_INVALID_ARGUMENT;
     return decode_impl(q, nullptr, nullptr, nullptr, k_cache, v_cache, num_slots, page_table, page_table_rows,
+                       page_table_stride, table_idx, seq_len, batch, max_seq_len, num_q_heads, num_kv_heads,
+                       head_dim, scale, num_partitions, out, workspace, workspace_bytes, stream, group_first,
+                       prefix_len, num_groups);
+}
+
+mg_status mg_store_decode_attn_shared_prefix(const void *q, const void *k_new, const void *v_new,
+                                             const int32_t *out_loc, void *k_cache, void *v_cache,
+                                             int64_t num_slots, const int32_t *page_table,
+                                             int32_t page_table_rows, int32_t page_table_stride,
+                                             const int32_t *table_idx, const int32_t *seq_len, int32_t batch,
+                                             int32_t max_seq_len, const int32_t *group_first,
+                                             const int32_t *prefix_len, int32_t num_groups,
+                                             int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                             float scale, int32_t num_partitions, void *out, void *workspace,
+                                             size_t workspace_bytes, void *stream) {
+    if (!k_new || !group_first || !prefix_len || num_groups <= 0) return MG_ERR_INVALID_ARGUMENT;
+    return decode_impl(q, k_new, v_new, out_loc, k_cache, v_cache, num_slots, page_table, page_table_rows,
                        page_table_stride, table_idx, seq_len, batch, max_seq_len, num_q_heads, num_kv_heads,
                        head_dim, scale, num_partitions, out, workspace, workspace_bytes, stream, group_first,
                        prefix_len, num_groups);

@@ -48,6 +48,9 @@ SIGNATURES = {
     "mg_decode_shared_prefix_workspace_bytes": (_SZ, [_I32, _I32, _I32, _I32, _I32, _I32, _I32]),
     "mg_decode_attn_shared_prefix": (ctypes.c_int, [_P, _P, _P, _I64, _P, _I32, _I32, _P, _P, _I32, _I32, _P, _P,
                                                     _I32, _I32, _I32, _I32, _F32, _I32, _P, _P, _SZ, _P]),
+    "mg_store_decode_attn_shared_prefix": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _P, _I32, _I32, _P, _P,
+                                                          _I32, _I32, _P, _P, _I32, _I32, _I32, _I32, _F32, _I32,
+                                                          _P, _P, _SZ, _P]),
     "mg_extend_attn": (ctypes.c_int, [_P, _P, _P, _I64, _P, _I32, _I32, _P, _P, _P, _P, _I32, _I32, _I32,
                                       _I32, _I32, _I32, _I32, _F32, _P, _P]),
     "mg_mixed_workspace_bytes": (_SZ, [_I32, _I32, _I32, _I32, _I32, _I32]),
@@ -271,6 +274,43 @@ def decode_attn_shared_prefix(q: torch.Tensor, k_cache: torch.Tensor, v_cache: t
     return out
 
 
+def store_decode_attn_shared_prefix(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
+                                    out_loc: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                                    page_table: torch.Tensor, table_idx: torch.Tensor, seq_len: torch.Tensor,
+                                    group_first: torch.Tensor, prefix_len: torch.Tensor, max_seq_len: int,
+                                    scale: float, num_partitions: int = 0, out: Optional[torch.Tensor] = None,
+                                    workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """store_kv(k_new, v_new, out_loc) then decode_attn_shared_prefix, fused
+    into one decode launch."""
+    b = q.shape[0] if isinstance(q, torch.Tensor) and q.dim() == 3 else -1
+    if not isinstance(prefix_len, torch.Tensor) or prefix_len.dim() != 1:
+        raise ValueError("store_decode_attn_shared_prefix: prefix_len must be [num_groups]")
+    ng = prefix_len.shape[0]
+    _attention_shapes("store_decode_attn_shared_prefix", q, k_cache, v_cache, page_table, out,
+                      {"table_idx": (table_idx, (b,)), "seq_len": (seq_len, (b,)),
+                       "group_first": (group_first, (ng + 1,))})
+    b, hq, d = q.shape
+    hkv = k_cache.shape[1]
+    if k_new.shape != (b, hkv, d) or v_new.shape != k_new.shape or out_loc.shape != (b,):
+        raise ValueError("store_decode_attn_shared_prefix: one new token per request expected")
+    if out is None:
+        out = torch.empty_like(q)
+    need = decode_shared_prefix_workspace_bytes(b, ng, hq, hkv, max_seq_len, num_partitions, d)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = _dev(workspace, torch.uint8, "workspace") if workspace is not None else None
+    ws_bytes = workspace.numel() if workspace is not None else 0
+    _check(load().mg_store_decode_attn_shared_prefix(
+        _dev(q, torch.bfloat16, "q"), _dev(k_new, torch.bfloat16, "k_new"), _dev(v_new, torch.bfloat16, "v_new"),
+        _dev(out_loc, torch.int32, "out_loc"), _dev(k_cache, torch.bfloat16, "k_cache"),
+        _dev(v_cache, torch.bfloat16, "v_cache"), k_cache.shape[0], _dev(page_table, torch.int32, "page_table"),
+        page_table.shape[0], page_table.shape[1], _dev(table_idx, torch.int32, "table_idx"),
+        _dev(seq_len, torch.int32, "seq_len"), b, max_seq_len, _dev(group_first, torch.int32, "group_first"),
+        _dev(prefix_len, torch.int32, "prefix_len"), ng, hq, hkv, d, float(scale), num_partitions,
+        _dev(out, torch.bfloat16, "out"), ws_ptr, ws_bytes, _stream(stream)), "mg_store_decode_attn_shared_prefix")
+    return out
+
+
 def extend_attn(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, page_table: torch.Tensor,
                 table_idx: torch.Tensor, cached_len: torch.Tensor, seq_len: torch.Tensor,
                 q_offset: torch.Tensor, max_q_len: int, max_seq_len: int, scale: float,
@@ -338,12 +378,13 @@ def mixed_attn(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, pa
     return out
 
 
-# Per-SM rates the split estimate works with, measured on B200 with this
-# library's kernels: a 128-key tile of an extend item (two Q tiles, causal
-# edge tiles counted whole) every ~3.6 us per SM, and ~39 GB/s of K/V per SM
-# for the decode kernel (5.8 TB/s over 148 SMs).
+# Rates the split estimate works with, measured on B200 with this library's
+# kernels: a 128-key tile of an extend item (two Q tiles, causal edge tiles
+# counted whole) every ~3.6 us per SM; the decode kernel's K/V stream at up to
+# ~52 GB/s per SM and ~5.6 TB/s in all (HBM).
 _EXTEND_TILE_S = 3.6e-6
-_DECODE_SM_BYTES_PER_S = 39e9
+_DECODE_SM_BYTES_PER_S = 52e9
+_DECODE_HBM_BYTES_PER_S = 5.6e12
 
 
 def mixed_extend_ctas(cached_len, seq_len, num_q_heads: int, num_kv_heads: int, sms: int,
@@ -351,8 +392,9 @@ def mixed_extend_ctas(cached_len, seq_len, num_q_heads: int, num_kv_heads: int, 
     """How many SMs mg_mixed_attn should give the extend kernel so that it and
     the decode kernel finish together, from the batch's host-side lengths (the
     scheduler that formed the batch has them): the extend items' KV tiles
-    against the one-token requests' K/V bytes, at the per-SM rates above.
-    0 when the batch has no prompt chunk or no one-token request."""
+    against the one-token requests' K/V bytes at the rates above; the split
+    whose later kernel ends first.  0 when the batch has no prompt chunk or no
+    one-token request."""
     g = num_q_heads // num_kv_heads
     span = 2 * (128 // g)  # tokens of a q block
     tiles, dec_bytes = 0, 0
@@ -366,9 +408,12 @@ def mixed_extend_ctas(cached_len, seq_len, num_q_heads: int, num_kv_heads: int, 
                 tiles += -(-(c + min(t0 + span, n)) // 128) * num_kv_heads
     if tiles == 0 or dec_bytes == 0:
         return 0
-    ext_s = tiles * _EXTEND_TILE_S
-    dec_s = dec_bytes / _DECODE_SM_BYTES_PER_S
-    return max(1, min(sms - 1, round(sms * ext_s / (ext_s + dec_s))))
+
+    def finish(e):  # when the later of the two kernels ends with e SMs for extend
+        ext = tiles * _EXTEND_TILE_S / e
+        dec = dec_bytes / min(_DECODE_HBM_BYTES_PER_S, (sms - e) * _DECODE_SM_BYTES_PER_S)
+        return max(ext, dec)
+    return min(range(1, sms), key=finish)
 
 
 STATIC_WORKSPACE_BYTES = 16 << 20  # MG_DECODE_STATIC_WORKSPACE_BYTES in include/mg.h

@@ -1,4 +1,5 @@
-"""GPU: decode over shared prefixes read once per group (mg_decode_attn_shared_prefix).
+"""GPU: decode over shared prefixes read once per group (mg_decode_attn_shared_prefix,
+and mg_store_decode_attn_shared_prefix with the KV store fused in).
 
 Requests that share the beginning of their history, as a radix prefix cache
 hands it out ("Mini-SGLang" tag page, KV Cache post), have page-table rows that
@@ -13,7 +14,7 @@ import numpy as np
 import pytest
 import torch
 
-from mg_testlib import GpuStep, assert_matches_oracle, oracle_decode
+from mg_testlib import GpuStep, assert_matches_oracle, host_pools_after_store, oracle_decode
 from paged_kv_attention_mg_b200 import mg
 from paged_kv_attention_mg_b200 import workload as wl
 
@@ -126,6 +127,60 @@ def test_shared_prefix_workload_full_size():
     req = sorted({0, 1, 7, 8, 30, 63, int(np.argmax(step.seq_len.numpy()))})
     assert_matches_oracle(out, oracle_decode(step, data, requests=req), "shared_prefix_decode")
     assert torch.isfinite(out.float()).all()
+
+
+def _run_fused(g: GpuStep, step, parts=0, group_first=None, prefix_len=None):
+    gf = (step.group_first if group_first is None else group_first).cuda()
+    pl = (step.prefix_len if prefix_len is None else prefix_len).cuda()
+    return mg.store_decode_attn_shared_prefix(g.q, g.k_new, g.v_new, g.out_loc, g.k_cache, g.v_cache, g.page_table,
+                                              g.table_idx, g.seq_len, gf, pl, step.max_seq_len, g.scale,
+                                              num_partitions=parts)
+
+
+@pytest.mark.parametrize("parts", [0, 1, 37])
+def test_fused_store_shared_prefix_matches_oracle_and_stores(parts):
+    """The KV store fused into the shared-prefix decode: the result is the
+    oracle's over the pool after the store, and the pool afterwards is, bit
+    for bit, the one mg_store_kv leaves (the new tokens lie after every
+    group's prefix, in each request's own keys)."""
+    step, data = _grouped_case(LENGTHS, GROUPS, 32, 8, seed=615)
+    g = GpuStep(step, data)  # pools before the store
+    out = _run_fused(g, step, parts)
+    assert mg.read_device_error() == 0
+    assert_matches_oracle(out, oracle_decode(step, data), f"fused shared prefix, {parts} workers")
+    k_ref, v_ref = host_pools_after_store(step, data)
+    assert torch.equal(g.k_cache.cpu().view(torch.int16), k_ref.view(torch.int16))
+    assert torch.equal(g.v_cache.cpu().view(torch.int16), v_ref.view(torch.int16))
+
+
+def test_fused_store_shared_prefix_with_malformed_groups():
+    """A malformed group's members are served as plain requests; their new
+    tokens are stored all the same."""
+    step, data = _grouped_case(LENGTHS, GROUPS, 32, 8, seed=616)
+    g = GpuStep(step, data)
+    mg.read_device_error()
+    gf = torch.tensor([0, 5, 8, 12, 13, 14], dtype=torch.int32)  # five members of group 4: too many
+    pl = torch.tensor([1500, 1500, 1500, 0, 0], dtype=torch.int32)
+    out = _run_fused(g, step, group_first=gf, prefix_len=pl)
+    assert mg.read_device_error() & mg.DEVERR_LENGTH
+    assert_matches_oracle(out, oracle_decode(step, data), "fused, a group with too many members")
+    k_ref, v_ref = host_pools_after_store(step, data)
+    assert torch.equal(g.k_cache.cpu().view(torch.int16), k_ref.view(torch.int16))
+    assert torch.equal(g.v_cache.cpu().view(torch.int16), v_ref.view(torch.int16))
+
+
+def test_fused_store_shared_prefix_workload_full_size():
+    spec = wl.BY_NAME["shared_prefix_decode"]
+    step = wl.make_step(spec)
+    data = wl.make_layer(step)
+    g = GpuStep(step, data)
+    out = _run_fused(g, step)
+    assert mg.read_device_error() == 0
+    req = sorted({0, 1, 7, 8, 30, 63, int(np.argmax(step.seq_len.numpy()))})
+    assert_matches_oracle(out, oracle_decode(step, data, requests=req), "fused shared_prefix_decode")
+    loc = step.out_loc.long()
+    assert torch.equal(g.k_cache[loc.cuda()].cpu().view(torch.int16), data.k_new.view(torch.int16))
+    assert torch.equal(g.v_cache[loc.cuda()].cpu().view(torch.int16), data.v_new.view(torch.int16))
 
 
 def test_shared_prefix_host_errors():
