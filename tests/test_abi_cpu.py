@@ -120,6 +120,23 @@ def test_shared_prefix_workspace_and_host_validation(lib):
     assert lib.mg_decode_attn_shared_prefix(*args, 4096, 4096, 2, *small) == 4     # workspace too small
 
 
+def test_mixed_extend_ctas_split_estimate():
+    """mixed_extend_ctas (host logic, no device): no split without both kinds of
+    request, a split inside [1, sms - 1] otherwise, and more SMs for the extend
+    kernel as the prompt chunks grow against the same decode rows."""
+    dec_c, dec_s = [1000] * 50, [1001] * 50
+    assert mg.mixed_extend_ctas(dec_c, dec_s, 16, 8, 148) == 0                  # decode only
+    assert mg.mixed_extend_ctas([0, 100], [512, 900], 16, 8, 148) == 0          # chunks only
+    assert mg.mixed_extend_ctas([5], [5], 16, 8, 148) == 0                      # nothing new
+    prev = 0
+    for n in (64, 256, 1024, 4096, 16384):
+        e = mg.mixed_extend_ctas([0] + dec_c, [n] + dec_s, 16, 8, 148)
+        assert 1 <= e <= 147 and e >= prev
+        prev = e
+    assert prev > 74  # a chunk far heavier than the decode rows gets most of the SMs
+    assert mg.mixed_extend_ctas([0] + dec_c, [256] + dec_s, 16, 8, 2) == 1     # two SMs: one each
+
+
 def test_mixed_attn_host_validation(lib):
     assert lib.mg_mixed_workspace_bytes(8, 32, 4, 128, 32768, 1000) == lib.mg_decode_workspace_bytes(8, 32, 4, 128,
                                                                                                        32768, 1000)

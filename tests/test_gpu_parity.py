@@ -546,6 +546,46 @@ def test_mixed_attn_on_the_mixed_workload():
     assert_matches_oracle(split, oracle_extend(step, data, requests=req), "mixed_attn split, mixed_prefill_decode")
 
 
+def test_mixed_attn_split_under_graph_capture():
+    """The split call (extend kernel on a side stream forked and joined with
+    events) captured in a CUDA graph and replayed gives the eager call's
+    output bit for bit, on fresh inputs copied into the captured buffers."""
+    spec = wl.BY_NAME["mixed_prefill_decode"]
+    step = wl.make_step(spec)
+    data = wl.make_layer(step)
+    g = GpuStep(step, data)
+    g.store()
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    ectas = mg.mixed_extend_ctas(step.cached_len.tolist(), step.seq_len.tolist(), spec.num_q_heads,
+                                 spec.num_kv_heads, sms)
+    ws = torch.empty(mg.mixed_workspace_bytes(step.batch, spec.num_q_heads, spec.num_kv_heads, step.max_seq_len),
+                     dtype=torch.uint8, device="cuda")
+    out = torch.empty_like(g.q)
+
+    def call():
+        mg.mixed_attn(g.q, g.k_cache, g.v_cache, g.page_table, g.table_idx, g.cached_len, g.seq_len, g.q_offset,
+                      step.max_q_len, step.max_seq_len, g.scale, extend_ctas=ectas, out=out, workspace=ws)
+    call()  # eager, also creates the library's side stream before the capture
+    torch.cuda.synchronize()
+    q0 = g.q.clone()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        call()
+    q1 = torch.randn(g.q.shape, generator=torch.Generator().manual_seed(77)).to(torch.bfloat16).cuda()
+    for q in (q0, q1):
+        g.q.copy_(q)
+        out.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        replayed = out.clone()
+        out.zero_()
+        call()
+        torch.cuda.synchronize()
+        assert mg.read_device_error() == 0
+        assert torch.equal(replayed, out)
+    del graph
+
+
 # --------------------------------------------------------------------------- shared prefix
 
 def test_decode_and_extend_over_a_shared_prefix():
