@@ -15,7 +15,9 @@
 //     contiguous share of the units (floor(w T / W) .. floor((w+1) T / W)), so
 //     all workers finish together whatever the length mix (no tail of long
 //     splits).  A worker's share covers one or a few "segments" (its part of a
-//     pair).
+//     pair).  Two CTAs of 4 warps per SM by default, so each SM sub-partition
+//     holds two workers (with one 7-warp CTA the worker alone on its
+//     sub-partition ran ahead of the others and the call ended with the slowest).
 //   * two prefetch distances per worker: the page-table entries of tile
 //     k + IDX_AHEAD are copied (4-byte cp.async) into a per-warp index ring, and
 //     tile k + STAGES - 1 is gathered (16-byte cp.async, two 256-byte rows per
@@ -32,11 +34,14 @@
 //     one per group (the group's common prefix keys, its members' q rows
 //     stacked, up to 16 rows = two n-tiles), then one per request (its keys
 //     after the prefix); the merge combines a request's own partials with its
-//     group's.  Mixed-batch mode (row_map): only the one-token requests count
-//     units, each writing the output row q_offset[r].
-//   * fused store (mg_store_decode_attn): the new token (position L-1) is read
-//     from k_new / v_new instead of the pool, and the worker that owns that tile
-//     writes it to its pool slot from shared memory once the tile has landed.
+//     group's.  The groups' ranges and checked prefixes are copied into shared
+//     memory once per CTA.  Mixed-batch mode (row_map): only the one-token
+//     requests count units, each writing the output row q_offset[r].
+//   * fused store (mg_store_decode_attn, mg_store_decode_attn_shared_prefix):
+//     the new token (position L-1) is read from k_new / v_new instead of the
+//     pool, and the worker that owns that tile (in shared-prefix mode, the last
+//     tile of the request's own keys) writes it to its pool slot from shared
+//     memory once the tile has landed.
 //   * a segment that is a whole pair writes bf16 output directly; otherwise it
 //     writes (O / l, m + log2 l) partials to slot (pair + worker), a slot that
 //     is unique because along the unit sequence either the pair or the worker
