@@ -169,6 +169,24 @@ def test_decode_split_count_independence_and_determinism():
     assert torch.equal(c, c2)
 
 
+@pytest.mark.parametrize("batch", [1000, 2000])
+def test_decode_batch_over_one_scan_chunk(batch):
+    """More requests than one prologue scan chunk holds (the second pass then
+    scans every chunk that overlaps a CTA's workers instead of reusing the
+    first pass), plain and fused."""
+    rng = np.random.default_rng(batch)
+    lengths = [int(x) for x in rng.integers(1, 200, size=batch)]
+    step, data = _custom("decode", [L - 1 for L in lengths], lengths, 16, 8, seed=batch + 3)
+    g = GpuStep(step, data)
+    req = _sample(step, k=12, seed=batch)
+    out = g.store_decode()
+    assert mg.read_device_error() == 0
+    assert_matches_oracle(out, oracle_decode(step, data, requests=req), f"fused, batch {batch}")
+    out2 = g.decode()  # the pools now hold the stored tokens
+    assert mg.read_device_error() == 0
+    assert_matches_oracle(out2, oracle_decode(step, data, requests=req), f"plain, batch {batch}")
+
+
 def test_decode_with_larger_max_seq_len_hint():
     step, data = _custom("decode", [99, 5], [100, 6], 16, 8, seed=6)
     g = GpuStep(step, data)

@@ -129,6 +129,23 @@ def test_shared_prefix_workload_full_size():
     assert torch.isfinite(out.float()).all()
 
 
+@pytest.mark.parametrize("groups", [100, 150])
+def test_many_groups_cached_and_not(groups):
+    """Many small groups: up to 128 have their ranges and prefixes checked once
+    into shared memory, more are looked up in global memory; both give the
+    oracle's result (sampled requests)."""
+    rng = np.random.default_rng(groups)
+    lengths = [int(x) for x in 200 + rng.integers(1, 300, size=2 * groups)]
+    grp = [(2 * i, 2, 150 + (i % 40)) for i in range(groups)]
+    step, data = _grouped_case(lengths, grp, 16, 8, seed=620 + groups)
+    g = GpuStep(step, data)
+    g.store()
+    out = _run(g, step)
+    assert mg.read_device_error() == 0
+    req = sorted({0, 1, 2, 77, 128, 129, 2 * groups - 1} & set(range(step.batch)))
+    assert_matches_oracle(out, oracle_decode(step, data, requests=req), f"{groups} groups")
+
+
 def _run_fused(g: GpuStep, step, parts=0, group_first=None, prefix_len=None):
     gf = (step.group_first if group_first is None else group_first).cuda()
     pl = (step.prefix_len if prefix_len is None else prefix_len).cuda()
