@@ -393,6 +393,22 @@ def test_extend_full_size_sampled():
     assert torch.isfinite(out.float()).all()
 
 
+@pytest.mark.parametrize("cached,seq,hq,hkv", [
+    ([30000, 5], [30070, 40], 16, 8),     # a chunk after a 30k-token history: 235 KV tiles an item
+    ([0, 100], [2048, 101], 32, 4),       # a 2048-token fresh prompt (many q blocks) beside one token
+    ([16000], [16070], 64, 8),            # group 8: 16 tokens a Q tile, ragged last q block
+])
+def test_extend_long_items(cached, seq, hq, hkv):
+    """Items far longer than the chunked-prefill workload's: long KV loops per
+    item and prompts of many q blocks, checked against the oracle."""
+    step, data = _custom("extend", cached, seq, hq, hkv, seed=sum(seq) % 1000 + 5)
+    g = GpuStep(step, data)
+    g.store()
+    out = g.extend()
+    assert mg.read_device_error() == 0
+    assert_matches_oracle(out, oracle_extend(step, data), f"extend long {cached}->{seq} hq {hq} hkv {hkv}")
+
+
 def test_extend_single_token_matches_decode_kernel():
     lengths = [5, 64, 129, 300]
     step, data = _custom("decode", [L - 1 for L in lengths], lengths, 16, 8, seed=12)
