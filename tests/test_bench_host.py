@@ -67,3 +67,42 @@ def test_reference_arm_line_on_a_small_workload(monkeypatch, capsys):
     assert line["impl"] == "reference" and line["unit"] == "GB/s" and line["value"] > 0
     assert line["config"]["workload"] == "tiny_decode" and line["cpu_baseline"]["cores"] == 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["steps"] == 2 and line["warmup"] == 1
+
+
+def test_committed_bench_lines_follow_the_contract():
+    """Every bench line committed under profiles/ carries the keys the bench
+    contract asks for, and its traffic figure is the one profiles/traffic.json
+    holds for its workload at the same kernel-source digest (never a figure
+    taken on other kernels)."""
+    import glob
+    import json
+    import os
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    traffic = json.load(open(os.path.join(root, "profiles", "traffic.json")))
+    paths = sorted(glob.glob(os.path.join(root, "profiles", "bench_*.json")))
+    assert paths
+    for path in paths:
+        line = json.loads(open(path).read())
+        for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                    "scaling", "vs_baseline", "dtype", "data", "config", "e2e", "cpu_baseline"):
+            assert key in line, (path, key)
+        assert line["warmup"] >= 3 and line["steps"] >= 1, path
+        e2e = line["e2e"]
+        assert {"value", "unit"} <= set(e2e), path
+        cpu = line["cpu_baseline"]
+        assert {"value", "unit", "cores", "kind", "sample"} <= set(cpu) and cpu["kind"] == "oracle", path
+        if line.get("impl") == "reference":
+            continue
+        assert "workload" in line["config"], path
+        assert line["gpu_launches"] > 0, path
+        clocks = line["clocks"]
+        assert {"sm_mhz", "sm_max_mhz", "reasons"} <= set(clocks), path
+        assert not {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"} & set(clocks["reasons"]), path
+        assert {"h2d_bytes_per_step", "d2h_bytes_per_step"} <= set(e2e), path
+        roof = line["roofline"]
+        assert {"bound", "achieved", "peak", "unit", "frac", "traffic"} <= set(roof), path
+        assert abs(roof["frac"] - roof["achieved"] / roof["peak"]) < 1e-3, path
+        if roof["traffic"] is not None:
+            key = line["config"]["workload"] + (":plain" if "plain" in os.path.basename(path) else "")
+            assert traffic[key]["source_digest"] == line["kernel_source_digest"], path
+            assert traffic[key]["dram_bytes_per_launch"] == roof["traffic"], path
